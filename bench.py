@@ -1,0 +1,470 @@
+#!/usr/bin/env python3
+"""Benchmark: MoE-layer tokens/s on B200 (route -> layout -> dispatch -> expert FFN -> combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
+
+One step = one full layer forward (every stage) over one batch of T tokens.
+Default workload: the Mixtral-shaped layer (T=4096, d=4096, E=8, top-2,
+f=14336, bf16 router linear, softmax top-2 renormalised), synthetic seeded
+inputs.  Multi-GPU runs are replicas (one process per GPU, each with its own
+token batch and a full copy of the weights, no data-path collective): weak
+scaling, value = all ranks' tokens / the slowest rank's time.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+(the only reference this method has) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from combine_moe_route_14_b200 import inputs as I  # noqa: E402
+
+METRIC = "MoE-layer tokens/s on 1 B200; HBM GB/s (dispatch/combine), TC util (GEMM)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# sampled tokens per oracle call: cpu_baseline leg / reference arm
+ORACLE_SAMPLE = {"mixtral": (256, 32), "skewed_top1": (256, 32), "skewed_top1_harsh": (256, 32),
+                 "fine_grained": (32, 8), "tiny": (256, 256), "decode_16": (16, 16),
+                 "decode_64": (64, 32), "decode_256": (256, 32), "decode_1024": (256, 32)}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ----------------------------------------------------------------------------
+# bookkeeping: algorithmic bytes / flops per stage
+# ----------------------------------------------------------------------------
+def stage_model(cfg, counts=None):
+    """Algorithmic work of each stage for one forward (bytes moved that the math needs)."""
+    T, d, E, k, f, R = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.R
+    E_act = E if counts is None else int((np.asarray(counts) > 0).sum())
+    m = {}
+    if cfg.router == "weights":
+        m["router_logits"] = {"bytes": T * d * 2 + E * d * 2 + T * E * 4, "flops": 2 * T * d * E}
+    m["route"] = {"bytes": T * E * 4 + R * 8}
+    m["layout"] = {"bytes": R * 4 + R * 8 + (2 * E + 1) * 4}
+    m["dispatch"] = {"bytes": T * d * 2 + R * d * 2 + R * 4}
+    m["gemm1"] = {"flops": 2 * R * d * f, "bytes": E_act * f * d * 2 + R * d * 2 + R * f * 2}
+    m["gemm2"] = {"flops": 2 * R * d * f, "bytes": E_act * d * f * 2 + R * f * 2 + R * d * 2}
+    m["combine"] = {"bytes": R * d * 2 + R * 8 + T * d * 2}
+    return m
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return {k: float(j[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it still matches the source.
+
+    profiles/<kernel>_<workload>.md carries 'traffic_bytes_per_launch:' and
+    'source_sha256:' lines; a changed kernel source voids the figure.
+    """
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    src = os.path.join(ROOT, "combine_moe_route_14_b200", "csrc", "grouped_gemm.cu")
+    if not os.path.exists(path) or not os.path.exists(src):
+        return None
+    text = open(path).read()
+    mt = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    ms = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    if not mt or not ms:
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != ms.group(1):
+        return None
+    return float(mt.group(1))
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                clk, cmax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            mx = cmax
+            active = parts[4]
+            if clk > 0:
+                sm.append(clk)
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+            del active
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline leg and the reference arm)
+# ----------------------------------------------------------------------------
+def _bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def host_inputs(cfg, seed):
+    """Inputs as host arrays (bf16 bits / fp32) for the oracle; weights made on a GPU if present."""
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = I.make_layer_inputs(cfg, seed, device=dev)
+    out = {"X": _bits(inp["X"]), "W1": _bits(inp["W1"]), "W2": _bits(inp["W2"]),
+           "logits": None if inp["logits"] is None else inp["logits"].numpy(),
+           "Wr": None if inp["Wr"] is None else _bits(inp["Wr"])}
+    del inp
+    return out
+
+
+def oracle_step(O, cfg, h, S):
+    """The oracle over a bounded sample: the first S tokens of the batch, all stages."""
+    X = h["X"][:S]
+    L = None if h["logits"] is None else h["logits"][:S]
+    return O.layer_forward(X, h["W1"], h["W2"], cfg.k, cfg.score, cfg.renormalize, logits=L,
+                           Wr_bits=h["Wr"])
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def time_oracle(cfg, h, S, reps=1):
+    from oracle import moe_oracle as O
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle_step(O, cfg, h, S)
+    dt = time.perf_counter() - t0
+    return S * reps / dt, dt
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+def run_ours(args, cfg, rank, world, local_rank):
+    import combine_moe_route_14_b200 as moe
+    from combine_moe_route_14_b200 import build as B
+
+    if rank == 0:
+        B.build()
+    if world > 1:
+        torch.distributed.barrier()
+    moe.load_library()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    inp = I.make_layer_inputs(cfg, args.seed, device=dev)  # weights: same on every rank
+    X_host = inp["X"] if rank == 0 else I.random_bf16((cfg.T, cfg.d), args.seed + 1000 * rank, "X")
+    X = X_host.to(dev)
+    logits = inp["logits"].to(dev) if inp["logits"] is not None else None
+    Wr = inp["Wr"].to(dev) if inp["Wr"] is not None else None
+    layer = moe.MoeLayer(inp["W1"], inp["W2"], cfg.k, cfg.score, cfg.renormalize, Wr=Wr)
+    Y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
+    counts = torch.empty((cfg.E,), dtype=torch.int32, device=dev)
+    ws = layer.workspace(cfg.T)
+
+    def step():
+        layer(X, logits=logits, Y=Y, counts_out=counts)
+
+    def sync_all():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    sync_all()
+    bits = moe.moe_device_status(clear=True)
+    if bits:
+        raise RuntimeError(f"device status bits {bits} after warm-up")
+
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.__enter__()
+    try:
+        # ---- value: K whole-layer forwards, inputs resident in HBM
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        sync_all()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        sync_all()
+        t_ms = max_over_ranks(e0.elapsed_time(e1))
+
+        # ---- per-stage times: the same kernels, launched stage by stage with events between
+        stage_names = (["router_logits"] if Wr is not None else []) + [
+            "route", "layout", "dispatch", "gemm1", "gemm2", "combine"]
+        R = cfg.R
+        L_buf = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev) if Wr is not None else logits
+        idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
+        g = torch.empty((cfg.T, cfg.k), dtype=torch.float32, device=dev)
+        offs = torch.empty((cfg.E + 1,), dtype=torch.int32, device=dev)
+        row_of = torch.empty((R,), dtype=torch.int32, device=dev)
+        src_of = torch.empty((R,), dtype=torch.int32, device=dev)
+        lws = torch.empty(max(16, moe.moe_layout_workspace_size(cfg.T, cfg.E, cfg.k)),
+                          dtype=torch.uint8, device=dev)
+        Xe = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=dev)
+        H = torch.empty((R, cfg.f), dtype=torch.bfloat16, device=dev)
+        Ye = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=dev)
+        fns = {
+            "router_logits": lambda: moe.moe_router_logits(X, Wr, logits=L_buf),
+            "route": lambda: moe.moe_route(L_buf, cfg.k, cfg.score, cfg.renormalize, idx, g),
+            "layout": lambda: moe.moe_layout(idx, cfg.E, counts, offs, row_of, src_of, lws),
+            "dispatch": lambda: moe.moe_dispatch(X, src_of, cfg.k, Xe),
+            "gemm1": lambda: moe.moe_expert_gemm(Xe, offs, inp["W1"], True, H),
+            "gemm2": lambda: moe.moe_expert_gemm(H, offs, inp["W2"], False, Ye),
+            "combine": lambda: moe.moe_combine(Ye, row_of, g, Y),
+        }
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stage_names) + 1)]
+               for _ in range(args.steps)]
+        sync_all()
+        for s in range(args.steps):
+            evs[s][0].record(stream)
+            for i, n in enumerate(stage_names):
+                fns[n]()
+                evs[s][i + 1].record(stream)
+        sync_all()
+        stage_ms = {n: float(np.mean([evs[s][i].elapsed_time(evs[s][i + 1])
+                                      for s in range(args.steps)]))
+                    for i, n in enumerate(stage_names)}
+        staged_total_ms = sum(stage_ms.values())
+
+        # ---- e2e: host buffers in, host buffer out, copies inside the timed region
+        X_pin = X_host.pin_memory()
+        L_pin = inp["logits"].pin_memory() if logits is not None else None
+        Y_pin = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16).pin_memory()
+        X_dev2 = torch.empty_like(X)
+        L_dev2 = torch.empty_like(logits) if logits is not None else None
+        h2d = X_pin.numel() * 2 + (L_pin.numel() * 4 if L_pin is not None else 0)
+        d2h = Y_pin.numel() * 2
+
+        def e2e_step():
+            X_dev2.copy_(X_pin, non_blocking=True)
+            if L_pin is not None:
+                L_dev2.copy_(L_pin, non_blocking=True)
+            layer(X_dev2, logits=L_dev2, Y=Y, counts_out=counts)
+            Y_pin.copy_(Y, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        sync_all()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        f1.record(stream)
+        sync_all()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    finally:
+        if sampler:
+            sampler.__exit__(None, None, None)
+
+    bits = moe.moe_device_status(clear=True)
+    if bits:
+        raise RuntimeError(f"device status bits {bits} after the timed region")
+
+    # ---- roofline of the dominant kernel
+    counts_h = counts.cpu().numpy()
+    model = stage_model(cfg, counts_h)
+    dom = max(stage_ms, key=lambda n: stage_ms[n])
+    peaks, peak_src = load_peaks()
+    long_region = (t_ms + staged_total_ms * args.steps) > 1000.0
+    per = model[dom]
+    dur_s = stage_ms[dom] / 1e3
+    if "flops" in per and per["flops"] / max(per["bytes"], 1) > (
+            peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9):
+        peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": per["flops"] / dur_s / 1e12, "peak": peak,
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": per["bytes"] / dur_s / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_src} ({'sustained' if long_region and roof['bound'] == 'tensor' else 'burst'})"
+    kname = {"gemm1": "grouped_gemm_gelu", "gemm2": "grouped_gemm"}.get(dom, dom)
+    tr = ncu_traffic(kname, cfg.name)
+    roof["traffic"] = tr
+    roof["algorithmic_bytes"] = per["bytes"]
+
+    stages = {}
+    for n, ms in stage_ms.items():
+        st = {"us": ms * 1e3}
+        if "bytes" in model[n]:
+            st["GB/s"] = model[n]["bytes"] / (ms / 1e3) / 1e9
+            st["hbm_frac"] = st["GB/s"] / peaks["hbm_gbs"]
+        if "flops" in model[n]:
+            st["TFLOP/s"] = model[n]["flops"] / (ms / 1e3) / 1e12
+        stages[n] = st
+
+    total_tokens = cfg.T * args.steps * world
+    value = total_tokens / (t_ms / 1e3)
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                   "f": cfg.f, "router": cfg.router, "score": cfg.score,
+                   "renormalize": cfg.renormalize, "tokens_per_gpu": cfg.T,
+                   "parallelism": f"replicas x{world} (no collective)",
+                   "l2": f"inputs larger than L2: each step streams "
+                         f"{2 * cfg.E * cfg.d * cfg.f * 2 / 1e9:.2f} GB of expert weights"},
+        "roofline": roof,
+        "stages": stages,
+        "expert_counts": {"max": int(counts_h.max()), "mean": float(counts_h.mean()),
+                          "min": int(counts_h.min())},
+        "e2e": {"value": cfg.T * args.steps * world / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * moe.moe_kernel_launches_per_forward(
+            moe.make_desc(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.score, cfg.renormalize),
+            Wr is not None),
+        "clocks": sampler.summary() if sampler else None,
+    }
+    del X, logits, Wr, layer, inp, ws, Xe, H, Ye
+    torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="mixtral", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = I.workload(args.workload)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        S_base, S = ORACLE_SAMPLE.get(cfg.name, (64, 16))
+        h = host_inputs(cfg, args.seed)
+        for _ in range(args.warmup):
+            time_oracle(cfg, h, S)
+        v, dt = time_oracle(cfg, h, S, reps=args.steps)
+        cores = blas_threads()
+        res = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+               "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+               "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+               "impl": "reference",
+               "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+                          "f": cfg.f, "router": cfg.router, "score": cfg.score,
+                          "renormalize": cfg.renormalize},
+               "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"first {S} of the {cfg.T} tokens per step, all stages"},
+               "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
+                       "d2h_bytes_per_step": 0}}
+        print(json.dumps(res), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, cfg, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            S_base, _ = ORACLE_SAMPLE.get(cfg.name, (64, 16))
+            h = host_inputs(cfg, args.seed)
+            v, dt = time_oracle(cfg, h, S_base)
+            res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(),
+                                   "kind": "oracle",
+                                   "sample": f"first {S_base} of the {cfg.T} tokens, all stages, "
+                                             f"one run ({dt:.1f} s)"}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

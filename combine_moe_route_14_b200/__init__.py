@@ -1,1 +1,326 @@
-"""B200-native MoE layer: route -> layout -> dispatch -> expert FFN -> combine."""
+"""B200-native MoE layer: route -> layout -> dispatch -> expert FFN -> combine.
+
+A thin Python binding over the C ABI of ``libmoe.so`` (``include/moe.h``).
+Functions carry the C names; they check tensor dtypes, shapes and devices,
+allocate outputs with torch when none are given, and pass device pointers
+and the current CUDA stream.  Every step of the layer runs in the library's
+CUDA kernels: there is no CPU or PyTorch fallback, and a missing library is
+an error.
+
+Build the library first:  ``python -m combine_moe_route_14_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "MoeError", "LayerDesc", "load_library", "library_path",
+    "moe_router_logits", "moe_route", "moe_layout_workspace_size", "moe_layout",
+    "moe_dispatch", "moe_expert_gemm", "moe_expert_ffn", "moe_combine",
+    "moe_workspace_size", "moe_layer_forward", "moe_device_status",
+    "moe_kernel_launches_per_forward", "MoeLayer", "SCORES",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libmoe.so")
+_lib = None
+_lock = threading.Lock()
+
+SCORES = {"softmax": 0, "sigmoid": 1}
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
+          4: "MOE_ERR_DEVICE"}
+DEV_BITS = {1: "MOE_DEV_BAD_EXPERT_ID", 2: "MOE_DEV_TIMEOUT", 4: "MOE_DEV_BAD_ROW"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class LayerDesc(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("f", ctypes.c_int32), ("score", ctypes.c_int32),
+                ("renormalize", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int32
+_SIG = {
+    "moe_router_logits": ([_P, _P, _I, _I, _I, _P, _P], ctypes.c_int),
+    "moe_route": ([_P, _I, _I, _I, _I, _I, _P, _P, _P], ctypes.c_int),
+    "moe_layout_workspace_size": ([_I, _I, _I], ctypes.c_size_t),
+    "moe_layout": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_dispatch": ([_P, _P, _I, _I, _I, _P, _P], ctypes.c_int),
+    "moe_expert_gemm": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
+    "moe_expert_ffn": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P], ctypes.c_int),
+    "moe_combine": ([_P, _P, _P, _I, _I, _I, _P, _P], ctypes.c_int),
+    "moe_workspace_size": ([ctypes.POINTER(LayerDesc)], ctypes.c_size_t),
+    "moe_layer_forward": ([ctypes.POINTER(LayerDesc), _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                           ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_last_error_string": ([], ctypes.c_char_p),
+    "moe_device_status": ([ctypes.POINTER(ctypes.c_uint32), _I], ctypes.c_int),
+    "moe_kernel_launches_per_forward": ([ctypes.POINTER(LayerDesc), _I], ctypes.c_int32),
+}
+
+
+def load_library():
+    """Load libmoe.so (raises if it has not been built: there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise MoeError(3, f"{_LIB_PATH} is missing; build it with "
+                                  "`python -m combine_moe_route_14_b200.build`")
+            lib = ctypes.CDLL(_LIB_PATH)
+            for name, (args, res) in _SIG.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = lib
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        msg = load_library().moe_last_error_string().decode(errors="replace")
+        raise MoeError(status, msg)
+
+
+def _stream(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t, name, dtype, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must live on a CUDA device")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _out(t, name, dtype, shape, device):
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    return _need(t, name, dtype, shape, device)
+
+
+def _score(score) -> int:
+    return SCORES[score] if isinstance(score, str) else int(score)
+
+
+# ----------------------------------------------------------------------------
+# stages
+# ----------------------------------------------------------------------------
+def moe_router_logits(X, Wr, logits=None, stream=None):
+    lib = load_library()
+    T, d = X.shape
+    E = Wr.shape[0]
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (T, d))
+    _need(Wr, "Wr", torch.bfloat16, (E, d), dev)
+    logits = _out(logits, "logits", torch.float32, (T, E), dev)
+    _check(lib.moe_router_logits(_ptr(X), _ptr(Wr), T, d, E, _ptr(logits), _stream(stream, dev)))
+    return logits
+
+
+def moe_route(logits, k, score="softmax", renormalize=True, topk_idx=None, gates=None,
+              stream=None):
+    lib = load_library()
+    T, E = logits.shape
+    dev = logits.device
+    _need(logits, "logits", torch.float32, (T, E))
+    topk_idx = _out(topk_idx, "topk_idx", torch.int32, (T, k), dev)
+    gates = _out(gates, "gates", torch.float32, (T, k), dev)
+    _check(lib.moe_route(_ptr(logits), T, E, k, _score(score), int(bool(renormalize)),
+                         _ptr(topk_idx), _ptr(gates), _stream(stream, dev)))
+    return topk_idx, gates
+
+
+def moe_layout_workspace_size(T, E, k) -> int:
+    return int(load_library().moe_layout_workspace_size(T, E, k))
+
+
+def moe_layout(topk_idx, E, counts=None, offsets=None, row_of=None, src_of=None, ws=None,
+               stream=None):
+    lib = load_library()
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    R = T * k
+    counts = _out(counts, "counts", torch.int32, (E,), dev)
+    offsets = _out(offsets, "offsets", torch.int32, (E + 1,), dev)
+    row_of = _out(row_of, "row_of", torch.int32, (R,), dev)
+    src_of = _out(src_of, "src_of", torch.int32, (R,), dev)
+    need = moe_layout_workspace_size(T, E, k)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _check(lib.moe_layout(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(row_of),
+                          _ptr(src_of), _ptr(ws), ws.numel(), _stream(stream, dev)))
+    return counts, offsets, row_of, src_of
+
+
+def moe_dispatch(X, src_of, k, Xe=None, stream=None):
+    lib = load_library()
+    T, d = X.shape
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (T, d))
+    _need(src_of, "src_of", torch.int32, (T * k,), dev)
+    Xe = _out(Xe, "Xe", torch.bfloat16, (T * k, d), dev)
+    _check(lib.moe_dispatch(_ptr(X), _ptr(src_of), T, d, k, _ptr(Xe), _stream(stream, dev)))
+    return Xe
+
+
+def moe_expert_gemm(A, offsets, W, gelu, out=None, stream=None):
+    lib = load_library()
+    R, K = A.shape
+    E, N, K2 = W.shape
+    dev = A.device
+    if K2 != K:
+        raise ValueError("W's last dim must equal A's")
+    _need(A, "A", torch.bfloat16, (R, K))
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(W, "W", torch.bfloat16, (E, N, K), dev)
+    out = _out(out, "out", torch.bfloat16, (R, N), dev)
+    _check(lib.moe_expert_gemm(_ptr(A), _ptr(offsets), _ptr(W), E, R, N, K, int(bool(gelu)),
+                               _ptr(out), _stream(stream, dev)))
+    return out
+
+
+def moe_expert_ffn(Xe, offsets, W1, W2, H=None, Ye=None, stream=None):
+    lib = load_library()
+    R, d = Xe.shape
+    E, f, _ = W1.shape
+    dev = Xe.device
+    _need(Xe, "Xe", torch.bfloat16, (R, d))
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(W1, "W1", torch.bfloat16, (E, f, d), dev)
+    _need(W2, "W2", torch.bfloat16, (E, d, f), dev)
+    H = _out(H, "H", torch.bfloat16, (R, f), dev)
+    Ye = _out(Ye, "Ye", torch.bfloat16, (R, d), dev)
+    _check(lib.moe_expert_ffn(_ptr(Xe), _ptr(offsets), _ptr(W1), _ptr(W2), E, R, d, f, _ptr(H),
+                              _ptr(Ye), _stream(stream, dev)))
+    return H, Ye
+
+
+def moe_combine(Ye, row_of, gates, Y=None, stream=None):
+    lib = load_library()
+    T, k = gates.shape
+    R, d = Ye.shape
+    dev = Ye.device
+    if R != T * k:
+        raise ValueError("Ye must have T*k rows")
+    _need(Ye, "Ye", torch.bfloat16, (R, d))
+    _need(row_of, "row_of", torch.int32, (R,), dev)
+    _need(gates, "gates", torch.float32, (T, k), dev)
+    Y = _out(Y, "Y", torch.bfloat16, (T, d), dev)
+    _check(lib.moe_combine(_ptr(Ye), _ptr(row_of), _ptr(gates), T, d, k, _ptr(Y),
+                           _stream(stream, dev)))
+    return Y
+
+
+# ----------------------------------------------------------------------------
+# whole layer
+# ----------------------------------------------------------------------------
+def make_desc(T, d, E, k, f, score="softmax", renormalize=True) -> LayerDesc:
+    return LayerDesc(T, d, E, k, f, _score(score), int(bool(renormalize)), 0)
+
+
+def moe_workspace_size(desc: LayerDesc) -> int:
+    return int(load_library().moe_workspace_size(ctypes.byref(desc)))
+
+
+def moe_kernel_launches_per_forward(desc: LayerDesc, with_router: bool) -> int:
+    return int(load_library().moe_kernel_launches_per_forward(ctypes.byref(desc),
+                                                              int(bool(with_router))))
+
+
+def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=None, Wr=None,
+                      Y=None, topk_idx_out=None, gates_out=None, counts_out=None, ws=None,
+                      stream=None):
+    lib = load_library()
+    T, d = X.shape
+    E, f, _ = W1.shape
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (T, d))
+    _need(W1, "W1", torch.bfloat16, (E, f, d), dev)
+    _need(W2, "W2", torch.bfloat16, (E, d, f), dev)
+    if logits is not None:
+        _need(logits, "logits", torch.float32, (T, E), dev)
+    if Wr is not None:
+        _need(Wr, "Wr", torch.bfloat16, (E, d), dev)
+    Y = _out(Y, "Y", torch.bfloat16, (T, d), dev)
+    if topk_idx_out is not None:
+        _need(topk_idx_out, "topk_idx_out", torch.int32, (T, k), dev)
+    if gates_out is not None:
+        _need(gates_out, "gates_out", torch.float32, (T, k), dev)
+    if counts_out is not None:
+        _need(counts_out, "counts_out", torch.int32, (E,), dev)
+    desc = make_desc(T, d, E, k, f, score, renormalize)
+    if ws is None:
+        ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _check(lib.moe_layer_forward(ctypes.byref(desc), _ptr(X), _ptr(logits), _ptr(Wr), _ptr(W1),
+                                 _ptr(W2), _ptr(Y), _ptr(topk_idx_out), _ptr(gates_out),
+                                 _ptr(counts_out), _ptr(ws), ws.numel(), _stream(stream, dev)))
+    return Y
+
+
+def moe_device_status(clear: bool = True) -> int:
+    """Synchronise the current device and return its sticky MOE_DEV_* bits."""
+    lib = load_library()
+    bits = ctypes.c_uint32(0)
+    st = lib.moe_device_status(ctypes.byref(bits), int(bool(clear)))
+    if st not in (0, 4):
+        _check(st)
+    return int(bits.value)
+
+
+class MoeLayer:
+    """A layer's weights plus a reusable workspace (allocation stays outside the call)."""
+
+    def __init__(self, W1, W2, k, score="softmax", renormalize=True, Wr=None):
+        self.W1, self.W2, self.Wr = W1, W2, Wr
+        self.k, self.score, self.renormalize = k, score, renormalize
+        self.E, self.f, self.d = W1.shape
+        self._ws = None
+
+    def workspace(self, T):
+        desc = make_desc(T, self.d, self.E, self.k, self.f, self.score, self.renormalize)
+        need = max(moe_workspace_size(desc), 16)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=self.W1.device)
+        return self._ws
+
+    def __call__(self, X, logits=None, Y=None, topk_idx_out=None, gates_out=None,
+                 counts_out=None, stream=None):
+        return moe_layer_forward(X, self.W1, self.W2, self.k, self.score, self.renormalize,
+                                 logits=logits, Wr=None if logits is not None else self.Wr,
+                                 Y=Y, topk_idx_out=topk_idx_out, gates_out=gates_out,
+                                 counts_out=counts_out, ws=self.workspace(X.shape[0]),
+                                 stream=stream)

@@ -1,0 +1,373 @@
+// The C ABI of libmoe.so (declared in include/moe.h): argument validation,
+// per-device state, workspace layout and the fused layer forward.
+#include <cuda_runtime.h>
+
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "launch.h"
+
+// Sticky per-device status word set by kernels (MOE_DEV_* bits).
+__device__ uint32_t g_moe_device_status;
+
+namespace moe {
+namespace {
+
+thread_local std::string g_last_error;
+
+moe_status fail(moe_status s, const std::string& msg) {
+  g_last_error = msg;
+  return s;
+}
+
+moe_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOE_ERR_CUDA, std::string(where) + ": " + cudaGetErrorName(e) + " (" +
+                                cudaGetErrorString(e) + ")");
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
+cudaError_t g_dev_err[kMaxDevices];
+
+}  // namespace
+
+const DeviceInfo* current_device_info(std::string* err) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    *err = std::string("cudaGetDevice: ") + cudaGetErrorString(e);
+    return nullptr;
+  }
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = "device ordinal out of range";
+    return nullptr;
+  }
+  std::call_once(g_dev_once[dev], [dev] {
+    DeviceInfo& d = g_dev[dev];
+    d.device = dev;
+    cudaError_t e1 = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    void* p = nullptr;
+    cudaError_t e2 = cudaGetSymbolAddress(&p, g_moe_device_status);
+    d.status = static_cast<uint32_t*>(p);
+    g_dev_err[dev] = e1 != cudaSuccess ? e1 : e2;
+  });
+  if (g_dev_err[dev] != cudaSuccess) {
+    *err = std::string("device set-up: ") + cudaGetErrorString(g_dev_err[dev]);
+    return nullptr;
+  }
+  return &g_dev[dev];
+}
+
+}  // namespace moe
+
+using moe::cuda_fail;
+using moe::fail;
+
+namespace {
+
+moe_status get_dev(const moe::DeviceInfo** out) {
+  std::string err;
+  *out = moe::current_device_info(&err);
+  if (!*out) return fail(MOE_ERR_CUDA, err);
+  return MOE_OK;
+}
+
+moe_status check_ET(int32_t T, int32_t E, int32_t k) {
+  if (T < 0) return fail(MOE_ERR_INVALID_ARG, "T must be >= 0");
+  if (E < 1) return fail(MOE_ERR_INVALID_ARG, "E must be >= 1");
+  if (k < 1 || k > E) return fail(MOE_ERR_INVALID_ARG, "k must be in [1, E]");
+  if (E > moe::kMaxExperts) return fail(MOE_ERR_UNSUPPORTED, "E > 1024 is not supported");
+  if (k > moe::kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k > 16 is not supported");
+  if ((int64_t)T * k >= (1ll << 30)) return fail(MOE_ERR_UNSUPPORTED, "T*k must be < 2^30");
+  return MOE_OK;
+}
+
+moe_status check_dim(int32_t v, const char* name) {
+  if (v < 1) return fail(MOE_ERR_INVALID_ARG, std::string(name) + " must be >= 1");
+  if (v % 8) return fail(MOE_ERR_UNSUPPORTED, std::string(name) + " must be a multiple of 8");
+  return MOE_OK;
+}
+
+moe_status check_ptr(const void* p, const char* name) {
+  if (!p) return fail(MOE_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  if (!moe::aligned16(p)) return fail(MOE_ERR_INVALID_ARG, std::string(name) + " is not 16-byte aligned");
+  return MOE_OK;
+}
+
+moe_status check_ptr4(const void* p, const char* name) {
+  if (!p) return fail(MOE_ERR_INVALID_ARG, std::string(name) + " is NULL");
+  if (reinterpret_cast<uintptr_t>(p) & 3u)
+    return fail(MOE_ERR_INVALID_ARG, std::string(name) + " is not 4-byte aligned");
+  return MOE_OK;
+}
+
+#define MOE_TRY(x)                \
+  do {                            \
+    moe_status _s = (x);          \
+    if (_s != MOE_OK) return _s;  \
+  } while (0)
+
+#define MOE_CUDA(x, where)                        \
+  do {                                            \
+    cudaError_t _e = (x);                         \
+    if (_e != cudaSuccess) return cuda_fail(_e, where); \
+  } while (0)
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+// Workspace of the fused forward: sub-buffers, each 256-byte aligned.
+struct LayerWs {
+  size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, total;
+};
+
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+LayerWs layer_ws(const moe_layer_desc& d) {
+  LayerWs w;
+  const size_t T = (size_t)d.T, R = (size_t)d.T * d.k;
+  size_t o = 0;
+  w.logits = o;  o += up256(T * d.E * sizeof(float));
+  w.idx = o;     o += up256(R * sizeof(int32_t));
+  w.gates = o;   o += up256(R * sizeof(float));
+  w.counts = o;  o += up256((size_t)d.E * sizeof(int32_t));
+  w.offsets = o; o += up256((size_t)(d.E + 1) * sizeof(int32_t));
+  w.row_of = o;  o += up256(R * sizeof(int32_t));
+  w.src_of = o;  o += up256(R * sizeof(int32_t));
+  w.layout = o;  o += up256(moe::layout_workspace_bytes((int64_t)R, d.E));
+  w.Xe = o;      o += up256(R * d.d * 2);
+  w.H = o;       o += up256(R * d.f * 2);
+  w.Ye = o;      o += up256(R * d.d * 2);
+  w.total = o;
+  return w;
+}
+
+moe_status check_desc(const moe_layer_desc* desc) {
+  if (!desc) return fail(MOE_ERR_INVALID_ARG, "desc is NULL");
+  MOE_TRY(check_ET(desc->T, desc->E, desc->k));
+  MOE_TRY(check_dim(desc->d, "d"));
+  MOE_TRY(check_dim(desc->f, "f"));
+  if (desc->score != MOE_SCORE_SOFTMAX && desc->score != MOE_SCORE_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "unknown score");
+  if (desc->renormalize != 0 && desc->renormalize != 1)
+    return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
+  if (desc->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved must be 0");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_last_error_string(void) { return moe::g_last_error.c_str(); }
+
+moe_status moe_device_status(uint32_t* bits, int32_t clear) {
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(cudaDeviceSynchronize(), "cudaDeviceSynchronize");
+  uint32_t v = 0;
+  MOE_CUDA(cudaMemcpy(&v, dev->status, sizeof(v), cudaMemcpyDeviceToHost), "read status");
+  if (clear) MOE_CUDA(cudaMemset(dev->status, 0, sizeof(uint32_t)), "clear status");
+  if (bits) *bits = v;
+  if (v) return fail(MOE_ERR_DEVICE, "device status bits set: " + std::to_string(v));
+  return MOE_OK;
+}
+
+moe_status moe_router_logits(const void* X, const void* Wr, int32_t T, int32_t d, int32_t E,
+                             float* logits, void* stream) {
+  MOE_TRY(check_ET(T, E, 1));
+  MOE_TRY(check_dim(d, "d"));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr(X, "X"));
+  MOE_TRY(check_ptr(Wr, "Wr"));
+  MOE_TRY(check_ptr4(logits, "logits"));
+  MOE_CUDA(moe::launch_router_logits(X, Wr, T, d, E, logits, as_stream(stream)), "router_logits");
+  return MOE_OK;
+}
+
+moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
+                     int32_t renormalize, int32_t* topk_idx, float* gates, void* stream) {
+  MOE_TRY(check_ET(T, E, k));
+  if (score != MOE_SCORE_SOFTMAX && score != MOE_SCORE_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "unknown score");
+  if (renormalize != 0 && renormalize != 1)
+    return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr4(logits, "logits"));
+  MOE_TRY(check_ptr4(topk_idx, "topk_idx"));
+  MOE_TRY(check_ptr4(gates, "gates"));
+  MOE_CUDA(moe::launch_route(logits, T, E, k, score, renormalize, topk_idx, gates,
+                             as_stream(stream)),
+           "route");
+  return MOE_OK;
+}
+
+size_t moe_layout_workspace_size(int32_t T, int32_t E, int32_t k) {
+  if (T < 0 || E < 1 || k < 1) return 0;
+  return up256(moe::layout_workspace_bytes((int64_t)T * k, E));
+}
+
+moe_status moe_layout(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k, int32_t* counts,
+                      int32_t* offsets, int32_t* row_of, int32_t* src_of, void* ws,
+                      size_t ws_bytes, void* stream) {
+  MOE_TRY(check_ET(T, E, k));
+  MOE_TRY(check_ptr4(counts, "counts"));
+  MOE_TRY(check_ptr4(offsets, "offsets"));
+  const size_t need = moe_layout_workspace_size(T, E, k);
+  if (T > 0) {
+    MOE_TRY(check_ptr4(topk_idx, "topk_idx"));
+    MOE_TRY(check_ptr4(row_of, "row_of"));
+    MOE_TRY(check_ptr4(src_of, "src_of"));
+  }
+  if (ws_bytes < need) return fail(MOE_ERR_INVALID_ARG, "workspace too small");
+  if (need > 0) MOE_TRY(check_ptr(ws, "ws"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {  // every expert empty
+    MOE_CUDA(cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), s), "memset counts");
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s), "memset offsets");
+    return MOE_OK;
+  }
+  MOE_CUDA(moe::launch_layout(topk_idx, T * k, E, counts, offsets, row_of, src_of, ws, *dev, s),
+           "layout");
+  return MOE_OK;
+}
+
+moe_status moe_dispatch(const void* X, const int32_t* src_of, int32_t T, int32_t d, int32_t k,
+                        void* Xe, void* stream) {
+  if (T < 0 || k < 1) return fail(MOE_ERR_INVALID_ARG, "need T >= 0 and k >= 1");
+  if (k > moe::kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k > 16 is not supported");
+  if ((int64_t)T * k >= (1ll << 30)) return fail(MOE_ERR_UNSUPPORTED, "T*k must be < 2^30");
+  MOE_TRY(check_dim(d, "d"));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr(X, "X"));
+  MOE_TRY(check_ptr4(src_of, "src_of"));
+  MOE_TRY(check_ptr(Xe, "Xe"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(moe::launch_dispatch(X, src_of, T, d, k, Xe, *dev, as_stream(stream)), "dispatch");
+  return MOE_OK;
+}
+
+moe_status moe_expert_gemm(const void* A, const int32_t* offsets, const void* W, int32_t E,
+                           int32_t R, int32_t N, int32_t K, int32_t gelu, void* out,
+                           void* stream) {
+  if (E < 1) return fail(MOE_ERR_INVALID_ARG, "E must be >= 1");
+  if (E > moe::kMaxExperts) return fail(MOE_ERR_UNSUPPORTED, "E > 1024 is not supported");
+  if (R < 0) return fail(MOE_ERR_INVALID_ARG, "R must be >= 0");
+  if (R >= (1 << 30)) return fail(MOE_ERR_UNSUPPORTED, "R must be < 2^30");
+  MOE_TRY(check_dim(N, "N"));
+  MOE_TRY(check_dim(K, "K"));
+  if ((int64_t)E * N >= (1ll << 31)) return fail(MOE_ERR_UNSUPPORTED, "E*N must be < 2^31");
+  if (gelu != 0 && gelu != 1) return fail(MOE_ERR_INVALID_ARG, "gelu must be 0 or 1");
+  if (R == 0) return MOE_OK;
+  MOE_TRY(check_ptr(A, "A"));
+  MOE_TRY(check_ptr4(offsets, "offsets"));
+  MOE_TRY(check_ptr(W, "W"));
+  MOE_TRY(check_ptr(out, "out"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  std::string err;
+  cudaError_t e = moe::launch_grouped_gemm(A, offsets, W, E, R, N, K, gelu != 0, out, *dev,
+                                           as_stream(stream), &err);
+  if (e != cudaSuccess) {
+    if (!err.empty()) return fail(MOE_ERR_CUDA, "expert_gemm: " + err);
+    return cuda_fail(e, "expert_gemm");
+  }
+  return MOE_OK;
+}
+
+moe_status moe_expert_ffn(const void* Xe, const int32_t* offsets, const void* W1, const void* W2,
+                          int32_t E, int32_t R, int32_t d, int32_t f, void* H, void* Ye,
+                          void* stream) {
+  MOE_TRY(moe_expert_gemm(Xe, offsets, W1, E, R, f, d, 1, H, stream));
+  return moe_expert_gemm(H, offsets, W2, E, R, d, f, 0, Ye, stream);
+}
+
+moe_status moe_combine(const void* Ye, const int32_t* row_of, const float* gates, int32_t T,
+                       int32_t d, int32_t k, void* Y, void* stream) {
+  if (T < 0 || k < 1) return fail(MOE_ERR_INVALID_ARG, "need T >= 0 and k >= 1");
+  if (k > moe::kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k > 16 is not supported");
+  if ((int64_t)T * k >= (1ll << 30)) return fail(MOE_ERR_UNSUPPORTED, "T*k must be < 2^30");
+  MOE_TRY(check_dim(d, "d"));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr(Ye, "Ye"));
+  MOE_TRY(check_ptr4(row_of, "row_of"));
+  MOE_TRY(check_ptr4(gates, "gates"));
+  MOE_TRY(check_ptr(Y, "Y"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(moe::launch_combine(Ye, row_of, gates, T, d, k, Y, *dev, as_stream(stream)), "combine");
+  return MOE_OK;
+}
+
+size_t moe_workspace_size(const moe_layer_desc* desc) {
+  if (check_desc(desc) != MOE_OK) return 0;
+  return layer_ws(*desc).total;
+}
+
+int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with_router) {
+  if (check_desc(desc) != MOE_OK || desc->T == 0) return 0;
+  // [router linear] + route + layout + dispatch + 2 GEMMs + combine
+  return (with_router ? 1 : 0) + 1 + moe::layout_kernel_count((int64_t)desc->T * desc->k) + 1 +
+         2 + 1;
+}
+
+moe_status moe_layer_forward(const moe_layer_desc* desc, const void* X, const float* logits,
+                             const void* Wr, const void* W1, const void* W2, void* Y,
+                             int32_t* topk_idx_out, float* gates_out, int32_t* counts_out,
+                             void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc d = *desc;
+  if ((logits == nullptr) == (Wr == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "give exactly one of logits and Wr");
+  if (d.T == 0) return MOE_OK;
+  if ((int64_t)d.E * d.f >= (1ll << 31) || (int64_t)d.E * d.d >= (1ll << 31))
+    return fail(MOE_ERR_UNSUPPORTED, "E*f and E*d must be < 2^31");
+  MOE_TRY(check_ptr(X, "X"));
+  if (logits) MOE_TRY(check_ptr4(logits, "logits"));
+  if (Wr) MOE_TRY(check_ptr(Wr, "Wr"));
+  MOE_TRY(check_ptr(W1, "W1"));
+  MOE_TRY(check_ptr(W2, "W2"));
+  MOE_TRY(check_ptr(Y, "Y"));
+  if (topk_idx_out) MOE_TRY(check_ptr4(topk_idx_out, "topk_idx_out"));
+  if (gates_out) MOE_TRY(check_ptr4(gates_out, "gates_out"));
+  if (counts_out) MOE_TRY(check_ptr4(counts_out, "counts_out"));
+  const LayerWs w = layer_ws(d);
+  if (ws_bytes < w.total) return fail(MOE_ERR_INVALID_ARG, "workspace too small");
+  MOE_TRY(check_ptr(ws, "ws"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  cudaStream_t s = as_stream(stream);
+  char* base = static_cast<char*>(ws);
+  float* L = logits ? const_cast<float*>(logits) : reinterpret_cast<float*>(base + w.logits);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+  float* gates = gates_out ? gates_out : reinterpret_cast<float*>(base + w.gates);
+  int32_t* counts = counts_out ? counts_out : reinterpret_cast<int32_t*>(base + w.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + w.offsets);
+  int32_t* row_of = reinterpret_cast<int32_t*>(base + w.row_of);
+  int32_t* src_of = reinterpret_cast<int32_t*>(base + w.src_of);
+  void* lws = base + w.layout;
+  void* Xe = base + w.Xe;
+  void* H = base + w.H;
+  void* Ye = base + w.Ye;
+  const int R = d.T * d.k;
+
+  if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, s), "router_logits");
+  MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, idx, gates, s), "route");
+  MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s), "layout");
+  MOE_CUDA(moe::launch_dispatch(X, src_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+  std::string err;
+  cudaError_t e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err);
+  if (e != cudaSuccess) return err.empty() ? cuda_fail(e, "gemm1") : fail(MOE_ERR_CUDA, "gemm1: " + err);
+  e = moe::launch_grouped_gemm(H, offsets, W2, d.E, R, d.d, d.f, false, Ye, *dev, s, &err);
+  if (e != cudaSuccess) return err.empty() ? cuda_fail(e, "gemm2") : fail(MOE_ERR_CUDA, "gemm2: " + err);
+  MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
+  return MOE_OK;
+}
+
+}  // extern "C"

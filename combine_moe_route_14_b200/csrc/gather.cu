@@ -1,0 +1,168 @@
+// Dispatch (token -> its k expert rows) and combine (gate-weighted sum of a
+// token's k expert rows).
+//
+// DySHARP review (marsggbo) §1: dispatch sends the same token data to each of
+// its k experts; combine reduces the k results into one.  ThunderEP PCIe
+// blog §1.1 and §2.1: the gate values weight the combine sum.
+//
+// Both are pure HBM streams of bf16 rows (d*2 bytes each): one warp moves one
+// row (dispatch) or produces one row (combine) with 16-byte vector accesses,
+// several loads in flight per lane before the dependent stores.  Grids are
+// sized to a multiple of the SM count and walk rows grid-stride.
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+constexpr int kGatherWarps = 8;  // warps per CTA
+constexpr int kCopyUnroll = 8;   // 16-byte vectors in flight per lane
+
+// Xe[r, :] = X[src_of[r] / k, :]
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    dispatch_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ src_of, int R,
+                    int k, int row_vecs, uint4* __restrict__ Xe, uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * kGatherWarps;
+  for (int r = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); r < R; r += nwarps) {
+    const int s = __ldg(src_of + r);
+    if (s < 0 || s >= R) {
+      if (lane == 0) flag_error(status, MOE_DEV_BAD_ROW);
+      continue;
+    }
+    const uint4* src = X + (size_t)(s / k) * row_vecs;
+    uint4* dst = Xe + (size_t)r * row_vecs;
+    for (int c0 = 0; c0 < row_vecs; c0 += 32 * kCopyUnroll) {
+      uint4 v[kCopyUnroll];
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_vecs) v[u] = ld_stream_v4(src + c);
+      }
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_vecs) dst[c] = v[u];
+      }
+    }
+  }
+}
+
+// Y[t, :] = bf16( sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :] ), fp32 sum in slot order.
+// kK > 0: k known at compile time; kK == 0: runtime k (<= kMaxTopK).
+template <int kK>
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    combine_kernel(const uint4* __restrict__ Ye, const int32_t* __restrict__ row_of,
+                   const float* __restrict__ gates, int T, int R, int k_rt, int row_vecs,
+                   uint4* __restrict__ Y, uint32_t* status) {
+  constexpr int kSlots = kK > 0 ? kK : kMaxTopK;
+  constexpr int kUnroll = kK > 0 ? (kK >= 4 ? 2 : 4) : 1;
+  const int k = kK > 0 ? kK : k_rt;
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * kGatherWarps;
+  for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
+    // lanes j < k fetch slot j's row and gate; broadcast below
+    int my_row = 0;
+    float my_gate = 0.f;
+    if (lane < k) {
+      my_row = __ldg(row_of + (size_t)t * k + lane);
+      my_gate = __ldg(gates + (size_t)t * k + lane);
+      if (my_row < 0 || my_row >= R) {
+        flag_error(status, MOE_DEV_BAD_ROW);
+        my_row = -1;
+      }
+    }
+    const bool bad = __any_sync(0xffffffffu, lane < k && my_row < 0);
+    if (bad) continue;
+    const uint4* src[kSlots];
+    float g[kSlots];
+#pragma unroll
+    for (int j = 0; j < kSlots; ++j) {
+      const int rj = __shfl_sync(0xffffffffu, my_row, j);
+      g[j] = __shfl_sync(0xffffffffu, my_gate, j);
+      src[j] = Ye + (size_t)rj * row_vecs;
+    }
+    uint4* dst = Y + (size_t)t * row_vecs;
+    for (int c0 = 0; c0 < row_vecs; c0 += 32 * kUnroll) {
+      uint4 v[kUnroll][kSlots];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int c = c0 + u * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < kSlots; ++j)
+          if (j < k && c < row_vecs) v[u][j] = ld_stream_v4(src[j] + c);
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c >= row_vecs) continue;
+        float acc[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+#pragma unroll
+        for (int j = 0; j < kSlots; ++j) {
+          if (j < k) {
+            const uint4 w = v[u][j];
+            acc[0] = fmaf(g[j], bf16_lo(w.x), acc[0]);
+            acc[1] = fmaf(g[j], bf16_hi(w.x), acc[1]);
+            acc[2] = fmaf(g[j], bf16_lo(w.y), acc[2]);
+            acc[3] = fmaf(g[j], bf16_hi(w.y), acc[3]);
+            acc[4] = fmaf(g[j], bf16_lo(w.z), acc[4]);
+            acc[5] = fmaf(g[j], bf16_hi(w.z), acc[5]);
+            acc[6] = fmaf(g[j], bf16_lo(w.w), acc[6]);
+            acc[7] = fmaf(g[j], bf16_hi(w.w), acc[7]);
+          }
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        dst[c] = o;
+      }
+    }
+  }
+}
+
+static int gather_grid(int rows, const DeviceInfo& dev) {
+  // up to 8 resident CTAs of 8 warps per SM; never more CTAs than rows need
+  const int need = (rows + kGatherWarps - 1) / kGatherWarps;
+  const int cap = dev.sm_count * 8;
+  return need < cap ? need : cap;
+}
+
+cudaError_t launch_dispatch(const void* X, const int32_t* src_of, int T, int d, int k, void* Xe,
+                            const DeviceInfo& dev, cudaStream_t stream) {
+  const int R = T * k;
+  if (R == 0) return cudaSuccess;
+  dispatch_kernel<<<gather_grid(R, dev), kGatherWarps * 32, 0, stream>>>(
+      static_cast<const uint4*>(X), src_of, R, k, d / 8, static_cast<uint4*>(Xe), dev.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* Ye, const int32_t* row_of, const float* gates, int T,
+                           int d, int k, void* Y, const DeviceInfo& dev, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const int grid = gather_grid(T, dev);
+  const uint4* ye = static_cast<const uint4*>(Ye);
+  uint4* y = static_cast<uint4*>(Y);
+  const int R = T * k;
+  switch (k) {
+    case 1:
+      combine_kernel<1><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      break;
+    case 2:
+      combine_kernel<2><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      break;
+    case 4:
+      combine_kernel<4><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      break;
+    case 8:
+      combine_kernel<8><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      break;
+    default:
+      combine_kernel<0><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,53 @@
+// Host-side launch wrappers of libmoe.so (internal; the public ABI is include/moe.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+namespace moe {
+
+// Limits checked by the ABI before any launch.
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxTopK = 16;
+
+// Per-device facts the launchers need, filled once per device.
+struct DeviceInfo {
+  int device = -1;
+  int sm_count = 0;
+  uint32_t* status = nullptr;  // device address of the sticky status word
+};
+
+// Returns the info of the current device, initialising it on first use
+// (cudaGetSymbolAddress, attribute queries).  nullptr on a CUDA error, with
+// the message in *err.
+const DeviceInfo* current_device_info(std::string* err);
+
+cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, int E, float* L,
+                                 cudaStream_t stream);
+
+cudaError_t launch_route(const float* L, int T, int E, int k, int score, int renormalize,
+                         int32_t* idx, float* gates, cudaStream_t stream);
+
+size_t layout_workspace_bytes(int64_t R, int E);
+// Number of kernels launch_layout issues for R slots.
+int layout_kernel_count(int64_t R);
+cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int32_t* offsets,
+                          int32_t* row_of, int32_t* src_of, void* ws, const DeviceInfo& dev,
+                          cudaStream_t stream);
+
+cudaError_t launch_dispatch(const void* X, const int32_t* src_of, int T, int d, int k, void* Xe,
+                            const DeviceInfo& dev, cudaStream_t stream);
+
+cudaError_t launch_combine(const void* Ye, const int32_t* row_of, const float* gates, int T,
+                           int d, int k, void* Y, const DeviceInfo& dev, cudaStream_t stream);
+
+// Grouped GEMM over per-expert row blocks (tcgen05 + TMA).  On a failure to
+// build the TMA descriptors, returns cudaErrorInvalidValue with *err set.
+cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const void* W, int E,
+                                int R, int N, int K, bool gelu, void* out,
+                                const DeviceInfo& dev, cudaStream_t stream, std::string* err);
+
+}  // namespace moe

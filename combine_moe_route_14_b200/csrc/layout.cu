@@ -1,0 +1,332 @@
+// Layout: per-expert histogram, exclusive scan and the logical -> layout table.
+//
+// DySHARP review (marsggbo) §3.1 item 3: the destination keeps an AL table
+// from the logical i-th token to its position in a dense per-expert tensor,
+// allocating layout blocks incrementally, and combine reads rows back through
+// the same table.  ThunderEP PCIe blog §2.2: tokens for the same expert are
+// grouped into one contiguous block.
+//
+// With R = T*k slots, slot i = t*k + j bound for expert e_i:
+//   counts[e]  = #{i : e_i = e},  offsets = exclusive scan of counts,
+//   row_of[i]  = offsets[e_i] + #{i' < i : e_i' = e_i},  src_of[row_of[i]] = i.
+// This is a stable counting sort of the slots by expert id.  It is
+// deterministic: ranks come from warp match/popc over items in order, never
+// from the order in which atomics land.
+//
+// Two paths:
+//  * R <= kSingleMax: one CTA does everything (one launch; decode sizes).
+//  * larger R: tiles of kTile slots.  Kernel 1 builds a block-level histogram
+//    per tile and adds it into counts.  Kernel 2 takes tiles in launch order
+//    (an atomic ticket), finds each tile's per-expert base with a decoupled
+//    look-back over the preceding tiles (Merrill & Garland, "Single-pass
+//    Parallel Prefix Scan with Decoupled Look-back", 2016), and scatters.
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+
+constexpr int kLayoutThreads = 512;                 // 16 warps
+constexpr int kLayoutWarps = kLayoutThreads / 32;
+constexpr int kTile = 8192;                          // slots per tile (multi-CTA path)
+constexpr int kSingleMax = 16384;                    // slots handled by the one-CTA path
+
+// Look-back status word: bits 31-30 = flag, bits 29-0 = count (R < 2^30).
+constexpr uint32_t kFlagAggregate = 1u << 30;
+constexpr uint32_t kFlagInclusive = 2u << 30;
+constexpr uint32_t kValueMask = (1u << 30) - 1u;
+
+// Reads the expert id of slot i (or -1 past the end / out of range).
+__device__ __forceinline__ int load_key(const int32_t* idx, int i, int end, int E,
+                                        uint32_t* status) {
+  if (i >= end) return -1;
+  const int e = __ldg(idx + i);
+  if (e < 0 || e >= E) {
+    flag_error(status, MOE_DEV_BAD_EXPERT_ID);
+    return -1;
+  }
+  return e;
+}
+
+// Per-warp histogram of the slots [begin, end) owned by this warp, walked in
+// 32-slot chunks.  warp_hist is this warp's row of E counters.
+__device__ __forceinline__ void warp_histogram(const int32_t* idx, int begin, int end, int E,
+                                               int* warp_hist, uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  for (int c = begin; c < end; c += 32) {
+    const int key = load_key(idx, c + lane, end, E, status);
+    const uint32_t peers = __match_any_sync(0xffffffffu, key);
+    const int leader = __ffs(peers) - 1;
+    if (key >= 0 && lane == leader) warp_hist[key] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// Second walk over the same slots: stable rank within the warp's running
+// counts, then row = base[key] + warp_run[key] + rank-in-chunk.
+__device__ __forceinline__ void warp_scatter(const int32_t* idx, int begin, int end, int E,
+                                             int* warp_run, const int* base, int32_t* row_of,
+                                             int32_t* src_of, uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int c = begin; c < end; c += 32) {
+    const int i = c + lane;
+    const int key = load_key(idx, i, end, E, nullptr);  // already flagged by the histogram
+    const uint32_t peers = __match_any_sync(0xffffffffu, key);
+    int row = 0;
+    if (key >= 0) row = base[key] + warp_run[key] + __popc(peers & lt_mask);
+    __syncwarp();
+    const int leader = __ffs(peers) - 1;
+    if (key >= 0 && lane == leader) warp_run[key] += __popc(peers);
+    if (key >= 0) {
+      row_of[i] = row;
+      src_of[row] = i;
+    } else if (i < end) {
+      row_of[i] = -1;  // a bad expert id has no row
+    }
+    __syncwarp();
+  }
+  (void)status;
+}
+
+// In-place exclusive scan of s[0..n) by the whole CTA (n <= 2 * blockDim).
+// Returns the total.  Uses `tmp` (>= kLayoutWarps ints) as scratch.
+__device__ int block_exclusive_scan(int* s, int n, int* tmp) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n + blockDim.x - 1) / blockDim.x;  // <= 2
+  const int b = tid * per;
+  int local = 0;
+  for (int q = 0; q < per; ++q)
+    if (b + q < n) local += s[b + q];
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < (int)(blockDim.x >> 5) ? tmp[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += y;
+    }
+    if (lane < (int)(blockDim.x >> 5)) tmp[lane] = wi - w;  // exclusive warp base
+    if (lane == 31) tmp[32] = wi;                            // total
+  }
+  __syncthreads();
+  int run = tmp[warp] + incl - local;
+  for (int q = 0; q < per; ++q)
+    if (b + q < n) {
+      const int v = s[b + q];
+      s[b + q] = run;
+      run += v;
+    }
+  const int total = tmp[32];
+  __syncthreads();
+  return total;
+}
+
+// Per-expert exclusive scan across the warps of the CTA: hist[w][e] becomes
+// the count of expert e in warps < w; returns through agg[e] the CTA total.
+__device__ void scan_over_warps(int* hist, int E, int* agg) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < kLayoutWarps; ++w) {
+      const int c = hist[w * E + e];
+      hist[w * E + e] = run;
+      run += c;
+    }
+    agg[e] = run;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// one-CTA path
+// smem: hist[kLayoutWarps][E] | base[E+1] | tmp[33]
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLayoutThreads)
+    layout_single_kernel(const int32_t* __restrict__ idx, int R, int E, int32_t* counts,
+                         int32_t* offsets, int32_t* row_of, int32_t* src_of, uint32_t* status) {
+  extern __shared__ int smem_i[];
+  int* hist = smem_i;
+  int* base = hist + kLayoutWarps * E;
+  int* tmp = base + E + 1;
+  for (int i = threadIdx.x; i < kLayoutWarps * E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  const int per_warp = ((R + kLayoutWarps * 32 - 1) / (kLayoutWarps * 32)) * 32;
+  const int begin = min(R, warp * per_warp), end = min(R, begin + per_warp);
+  warp_histogram(idx, begin, end, E, hist + warp * E, status);
+  __syncthreads();
+  scan_over_warps(hist, E, base);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = base[e];
+  __syncthreads();
+  const int total = block_exclusive_scan(base, E, tmp);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = base[e];
+  if (threadIdx.x == 0) offsets[E] = total;
+  warp_scatter(idx, begin, end, E, hist + warp * E, base, row_of, src_of, status);
+}
+
+// ---------------------------------------------------------------------------
+// multi-CTA path, kernel 1: block histogram of one tile, added into counts
+// (counts zeroed by the host before).  Also clears this tile's look-back
+// status row and, in tile 0, the ticket counter for kernel 2.
+// smem: hist[E]
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLayoutThreads)
+    layout_hist_kernel(const int32_t* __restrict__ idx, int R, int E, int32_t* counts,
+                       uint32_t* lookback, uint32_t* ticket, uint32_t* status) {
+  extern __shared__ int smem_i[];
+  int* hist = smem_i;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    hist[e] = 0;
+    lookback[(size_t)blockIdx.x * E + e] = 0u;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;
+  __syncthreads();
+  const int tile_begin = blockIdx.x * kTile;
+  const int tile_end = min(R, tile_begin + kTile);
+  for (int i = tile_begin + threadIdx.x; i < tile_end; i += blockDim.x) {
+    const int e = load_key(idx, i, tile_end, E, status);
+    if (e >= 0) atomicAdd(&hist[e], 1);  // order of adds does not matter for a count
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (hist[e]) atomicAdd(counts + e, hist[e]);
+}
+
+// ---------------------------------------------------------------------------
+// multi-CTA path, kernel 2: per-tile stable ranks + decoupled look-back.
+// smem: hist[kLayoutWarps][E] | agg[E] | base[E+1] | tmp[33] | tile id
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLayoutThreads)
+    layout_scatter_kernel(const int32_t* __restrict__ idx, int R, int E,
+                          const int32_t* __restrict__ counts, int32_t* offsets, int32_t* row_of,
+                          int32_t* src_of, uint32_t* lookback, uint32_t* ticket,
+                          uint32_t* status) {
+  extern __shared__ int smem_i[];
+  int* hist = smem_i;
+  int* agg = hist + kLayoutWarps * E;
+  int* base = agg + E;
+  int* tmp = base + E + 1;
+  int* s_tile = tmp + 33;
+  if (threadIdx.x == 0) *s_tile = (int)atomicAdd(ticket, 1u);
+  for (int i = threadIdx.x; i < kLayoutWarps * E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  const int tile = *s_tile;
+  const int tile_begin = tile * kTile;
+  const int tile_end = min(R, tile_begin + kTile);
+  const int warp = threadIdx.x >> 5;
+  const int n = tile_end - tile_begin;
+  const int per_warp = ((n + kLayoutWarps * 32 - 1) / (kLayoutWarps * 32)) * 32;
+  const int begin = min(tile_end, tile_begin + warp * per_warp);
+  const int end = min(tile_end, begin + per_warp);
+  warp_histogram(idx, begin, end, E, hist + warp * E, nullptr);  // kernel 1 flagged bad ids
+  __syncthreads();
+  scan_over_warps(hist, E, agg);
+  __syncthreads();
+
+  // Decoupled look-back, one thread per expert: publish this tile's
+  // aggregate, sum predecessors until an inclusive prefix is found, publish
+  // the inclusive prefix.  Waits are bounded.
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    uint32_t* my = lookback + (size_t)tile * E + e;
+    const uint32_t a = (uint32_t)agg[e];
+    if (tile == 0) {
+      st_release_gpu(my, kFlagInclusive | a);
+      agg[e] = 0;  // exclusive prefix of tile 0
+      continue;
+    }
+    st_release_gpu(my, kFlagAggregate | a);
+    uint32_t excl = 0;
+    int pred = tile - 1;
+    uint64_t t0 = 0;
+    uint32_t spins = 0;
+    while (pred >= 0) {
+      const uint32_t s = ld_acquire_gpu(lookback + (size_t)pred * E + e);
+      const uint32_t flag = s & ~kValueMask;
+      if (flag == kFlagInclusive) {
+        excl += s & kValueMask;
+        break;
+      }
+      if (flag == kFlagAggregate) {
+        excl += s & kValueMask;
+        --pred;
+        continue;
+      }
+      // predecessor not published yet: it started earlier (ticket order), so
+      // it is running; wait, but not forever
+      if (spins == 0) t0 = globaltimer_ns();
+      if ((++spins & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+        flag_error(status, MOE_DEV_TIMEOUT);
+        break;
+      }
+      __nanosleep(32);
+    }
+    st_release_gpu(my, kFlagInclusive | ((excl + a) & kValueMask));
+    agg[e] = (int)excl;  // this tile's per-expert base among earlier tiles
+  }
+  // offsets from the complete counts (kernel 1 finished before this launch)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) base[e] = counts[e];
+  __syncthreads();
+  const int total = block_exclusive_scan(base, E, tmp);
+  if (tile == 0) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = base[e];
+    if (threadIdx.x == 0) offsets[E] = total;
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) base[e] += agg[e];
+  __syncthreads();
+  warp_scatter(idx, begin, end, E, hist + warp * E, base, row_of, src_of, status);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static int num_tiles(int64_t R) { return (int)((R + kTile - 1) / kTile); }
+
+int layout_kernel_count(int64_t R) { return R <= kSingleMax ? 1 : 2; }
+
+size_t layout_workspace_bytes(int64_t R, int E) {
+  if (R <= kSingleMax) return 0;
+  return 256 + (size_t)num_tiles(R) * (size_t)E * sizeof(uint32_t);
+}
+
+cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int32_t* offsets,
+                          int32_t* row_of, int32_t* src_of, void* ws, const DeviceInfo& dev,
+                          cudaStream_t stream) {
+  if (R <= kSingleMax) {
+    const size_t smem = (size_t)(kLayoutWarps * E + E + 1 + 33) * sizeof(int);
+    if (smem > 48 * 1024) {
+      cudaError_t err = cudaFuncSetAttribute(layout_single_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (err != cudaSuccess) return err;
+    }
+    layout_single_kernel<<<1, kLayoutThreads, smem, stream>>>(idx, R, E, counts, offsets, row_of,
+                                                              src_of, dev.status);
+    return cudaGetLastError();
+  }
+  uint32_t* ticket = static_cast<uint32_t*>(ws);
+  uint32_t* lookback = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 256);
+  const int tiles = num_tiles(R);
+  cudaError_t err = cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), stream);
+  if (err != cudaSuccess) return err;
+  layout_hist_kernel<<<tiles, kLayoutThreads, (size_t)E * sizeof(int), stream>>>(
+      idx, R, E, counts, lookback, ticket, dev.status);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const size_t smem = (size_t)(kLayoutWarps * E + E + E + 1 + 33 + 1) * sizeof(int);
+  if (smem > 48 * 1024) {
+    err = cudaFuncSetAttribute(layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+    if (err != cudaSuccess) return err;
+  }
+  layout_scatter_kernel<<<tiles, kLayoutThreads, smem, stream>>>(
+      idx, R, E, counts, offsets, row_of, src_of, lookback, ticket, dev.status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,211 @@
+/*
+ * moe.h -- C ABI of libmoe.so: one Mixture-of-Experts layer on one B200 (sm_100a).
+ *
+ * The layer, as the source pages describe it (DySHARP review, marsggbo, §1 and
+ * §3.1-3.2; "ThunderEP" PCIe blog, dpshk.com, §1.1 and §2.1-2.2; GPT-4 "2%"
+ * article, CSDN, §2.3, §3.1 table and §4.1):
+ *
+ *   route     a router scores each token, picks its top-k experts and a gate
+ *             value per chosen expert;
+ *   layout    tokens bound for the same expert are grouped into one dense,
+ *             contiguous block: a table maps the logical i-th (token, slot) to
+ *             its layout row (DySHARP §3.1 item 3, the AL table);
+ *   dispatch  the same token row is copied to each of its k experts;
+ *   expert    each expert applies Linear(d->f), GELU, Linear(f->d);
+ *   combine   the k expert outputs of a token are reduced into one row,
+ *             weighted by the gates.
+ *
+ * Conventions for every entry point
+ *   - Tensor arguments are DEVICE pointers owned by the caller, row-major and
+ *     contiguous, 16-byte aligned.  bf16 data is passed as void* holding
+ *     IEEE bfloat16 (the __nv_bfloat16 layout); indices are int32, gates and
+ *     logits fp32.
+ *   - Every call is asynchronous and stream-ordered on `stream` (a
+ *     cudaStream_t, passed as void*; NULL = the legacy default stream).  No
+ *     call synchronises the host or copies data to it (only
+ *     moe_device_status does, on request), so sequences of calls can be
+ *     captured in a CUDA graph.  Sizes that depend on the routing (per-expert
+ *     counts, offsets) stay in device memory.
+ *   - The library never allocates device memory.  Scratch space is a caller
+ *     workspace of at least the size the matching *_workspace_size returns.
+ *   - Arguments are validated on the host before any launch.  A rejected call
+ *     launches nothing and returns MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED;
+ *     moe_last_error_string() then describes the problem.
+ *   - Kernels that meet bad data (an expert id outside [0, E)) or a wait that
+ *     runs past its time limit set a sticky bit in a per-device status word
+ *     instead of trapping; read it with moe_device_status().
+ *   - Limits: 1 <= E <= 1024, 1 <= k <= min(E, 16), d % 8 == 0, f % 8 == 0,
+ *     T*k < 2^30.  T == 0 is a valid no-op.
+ *   - Threads may call the library concurrently; calls on streams that run at
+ *     the same time must not share output buffers or workspaces.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, negative size, k > E, short workspace, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2, /* valid, but outside the limits above (d % 8 != 0, E > 1024, ...) */
+  MOE_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  MOE_ERR_DEVICE = 4       /* moe_device_status found a bit set by a kernel */
+} moe_status;
+
+typedef enum moe_score {
+  MOE_SCORE_SOFTMAX = 0, /* p_e = softmax over the E logits */
+  MOE_SCORE_SIGMOID = 1  /* s_e = 1 / (1 + exp(-logit_e)) */
+} moe_score;
+
+/* Bits of the per-device status word (moe_device_status). */
+#define MOE_DEV_BAD_EXPERT_ID 0x1u /* an expert id outside [0, E) reached layout / dispatch */
+#define MOE_DEV_TIMEOUT       0x2u /* a bounded device-side wait gave up; outputs are invalid */
+#define MOE_DEV_BAD_ROW       0x4u /* a row index outside [0, T*k) reached dispatch / combine */
+
+/* Shape and routing recipe of one layer. */
+typedef struct moe_layer_desc {
+  int32_t T;           /* tokens */
+  int32_t d;           /* model dim */
+  int32_t E;           /* experts */
+  int32_t k;           /* experts per token */
+  int32_t f;           /* FFN hidden dim */
+  int32_t score;       /* moe_score */
+  int32_t renormalize; /* 1: gates renormalised over the chosen k; 0: plain probability */
+  int32_t reserved;    /* must be 0 */
+} moe_layer_desc;
+
+/* ---------------------------------------------------------------------------
+ * moe_router_logits -- the router linear layer (GPT-4 "2%" article §4.1:
+ * logits = router_proj(h); §3.1 table: the router maps a token to one logit
+ * per expert).
+ *   logits[t, e] = sum_c X[t, c] * Wr[e, c], accumulated in fp32.
+ *   X [T, d] bf16, Wr [E, d] bf16 (nn.Linear [out, in] layout), logits [T, E] fp32.
+ * ------------------------------------------------------------------------- */
+moe_status moe_router_logits(const void* X, const void* Wr, int32_t T, int32_t d, int32_t E,
+                             float* logits, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_route -- scores, top-k and gates (GPT-4 "2%" article §2.3 and §4.1:
+ * softmax over the logits, then top-k; ThunderEP blog §1.1: top-1 / top-2
+ * routing, §2.1: top-k indices and gate values drive the combine).
+ *   Per token t: the k experts with the largest logit, in descending order,
+ *   ties broken toward the lower expert id (selection on the fp32 logit equals
+ *   selection on the score, which is strictly increasing in it).
+ *   Gates, for chosen logits L_0 >= ... >= L_{k-1}:
+ *     SOFTMAX, renormalize=1: exp(L_j - L_0) / sum_{i<k} exp(L_i - L_0)
+ *     SOFTMAX, renormalize=0: exp(L_j - L_0) / sum_{e<E} exp(L_e - L_0)
+ *     SIGMOID, renormalize=1: s_j / sum_{i<k} s_i,  s = 1/(1+exp(-L))
+ *     SIGMOID, renormalize=0: s_j
+ *   logits [T, E] fp32 (finite; NaN/inf give unspecified choices);
+ *   topk_idx [T, k] int32, gates [T, k] fp32.
+ * ------------------------------------------------------------------------- */
+moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
+                     int32_t renormalize, int32_t* topk_idx, float* gates, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_layout -- per-expert histogram, exclusive scan and the logical->layout
+ * table (DySHARP §3.1 item 3: an AL table translates the logical i-th token to
+ * its position in a dense per-expert tensor, layout blocks being allocated
+ * incrementally; combine reuses the same table.  ThunderEP §2.2: tokens for
+ * the same expert are grouped contiguously).
+ *   With R = T*k and logical slot i = t*k + j, e_i = topk_idx[i]:
+ *     counts[e]   = #{i : e_i == e}
+ *     offsets[e]  = sum_{e' < e} counts[e'],  offsets[E] = R
+ *     row_of[i]   = offsets[e_i] + #{i' < i : e_i' == e_i}   (stable by token)
+ *     src_of[row_of[i]] = i
+ *   topk_idx [T, k] int32 in [0, E) (others set MOE_DEV_BAD_EXPERT_ID and are
+ *   skipped); counts [E], offsets [E+1], row_of [R], src_of [R] int32.
+ *   ws: at least moe_layout_workspace_size(T, E, k) bytes; its contents are
+ *   scratch (look-back status words for the multi-block scan).
+ * ------------------------------------------------------------------------- */
+size_t moe_layout_workspace_size(int32_t T, int32_t E, int32_t k);
+moe_status moe_layout(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k, int32_t* counts,
+                      int32_t* offsets, int32_t* row_of, int32_t* src_of, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_dispatch -- copy each token to its k experts' rows (DySHARP §1: the same
+ * token data goes to each of its k experts; ThunderEP §1.1).
+ *   Xe[r, :] = X[src_of[r] / k, :]   for r in [0, T*k).
+ *   X [T, d] bf16, src_of [T*k] int32, Xe [T*k, d] bf16.
+ * ------------------------------------------------------------------------- */
+moe_status moe_dispatch(const void* X, const int32_t* src_of, int32_t T, int32_t d, int32_t k,
+                        void* Xe, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_expert_gemm -- one grouped expert linear layer over variable-size row
+ * blocks (GPT-4 "2%" article §3.1 table: each expert is Linear -> GELU ->
+ * Linear; DySHARP §3.2: GEMM-1 then GEMM-2 per expert).
+ *   For each expert e and row r in [offsets[e], offsets[e+1]):
+ *     out[r, n] = act( sum_c A[r, c] * W[e, n, c] ),  act = GELU (exact erf
+ *     form, 0.5 x (1 + erf(x / sqrt 2))) when gelu != 0, identity otherwise;
+ *   accumulated in fp32 on the tensor cores, rounded once to bf16.
+ *   A [R, K] bf16, offsets [E+1] int32 (non-decreasing, offsets[E] <= R),
+ *   W [E, N, K] bf16, out [R, N] bf16.  Rows at or past offsets[E] are not
+ *   written.  K % 8 == 0, N % 8 == 0.
+ * ------------------------------------------------------------------------- */
+moe_status moe_expert_gemm(const void* A, const int32_t* offsets, const void* W, int32_t E,
+                           int32_t R, int32_t N, int32_t K, int32_t gelu, void* out,
+                           void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_expert_ffn -- both expert layers:  H = GELU(Xe W1[e]^T),  Ye = H W2[e]^T.
+ *   Xe [R, d] bf16, offsets [E+1], W1 [E, f, d] bf16, W2 [E, d, f] bf16,
+ *   H [R, f] bf16 (output, kept), Ye [R, d] bf16.
+ * ------------------------------------------------------------------------- */
+moe_status moe_expert_ffn(const void* Xe, const int32_t* offsets, const void* W1, const void* W2,
+                          int32_t E, int32_t R, int32_t d, int32_t f, void* H, void* Ye,
+                          void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_combine -- gate-weighted reduction of each token's k expert outputs
+ * (DySHARP §1: the k results are summed into one; ThunderEP §2.1: the gate
+ * values weight the combine sum).
+ *   Y[t, :] = bf16( sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :] ),
+ *   summed in fp32 in slot order j = 0..k-1.
+ *   Ye [T*k, d] bf16, row_of [T*k] int32, gates [T, k] fp32, Y [T, d] bf16.
+ * ------------------------------------------------------------------------- */
+moe_status moe_combine(const void* Ye, const int32_t* row_of, const float* gates, int32_t T,
+                       int32_t d, int32_t k, void* Y, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_layer_forward -- the whole layer in one call: [router_logits] -> route ->
+ * layout -> dispatch -> GEMM-1 + GELU -> GEMM-2 -> combine, all on `stream`,
+ * no host synchronisation.
+ *   Exactly one of `logits` ([T, E] fp32) and `Wr` ([E, d] bf16) is non-NULL.
+ *   X [T, d] bf16, W1 [E, f, d], W2 [E, d, f] bf16, Y [T, d] bf16.
+ *   topk_idx_out [T, k], gates_out [T, k], counts_out [E]: optional copies
+ *   of the routing (NULL to skip).
+ *   ws: at least moe_workspace_size(desc) bytes.
+ * ------------------------------------------------------------------------- */
+size_t moe_workspace_size(const moe_layer_desc* desc);
+moe_status moe_layer_forward(const moe_layer_desc* desc, const void* X, const float* logits,
+                             const void* Wr, const void* W1, const void* W2, void* Y,
+                             int32_t* topk_idx_out, float* gates_out, int32_t* counts_out,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Diagnostics.
+ *   moe_last_error_string: a description of the last failed call on this
+ *   host thread ("" if none).  The pointer stays valid until the next call.
+ *   moe_device_status: synchronises the current device, then stores the
+ *   sticky MOE_DEV_* bits into *bits (clearing them when clear != 0).  Returns
+ *   MOE_ERR_DEVICE when any bit was set, MOE_OK otherwise.
+ *   moe_kernel_launches_per_forward: the number of kernels moe_layer_forward
+ *   launches for this shape, with (with_router != 0) or without the router
+ *   linear (for launch accounting; memsets excluded).
+ * ------------------------------------------------------------------------- */
+const char* moe_last_error_string(void);
+moe_status moe_device_status(uint32_t* bits, int32_t clear);
+int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with_router);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,115 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import combine_moe_route_14_b200 as moe
+from combine_moe_route_14_b200 import build as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "moe.h")
+OK, INVALID, UNSUPPORTED = 0, 1, 2
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return moe.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_layer_calls():
+    names = declared_functions()
+    for n in ("moe_route", "moe_layout", "moe_dispatch", "moe_expert_ffn", "moe_combine",
+              "moe_layer_forward", "moe_router_logits", "moe_expert_gemm"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_declared_symbol():
+    sig = set(moe._SIG)
+    assert set(declared_functions()) <= sig
+
+
+def _err(lib):
+    return lib.moe_last_error_string().decode()
+
+
+N = None
+
+
+def test_route_rejects_bad_args(lib):
+    assert lib.moe_route(N, 4, 8, 2, 0, 1, N, N, N) == INVALID          # null pointers
+    assert lib.moe_route(N, 4, 8, 9, 0, 1, N, N, N) == INVALID          # k > E
+    assert "k must be" in _err(lib)
+    assert lib.moe_route(N, -1, 8, 2, 0, 1, N, N, N) == INVALID         # T < 0
+    assert lib.moe_route(N, 4, 2048, 2, 0, 1, N, N, N) == UNSUPPORTED   # E > 1024
+    assert lib.moe_route(N, 4, 64, 32, 0, 1, N, N, N) == UNSUPPORTED    # k > 16
+    assert lib.moe_route(N, 4, 8, 2, 7, 1, N, N, N) == INVALID          # unknown score
+    assert lib.moe_route(N, 0, 8, 2, 0, 1, N, N, N) == OK               # T == 0: no-op
+
+
+def test_misaligned_pointer_is_rejected(lib):
+    assert lib.moe_route(ctypes.c_void_p(0x1002), 4, 8, 2, 0, 1, ctypes.c_void_p(0x1000),
+                         ctypes.c_void_p(0x1000), N) == INVALID
+    assert "aligned" in _err(lib)
+    assert lib.moe_dispatch(ctypes.c_void_p(0x1008), ctypes.c_void_p(0x2000), 4, 64, 2,
+                            ctypes.c_void_p(0x3000), N) == INVALID
+
+
+def test_dims_must_be_multiples_of_8(lib):
+    assert lib.moe_dispatch(N, N, 4, 12, 2, N, N) == UNSUPPORTED
+    assert lib.moe_combine(N, N, N, 4, 100, 2, N, N) == UNSUPPORTED
+    assert lib.moe_expert_gemm(N, N, N, 8, 16, 12, 64, 0, N, N) == UNSUPPORTED
+    assert lib.moe_expert_gemm(N, N, N, 8, 16, 64, 0, 0, N, N) == INVALID
+
+
+def test_layout_rejects_short_workspace(lib):
+    p = ctypes.c_void_p(0x10000)
+    need = lib.moe_layout_workspace_size(8192, 256, 8)
+    assert need > 0  # the multi-block scan needs look-back words
+    assert lib.moe_layout(p, 8192, 256, 8, p, p, p, p, p, need - 1, N) == INVALID
+    assert "workspace" in _err(lib)
+    assert lib.moe_layout_workspace_size(16, 8, 2) == 0  # one-block path needs none
+
+
+def test_layer_workspace_and_desc_checks(lib):
+    d = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 0)
+    ws = lib.moe_workspace_size(ctypes.byref(d))
+    R = 4096 * 2
+    assert ws >= R * 4096 * 2 * 2 + R * 14336 * 2  # Xe + Ye + H at least
+    bad = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 7)
+    assert lib.moe_workspace_size(ctypes.byref(bad)) == 0
+    p = ctypes.c_void_p(0x10000)
+    # both logits and Wr given
+    assert lib.moe_layer_forward(ctypes.byref(d), p, p, p, p, p, p, N, N, N, p, ws, N) == INVALID
+    # short workspace
+    assert lib.moe_layer_forward(ctypes.byref(d), p, p, N, p, p, p, N, N, N, p, ws - 1,
+                                 N) == INVALID
+    assert lib.moe_layer_forward(N, p, p, N, p, p, p, N, N, N, p, ws, N) == INVALID
+
+
+def test_launch_count(lib):
+    d = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 0)
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 1) == 7
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 0) == 6
+    d4 = moe.LayerDesc(8192, 7168, 256, 8, 2048, 1, 1, 0)
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d4), 0) == 7  # two-kernel layout
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(moe, "_lib", None)
+    monkeypatch.setattr(moe, "_LIB_PATH", str(tmp_path / "libmoe.so"))
+    with pytest.raises(moe.MoeError):
+        moe.load_library()

@@ -1,0 +1,358 @@
+"""CUDA path vs the CPU oracle, stage by stage and end to end (needs a B200).
+
+Bars:
+  * indices, counts, offsets, the permutation and dispatched rows: bit-exact;
+  * floats: max|out - ref| <= 2e-2 * max|ref| + 1e-3 (bf16 I/O, fp32 accumulate),
+    plus tighter per-stage bounds where the arithmetic fixes one;
+  * router logits: the fp32 dot-product error bound gamma_d * sum|x w|.
+Inputs are seeded (combine_moe_route_14_b200.inputs); the oracle never sees a
+value produced by the CUDA path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import combine_moe_route_14_b200 as moe
+from combine_moe_route_14_b200 import inputs as I
+from oracle import moe_oracle as O
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    if t.dtype == torch.bfloat16:
+        return O.bf16_to_f64(bits(t))
+    return t.detach().cpu().double().numpy()
+
+
+def assert_close(out, ref, what, rel=2e-2, abs_=1e-3):
+    out = np.asarray(out, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert out.shape == ref.shape, (what, out.shape, ref.shape)
+    err = float(np.abs(out - ref).max()) if ref.size else 0.0
+    tol = O.tolerance(ref, rel, abs_)
+    assert err <= tol, f"{what}: max|err| {err:.3e} > tol {tol:.3e}"
+    return err
+
+
+@pytest.fixture(autouse=True)
+def _status_clean(cuda_lib):
+    moe.moe_device_status(clear=True)
+    yield
+    assert moe.moe_device_status(clear=True) == 0, "a kernel raised a device status bit"
+
+
+class LazyExperts:
+    """W[e] fetched from the device one expert at a time, as bf16 bits."""
+
+    def __init__(self, W):
+        self.W = W
+        self.shape = tuple(W.shape)
+
+    def __getitem__(self, e):
+        return bits(self.W[e])
+
+
+# ----------------------------------------------------------------------------
+# route
+# ----------------------------------------------------------------------------
+ROUTE_CASES = [
+    # (T, E, k, score, renorm, kind)
+    (256, 8, 2, "softmax", 1, "normal"),
+    (4096, 8, 1, "softmax", 1, "normal"),
+    (8192, 256, 8, "sigmoid", 1, "normal"),
+    (777, 64, 6, "softmax", 0, "normal"),
+    (333, 40, 3, "sigmoid", 0, "normal"),
+    (500, 8, 2, "softmax", 1, "ties"),
+    (500, 256, 8, "sigmoid", 1, "ties"),
+    (64, 1024, 16, "softmax", 1, "ties"),
+    (64, 1024, 16, "softmax", 0, "normal"),
+    (100, 5, 5, "softmax", 1, "normal"),
+    (1, 1, 1, "softmax", 1, "normal"),
+    (37, 33, 2, "softmax", 1, "ties"),
+]
+
+
+def _logits(T, E, kind, seed=0):
+    L = I.random_f32((T, E), seed, f"route{T}x{E}")
+    if kind == "ties":  # few distinct values, signed zeros included
+        L = torch.round(L * 2) / 2
+        L[L == 0] = torch.where(torch.rand(int((L == 0).sum()), generator=torch.Generator().manual_seed(1)) < 0.5,
+                                torch.tensor(-0.0), torch.tensor(0.0))
+    return L
+
+
+@pytest.mark.parametrize("T,E,k,score,renorm,kind", ROUTE_CASES)
+def test_route_parity(T, E, k, score, renorm, kind):
+    L = _logits(T, E, kind)
+    idx, g = moe.moe_route(L.to(DEV), k, score, renorm)
+    ref_idx, ref_g = O.route(L.numpy(), k, score, renorm)
+    assert np.array_equal(idx.cpu().numpy(), ref_idx)
+    # fp32 exp / division against float64: a few ulp of values in [0, 1]
+    np.testing.assert_allclose(g.cpu().numpy(), ref_g, rtol=2e-6, atol=2e-7)
+
+
+# ----------------------------------------------------------------------------
+# router linear
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("T,d,E", [(4096, 4096, 8), (16, 4096, 8), (300, 136, 3), (77, 512, 40),
+                                   (1, 8, 1)])
+def test_router_logits_parity(T, d, E):
+    X = I.random_bf16((T, d), 1, "X")
+    Wr = I.random_bf16((E, d), 1, "Wr", 0.02)
+    L = moe.moe_router_logits(X.to(DEV), Wr.to(DEV)).cpu().double().numpy()
+    x, w = O.bf16_to_f64(bits(X)), O.bf16_to_f64(bits(Wr))
+    ref = O.router_logits(x, w)
+    u = 2.0 ** -24
+    gamma = d * u / (1 - d * u)
+    bound = gamma * (np.abs(x) @ np.abs(w).T) + 1e-30
+    assert (np.abs(L - ref) <= bound).all(), float((np.abs(L - ref) / bound).max())
+
+
+# ----------------------------------------------------------------------------
+# layout
+# ----------------------------------------------------------------------------
+LAYOUT_CASES = [
+    # (T, E, k, skew)
+    (256, 8, 2, 0.0),
+    (4096, 8, 2, 0.0),        # 8192 slots: one-block path
+    (4096, 8, 1, 2.5),        # skewed
+    (8192, 256, 8, 0.0),      # 65536 slots: histogram + decoupled look-back
+    (8193, 256, 2, 0.0),      # 16386 slots: just past the one-block limit, ragged last tile
+    (20000, 7, 3, 1.0),       # several tiles, few experts
+    (10, 256, 4, 0.0),        # mostly empty experts
+    (3000, 1024, 16, 0.0),    # max experts and k, multi-block
+    (50, 1024, 2, 0.0),
+    (1, 1, 1, 0.0),
+    (999, 1, 1, 0.0),
+]
+
+
+@pytest.mark.parametrize("T,E,k,skew", LAYOUT_CASES)
+def test_layout_parity(T, E, k, skew):
+    idx = I.random_topk(T, E, k, 5, skew=skew)
+    counts, offsets, row_of, src_of = moe.moe_layout(idx.to(DEV), E)
+    rc, ro, rr, rs = O.layout(idx.numpy(), E)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(row_of.cpu().numpy(), rr)
+    assert np.array_equal(src_of.cpu().numpy(), rs)
+
+
+def test_layout_repeatable_and_stable_under_reuse():
+    """Same workspace twice (look-back words must be re-armed each call)."""
+    T, E, k = 8192, 256, 8
+    idx = I.random_topk(T, E, k, 6).to(DEV)
+    ws = torch.empty(moe.moe_layout_workspace_size(T, E, k), dtype=torch.uint8, device=DEV)
+    a = [x.clone() for x in moe.moe_layout(idx, E, ws=ws)]
+    b = moe.moe_layout(idx, E, ws=ws)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_layout_flags_bad_expert_ids():
+    idx = I.random_topk(64, 8, 2, 7)
+    idx[3, 1] = 8
+    idx[10, 0] = -1
+    counts, offsets, row_of, src_of = moe.moe_layout(idx.to(DEV), 8)
+    assert moe.moe_device_status(clear=True) & 1  # MOE_DEV_BAD_EXPERT_ID
+    rc = row_of.cpu().numpy()
+    assert rc[3 * 2 + 1] == -1 and rc[10 * 2] == -1
+    assert counts.sum().item() == 64 * 2 - 2
+
+
+# ----------------------------------------------------------------------------
+# dispatch / combine
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("T,d,E,k", [(256, 128, 8, 2), (4096, 4096, 8, 2), (8192, 7168, 256, 8),
+                                     (33, 8, 4, 3), (100, 4104, 16, 5), (5, 2056, 3, 1)])
+def test_dispatch_bit_exact(T, d, E, k):
+    X = I.random_bf16((T, d), 2, "X")
+    idx = I.random_topk(T, E, k, 2)
+    _, _, _, rs = O.layout(idx.numpy(), E)
+    Xe = moe.moe_dispatch(X.to(DEV), torch.from_numpy(rs).to(DEV), k)
+    ref = O.dispatch(bits(X), rs, k)
+    assert np.array_equal(bits(Xe), ref)
+
+
+@pytest.mark.parametrize("T,d,E,k", [(256, 128, 8, 2), (4096, 4096, 8, 2), (8192, 7168, 256, 8),
+                                     (33, 8, 4, 3), (100, 4104, 16, 5), (50, 64, 16, 16),
+                                     (7, 24, 12, 11), (4096, 4096, 8, 1)])
+def test_combine_parity(T, d, E, k):
+    Ye = I.random_bf16((T * k, d), 3, "Ye")
+    idx = I.random_topk(T, E, k, 3)
+    _, _, rr, _ = O.layout(idx.numpy(), E)
+    L = I.random_f32((T, E), 3, "L")
+    _, g = O.route(L.numpy(), k)
+    g32 = torch.from_numpy(g.astype(np.float32))
+    Y = moe.moe_combine(Ye.to(DEV), torch.from_numpy(rr).to(DEV), g32.to(DEV))
+    ref = O.combine(O.bf16_to_f64(bits(Ye)), rr, g32.double().numpy(), k)
+    out = f64(Y)
+    assert_close(out, ref, "combine")
+    # one bf16 rounding of an fp32 sum: |err| <= 2^-8 |ref| + fp32 slack
+    slack = 1e-6 * (np.abs(g32.double().numpy()).sum(1, keepdims=True) * 8)
+    assert (np.abs(out - ref) <= 2.0 ** -8 * np.abs(ref) + slack).all()
+
+
+def test_identity_experts_return_input():
+    """combine(dispatch(X)) with Ye = Xe returns X * sum(g) = X (renormalised)."""
+    T, d, E, k = 1000, 256, 8, 2
+    X = I.random_bf16((T, d), 4, "X").to(DEV)
+    L = I.random_f32((T, E), 4, "L").to(DEV)
+    idx, g = moe.moe_route(L, k)
+    _, _, row_of, src_of = moe.moe_layout(idx, E)
+    Y = moe.moe_combine(moe.moe_dispatch(X, src_of, k), row_of, g)
+    assert_close(f64(Y), f64(X), "identity", rel=2.0 ** -7, abs_=0)
+
+
+# ----------------------------------------------------------------------------
+# grouped GEMM / expert FFN
+# ----------------------------------------------------------------------------
+def _gemm_case(counts, N, K, gelu, seed=8, std_w=0.05):
+    counts = np.asarray(counts)
+    E = len(counts)
+    R = int(counts.sum())
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    A = I.random_bf16((max(R, 1), K), seed, "A")[:R]
+    W = I.random_bf16((E, N, K), seed, "W", std_w)
+    out = torch.full((R, N), float("nan"), dtype=torch.bfloat16, device=DEV)
+    moe.moe_expert_gemm(A.to(DEV), torch.from_numpy(offsets).to(DEV), W.to(DEV), gelu, out=out)
+    a = O.bf16_to_f64(bits(A))
+    ref = np.zeros((R, N))
+    for e in range(E):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            w = O.bf16_to_f64(bits(W[e]))
+            ref[lo:hi] = O.expert_gemm1(a[lo:hi], w) if gelu else O.expert_gemm2(a[lo:hi], w)
+    return f64(out), ref
+
+
+GEMM_CASES = [
+    # (counts per expert, N, K, gelu)
+    ([64] * 8, 256, 128, True),                       # tiny layer, GEMM-1 shape
+    ([64] * 8, 128, 256, False),                      # tiny layer, GEMM-2 shape
+    ([0, 1, 15, 16, 17, 31, 33, 255, 256, 257, 300, 0], 256, 192, True),  # ragged blocks
+    ([700], 384, 512, False),                         # one expert, several token blocks
+    ([40, 0, 0, 90], 136, 72, True),                  # N and K tails (not multiples of 128 / 64)
+    ([5, 3], 8, 8, False),                            # smallest dims
+    ([128] * 3, 1024, 1024, True),
+    ([1] * 64, 256, 256, False),                      # many one-row experts
+]
+
+
+@pytest.mark.parametrize("counts,N,K,gelu", GEMM_CASES)
+def test_expert_gemm_parity(counts, N, K, gelu):
+    out, ref = _gemm_case(counts, N, K, gelu)
+    assert not np.isnan(out).any()
+    assert_close(out, ref, "gemm")
+    # bf16 output rounding plus fp32 accumulation: far inside the bar
+    assert_close(out, ref, "gemm (tight)", rel=1e-2, abs_=1e-3)
+
+
+def test_expert_gemm_leaves_rows_past_offsets_alone():
+    counts = np.array([10, 20])
+    offsets = torch.tensor([0, 10, 30], dtype=torch.int32, device=DEV)
+    A = I.random_bf16((40, 64), 9, "A").to(DEV)
+    W = I.random_bf16((2, 128, 64), 9, "W", 0.05).to(DEV)
+    out = torch.full((40, 128), 7.0, dtype=torch.bfloat16, device=DEV)
+    moe.moe_expert_gemm(A, offsets, W, True, out=out)
+    assert (out[30:] == 7.0).all()
+
+
+def test_expert_ffn_tiny_matches_oracle():
+    cfg = I.workload("tiny")
+    inp = I.make_layer_inputs(cfg, 0, device=DEV)
+    Xe_bits = I.random_bf16((cfg.R, cfg.d), 0, "Xe")
+    idx = I.random_topk(cfg.T, cfg.E, cfg.k, 0)
+    rc, ro, _, _ = O.layout(idx.numpy(), cfg.E)
+    H, Ye = moe.moe_expert_ffn(Xe_bits.to(DEV), torch.from_numpy(ro).to(DEV), inp["W1"], inp["W2"])
+    rH, rYe = O.expert_ffn(O.bf16_to_f64(bits(Xe_bits)), ro, bits(inp["W1"]), bits(inp["W2"]))
+    assert_close(f64(H), rH, "H")
+    assert_close(f64(Ye), rYe, "Ye")
+
+
+# ----------------------------------------------------------------------------
+# whole layer
+# ----------------------------------------------------------------------------
+def _run_layer(inp, cfg):
+    dev_in = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    layer = moe.MoeLayer(dev_in["W1"], dev_in["W2"], cfg.k, cfg.score, cfg.renormalize,
+                         Wr=dev_in["Wr"])
+    T = cfg.T
+    idx = torch.empty((T, cfg.k), dtype=torch.int32, device=DEV)
+    g = torch.empty((T, cfg.k), dtype=torch.float32, device=DEV)
+    counts = torch.empty((cfg.E,), dtype=torch.int32, device=DEV)
+    Y = layer(dev_in["X"], logits=dev_in["logits"], topk_idx_out=idx, gates_out=g,
+              counts_out=counts)
+    torch.cuda.synchronize()
+    return Y, idx, g, counts, layer
+
+
+def test_layer_tiny_full_parity():
+    cfg = I.workload("tiny")
+    inp = I.make_layer_inputs(cfg, 0, device=DEV)
+    Y, idx, g, counts, _ = _run_layer(inp, cfg)
+    ref = O.layer_forward(bits(inp["X"]), bits(inp["W1"]), bits(inp["W2"]), cfg.k, cfg.score,
+                          cfg.renormalize, logits=inp["logits"].numpy())
+    assert np.array_equal(idx.cpu().numpy(), ref["topk_idx"])
+    assert np.array_equal(counts.cpu().numpy(), ref["counts"])
+    np.testing.assert_allclose(g.cpu().numpy(), ref["gates"], rtol=2e-6, atol=2e-7)
+    assert_close(f64(Y), ref["Y"], "Y")
+
+
+def test_layer_deterministic():
+    cfg = I.workload("tiny")
+    inp = I.make_layer_inputs(cfg, 1, device=DEV)
+    Y1 = _run_layer(inp, cfg)[0].clone()
+    Y2 = _run_layer(inp, cfg)[0]
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+
+
+def _sample_tokens(T, n, seed=0):
+    rng = np.random.default_rng(seed)
+    pick = set([0, T - 1]) | set(rng.choice(T, size=min(T, n), replace=False).tolist())
+    return np.array(sorted(pick))
+
+
+def _near_ties(L, k, eps):
+    """Tokens whose k-th and (k+1)-th logits lie within eps (routing there is a coin toss)."""
+    if L.shape[1] <= k:
+        return np.zeros(L.shape[0], bool)
+    s = -np.sort(-L, axis=1)
+    return (s[:, k - 1] - s[:, k]) <= eps
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,nsample", [("skewed_top1", 48), ("skewed_top1_harsh", 24),
+                                          ("fine_grained", 12), ("mixtral", 32),
+                                          ("decode_16", 16), ("decode_64", 24),
+                                          ("decode_256", 24), ("decode_1024", 24)])
+def test_layer_full_size_sampled(name, nsample):
+    cfg = I.workload(name)
+    inp = I.make_layer_inputs(cfg, 0, device=DEV)
+    Y, idx, g, counts, layer = _run_layer(inp, cfg)
+    X_bits = bits(inp["X"])
+    gi = idx.cpu().numpy()
+    if cfg.router == "weights":
+        # oracle's own logits (float64 -> fp32) and routing; near-ties may differ
+        Lref = O.router_logits(O.bf16_to_f64(X_bits), O.bf16_to_f64(bits(inp["Wr"]))).astype(np.float32)
+        x = O.bf16_to_f64(X_bits)
+        w = O.bf16_to_f64(bits(inp["Wr"]))
+        eps = 2 * (cfg.d * 2.0 ** -24) * float((np.abs(x) @ np.abs(w).T).max())
+        ties = _near_ties(Lref.astype(np.float64), cfg.k, eps)
+    else:
+        Lref = inp["logits"].numpy()
+        ties = np.zeros(cfg.T, bool)
+    ref_idx, ref_g = O.route(Lref, cfg.k, cfg.score, cfg.renormalize)
+    mism = np.any(gi != ref_idx, axis=1)
+    assert not (mism & ~ties).any(), f"{int((mism & ~ties).sum())} tokens routed differently"
+    assert np.array_equal(counts.cpu().numpy()[None], np.bincount(gi.ravel(), minlength=cfg.E)[None])
+    toks = np.array([t for t in _sample_tokens(cfg.T, nsample) if not ties[t]])
+    ref = O.layer_forward_tokens(X_bits, LazyExperts(inp["W1"]), LazyExperts(inp["W2"]), ref_idx,
+                                 ref_g, toks)
+    assert_close(f64(Y[torch.from_numpy(toks).to(DEV)]), ref, f"{name} Y")

@@ -20,6 +20,7 @@ import torch
 __all__ = [
     "MoeError", "LayerDesc", "load_library", "library_path",
     "moe_router_logits", "moe_route", "moe_layout_workspace_size", "moe_layout",
+    "moe_layout_static",
     "moe_dispatch", "moe_expert_gemm", "moe_expert_ffn", "moe_combine",
     "moe_workspace_size", "moe_layer_forward", "moe_device_status",
     "moe_kernel_launches_per_forward", "MoeLayer", "SCORES",
@@ -59,6 +60,7 @@ _SIG = {
     "moe_route": ([_P, _I, _I, _I, _I, _I, _P, _P, _P], ctypes.c_int),
     "moe_layout_workspace_size": ([_I, _I, _I], ctypes.c_size_t),
     "moe_layout": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_layout_static": ([_P, _I, _I, _I, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_dispatch": ([_P, _P, _I, _I, _I, _P, _P], ctypes.c_int),
     "moe_expert_gemm": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
     "moe_expert_ffn": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P], ctypes.c_int),
@@ -182,6 +184,27 @@ def moe_layout(topk_idx, E, counts=None, offsets=None, row_of=None, src_of=None,
     _need(ws, "ws", torch.uint8, None, dev)
     _check(lib.moe_layout(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets), _ptr(row_of),
                           _ptr(src_of), _ptr(ws), ws.numel(), _stream(stream, dev)))
+    return counts, offsets, row_of, src_of
+
+
+def moe_layout_static(topk_idx, E, counts=None, offsets=None, row_of=None, src_of=None,
+                      stream=None):
+    """moe_layout with the scratch kept in the library's own static device array.
+
+    For callers that cannot allocate device memory for a workspace; see
+    include/moe.h.  Calls that may overlap on the GPU race on the shared array.
+    """
+    lib = load_library()
+    T, k = topk_idx.shape
+    dev = topk_idx.device
+    _need(topk_idx, "topk_idx", torch.int32, (T, k))
+    R = T * k
+    counts = _out(counts, "counts", torch.int32, (E,), dev)
+    offsets = _out(offsets, "offsets", torch.int32, (E + 1,), dev)
+    row_of = _out(row_of, "row_of", torch.int32, (R,), dev)
+    src_of = _out(src_of, "src_of", torch.int32, (R,), dev)
+    _check(lib.moe_layout_static(_ptr(topk_idx), T, E, k, _ptr(counts), _ptr(offsets),
+                                 _ptr(row_of), _ptr(src_of), _stream(stream, dev)))
     return counts, offsets, row_of, src_of
 
 

@@ -35,6 +35,11 @@ cudaError_t g_dev_err[kMaxDevices];
 
 }  // namespace
 
+int set_last_error(int status, const std::string& msg) {
+  g_last_error = msg;
+  return status;
+}
+
 const DeviceInfo* current_device_info(std::string* err) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -50,4 +50,7 @@ cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const voi
                                 int R, int N, int K, bool gelu, void* out,
                                 const DeviceInfo& dev, cudaStream_t stream, std::string* err);
 
+// Records `msg` as this thread's moe_last_error_string() and returns `status`.
+int set_last_error(int status, const std::string& msg);
+
 }  // namespace moe

@@ -129,6 +129,32 @@ moe_status moe_layout(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k, 
                       size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_layout_static -- moe_layout without a workspace argument, for callers
+ * that cannot allocate device memory.  The pages have no counterpart: this
+ * is a convenience of this library, not a step of the method.
+ *   Some callers have no way to get scratch memory on the GPU: code running
+ *   inside another framework's callback that is handed only the tensors it
+ *   works on, with no allocator; or code that must not allocate after
+ *   start-up.  This variant keeps the layout's scratch (the multi-block
+ *   scan's look-back words and tile ticket) in a 1 MiB array inside the
+ *   library, which every GPU that loads the library holds until the process
+ *   exits.  It allocates nothing and calls no allocating routine.
+ *   Same arguments and results as moe_layout, minus ws / ws_bytes.  Shapes
+ *   whose scratch would exceed 1 MiB (moe_layout_workspace_size(T, E, k) >
+ *   1048576, e.g. more than about 2 million slots with 1024 experts) are
+ *   rejected with MOE_ERR_UNSUPPORTED before any launch.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  Every call on a device shares the one array
+ *   and leaves its contents behind; the kernels re-arm what must start at
+ *   zero on each call.  Calls whose kernels may overlap on the GPU (other
+ *   streams, other host threads) race on the array: serialise them.
+ * ------------------------------------------------------------------------- */
+moe_status moe_layout_static(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k,
+                             int32_t* counts, int32_t* offsets, int32_t* row_of, int32_t* src_of,
+                             void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_dispatch -- copy each token to its k experts' rows (DySHARP §1: the same
  * token data goes to each of its k experts; ThunderEP §1.1).
  *   Xe[r, :] = X[src_of[r] / k, :]   for r in [0, T*k).

@@ -6,7 +6,7 @@
 //
 //   out[r, n] = act( sum_c A[r, c] * W[e, n, c] )   for r in expert e's block
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM, 10 warps):
 //   * Operand roles are swapped with respect to the usual token-major GEMM:
 //     128 weight rows (output features) form the MMA's M side, and up to 256
 //     token rows of one expert form its N side.  N is chosen per tile at run
@@ -14,9 +14,11 @@
 //     ceil(c/16)*16 columns of MMA work instead of a full 128-row tile.
 //   * warp 0 (one lane) streams K-blocks of 64 through a 4-stage ring with
 //     TMA (128-byte swizzle), warp 1 (one lane) issues tcgen05.mma into one
-//     of two TMEM accumulators (2 x 256 fp32 columns), warps 2-5 drain the
+//     of two TMEM accumulators (2 x 256 fp32 columns), warps 2-9 drain the
 //     other accumulator (tcgen05.ld), apply GELU, round to bf16, transpose
-//     through shared memory and store token rows.  Mainloop and epilogue of
+//     through shared memory and store token rows.  Each epilogue warp owns
+//     one TMEM lane quarter (32 features) and one half of the tile's tokens,
+//     so every SM sub-partition runs two of them.  Mainloop and epilogue of
 //     consecutive tiles overlap.
 //   * The tile list comes from the per-expert offsets in device memory: no
 //     host synchronisation.  Tiles are ordered (expert, feature block, token
@@ -41,8 +43,8 @@ constexpr int A_STAGE = BM * BK * 2;         // 16 KB
 constexpr int B_STAGE = BN * BK * 2;         // 32 KB
 constexpr int B_BOX_ROWS = 32;
 constexpr int B_BOX = B_BOX_ROWS * BK * 2;   // 4 KB
-constexpr int EPI_WARPS = 4;
-constexpr int THREADS = 64 + EPI_WARPS * 32; // producer, MMA, 4 epilogue warps
+constexpr int EPI_WARPS = 8;                 // two per SM sub-partition
+constexpr int THREADS = 64 + EPI_WARPS * 32; // producer, MMA, 8 epilogue warps
 constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int XPOSE = EPI_WARPS * 32 * 32 * 2;  // per-warp 32x32 bf16 transpose tile
 constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
@@ -92,8 +94,23 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
   return __all_sync(0xffffffffu, ok);
 }
 
+// GELU(x) = x * Phi(x), Phi the standard normal CDF (the exact, erf-based
+// GELU).  With z = |x| / sqrt(2), Phi(-|x|) = erfc(z) / 2, and erfc is
+// evaluated with the rational approximation of Abramowitz & Stegun,
+// "Handbook of Mathematical Functions", eq. 7.1.26 (Hastings):
+//   erfc(z) ~= (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),
+//   t = 1 / (1 + p z),  |error| <= 1.5e-7 for z >= 0.
+// Then Phi(x) = 1 - Phi(-|x|) for x >= 0.  The result is within a few 1e-7
+// of the exact GELU relative to |x|, far below one bf16 ulp of the output.
 __device__ __forceinline__ float gelu_erf(float x) {
-  return 0.5f * x * (1.f + erff(x * 0.70710678118654752440f));
+  const float z = fabsf(x) * 0.70710678118654752440f;
+  const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+  float p = fmaf(1.061405429f, t, -1.453152027f);
+  p = fmaf(p, t, 1.421413741f);
+  p = fmaf(p, t, -0.284496736f);
+  p = fmaf(p, t, 0.254829592f);
+  const float q = 0.5f * p * t * __expf(-z * z);  // Phi(-|x|)
+  return x * (x >= 0.f ? 1.0f - q : q);
 }
 
 __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
@@ -187,7 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     const uint64_t pol_tokens = l2_policy_evict_last();   // re-read by every feature block
-    const uint64_t pol_weights = l2_policy_evict_first(); // read by one wave of CTAs
+    const uint64_t pol_weights = l2_policy_evict_normal(); // shared by the CTAs of one feature block
     int s = 0;
     uint32_t ph = 0;
     uint32_t issued = 0;  // bit s: stage s has a load in flight or landed
@@ -270,7 +287,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;              // TMEM lane quarter this warp may access
+    const int half = (warp - 2) >> 2;    // which 128 of the tile's 256 token columns
     uint16_t* xp = sX + (warp - 2) * 32 * 32;
     uint16_t* out = args.out;
     const int N = args.N;
@@ -283,7 +301,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after_sync();
       const int fbase = t.fb * BM + q * 32;  // this warp's 32 output features
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      for (int c0 = 0; c0 < t.ntok; c0 += 32) {
+      const int c_end = min(t.ntok, half * (BN / 2) + BN / 2);
+      for (int c0 = half * (BN / 2); c0 < c_end; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + (uint32_t)c0, v);
         tmem_wait_ld();

@@ -356,3 +356,25 @@ def test_layer_full_size_sampled(name, nsample):
     ref = O.layer_forward_tokens(X_bits, LazyExperts(inp["W1"]), LazyExperts(inp["W2"]), ref_idx,
                                  ref_g, toks)
     assert_close(f64(Y[torch.from_numpy(toks).to(DEV)]), ref, f"{name} Y")
+
+
+def test_gemm_gelu_is_exact_to_bf16():
+    """Identity weights make the GEMM output GELU(x) itself.  The kernel's erf
+    approximation (Abramowitz & Stegun 7.1.26, |erfc error| <= 1.5e-7) adds at
+    most 0.75e-7 * |x| to the exact GELU, so the output must equal the exact
+    GELU rounded to bf16 up to half an ulp plus that term (a last-place flip
+    where the exact value sits next to a rounding midpoint)."""
+    K = 64
+    xs = torch.linspace(-9, 9, 64 * K, dtype=torch.float32).reshape(64, K)
+    A = xs.to(torch.bfloat16)
+    W = torch.eye(K, dtype=torch.bfloat16).reshape(1, K, K)
+    offsets = torch.tensor([0, 64], dtype=torch.int32, device=DEV)
+    out = moe.moe_expert_gemm(A.to(DEV), offsets, W.to(DEV), True)
+    x = O.bf16_to_f64(bits(A))
+    ref = O.gelu(x)
+    got = f64(out)
+    bound = 2.0 ** -8 * np.abs(ref) + 1e-7 * np.abs(x) + 1e-30
+    assert (np.abs(got - ref) <= bound).all(), float((np.abs(got - ref) / bound).max())
+    big = np.abs(ref) > 1e-3  # where bf16 resolution dominates: the rounded value itself
+    ref_bits = I.f32_to_bf16_bits(ref.astype(np.float32))
+    assert (bits(out)[big] == ref_bits[big]).mean() >= 0.99

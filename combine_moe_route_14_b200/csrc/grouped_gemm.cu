@@ -34,25 +34,35 @@
 namespace moe {
 
 namespace gg {
-constexpr int BM = 128;                      // weight rows per tile (UMMA M)
+constexpr int BM = 128;                      // weight rows per CTA (UMMA M per CTA)
 constexpr int BN = 256;                      // token rows per tile, at most (UMMA N)
 constexpr int BK = 64;                       // K per stage: one 128-byte swizzled bf16 row
 constexpr int UMMA_K = 16;                   // K per tcgen05.mma (kind::f16)
-constexpr int STAGES = 4;
-constexpr int A_STAGE = BM * BK * 2;         // 16 KB
-constexpr int B_STAGE = BN * BK * 2;         // 32 KB
+constexpr int A_STAGE = BM * BK * 2;         // 16 KB of weight rows per CTA and stage
 constexpr int B_BOX_ROWS = 32;
 constexpr int B_BOX = B_BOX_ROWS * BK * 2;   // 4 KB
 constexpr int EPI_WARPS = 8;                 // two per SM sub-partition
 constexpr int THREADS = 64 + EPI_WARPS * 32; // producer, MMA, 8 epilogue warps
 constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int XPOSE = EPI_WARPS * 32 * 32 * 2;  // per-warp 32x32 bf16 transpose tile
-constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
 constexpr uint64_t kDrainLimitNs = 20ull * 1000ull * 1000ull;  // 20 ms
 
+// kPair = 1: one CTA computes a 128-feature x N-token tile (cta_group::1).
+// kPair = 2: a cluster of two CTAs computes a 256-feature x N-token tile with
+//   the paired MMA (cta_group::2, M = 256): each CTA stages its own 128
+//   weight rows and half of the token rows, so per-SM shared-memory traffic
+//   and L2 reads per FLOP are a third lower, and 6 stages fit.
+template <int kPair> struct Cfg {
+  static constexpr int STAGES = kPair == 2 ? 6 : 4;
+  static constexpr int B_STAGE = (BN / kPair) * BK * 2;  // token rows this CTA stages
+  static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
+  static constexpr int FEAT = BM * kPair;                // output features per tile
+};
+
+template <int kPair>
 __host__ __device__ constexpr size_t smem_bytes(int E) {
-  return 1024 /* alignment slack */ + (size_t)STAGES * (A_STAGE + B_STAGE) + XPOSE +
-         NUM_BARS * 8 + 16 + (size_t)3 * (E + 1) * sizeof(int);
+  return 1024 /* alignment slack */ + (size_t)Cfg<kPair>::STAGES * (A_STAGE + Cfg<kPair>::B_STAGE) +
+         XPOSE + Cfg<kPair>::NUM_BARS * 8 + 16 + (size_t)3 * (E + 1) * sizeof(int);
 }
 
 struct Args {
@@ -60,7 +70,7 @@ struct Args {
   uint16_t* out;           // [R, N] bf16
   uint32_t* status;
   int E, R, N, K;
-  int n_fblocks;           // ceil(N / BM)
+  int n_fblocks;           // ceil(N / features per tile)
   int num_kb;              // ceil(K / BK)
 };
 
@@ -100,8 +110,8 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
 // "Handbook of Mathematical Functions", eq. 7.1.26 (Hastings):
 //   erfc(z) ~= (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),
 //   t = 1 / (1 + p z),  |error| <= 1.5e-7 for z >= 0.
-// Then Phi(x) = 1 - Phi(-|x|) for x >= 0.  The result is within a few 1e-7
-// of the exact GELU relative to |x|, far below one bf16 ulp of the output.
+// Then Phi(x) = 1 - Phi(-|x|) for x >= 0.  The result is within 0.75e-7 * |x|
+// of the exact GELU, far below one bf16 ulp of the output.
 __device__ __forceinline__ float gelu_erf(float x) {
   const float z = fabsf(x) * 0.70710678118654752440f;
   const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
@@ -118,10 +128,13 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
-template <bool kGelu>
+template <bool kGelu, int kPair>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x, const Args args) {
+  using C = Cfg<kPair>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int B_STAGE = C::B_STAGE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -129,12 +142,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t* sB = sA + STAGES * A_STAGE;
   uint16_t* sX = reinterpret_cast<uint16_t*>(sB + STAGES * B_STAGE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sX) + XPOSE);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* tfull = bars + 2 * STAGES;
-  uint64_t* tempty = tfull + 2;
+  uint64_t* full = bars;               // used in the leader CTA: both CTAs' bytes land here
+  uint64_t* empty = bars + STAGES;     // per CTA: the MMAs have read this stage
+  uint64_t* tfull = bars + 2 * STAGES; // per CTA: accumulator ready
+  uint64_t* tempty = tfull + 2;        // leader CTA: both CTAs' epilogues drained it
   uint64_t* drain = tempty + 2;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   const int E = args.E;
   int* s_lo = reinterpret_cast<int*>(s_tmem + 4);
@@ -143,6 +156,9 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = kPair == 2 ? cluster_ctarank() : 0u;  // 0 = MMA leader
+  const int cid = blockIdx.x / kPair;                          // tile-scheduling unit
+  const int ncl = gridDim.x / kPair;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -151,7 +167,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], EPI_WARPS);
+      mbar_init(&tempty[a], kPair * EPI_WARPS);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -162,8 +178,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tm_x);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc<kPair>(s_tmem, TMEM_COLS);
+    tmem_relinquish<kPair>();
   }
   // Expert row ranges, clamped into [0, R) so that malformed offsets can
   // only produce wrong numbers, never out-of-range stores.
@@ -196,34 +212,42 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 31) s_start[E] = incl;
   }
   tc_fence_before_sync();
-  __syncthreads();
+  if (kPair == 2) cluster_sync();  // the peer's barriers are initialised before any remote use
+  else __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
   const int total_tiles = s_start[E];
+  // the leader's barriers as cluster addresses (the CTA's own when kPair == 1)
+  const uint32_t full_lead = kPair == 2 ? cluster_map(smem_u32(full), 0) : smem_u32(full);
+  const uint32_t tempty_lead = kPair == 2 ? cluster_map(smem_u32(tempty), 0) : smem_u32(tempty);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    const uint64_t pol_tokens = l2_policy_evict_last();   // re-read by every feature block
+    // ------------------------------------------------------------ producer (both CTAs)
+    const uint64_t pol_tokens = l2_policy_evict_last();    // re-read by every feature block
     const uint64_t pol_weights = l2_policy_evict_normal(); // shared by the CTAs of one feature block
     int s = 0;
     uint32_t ph = 0;
     uint32_t issued = 0;  // bit s: stage s has a load in flight or landed
     uint32_t last_ph = 0; // bit s: parity of the last load issued on stage s
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+    for (int tile = cid; ok && tile < total_tiles; tile += ncl) {
       const Tile t = decode(tile, s_start, s_lo, s_hi, E);
-      const int nbox = (t.ntok + B_BOX_ROWS - 1) / B_BOX_ROWS;
-      const uint32_t bytes = A_STAGE + nbox * B_BOX;
-      const int wy = t.e * args.N + t.fb * BM;
+      const int nmma = (t.ntok + 15) & ~15;
+      const int half = nmma / kPair;  // token rows staged by this CTA (a multiple of 8)
+      const int nbox = (half + B_BOX_ROWS - 1) / B_BOX_ROWS;
+      const uint32_t bytes = (uint32_t)kPair * (A_STAGE + nbox * B_BOX);
+      const int wy = t.e * args.N + t.fb * C::FEAT + (int)rank * BM;
+      const int by = t.row0 + (int)rank * half;
       for (int kb = 0; kb < args.num_kb; ++kb) {
         ok = warp_wait(&empty[s], ph ^ 1u, args.status, s_abort);
         if (!ok) break;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d(sA + s * A_STAGE, &tm_w, kb * BK, wy, &full[s], pol_weights);
+          const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes);
+          tma_load_2d_cg<kPair>(sA + s * A_STAGE, &tm_w, kb * BK, wy, fb_addr, pol_weights);
           for (int j = 0; j < nbox; ++j)
-            tma_load_2d(sB + s * B_STAGE + j * B_BOX, &tm_x, kb * BK, t.row0 + j * B_BOX_ROWS,
-                        &full[s], pol_tokens);
+            tma_load_2d_cg<kPair>(sB + s * B_STAGE + j * B_BOX, &tm_x, kb * BK,
+                                  by + j * B_BOX_ROWS, fb_addr, pol_tokens);
         }
         __syncwarp();
         issued |= 1u << s;
@@ -234,75 +258,86 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-    if (!ok) {  // let issued copies land before the CTA leaves
+    if (!ok && rank == 0) {  // let issued copies land before the CTA leaves
       int dummy = 0;
       for (int q = 0; q < STAGES; ++q)
         if ((issued >> q) & 1u)
           mbar_wait(&full[q], (last_ph >> q) & 1u, nullptr, (volatile int*)&dummy, kDrainLimitNs);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    int s = 0;
-    uint32_t ph = 0;
-    int it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++it) {
-      const Tile t = decode(tile, s_start, s_lo, s_hi, E);
-      const uint32_t nmma = (uint32_t)((t.ntok + 15) & ~15);
-      const uint32_t idesc = idesc_bf16_f32(BM, nmma);
-      const int acc = it & 1;
-      const uint32_t aph = (uint32_t)((it >> 1) & 1);
-      ok = warp_wait(&tempty[acc], aph ^ 1u, args.status, s_abort);
-      if (!ok) break;
-      tc_fence_after_sync();
-      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-      for (int kb = 0; kb < args.num_kb; ++kb) {
-        ok = warp_wait(&full[s], ph, args.status, s_abort);
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (rank == 0) {
+      const uint32_t empty_peer = kPair == 2 ? cluster_map(smem_u32(empty), 1) : 0u;
+      const uint32_t tfull_peer = kPair == 2 ? cluster_map(smem_u32(tfull), 1) : 0u;
+      int s = 0;
+      uint32_t ph = 0;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; ok && tile < total_tiles; tile += ncl, ++it) {
+        const Tile t = decode(tile, s_start, s_lo, s_hi, E);
+        const uint32_t nmma = (uint32_t)((t.ntok + 15) & ~15);
+        const uint32_t idesc = idesc_bf16_f32((uint32_t)C::FEAT, nmma);
+        const int acc = it & 1;
+        const uint32_t aph = (uint32_t)((it >> 1) & 1);
+        ok = warp_wait(&tempty[acc], aph ^ 1u, args.status, s_abort);
         if (!ok) break;
         tc_fence_after_sync();
-        if (lane == 0) {
-          const uint32_t a0 = smem_u32(sA + s * A_STAGE);
-          const uint32_t b0 = smem_u32(sB + s * B_STAGE);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < args.num_kb; ++kb) {
+          ok = warp_wait(&full[s], ph, args.status, s_abort);
+          if (!ok) break;
+          tc_fence_after_sync();
+          if (lane == 0) {
+            const uint32_t a0 = smem_u32(sA + s * A_STAGE);
+            const uint32_t b0 = smem_u32(sB + s * B_STAGE);
 #pragma unroll
-          for (int kk = 0; kk < BK / UMMA_K; ++kk)
-            tc_mma_bf16(d_tmem, smem_desc_k128(a0 + kk * UMMA_K * 2),
-                        smem_desc_k128(b0 + kk * UMMA_K * 2), idesc, (kb | kk) != 0 ? 1u : 0u);
-          tc_commit(&empty[s]);  // the stage is free once these MMAs have read it
+            for (int kk = 0; kk < BK / UMMA_K; ++kk)
+              tc_mma_bf16<kPair>(d_tmem, smem_desc_k128(a0 + kk * UMMA_K * 2),
+                                 smem_desc_k128(b0 + kk * UMMA_K * 2), idesc,
+                                 (kb | kk) != 0 ? 1u : 0u);
+            // the stage is free (in both CTAs) once these MMAs have read it
+            tc_commit<kPair>(smem_u32(&empty[s]));
+            if (kPair == 2) tc_commit<kPair>(empty_peer + (uint32_t)s * 8u);
+          }
+          __syncwarp();
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) {  // accumulator complete, in both CTAs
+          tc_commit<kPair>(smem_u32(&tfull[acc]));
+          if (kPair == 2) tc_commit<kPair>(tfull_peer + (uint32_t)acc * 8u);
         }
         __syncwarp();
-        if (++s == STAGES) {
-          s = 0;
-          ph ^= 1u;
-        }
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(&tfull[acc]);  // accumulator complete
-      __syncwarp();
-    }
-    if (!ok) {  // wait for every MMA already issued before TMEM is freed
-      if (lane == 0) tc_commit(drain);
-      __syncwarp();
-      int dummy = 0;
-      mbar_wait(drain, 0, nullptr, (volatile int*)&dummy, kDrainLimitNs);
+      if (!ok) {  // wait for every MMA already issued before TMEM is freed
+        if (lane == 0) tc_commit<kPair>(smem_u32(drain));
+        __syncwarp();
+        int dummy = 0;
+        mbar_wait(drain, 0, nullptr, (volatile int*)&dummy, kDrainLimitNs);
+      }
     }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;              // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;    // which 128 of the tile's 256 token columns
+    const int hsel = (warp - 2) >> 2;    // which 128 of the tile's 256 token columns
     uint16_t* xp = sX + (warp - 2) * 32 * 32;
     uint16_t* out = args.out;
     const int N = args.N;
     int it = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++it) {
+    for (int tile = cid; tile < total_tiles; tile += ncl, ++it) {
       const Tile t = decode(tile, s_start, s_lo, s_hi, E);
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       if (!warp_wait(&tfull[acc], aph, args.status, s_abort)) break;
       tc_fence_after_sync();
-      const int fbase = t.fb * BM + q * 32;  // this warp's 32 output features
+      // this warp's 32 output features
+      const int fbase = t.fb * C::FEAT + (int)rank * BM + q * 32;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const int c_end = min(t.ntok, half * (BN / 2) + BN / 2);
-      for (int c0 = half * (BN / 2); c0 < c_end; c0 += 32) {
+      const int c_end = min(t.ntok, hsel * (BN / 2) + BN / 2);
+      for (int c0 = hsel * (BN / 2); c0 < c_end; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + (uint32_t)c0, v);
         tmem_wait_ld();
@@ -328,14 +363,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) mbar_arrive_cluster(tempty_lead + (uint32_t)acc * 8u);
     }
   }
 
+  tc_fence_before_sync();
   __syncthreads();
+  if (kPair == 2) cluster_sync();  // no CTA leaves while its peer may still signal it
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc<kPair>(tmem_base, TMEM_COLS);
   }
 }
 
@@ -386,12 +423,67 @@ static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t
   return true;
 }
 
-static std::once_flag g_attr_once[64][2];
+struct KernelSlot {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  int max_clusters = 0;  // co-resident clusters (pairs) or CTAs of this kernel
+};
+static KernelSlot g_slots[64][4];
+
+template <bool kGelu, int kPair>
+static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
+                                  const gg::Args& args, long long max_tiles, const DeviceInfo& dev,
+                                  cudaStream_t stream) {
+  auto kern = gg::grouped_gemm_kernel<kGelu, kPair>;
+  const size_t smem_max = gg::smem_bytes<kPair>(kMaxExperts);  // one attribute for every E
+  const int slot = (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0);
+  KernelSlot& ks = g_slots[dev.device & 63][slot];
+  std::call_once(ks.once, [&] {
+    ks.err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
+    if (ks.err != cudaSuccess) return;
+    if (kPair == 2) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * dev.sm_count, 1, 1);
+      cfg.blockDim = dim3(gg::THREADS, 1, 1);
+      cfg.dynamicSmemBytes = smem_max;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      ks.err = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      ks.max_clusters = n;
+    } else {
+      ks.max_clusters = dev.sm_count;
+    }
+  });
+  if (ks.err != cudaSuccess) return ks.err;
+  if (ks.max_clusters < 1) return cudaErrorInvalidConfiguration;
+  const long long units = max_tiles < ks.max_clusters ? max_tiles : ks.max_clusters;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kPair;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(units * kPair), 1, 1);
+  cfg.blockDim = dim3(gg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = gg::smem_bytes<kPair>(args.E);
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, args);
+}
 
 cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const void* W, int E,
                                 int R, int N, int K, bool gelu, void* out,
                                 const DeviceInfo& dev, cudaStream_t stream, std::string* err) {
   if (R == 0 || N == 0) return cudaSuccess;
+  // Paired CTAs (256 features per tile) unless the layer is too narrow to fill them.
+  const int pair = N > gg::BM ? 2 : 1;
   CUtensorMap tm_w, tm_x;
   if (!make_map(&tm_w, W, (uint64_t)E * (uint64_t)N, (uint64_t)K, gg::BM, err) ||
       !make_map(&tm_x, A, (uint64_t)R, (uint64_t)K, gg::B_BOX_ROWS, err))
@@ -404,25 +496,16 @@ cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const voi
   args.R = R;
   args.N = N;
   args.K = K;
-  args.n_fblocks = (N + gg::BM - 1) / gg::BM;
+  args.n_fblocks = (N + gg::BM * pair - 1) / (gg::BM * pair);
   args.num_kb = (K + gg::BK - 1) / gg::BK;
-  const size_t smem = gg::smem_bytes(kMaxExperts);  // one attribute value for every E
-  cudaError_t e = cudaSuccess;
-  auto kern = gelu ? gg::grouped_gemm_kernel<true> : gg::grouped_gemm_kernel<false>;
-  if (dev.device >= 0 && dev.device < 64) {
-    std::call_once(g_attr_once[dev.device][gelu ? 1 : 0], [&] {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    });
-  } else {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  }
-  if (e != cudaSuccess) return e;
   // an upper bound on the tile count: every expert adds at most one partial token block
   const long long max_tiles =
       ((long long)(R + gg::BN - 1) / gg::BN + E) * (long long)args.n_fblocks;
-  const int grid = (int)(max_tiles < dev.sm_count ? max_tiles : dev.sm_count);
-  kern<<<grid, gg::THREADS, gg::smem_bytes(E), stream>>>(tm_w, tm_x, args);
-  return cudaGetLastError();
+  if (pair == 2)
+    return gelu ? launch_variant<true, 2>(tm_w, tm_x, args, max_tiles, dev, stream)
+                : launch_variant<false, 2>(tm_w, tm_x, args, max_tiles, dev, stream);
+  return gelu ? launch_variant<true, 1>(tm_w, tm_x, args, max_tiles, dev, stream)
+              : launch_variant<false, 1>(tm_w, tm_x, args, max_tiles, dev, stream);
 }
 
 }  // namespace moe

@@ -6,15 +6,16 @@
 //
 //   out[r, n] = act( sum_c A[r, c] * W[e, n, c] )   for r in expert e's block
 //
-// Design (one persistent CTA per SM, 10 warps):
+// Design (one persistent CTA per SM, 11 warps):
 //   * Operand roles are swapped with respect to the usual token-major GEMM:
 //     128 weight rows (output features) form the MMA's M side, and up to 256
 //     token rows of one expert form its N side.  N is chosen per tile at run
 //     time (a multiple of 16), so a ragged expert block of c rows costs
 //     ceil(c/16)*16 columns of MMA work instead of a full 128-row tile.
-//   * warp 0 (one lane) streams K-blocks of 64 through a 4-stage ring with
-//     TMA (128-byte swizzle), warp 1 (one lane) issues tcgen05.mma into one
-//     of two TMEM accumulators (2 x 256 fp32 columns), warps 2-9 drain the
+//   * warps 0 and 1 (one lane each) stream K-blocks of 64 of the weight and
+//     the token operand through a ring of stages with TMA (128-byte swizzle),
+//     warp 2 (one lane) issues tcgen05.mma into one of two TMEM
+//     accumulators (2 x 256 fp32 columns), warps 3-10 drain the
 //     other accumulator (tcgen05.ld), apply GELU, round to bf16, transpose
 //     through shared memory and store token rows.  Each epilogue warp owns
 //     one TMEM lane quarter (32 features) and one half of the tile's tokens,
@@ -41,8 +42,16 @@ constexpr int UMMA_K = 16;                   // K per tcgen05.mma (kind::f16)
 constexpr int A_STAGE = BM * BK * 2;         // 16 KB of weight rows per CTA and stage
 constexpr int B_BOX_ROWS = 32;
 constexpr int B_BOX = B_BOX_ROWS * BK * 2;   // 4 KB
+// Token rows a CTA stages for a full tile (256 tokens split over a pair, or
+// 128 with one CTA) are loaded with one 16 KB request instead of four 4 KB
+// ones, since TMA throughput grows with the request size; a half-tile of at
+// least kWideMin rows also takes the single request (over-fetching at most
+// 32 rows into the stage buffer, which holds 128).
+constexpr int B_WIDE_ROWS = 128;
+constexpr int kWideMin = 96;
 constexpr int EPI_WARPS = 8;                 // two per SM sub-partition
-constexpr int THREADS = 64 + EPI_WARPS * 32; // producer, MMA, 8 epilogue warps
+constexpr int EPI_WARP0 = 3;                 // warps 0-1 load, warp 2 issues MMAs
+constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int XPOSE = EPI_WARPS * 32 * 32 * 2;  // per-warp 32x32 bf16 transpose tile
 constexpr uint64_t kDrainLimitNs = 20ull * 1000ull * 1000ull;  // 20 ms
@@ -78,6 +87,12 @@ struct Tile {
   int e, fb, row0, ntok;
 };
 
+// Token blocks of an expert with c rows: ceil(c / 256) blocks of 256 rows,
+// the last one ragged.  (Splitting c evenly across the blocks was measured
+// slower: the kernel is bound by operand loads, and even blocks cost more
+// load requests than one ragged block.)
+__device__ __forceinline__ int token_blocks(int c) { return (c + BN - 1) / BN; }
+
 __device__ __forceinline__ Tile decode(int tile, const int* s_start, const int* s_lo,
                                        const int* s_hi, int E) {
   int lo = 0, hi = E - 1;
@@ -88,11 +103,12 @@ __device__ __forceinline__ Tile decode(int tile, const int* s_start, const int* 
   Tile t;
   t.e = lo;
   const int local = tile - s_start[lo];
-  const int ntb = (s_hi[lo] - s_lo[lo] + BN - 1) / BN;
+  const int c = s_hi[lo] - s_lo[lo];
+  const int ntb = token_blocks(c);
   t.fb = local / ntb;
   const int tb = local - t.fb * ntb;
   t.row0 = s_lo[lo] + tb * BN;
-  t.ntok = min(BN, s_hi[lo] - t.row0);
+  t.ntok = min(BN, c - tb * BN);
   return t;
 }
 
@@ -131,7 +147,8 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
 template <bool kGelu, int kPair>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
-                        const __grid_constant__ CUtensorMap tm_x, const Args args) {
+                        const __grid_constant__ CUtensorMap tm_x,
+                        const __grid_constant__ CUtensorMap tm_xw, const Args args) {
   using C = Cfg<kPair>;
   constexpr int STAGES = C::STAGES;
   constexpr int B_STAGE = C::B_STAGE;
@@ -162,7 +179,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], 2);  // the two producers of the leader CTA
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -176,8 +193,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 32) {
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_xw);
   }
-  if (warp == 1) {
+  if (warp == 2) {
     tmem_alloc<kPair>(s_tmem, TMEM_COLS);
     tmem_relinquish<kPair>();
   }
@@ -197,7 +215,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int per = (E + 31) / 32;
     const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
     int sum = 0;
-    for (int e = e0; e < e1; ++e) sum += ((s_hi[e] - s_lo[e] + BN - 1) / BN) * args.n_fblocks;
+    for (int e = e0; e < e1; ++e) sum += token_blocks(s_hi[e] - s_lo[e]) * args.n_fblocks;
     int incl = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -207,7 +225,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     int run = incl - sum;
     for (int e = e0; e < e1; ++e) {
       s_start[e] = run;
-      run += ((s_hi[e] - s_lo[e] + BN - 1) / BN) * args.n_fblocks;
+      run += token_blocks(s_hi[e] - s_lo[e]) * args.n_fblocks;
     }
     if (lane == 31) s_start[E] = incl;
   }
@@ -221,10 +239,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t full_lead = kPair == 2 ? cluster_map(smem_u32(full), 0) : smem_u32(full);
   const uint32_t tempty_lead = kPair == 2 ? cluster_map(smem_u32(tempty), 0) : smem_u32(tempty);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    const uint64_t pol_tokens = l2_policy_evict_last();    // re-read by every feature block
-    const uint64_t pol_weights = l2_policy_evict_normal(); // shared by the CTAs of one feature block
+  if (warp <= 1) {
+    // ------------------------------------------------------------ producers (both CTAs)
+    // Warp 0 streams the weight rows, warp 1 the token rows, each into the
+    // same ring of stages: two issuing threads keep twice as many TMA
+    // requests in flight as one.  In the leader CTA each arms the stage's
+    // barrier with the bytes of its operand in both CTAs of the pair.
+    const bool is_w = warp == 0;
+    const uint64_t pol = is_w ? l2_policy_evict_normal()  // shared by the CTAs of a feature block
+                              : l2_policy_evict_last();   // re-read by every feature block
     int s = 0;
     uint32_t ph = 0;
     uint32_t issued = 0;  // bit s: stage s has a load in flight or landed
@@ -234,8 +257,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const Tile t = decode(tile, s_start, s_lo, s_hi, E);
       const int nmma = (t.ntok + 15) & ~15;
       const int half = nmma / kPair;  // token rows staged by this CTA (a multiple of 8)
+      const bool wide = half >= kWideMin;
       const int nbox = (half + B_BOX_ROWS - 1) / B_BOX_ROWS;
-      const uint32_t bytes = (uint32_t)kPair * (A_STAGE + nbox * B_BOX);
+      const uint32_t bytes = is_w ? (uint32_t)(kPair * A_STAGE)
+                                  : (uint32_t)kPair * (wide ? B_WIDE_ROWS * BK * 2 : nbox * B_BOX);
       const int wy = t.e * args.N + t.fb * C::FEAT + (int)rank * BM;
       const int by = t.row0 + (int)rank * half;
       for (int kb = 0; kb < args.num_kb; ++kb) {
@@ -244,10 +269,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d_cg<kPair>(sA + s * A_STAGE, &tm_w, kb * BK, wy, fb_addr, pol_weights);
-          for (int j = 0; j < nbox; ++j)
-            tma_load_2d_cg<kPair>(sB + s * B_STAGE + j * B_BOX, &tm_x, kb * BK,
-                                  by + j * B_BOX_ROWS, fb_addr, pol_tokens);
+          if (is_w) {
+            tma_load_2d_cg<kPair>(sA + s * A_STAGE, &tm_w, kb * BK, wy, fb_addr, pol);
+          } else if (wide) {  // (nearly) a full half-tile: one large request
+            tma_load_2d_cg<kPair>(sB + s * B_STAGE, &tm_xw, kb * BK, by, fb_addr, pol);
+          } else {
+            for (int j = 0; j < nbox; ++j)
+              tma_load_2d_cg<kPair>(sB + s * B_STAGE + j * B_BOX, &tm_x, kb * BK,
+                                    by + j * B_BOX_ROWS, fb_addr, pol);
+          }
         }
         __syncwarp();
         issued |= 1u << s;
@@ -258,13 +288,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-    if (!ok && rank == 0) {  // let issued copies land before the CTA leaves
+    if (!ok && rank == 0 && is_w) {  // let issued copies land before the CTA leaves
       int dummy = 0;
       for (int q = 0; q < STAGES; ++q)
         if ((issued >> q) & 1u)
           mbar_wait(&full[q], (last_ph >> q) & 1u, nullptr, (volatile int*)&dummy, kDrainLimitNs);
     }
-  } else if (warp == 1) {
+  } else if (warp == 2) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (rank == 0) {
       const uint32_t empty_peer = kPair == 2 ? cluster_map(smem_u32(empty), 1) : 0u;
@@ -322,8 +352,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;              // TMEM lane quarter this warp may access
-    const int hsel = (warp - 2) >> 2;    // which 128 of the tile's 256 token columns
-    uint16_t* xp = sX + (warp - 2) * 32 * 32;
+    const int hsel = (warp - EPI_WARP0) >> 2;  // which 128 of the tile's 256 token columns
+    uint16_t* xp = sX + (warp - EPI_WARP0) * 32 * 32;
     uint16_t* out = args.out;
     const int N = args.N;
     int it = 0;
@@ -370,7 +400,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before_sync();
   __syncthreads();
   if (kPair == 2) cluster_sync();  // no CTA leaves while its peer may still signal it
-  if (warp == 1) {
+  if (warp == 2) {
     tc_fence_after_sync();
     tmem_dealloc<kPair>(tmem_base, TMEM_COLS);
   }
@@ -432,7 +462,7 @@ static KernelSlot g_slots[64][4];
 
 template <bool kGelu, int kPair>
 static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
-                                  const gg::Args& args, long long max_tiles, const DeviceInfo& dev,
+                                  const CUtensorMap& tm_xw, const gg::Args& args, long long max_tiles, const DeviceInfo& dev,
                                   cudaStream_t stream) {
   auto kern = gg::grouped_gemm_kernel<kGelu, kPair>;
   const size_t smem_max = gg::smem_bytes<kPair>(kMaxExperts);  // one attribute for every E
@@ -475,7 +505,7 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, args);
+  return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, tm_xw, args);
 }
 
 cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const void* W, int E,
@@ -484,9 +514,10 @@ cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const voi
   if (R == 0 || N == 0) return cudaSuccess;
   // Paired CTAs (256 features per tile) unless the layer is too narrow to fill them.
   const int pair = N > gg::BM ? 2 : 1;
-  CUtensorMap tm_w, tm_x;
+  CUtensorMap tm_w, tm_x, tm_xw;
   if (!make_map(&tm_w, W, (uint64_t)E * (uint64_t)N, (uint64_t)K, gg::BM, err) ||
-      !make_map(&tm_x, A, (uint64_t)R, (uint64_t)K, gg::B_BOX_ROWS, err))
+      !make_map(&tm_x, A, (uint64_t)R, (uint64_t)K, gg::B_BOX_ROWS, err) ||
+      !make_map(&tm_xw, A, (uint64_t)R, (uint64_t)K, gg::B_WIDE_ROWS, err))
     return cudaErrorInvalidValue;
   gg::Args args;
   args.offsets = offsets;
@@ -502,10 +533,10 @@ cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const voi
   const long long max_tiles =
       ((long long)(R + gg::BN - 1) / gg::BN + E) * (long long)args.n_fblocks;
   if (pair == 2)
-    return gelu ? launch_variant<true, 2>(tm_w, tm_x, args, max_tiles, dev, stream)
-                : launch_variant<false, 2>(tm_w, tm_x, args, max_tiles, dev, stream);
-  return gelu ? launch_variant<true, 1>(tm_w, tm_x, args, max_tiles, dev, stream)
-              : launch_variant<false, 1>(tm_w, tm_x, args, max_tiles, dev, stream);
+    return gelu ? launch_variant<true, 2>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
+                : launch_variant<false, 2>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream);
+  return gelu ? launch_variant<true, 1>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
+              : launch_variant<false, 1>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream);
 }
 
 }  // namespace moe

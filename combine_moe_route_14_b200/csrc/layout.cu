@@ -35,25 +35,29 @@ constexpr uint32_t kFlagAggregate = 1u << 30;
 constexpr uint32_t kFlagInclusive = 2u << 30;
 constexpr uint32_t kValueMask = (1u << 30) - 1u;
 
-// Reads the expert id of slot i (or -1 past the end / out of range).
-__device__ __forceinline__ int load_key(const int32_t* idx, int i, int end, int E,
-                                        uint32_t* status) {
-  if (i >= end) return -1;
-  const int e = __ldg(idx + i);
-  if (e < 0 || e >= E) {
-    flag_error(status, MOE_DEV_BAD_EXPERT_ID);
-    return -1;
+// Copies the expert ids of slots [begin, end) into shared memory (one
+// coalesced pass, all loads in flight together), replacing ids outside
+// [0, E) by -1 and flagging them.
+__device__ __forceinline__ void stage_keys(const int32_t* idx, int begin, int end, int E,
+                                           int* keys, uint32_t* status) {
+  for (int i = begin + threadIdx.x; i < end; i += blockDim.x) {
+    int e = __ldg(idx + i);
+    if (e < 0 || e >= E) {
+      if (status) flag_error(status, MOE_DEV_BAD_EXPERT_ID);
+      e = -1;
+    }
+    keys[i - begin] = e;
   }
-  return e;
 }
 
-// Per-warp histogram of the slots [begin, end) owned by this warp, walked in
-// 32-slot chunks.  warp_hist is this warp's row of E counters.
-__device__ __forceinline__ void warp_histogram(const int32_t* idx, int begin, int end, int E,
-                                               int* warp_hist, uint32_t* status) {
+// Per-warp histogram of the staged slots [begin, end) (indices into `keys`)
+// owned by this warp, walked in 32-slot chunks.  warp_hist is this warp's
+// row of E counters.
+__device__ __forceinline__ void warp_histogram(const int* keys, int begin, int end,
+                                               int* warp_hist) {
   const int lane = threadIdx.x & 31;
   for (int c = begin; c < end; c += 32) {
-    const int key = load_key(idx, c + lane, end, E, status);
+    const int key = c + lane < end ? keys[c + lane] : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, key);
     const int leader = __ffs(peers) - 1;
     if (key >= 0 && lane == leader) warp_hist[key] += __popc(peers);
@@ -62,15 +66,16 @@ __device__ __forceinline__ void warp_histogram(const int32_t* idx, int begin, in
 }
 
 // Second walk over the same slots: stable rank within the warp's running
-// counts, then row = base[key] + warp_run[key] + rank-in-chunk.
-__device__ __forceinline__ void warp_scatter(const int32_t* idx, int begin, int end, int E,
+// counts, then row = base[key] + warp_run[key] + rank-in-chunk.  `first` is
+// the global slot number of keys[0].
+__device__ __forceinline__ void warp_scatter(const int* keys, int first, int begin, int end,
                                              int* warp_run, const int* base, int32_t* row_of,
-                                             int32_t* src_of, uint32_t* status) {
+                                             int32_t* src_of) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt_mask = (1u << lane) - 1u;
   for (int c = begin; c < end; c += 32) {
-    const int i = c + lane;
-    const int key = load_key(idx, i, end, E, nullptr);  // already flagged by the histogram
+    const int li = c + lane;
+    const int key = li < end ? keys[li] : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, key);
     int row = 0;
     if (key >= 0) row = base[key] + warp_run[key] + __popc(peers & lt_mask);
@@ -78,14 +83,13 @@ __device__ __forceinline__ void warp_scatter(const int32_t* idx, int begin, int 
     const int leader = __ffs(peers) - 1;
     if (key >= 0 && lane == leader) warp_run[key] += __popc(peers);
     if (key >= 0) {
-      row_of[i] = row;
-      src_of[row] = i;
-    } else if (i < end) {
-      row_of[i] = -1;  // a bad expert id has no row
+      row_of[first + li] = row;
+      src_of[row] = first + li;
+    } else if (li < end) {
+      row_of[first + li] = -1;  // a bad expert id has no row
     }
     __syncwarp();
   }
-  (void)status;
 }
 
 // In-place exclusive scan of s[0..n) by the whole CTA (n <= 2 * blockDim).
@@ -145,21 +149,23 @@ __device__ void scan_over_warps(int* hist, int E, int* agg) {
 
 // ---------------------------------------------------------------------------
 // one-CTA path
-// smem: hist[kLayoutWarps][E] | base[E+1] | tmp[33]
+// smem: keys[R] | hist[kLayoutWarps][E] | base[E+1] | tmp[33]
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kLayoutThreads)
     layout_single_kernel(const int32_t* __restrict__ idx, int R, int E, int32_t* counts,
                          int32_t* offsets, int32_t* row_of, int32_t* src_of, uint32_t* status) {
   extern __shared__ int smem_i[];
-  int* hist = smem_i;
+  int* keys = smem_i;
+  int* hist = keys + R;
   int* base = hist + kLayoutWarps * E;
   int* tmp = base + E + 1;
+  stage_keys(idx, 0, R, E, keys, status);
   for (int i = threadIdx.x; i < kLayoutWarps * E; i += blockDim.x) hist[i] = 0;
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   const int per_warp = ((R + kLayoutWarps * 32 - 1) / (kLayoutWarps * 32)) * 32;
   const int begin = min(R, warp * per_warp), end = min(R, begin + per_warp);
-  warp_histogram(idx, begin, end, E, hist + warp * E, status);
+  warp_histogram(keys, begin, end, hist + warp * E);
   __syncthreads();
   scan_over_warps(hist, E, base);
   __syncthreads();
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int total = block_exclusive_scan(base, E, tmp);
   for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = base[e];
   if (threadIdx.x == 0) offsets[E] = total;
-  warp_scatter(idx, begin, end, E, hist + warp * E, base, row_of, src_of, status);
+  warp_scatter(keys, 0, begin, end, hist + warp * E, base, row_of, src_of);
 }
 
 // ---------------------------------------------------------------------------
@@ -191,8 +197,9 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int tile_begin = blockIdx.x * kTile;
   const int tile_end = min(R, tile_begin + kTile);
   for (int i = tile_begin + threadIdx.x; i < tile_end; i += blockDim.x) {
-    const int e = load_key(idx, i, tile_end, E, status);
-    if (e >= 0) atomicAdd(&hist[e], 1);  // order of adds does not matter for a count
+    const int e = __ldg(idx + i);
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);  // order of adds does not matter for a count
+    else flag_error(status, MOE_DEV_BAD_EXPERT_ID);
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -201,7 +208,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
 
 // ---------------------------------------------------------------------------
 // multi-CTA path, kernel 2: per-tile stable ranks + decoupled look-back.
-// smem: hist[kLayoutWarps][E] | agg[E] | base[E+1] | tmp[33] | tile id
+// smem: keys[kTile] | hist[kLayoutWarps][E] | agg[E] | base[E+1] | tmp[33] | tile id
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kLayoutThreads)
     layout_scatter_kernel(const int32_t* __restrict__ idx, int R, int E,
@@ -209,7 +216,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
                           int32_t* src_of, uint32_t* lookback, uint32_t* ticket,
                           uint32_t* status) {
   extern __shared__ int smem_i[];
-  int* hist = smem_i;
+  int* keys = smem_i;
+  int* hist = keys + kTile;
   int* agg = hist + kLayoutWarps * E;
   int* base = agg + E;
   int* tmp = base + E + 1;
@@ -220,12 +228,14 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int tile = *s_tile;
   const int tile_begin = tile * kTile;
   const int tile_end = min(R, tile_begin + kTile);
-  const int warp = threadIdx.x >> 5;
   const int n = tile_end - tile_begin;
+  stage_keys(idx, tile_begin, tile_end, E, keys, nullptr);  // kernel 1 flagged bad ids
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
   const int per_warp = ((n + kLayoutWarps * 32 - 1) / (kLayoutWarps * 32)) * 32;
-  const int begin = min(tile_end, tile_begin + warp * per_warp);
-  const int end = min(tile_end, begin + per_warp);
-  warp_histogram(idx, begin, end, E, hist + warp * E, nullptr);  // kernel 1 flagged bad ids
+  const int begin = min(n, warp * per_warp);
+  const int end = min(n, begin + per_warp);
+  warp_histogram(keys, begin, end, hist + warp * E);
   __syncthreads();
   scan_over_warps(hist, E, agg);
   __syncthreads();
@@ -280,7 +290,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x) base[e] += agg[e];
   __syncthreads();
-  warp_scatter(idx, begin, end, E, hist + warp * E, base, row_of, src_of, status);
+  warp_scatter(keys, tile_begin, begin, end, hist + warp * E, base, row_of, src_of);
 }
 
 // ---------------------------------------------------------------------------
@@ -299,7 +309,7 @@ cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int
                           int32_t* row_of, int32_t* src_of, void* ws, const DeviceInfo& dev,
                           cudaStream_t stream) {
   if (R <= kSingleMax) {
-    const size_t smem = (size_t)(kLayoutWarps * E + E + 1 + 33) * sizeof(int);
+    const size_t smem = (size_t)(R + kLayoutWarps * E + E + 1 + 33) * sizeof(int);
     if (smem > 48 * 1024) {
       cudaError_t err = cudaFuncSetAttribute(layout_single_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -318,7 +328,7 @@ cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int
       idx, R, E, counts, lookback, ticket, dev.status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  const size_t smem = (size_t)(kLayoutWarps * E + E + E + 1 + 33 + 1) * sizeof(int);
+  const size_t smem = (size_t)(kTile + kLayoutWarps * E + E + E + 1 + 33 + 1) * sizeof(int);
   if (smem > 48 * 1024) {
     err = cudaFuncSetAttribute(layout_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)smem);

@@ -16,13 +16,17 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // router linear: L[t, e] = sum_c X[t, c] * Wr[e, c]   (fp32 accumulate)
 //
-// One warp handles kTokPerWarp consecutive tokens and experts in groups of 8:
-// each lane owns 8 consecutive bf16 of the row per step (16-byte loads), keeps
-// kTokPerWarp x 8 fp32 partial sums, and the warp reduces them at the end.
-// Router weights are small (E*d*2 bytes) and stay in L1/L2.
+// HBM-bound on X (T*d*2 bytes).  A CTA of 8 warps takes 16 tokens, two per
+// warp; each lane owns 16-byte slices (8 bf16) of the row and keeps
+// kUnroll slices of both tokens in flight before the FMAs.  Router weights
+// (E*d*2 bytes) are staged once per CTA in shared memory when they fit,
+// else read through L1.  Experts are processed in groups of 8 (one partial
+// sum per token and expert per lane), then reduced across the warp.
 // ---------------------------------------------------------------------------
-constexpr int kTokPerWarp = 4;
 constexpr int kRouterWarps = 8;
+constexpr int kTokPerWarp = 2;
+constexpr int kRouterUnroll = 4;
+constexpr int kRouterSmemMax = 96 * 1024;
 
 __device__ __forceinline__ float dot8(const uint4& a, const uint4& b, float acc) {
   acc = fmaf(bf16_lo(a.x), bf16_lo(b.x), acc);
@@ -36,47 +40,67 @@ __device__ __forceinline__ float dot8(const uint4& a, const uint4& b, float acc)
   return acc;
 }
 
+template <bool kSmemW>
 __global__ void __launch_bounds__(kRouterWarps * 32)
     router_logits_kernel(const uint4* __restrict__ X, const uint4* __restrict__ Wr, int T,
                          int row_vecs, int E, float* __restrict__ L) {
-  const int warp = blockIdx.x * kRouterWarps + (threadIdx.x >> 5);
+  extern __shared__ uint4 s_w[];
+  if (kSmemW) {
+    const int n = E * row_vecs;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) s_w[i] = __ldg(Wr + i);
+    __syncthreads();
+  }
+  const uint4* W = kSmemW ? s_w : Wr;
   const int lane = threadIdx.x & 31;
-  const int t0 = warp * kTokPerWarp;
+  const int t0 = (blockIdx.x * kRouterWarps + (threadIdx.x >> 5)) * kTokPerWarp;
   if (t0 >= T) return;
-  const int ntok = min(kTokPerWarp, T - t0);
+  const bool two = t0 + 1 < T;
+  const uint4* x0 = X + (size_t)t0 * row_vecs;
+  const uint4* x1 = X + (size_t)(two ? t0 + 1 : t0) * row_vecs;
   for (int e0 = 0; e0 < E; e0 += 8) {
     const int ne = min(8, E - e0);
-    float acc[kTokPerWarp][8];
+    float acc0[8], acc1[8];
 #pragma unroll
-    for (int i = 0; i < kTokPerWarp; ++i)
+    for (int j = 0; j < 8; ++j) acc0[j] = acc1[j] = 0.f;
+    for (int c0 = lane; c0 < row_vecs; c0 += 32 * kRouterUnroll) {
+      uint4 a[kRouterUnroll], b[kRouterUnroll];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-    for (int c = lane; c < row_vecs; c += 32) {
-      uint4 xv[kTokPerWarp];
+      for (int u = 0; u < kRouterUnroll; ++u) {
+        const int c = c0 + u * 32;
+        if (c < row_vecs) {
+          a[u] = ld_stream_v4(x0 + c);
+          b[u] = ld_stream_v4(x1 + c);
+        }
+      }
 #pragma unroll
-      for (int i = 0; i < kTokPerWarp; ++i)
-        xv[i] = (i < ntok) ? ld_stream_v4(X + (size_t)(t0 + i) * row_vecs + c) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < kRouterUnroll; ++u) {
+        const int c = c0 + u * 32;
+        if (c < row_vecs) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < ne) {
-          const uint4 wv = __ldg(Wr + (size_t)(e0 + j) * row_vecs + c);
-#pragma unroll
-          for (int i = 0; i < kTokPerWarp; ++i) acc[i][j] = dot8(xv[i], wv, acc[i][j]);
+          for (int j = 0; j < 8; ++j) {
+            if (j < ne) {
+              const uint4 w = kSmemW ? W[(size_t)(e0 + j) * row_vecs + c]
+                                     : __ldg(W + (size_t)(e0 + j) * row_vecs + c);
+              acc0[j] = dot8(a[u], w, acc0[j]);
+              acc1[j] = dot8(b[u], w, acc1[j]);
+            }
+          }
         }
       }
     }
 #pragma unroll
-    for (int i = 0; i < kTokPerWarp; ++i)
+    for (int j = 0; j < 8; ++j) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float v = acc[i][j];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        acc[i][j] = v;
+      for (int off = 16; off > 0; off >>= 1) {
+        acc0[j] += __shfl_xor_sync(0xffffffffu, acc0[j], off);
+        acc1[j] += __shfl_xor_sync(0xffffffffu, acc1[j], off);
       }
-    if (lane == 0) {
-      for (int i = 0; i < ntok; ++i)
-        for (int j = 0; j < ne; ++j) L[(size_t)(t0 + i) * E + e0 + j] = acc[i][j];
+    }
+    // lane j < ne writes expert e0+j of token t0, lane 8+j of token t0+1
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (lane == j && j < ne) L[(size_t)t0 * E + e0 + j] = acc0[j];
+      if (two && lane == 8 + j && j < ne) L[(size_t)(t0 + 1) * E + e0 + j] = acc1[j];
     }
   }
 }
@@ -84,10 +108,22 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
 cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, int E, float* L,
                                  cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const int warps = (T + kTokPerWarp - 1) / kTokPerWarp;
-  const int blocks = (warps + kRouterWarps - 1) / kRouterWarps;
-  router_logits_kernel<<<blocks, kRouterWarps * 32, 0, stream>>>(
-      static_cast<const uint4*>(X), static_cast<const uint4*>(Wr), T, d / 8, E, L);
+  const int per_cta = kRouterWarps * kTokPerWarp;
+  const int blocks = (T + per_cta - 1) / per_cta;
+  const size_t wbytes = (size_t)E * d * 2;
+  const uint4* x = static_cast<const uint4*>(X);
+  const uint4* w = static_cast<const uint4*>(Wr);
+  if (wbytes <= (size_t)kRouterSmemMax) {
+    if (wbytes > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           kRouterSmemMax);
+      if (e != cudaSuccess) return e;
+    }
+    router_logits_kernel<true><<<blocks, kRouterWarps * 32, wbytes, stream>>>(x, w, T, d / 8, E, L);
+  } else {
+    router_logits_kernel<false><<<blocks, kRouterWarps * 32, 0, stream>>>(x, w, T, d / 8, E, L);
+  }
   return cudaGetLastError();
 }
 

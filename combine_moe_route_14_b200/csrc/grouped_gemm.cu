@@ -13,11 +13,13 @@
 //     time (a multiple of 16), so a ragged expert block of c rows costs
 //     ceil(c/16)*16 columns of MMA work instead of a full 128-row tile.
 //   * warps 0 and 1 (one lane each) stream K-blocks of 64 of the weight and
-//     the token operand through a ring of stages with TMA (128-byte swizzle),
+//     the token operand through a ring of 6-7 stages (as many as shared
+//     memory holds) with TMA (128-byte swizzle),
 //     warp 2 (one lane) issues tcgen05.mma into one of two TMEM
 //     accumulators (2 x 256 fp32 columns), warps 3-10 drain the
-//     other accumulator (tcgen05.ld), apply GELU, round to bf16, transpose
-//     through shared memory and store token rows.  Each epilogue warp owns
+//     other accumulator (tcgen05.ld), apply GELU, round to bf16 and store
+//     token rows (a warp writes 32 consecutive features of a row per store
+//     instruction).  Each epilogue warp owns
 //     one TMEM lane quarter (32 features) and one half of the tile's tokens,
 //     so every SM sub-partition runs two of them.  Mainloop and epilogue of
 //     consecutive tiles overlap.
@@ -53,7 +55,8 @@ constexpr int EPI_WARPS = 8;                 // two per SM sub-partition
 constexpr int EPI_WARP0 = 3;                 // warps 0-1 load, warp 2 issues MMAs
 constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
-constexpr int XPOSE = EPI_WARPS * 32 * 32 * 2;  // per-warp 32x32 bf16 transpose tile
+constexpr int MAX_STAGES = 8;                // barrier slots; the ring uses Args::stages of them
+constexpr size_t kSmemBudget = 232448;       // B200 opt-in shared memory per block
 constexpr uint64_t kDrainLimitNs = 20ull * 1000ull * 1000ull;  // 20 ms
 
 // kPair = 1: one CTA computes a 128-feature x N-token tile (cta_group::1).
@@ -62,16 +65,27 @@ constexpr uint64_t kDrainLimitNs = 20ull * 1000ull * 1000ull;  // 20 ms
 //   weight rows and half of the token rows, so per-SM shared-memory traffic
 //   and L2 reads per FLOP are a third lower, and 6 stages fit.
 template <int kPair> struct Cfg {
-  static constexpr int STAGES = kPair == 2 ? 6 : 4;
   static constexpr int B_STAGE = (BN / kPair) * BK * 2;  // token rows this CTA stages
-  static constexpr int NUM_BARS = 2 * STAGES + 4 + 1;
+  static constexpr int STAGE = A_STAGE + B_STAGE;
+  static constexpr int NUM_BARS = 2 * MAX_STAGES + 4 + 1;
   static constexpr int FEAT = BM * kPair;                // output features per tile
 };
 
+// Shared memory: the stage ring, barriers, and the per-expert tile table.
 template <int kPair>
-__host__ __device__ constexpr size_t smem_bytes(int E) {
-  return 1024 /* alignment slack */ + (size_t)Cfg<kPair>::STAGES * (A_STAGE + Cfg<kPair>::B_STAGE) +
-         XPOSE + Cfg<kPair>::NUM_BARS * 8 + 16 + (size_t)3 * (E + 1) * sizeof(int);
+__host__ __device__ constexpr size_t fixed_smem(int E) {
+  return 1024 /* alignment slack */ + Cfg<kPair>::NUM_BARS * 8 + 16 + (size_t)3 * (E + 1) * sizeof(int);
+}
+template <int kPair>
+__host__ __device__ constexpr size_t smem_bytes(int E, int stages) {
+  return fixed_smem<kPair>(E) + (size_t)stages * Cfg<kPair>::STAGE;
+}
+// As many stages as fit (more bytes in flight hide more load latency).
+template <int kPair>
+inline int stages_for(int E) {
+  const size_t avail = kSmemBudget - fixed_smem<kPair>(E);
+  const int n = (int)(avail / Cfg<kPair>::STAGE);
+  return n < MAX_STAGES ? n : MAX_STAGES;
 }
 
 struct Args {
@@ -81,6 +95,7 @@ struct Args {
   int E, R, N, K;
   int n_fblocks;           // ceil(N / features per tile)
   int num_kb;              // ceil(K / BK)
+  int stages;              // ring depth (<= MAX_STAGES)
 };
 
 struct Tile {
@@ -150,18 +165,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                         const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_xw, const Args args) {
   using C = Cfg<kPair>;
-  constexpr int STAGES = C::STAGES;
+  const int STAGES = args.stages;
   constexpr int B_STAGE = C::B_STAGE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * A_STAGE;
-  uint16_t* sX = reinterpret_cast<uint16_t*>(sB + STAGES * B_STAGE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sX) + XPOSE);
-  uint64_t* full = bars;               // used in the leader CTA: both CTAs' bytes land here
-  uint64_t* empty = bars + STAGES;     // per CTA: the MMAs have read this stage
-  uint64_t* tfull = bars + 2 * STAGES; // per CTA: accumulator ready
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  uint64_t* full = bars;                   // used in the leader CTA: both CTAs' bytes land here
+  uint64_t* empty = bars + MAX_STAGES;     // per CTA: the MMAs have read this stage
+  uint64_t* tfull = bars + 2 * MAX_STAGES; // per CTA: accumulator ready
   uint64_t* tempty = tfull + 2;        // leader CTA: both CTAs' epilogues drained it
   uint64_t* drain = tempty + 2;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
@@ -352,8 +366,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;              // TMEM lane quarter this warp may access
-    const int hsel = (warp - EPI_WARP0) >> 2;  // which 128 of the tile's 256 token columns
-    uint16_t* xp = sX + (warp - EPI_WARP0) * 32 * 32;
+    // which span of the tile's 256 token columns (EPI_WARPS / 4 spans)
+    constexpr int SPAN = BN / (EPI_WARPS / 4);
+    const int hsel = (warp - EPI_WARP0) >> 2;
     uint16_t* out = args.out;
     const int N = args.N;
     int it = 0;
@@ -363,33 +378,27 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       if (!warp_wait(&tfull[acc], aph, args.status, s_abort)) break;
       tc_fence_after_sync();
-      // this warp's 32 output features
-      const int fbase = t.fb * C::FEAT + (int)rank * BM + q * 32;
+      // this lane's output feature; the warp covers 32 consecutive features
+      const int f = t.fb * C::FEAT + (int)rank * BM + q * 32 + lane;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const int c_end = min(t.ntok, hsel * (BN / 2) + BN / 2);
-      for (int c0 = hsel * (BN / 2); c0 < c_end; c0 += 32) {
+      const int c_end = min(t.ntok, hsel * SPAN + SPAN);
+      for (int c0 = hsel * SPAN; c0 < c_end; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + (uint32_t)c0, v);
         tmem_wait_ld();
-        // v[j] = accumulator of feature (fbase + lane), token (c0 + j)
+        // v[j] = accumulator of feature f, token (c0 + j).  For a fixed j the
+        // warp writes 32 consecutive features of one token row: 64 contiguous
+        // bytes per store instruction, no shared-memory transpose needed.
+        const int jmax = min(32, t.ntok - c0);
+        uint16_t* col = out + (size_t)(t.row0 + c0) * N + f;
+        if (f < N) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          float x = __uint_as_float(v[j]);
-          if (kGelu) x = gelu_erf(x);
-          xp[j * 32 + lane] = to_bf16_bits(x);
-        }
-        __syncwarp();
-#pragma unroll
-        for (int pass = 0; pass < 4; ++pass) {
-          const int j = pass * 8 + (lane >> 2);
-          const int f0 = fbase + (lane & 3) * 8;
-          const int tok = c0 + j;
-          if (tok < t.ntok && f0 < N) {
-            const uint4 val = *reinterpret_cast<const uint4*>(xp + j * 32 + (lane & 3) * 8);
-            *reinterpret_cast<uint4*>(out + (size_t)(t.row0 + tok) * N + f0) = val;
+          for (int j = 0; j < 32; ++j) {
+            float x = __uint_as_float(v[j]);
+            if (kGelu) x = gelu_erf(x);
+            if (j < jmax) col[(size_t)j * N] = to_bf16_bits(x);
           }
         }
-        __syncwarp();
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -465,7 +474,7 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
                                   const CUtensorMap& tm_xw, const gg::Args& args, long long max_tiles, const DeviceInfo& dev,
                                   cudaStream_t stream) {
   auto kern = gg::grouped_gemm_kernel<kGelu, kPair>;
-  const size_t smem_max = gg::smem_bytes<kPair>(kMaxExperts);  // one attribute for every E
+  const size_t smem_max = gg::kSmemBudget;  // one attribute for every E
   const int slot = (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0);
   KernelSlot& ks = g_slots[dev.device & 63][slot];
   std::call_once(ks.once, [&] {
@@ -501,7 +510,7 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3((unsigned)(units * kPair), 1, 1);
   cfg.blockDim = dim3(gg::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = gg::smem_bytes<kPair>(args.E);
+  cfg.dynamicSmemBytes = gg::smem_bytes<kPair>(args.E, args.stages);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -529,6 +538,7 @@ cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const voi
   args.K = K;
   args.n_fblocks = (N + gg::BM * pair - 1) / (gg::BM * pair);
   args.num_kb = (K + gg::BK - 1) / gg::BK;
+  args.stages = pair == 2 ? gg::stages_for<2>(E) : gg::stages_for<1>(E);
   // an upper bound on the tile count: every expert adds at most one partial token block
   const long long max_tiles =
       ((long long)(R + gg::BN - 1) / gg::BN + E) * (long long)args.n_fblocks;

@@ -32,6 +32,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from combine_moe_route_14_b200 import inputs as I  # noqa: E402
+from combine_moe_route_14_b200 import replicas as Rp  # noqa: E402
 
 METRIC = "MoE-layer tokens/s on 1 B200; HBM GB/s (dispatch/combine), TC util (GEMM)"
 UNIT = "tokens/s"
@@ -227,7 +228,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
 
     inp = I.make_layer_inputs(cfg, args.seed, device=dev)  # weights: same on every rank
-    X_host = inp["X"] if rank == 0 else I.random_bf16((cfg.T, cfg.d), args.seed + 1000 * rank, "X")
+    X_host = inp["X"] if rank == 0 else I.random_bf16((cfg.T, cfg.d),
+                                                       Rp.replica_token_seed(args.seed, rank), "X")
     X = X_host.to(dev)
     logits = inp["logits"].to(dev) if inp["logits"] is not None else None
     Wr = inp["Wr"].to(dev) if inp["Wr"] is not None else None
@@ -245,11 +247,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             torch.distributed.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return Rp.max_over_ranks(x, device=dev)
 
     for _ in range(args.warmup):
         step()
@@ -354,20 +352,26 @@ def run_ours(args, cfg, rank, world, local_rank):
     model = stage_model(cfg, counts_h)
     dom = max(stage_ms, key=lambda n: stage_ms[n])
     peaks, peak_src = load_peaks()
-    long_region = (t_ms + staged_total_ms * args.steps) > 1000.0
+    clocks = sampler.summary() if sampler else None
+    capped = bool(clocks and "sw_power_cap" in clocks.get("reasons", []))
+    # The sustained peak is cuBLAS under the 1 kW power cap; a kernel timed
+    # inside a continuous step loop that ran under that cap is held to it.
+    sustained = capped or (t_ms + staged_total_ms * args.steps) > 1000.0
     per = model[dom]
     dur_s = stage_ms[dom] / 1e3
     if "flops" in per and per["flops"] / max(per["bytes"], 1) > (
             peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9):
-        peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": per["flops"] / dur_s / 1e12, "peak": peak,
                 "unit": "TFLOP/s"}
+        roof["frac_vs_burst"] = roof["achieved"] / peaks["bf16_tflops"]
     else:
         roof = {"bound": "hbm", "achieved": per["bytes"] / dur_s / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = dom
-    roof["peak_source"] = f"{peak_src} ({'sustained' if long_region and roof['bound'] == 'tensor' else 'burst'})"
+    roof["peak_source"] = (f"{peak_src} ("
+                           f"{'sustained: power cap active in the timed region' if sustained and roof['bound'] == 'tensor' else 'burst'})")
     kname = {"gemm1": "grouped_gemm_gelu", "gemm2": "grouped_gemm"}.get(dom, dom)
     tr = ncu_traffic(kname, cfg.name)
     roof["traffic"] = tr
@@ -383,8 +387,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             st["TFLOP/s"] = model[n]["flops"] / (ms / 1e3) / 1e12
         stages[n] = st
 
-    total_tokens = cfg.T * args.steps * world
-    value = total_tokens / (t_ms / 1e3)
+    value = Rp.weak_scaling_throughput(cfg.T, args.steps, world, t_ms)
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
@@ -399,12 +402,12 @@ def run_ours(args, cfg, rank, world, local_rank):
         "stages": stages,
         "expert_counts": {"max": int(counts_h.max()), "mean": float(counts_h.mean()),
                           "min": int(counts_h.min())},
-        "e2e": {"value": cfg.T * args.steps * world / (e2e_ms / 1e3), "unit": UNIT,
+        "e2e": {"value": Rp.weak_scaling_throughput(cfg.T, args.steps, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * moe.moe_kernel_launches_per_forward(
             moe.make_desc(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.score, cfg.renormalize),
             Wr is not None),
-        "clocks": sampler.summary() if sampler else None,
+        "clocks": clocks,
     }
     del X, logits, Wr, layer, inp, ws, Xe, H, Ye
     torch.cuda.empty_cache()

@@ -29,7 +29,13 @@ Readings where the pages are silent (each is also listed in the design notes):
   * gates: softmax over the chosen logits (= softmax over all experts
     renormalised over the chosen k), sigmoid scores renormalised, or, with
     renormalize=0, the plain softmax / sigmoid probability of each chosen
-    expert.  Temperature 1, no threshold, no capacity limit: R = T*k rows.
+    expert.  No capacity limit.
+  * routing variants ([GPT] §2.3, §4.1): scores use logits / temperature
+    (the top-k order is unchanged for temperature > 0); with a threshold
+    min_prob > 0, a chosen slot whose probability (softmax over all E, or
+    sigmoid) is not above min_prob is dropped: index -1, gate 0, no layout
+    row.  Renormalised gates divide by the sum over the kept slots.  Defaults
+    (temperature 1, no threshold) keep every slot: R = T*k rows.
   * rows inside an expert block are in ascending (token, slot) order; blocks
     are in expert order 0..E-1.
   * GELU is the exact erf form 0.5*x*(1+erf(x/sqrt 2)).
@@ -91,37 +97,45 @@ def topk_order(logits: np.ndarray, k: int) -> np.ndarray:
 
 
 def gates_from_logits(logits: np.ndarray, idx: np.ndarray, score: str,
-                      renormalize: int) -> np.ndarray:
-    """Gate value of each chosen slot, float64.
+                      renormalize: int, temperature: float = 1.0,
+                      min_prob: float = 0.0):
+    """Gate value of each chosen slot and whether the slot is kept, float64.
 
-    softmax:  p_e = exp(L_e - m) / sum_{e'} exp(L_e' - m)  over all E experts;
-              renormalised: p_j / sum_{chosen} p.
-    sigmoid:  s_e = 1 / (1 + exp(-L_e)); renormalised: s_j / sum_{chosen} s.
+    With z = logits / temperature:
+    softmax:  p_e = exp(z_e - m) / sum_{e'} exp(z_e' - m)  over all E experts;
+    sigmoid:  s_e = 1 / (1 + exp(-z_e)).
+    A slot is kept when min_prob <= 0 or its probability exceeds min_prob.
+    renormalize=1: gate = prob / sum of the kept slots' probs; else the prob.
+    Dropped slots get gate 0.  Returns (gates [T,k], keep [T,k] bool).
     """
-    L = np.asarray(logits, dtype=np.float64)
+    if not temperature > 0:
+        raise ValueError("temperature must be > 0")
+    L = np.asarray(logits, dtype=np.float64) / float(temperature)
     T, E = L.shape
-    k = idx.shape[1]
     chosen = np.take_along_axis(L, idx.astype(np.int64), axis=1)  # [T, k]
     if score == SOFTMAX:
         m = L.max(axis=1, keepdims=True)
-        num = np.exp(chosen - m)
-        if renormalize:
-            den = num.sum(axis=1, keepdims=True)
-        else:
-            den = np.exp(L - m).sum(axis=1, keepdims=True)
-        return num / den
-    if score == SIGMOID:
-        s = 1.0 / (1.0 + np.exp(-chosen))
-        if renormalize:
-            return s / s.sum(axis=1, keepdims=True)
-        return s
-    raise ValueError(f"unknown score {score!r}")
+        prob = np.exp(chosen - m) / np.exp(L - m).sum(axis=1, keepdims=True)
+    elif score == SIGMOID:
+        prob = 1.0 / (1.0 + np.exp(-chosen))
+    else:
+        raise ValueError(f"unknown score {score!r}")
+    keep = np.ones_like(prob, dtype=bool) if min_prob <= 0 else prob > min_prob
+    kept = np.where(keep, prob, 0.0)
+    if renormalize:
+        den = kept.sum(axis=1, keepdims=True)
+        gates = np.divide(kept, den, out=np.zeros_like(kept), where=den > 0)
+    else:
+        gates = kept
+    return gates, keep
 
 
-def route(logits, k: int, score: str = SOFTMAX, renormalize: int = 1):
-    """(topk_idx [T,k] int32, gates [T,k] float64)."""
+def route(logits, k: int, score: str = SOFTMAX, renormalize: int = 1,
+          temperature: float = 1.0, min_prob: float = 0.0):
+    """(topk_idx [T,k] int32 with -1 for dropped slots, gates [T,k] float64)."""
     idx = topk_order(logits, k)
-    return idx, gates_from_logits(logits, idx, score, renormalize)
+    gates, keep = gates_from_logits(logits, idx, score, renormalize, temperature, min_prob)
+    return np.where(keep, idx, -1).astype(np.int32), gates
 
 
 # ----------------------------------------------------------------------------
@@ -132,28 +146,33 @@ def layout(topk_idx, E: int):
 
     Walks the slots in logical order and hands each one the next free row of
     its expert's block (the incremental layout-block allocation of the AL
-    table).  Returns counts [E], offsets [E+1] (exclusive prefix sum,
-    offsets[E] = R), row_of [R] (logical -> layout) and src_of [R] (its
-    inverse, layout -> logical), all int32.
+    table).  Slot value -1 marks a dropped slot: it takes no row (row_of -1).
+    Returns counts [E], offsets [E+1] (exclusive prefix sum, offsets[E] =
+    number of kept slots), row_of [R] (logical -> layout) and src_of [R]
+    (layout -> logical for rows below offsets[E], -1 above), all int32.
     """
     flat = np.asarray(topk_idx, dtype=np.int64).reshape(-1)
     R = flat.size
-    if R and (flat.min() < 0 or flat.max() >= E):
+    if R and (flat.min() < -1 or flat.max() >= E):
         raise ValueError("expert id out of range")
     counts = np.zeros(E, dtype=np.int64)
     for e in flat:
-        counts[e] += 1
+        if e >= 0:
+            counts[e] += 1
     offsets = np.zeros(E + 1, dtype=np.int64)
     for e in range(E):
         offsets[e + 1] = offsets[e] + counts[e]
     cursor = offsets[:E].copy()
-    row_of = np.empty(R, dtype=np.int64)
+    row_of = np.full(R, -1, dtype=np.int64)
     for i in range(R):
         e = flat[i]
+        if e < 0:
+            continue
         row_of[i] = cursor[e]
         cursor[e] += 1
-    src_of = np.empty(R, dtype=np.int64)
-    src_of[row_of] = np.arange(R)
+    src_of = np.full(R, -1, dtype=np.int64)
+    kept = row_of >= 0
+    src_of[row_of[kept]] = np.arange(R)[kept]
     return (counts.astype(np.int32), offsets.astype(np.int32),
             row_of.astype(np.int32), src_of.astype(np.int32))
 
@@ -162,10 +181,14 @@ def layout(topk_idx, E: int):
 # a4: dispatch   [DYS] §1 (one token -> its k experts); [TEP] §1.1
 # ----------------------------------------------------------------------------
 def dispatch(X, src_of, k: int) -> np.ndarray:
-    """Xe[r, :] = X[src_of[r] // k, :]  (a copy; works on any dtype, bf16 bits included)."""
+    """Xe[r, :] = X[src_of[r] // k, :] for the layout's rows (src_of[r] >= 0); a copy,
+    on any dtype (bf16 bits included).  Rows past the kept slots are returned as zeros."""
     X = np.asarray(X)
     src = np.asarray(src_of, dtype=np.int64)
-    return X[src // k].copy()
+    out = np.zeros((src.size,) + X.shape[1:], dtype=X.dtype)
+    ok = src >= 0
+    out[ok] = X[src[ok] // k]
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -222,14 +245,17 @@ def _as_f64(w):
 # a7: combine   [DYS] §1 (k results reduced into one); [TEP] §1.1, §2.1
 # ----------------------------------------------------------------------------
 def combine(Ye, row_of, gates, k: int) -> np.ndarray:
-    """Y[t, :] = sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :]  (slot order), float64."""
+    """Y[t, :] = sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :]  (slot order), float64.
+
+    Dropped slots (row_of -1) contribute nothing."""
     Ye = np.asarray(Ye, np.float64)
     g = np.asarray(gates, np.float64)
     T = g.shape[0]
     rows = np.asarray(row_of, np.int64).reshape(T, k)
     Y = np.zeros((T, Ye.shape[1]))
     for j in range(k):
-        Y += g[:, j:j + 1] * Ye[rows[:, j]]
+        kept = rows[:, j] >= 0
+        Y[kept] += g[kept, j:j + 1] * Ye[rows[kept, j]]
     return Y
 
 
@@ -237,7 +263,7 @@ def combine(Ye, row_of, gates, k: int) -> np.ndarray:
 # the whole layer
 # ----------------------------------------------------------------------------
 def layer_forward(X_bits, W1_bits, W2_bits, k, score=SOFTMAX, renormalize=1,
-                  logits=None, Wr_bits=None):
+                  logits=None, Wr_bits=None, temperature=1.0, min_prob=0.0):
     """Full layer on the CPU.  Exactly one of ``logits`` (fp32) / ``Wr_bits`` is given.
 
     With router weights, the logits are computed in float64 and rounded to
@@ -253,7 +279,7 @@ def layer_forward(X_bits, W1_bits, W2_bits, k, score=SOFTMAX, renormalize=1,
         L = router_logits(X, bf16_to_f64(Wr_bits)).astype(np.float32)
     else:
         L = np.asarray(logits, dtype=np.float32)
-    idx, gates = route(L, k, score, renormalize)
+    idx, gates = route(L, k, score, renormalize, temperature, min_prob)
     counts, offsets, row_of, src_of = layout(idx, E)
     Xe = dispatch(X, src_of, k)
     H, Ye = expert_ffn(Xe, offsets, W1_bits, W2_bits)
@@ -281,7 +307,8 @@ def layer_forward_tokens(X_bits, W1_bits, W2_bits, topk_idx, gates, tokens):
     by_e = {}
     for n in range(len(tokens)):
         for j in range(k):
-            by_e.setdefault(int(idx[n, j]), []).append((n, j))
+            if idx[n, j] >= 0:  # dropped slots contribute nothing
+                by_e.setdefault(int(idx[n, j]), []).append((n, j))
     for e, pairs in sorted(by_e.items()):
         ns = np.array([p[0] for p in pairs])
         js = np.array([p[1] for p in pairs])

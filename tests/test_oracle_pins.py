@@ -98,6 +98,60 @@ def check_gates_closed_forms(route_fn):
     assert abs(g[0, 1] - 0.2689414213699951) < 1e-15
 
 
+def check_router_variants_library(route_fn):
+    """The router of [GPT] §4.1 written with torch: softmax(L / T), top-k,
+    probabilities not above the threshold masked to -1."""
+    L = I.random_f32((600, 16), 13, "variants")
+    for temp, thr in ((1.0, 0.0), (0.3, 0.05), (1.3, 0.1), (2.0, 0.2)):
+        probs = torch.softmax(L.double() / temp, dim=1)
+        vals, ids = torch.topk(probs, 4, dim=1, sorted=True)
+        mask = vals > thr
+        ref_idx = torch.where(mask, ids, torch.full_like(ids, -1)).numpy()
+        idx, g = route_fn(L.numpy(), 4, O.SOFTMAX, 0, temp, thr)
+        assert np.array_equal(idx, ref_idx), (temp, thr)
+        np.testing.assert_allclose(g, torch.where(mask, vals, 0.0).numpy(), rtol=1e-12, atol=1e-15)
+        idx, g = route_fn(L.numpy(), 4, O.SOFTMAX, 1, temp, thr)
+        kept = torch.where(mask, vals, 0.0)
+        den = kept.sum(1, keepdim=True)
+        ref = torch.where(den > 0, kept / den.clamp_min(1e-300), 0.0).numpy()
+        np.testing.assert_allclose(g, ref, rtol=1e-12, atol=1e-15)
+
+
+def check_router_variants_closed_forms(route_fn):
+    # temperature 2 on logits [0, 1]: softmax over both = logistic((1 - 0) / 2)
+    idx, g = route_fn(np.array([[0.0, 1.0]], np.float32), 2, O.SOFTMAX, 1, 2.0, 0.0)
+    assert list(idx[0]) == [1, 0]
+    assert abs(g[0, 0] - 1.0 / (1.0 + np.exp(-0.5))) < 1e-15
+    # probabilities 0.6 / 0.3 / 0.1 with threshold 0.2: the third slot is dropped
+    L = np.log(np.array([[0.6, 0.3, 0.1]]))
+    idx, g = route_fn(L, 3, O.SOFTMAX, 0, 1.0, 0.2)
+    assert list(idx[0]) == [0, 1, -1]
+    np.testing.assert_allclose(g[0], [0.6, 0.3, 0.0], rtol=1e-12, atol=1e-15)
+    idx, g = route_fn(L, 3, O.SOFTMAX, 1, 1.0, 0.2)
+    np.testing.assert_allclose(g[0], [2 / 3, 1 / 3, 0.0], rtol=1e-12)
+    # every slot below the threshold: all dropped, all gates 0
+    idx, g = route_fn(np.zeros((1, 8), np.float32), 2, O.SOFTMAX, 1, 1.0, 0.2)
+    assert list(idx[0]) == [-1, -1] and (g == 0).all()
+
+
+def test_router_variants_match_library():
+    check_router_variants_library(O.route)
+
+
+def test_router_variants_closed_forms():
+    check_router_variants_closed_forms(O.route)
+
+
+def test_combine_skips_dropped_slots():
+    Ye = np.arange(12, dtype=np.float64).reshape(3, 4)
+    row_of = np.array([0, -1, -1, -1, 2, 1], np.int32)  # T=3, k=2
+    g = np.array([[0.5, 0.5], [1.0, 1.0], [0.25, 0.75]])
+    Y = O.combine(Ye, row_of, g, 2)
+    np.testing.assert_array_equal(Y[0], 0.5 * Ye[0])
+    np.testing.assert_array_equal(Y[1], 0.0)               # every slot dropped
+    np.testing.assert_array_equal(Y[2], 0.25 * Ye[2] + 0.75 * Ye[1])
+
+
 def test_topk_bruteforce_ternary():
     check_topk_bruteforce(O.topk_order)
 
@@ -167,17 +221,36 @@ def check_layout_golden(layout_fn):
     assert row_of.tolist() == gd["row_of"]
 
 
-def check_layout_bruteforce(layout_fn, T=37, E=6, k=3, seed=1):
+def check_layout_dropped(layout_fn):
+    gd = _read_golden("layout_small.txt")
+    idx = np.array(gd["D_topk_idx"], np.int32).reshape(gd["T"][0], gd["k"][0])
+    counts, offsets, row_of, src_of = layout_fn(idx, gd["E"][0])
+    assert counts.tolist() == gd["D_counts"]
+    assert offsets.tolist() == gd["D_offsets"]
+    assert row_of.tolist() == gd["D_row_of"]
+    assert src_of.tolist() == gd["D_src_of"]
+
+
+def check_layout_bruteforce(layout_fn, T=37, E=6, k=3, seed=1, drop=0.0):
     idx = I.random_topk(T, E, k, seed).numpy()
+    if drop:
+        rng = np.random.default_rng(seed)
+        idx[rng.random(idx.shape) < drop] = -1
     counts, offsets, row_of, src_of = layout_fn(idx, E)
     flat = idx.reshape(-1)
     R = flat.size
     for i in range(R):
         e = flat[i]
-        before_block = sum(1 for i2 in range(R) if flat[i2] < e)
+        if e < 0:
+            assert row_of[i] == -1
+            continue
+        before_block = sum(1 for i2 in range(R) if 0 <= flat[i2] < e)
         before_in_block = sum(1 for i2 in range(i) if flat[i2] == e)
         assert row_of[i] == before_block + before_in_block
-    assert np.array_equal(src_of, np.argsort(flat, kind="stable"))
+    kept = int((flat >= 0).sum())
+    order = np.argsort(np.where(flat < 0, E, flat), kind="stable")  # dropped slots sort last
+    assert np.array_equal(src_of[:kept], order[:kept])
+    assert (src_of[kept:] == -1).all()
 
 
 def check_layout_invariants(layout_fn, T, E, k, seed, skew=0.0):
@@ -201,6 +274,11 @@ def test_layout_golden():
 
 def test_layout_bruteforce_rank_count():
     check_layout_bruteforce(O.layout)
+    check_layout_bruteforce(O.layout, T=41, E=5, k=3, seed=2, drop=0.3)
+
+
+def test_layout_dropped_slots_golden():
+    check_layout_dropped(O.layout)
 
 
 @pytest.mark.parametrize("T,E,k,skew", [(256, 8, 2, 0.0), (1000, 64, 4, 1.2), (50, 256, 8, 0.0),
@@ -406,6 +484,21 @@ def _combine_no_gate(Ye, row_of, gates, k):
     return O.combine(Ye, row_of, np.ones_like(np.asarray(gates, np.float64)), k)
 
 
+def _route_threshold_on_gates(L, k, score, renorm, temp=1.0, thr=0.0):
+    """Plausible mistake: threshold the renormalised gates instead of the probabilities."""
+    idx, g = O.route(L, k, score, renorm, temp, 0.0)
+    keep = g > thr if thr > 0 else np.ones_like(g, bool)
+    return np.where(keep, idx, -1).astype(np.int32), np.where(keep, g, 0.0)
+
+
+def _route_temperature_multiplies(L, k, score, renorm, temp=1.0, thr=0.0):
+    return O.route(L, k, score, renorm, 1.0 / temp, thr)
+
+
+def _layout_drop_counts_as_expert0(idx, E):
+    return O.layout(np.where(np.asarray(idx) < 0, 0, idx), E)
+
+
 def _layer_with(**repl):
     def fn(*a, **kw):
         saved = {n: getattr(O, n) for n in repl}
@@ -432,6 +525,9 @@ def _layer_with(**repl):
     ("gate dropped", lambda: check_identity_experts(O.route, O.layout, O.dispatch,
                                                     _combine_no_gate)),
     ("dense FFN with tanh GELU", lambda: check_dense_special_case(_layer_with(gelu=_gelu_tanh))),
+    ("threshold on gates", lambda: check_router_variants_library(_route_threshold_on_gates)),
+    ("temperature multiplies", lambda: check_router_variants_closed_forms(_route_temperature_multiplies)),
+    ("dropped slot counted", lambda: check_layout_dropped(_layout_drop_counts_as_expert0)),
 ])
 def test_planted_mistake_is_caught(name, run):
     with pytest.raises(AssertionError):

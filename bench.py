@@ -39,7 +39,7 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # sampled tokens per oracle call: cpu_baseline leg / reference arm
-ORACLE_SAMPLE = {"mixtral": (256, 32), "skewed_top1": (256, 32), "skewed_top1_harsh": (256, 32),
+ORACLE_SAMPLE = {"mixtral": (256, 32), "mixtral_threshold": (256, 32), "tiny_threshold": (256, 256), "skewed_top1": (256, 32), "skewed_top1_harsh": (256, 32),
                  "fine_grained": (32, 8), "tiny": (256, 256), "decode_16": (16, 16),
                  "decode_64": (64, 32), "decode_256": (256, 32), "decode_1024": (256, 32)}
 
@@ -188,7 +188,7 @@ def oracle_step(O, cfg, h, S):
     X = h["X"][:S]
     L = None if h["logits"] is None else h["logits"][:S]
     return O.layer_forward(X, h["W1"], h["W2"], cfg.k, cfg.score, cfg.renormalize, logits=L,
-                           Wr_bits=h["Wr"])
+                           Wr_bits=h["Wr"], temperature=cfg.temperature, min_prob=cfg.min_prob)
 
 
 def blas_threads():
@@ -233,7 +233,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     X = X_host.to(dev)
     logits = inp["logits"].to(dev) if inp["logits"] is not None else None
     Wr = inp["Wr"].to(dev) if inp["Wr"] is not None else None
-    layer = moe.MoeLayer(inp["W1"], inp["W2"], cfg.k, cfg.score, cfg.renormalize, Wr=Wr)
+    layer = moe.MoeLayer(inp["W1"], inp["W2"], cfg.k, cfg.score, cfg.renormalize, Wr=Wr,
+                         temperature=cfg.temperature, min_prob=cfg.min_prob)
     Y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
     counts = torch.empty((cfg.E,), dtype=torch.int32, device=dev)
     ws = layer.workspace(cfg.T)
@@ -287,7 +288,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         Ye = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=dev)
         fns = {
             "router_logits": lambda: moe.moe_router_logits(X, Wr, logits=L_buf),
-            "route": lambda: moe.moe_route(L_buf, cfg.k, cfg.score, cfg.renormalize, idx, g),
+            "route": lambda: moe.moe_route_ex(L_buf, cfg.k, cfg.score, cfg.renormalize,
+                                              cfg.temperature, cfg.min_prob, idx, g),
             "layout": lambda: moe.moe_layout(idx, cfg.E, counts, offs, row_of, src_of, lws),
             "dispatch": lambda: moe.moe_dispatch(X, src_of, cfg.k, Xe),
             "gemm1": lambda: moe.moe_expert_gemm(Xe, offs, inp["W1"], True, H),
@@ -394,14 +396,16 @@ def run_ours(args, cfg, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
                    "f": cfg.f, "router": cfg.router, "score": cfg.score,
-                   "renormalize": cfg.renormalize, "tokens_per_gpu": cfg.T,
+                   "renormalize": cfg.renormalize, "temperature": cfg.temperature,
+                   "min_prob": cfg.min_prob, "tokens_per_gpu": cfg.T,
                    "parallelism": f"replicas x{world} (no collective)",
                    "l2": f"inputs larger than L2: each step streams "
                          f"{2 * cfg.E * cfg.d * cfg.f * 2 / 1e9:.2f} GB of expert weights"},
         "roofline": roof,
         "stages": stages,
         "expert_counts": {"max": int(counts_h.max()), "mean": float(counts_h.mean()),
-                          "min": int(counts_h.min())},
+                          "min": int(counts_h.min()),
+                          "dropped_slots": int(cfg.R - counts_h.sum())},
         "e2e": {"value": Rp.weak_scaling_throughput(cfg.T, args.steps, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * moe.moe_kernel_launches_per_forward(

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "MoeError", "LayerDesc", "load_library", "library_path",
-    "moe_router_logits", "moe_route", "moe_layout_workspace_size", "moe_layout",
+    "moe_router_logits", "moe_route", "moe_route_ex", "moe_layout_workspace_size", "moe_layout",
     "moe_layout_static",
     "moe_dispatch", "moe_expert_gemm", "moe_expert_ffn", "moe_combine",
     "moe_workspace_size", "moe_layer_forward", "moe_device_status",
@@ -46,7 +46,8 @@ class MoeError(RuntimeError):
 class LayerDesc(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("f", ctypes.c_int32), ("score", ctypes.c_int32),
-                ("renormalize", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("renormalize", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("temperature", ctypes.c_float), ("min_prob", ctypes.c_float)]
 
 
 def library_path() -> str:
@@ -58,6 +59,8 @@ _I = ctypes.c_int32
 _SIG = {
     "moe_router_logits": ([_P, _P, _I, _I, _I, _P, _P], ctypes.c_int),
     "moe_route": ([_P, _I, _I, _I, _I, _I, _P, _P, _P], ctypes.c_int),
+    "moe_route_ex": ([_P, _I, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P],
+                     ctypes.c_int),
     "moe_layout_workspace_size": ([_I, _I, _I], ctypes.c_size_t),
     "moe_layout": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_layout_static": ([_P, _I, _I, _I, _P, _P, _P, _P, _P], ctypes.c_int),
@@ -160,6 +163,21 @@ def moe_route(logits, k, score="softmax", renormalize=True, topk_idx=None, gates
     gates = _out(gates, "gates", torch.float32, (T, k), dev)
     _check(lib.moe_route(_ptr(logits), T, E, k, _score(score), int(bool(renormalize)),
                          _ptr(topk_idx), _ptr(gates), _stream(stream, dev)))
+    return topk_idx, gates
+
+
+def moe_route_ex(logits, k, score="softmax", renormalize=True, temperature=1.0, min_prob=0.0,
+                 topk_idx=None, gates=None, stream=None):
+    """moe_route with a router temperature and a minimum-probability threshold (-1 = dropped)."""
+    lib = load_library()
+    T, E = logits.shape
+    dev = logits.device
+    _need(logits, "logits", torch.float32, (T, E))
+    topk_idx = _out(topk_idx, "topk_idx", torch.int32, (T, k), dev)
+    gates = _out(gates, "gates", torch.float32, (T, k), dev)
+    _check(lib.moe_route_ex(_ptr(logits), T, E, k, _score(score), int(bool(renormalize)),
+                            float(temperature), float(min_prob), _ptr(topk_idx), _ptr(gates),
+                            _stream(stream, dev)))
     return topk_idx, gates
 
 
@@ -270,8 +288,10 @@ def moe_combine(Ye, row_of, gates, Y=None, stream=None):
 # ----------------------------------------------------------------------------
 # whole layer
 # ----------------------------------------------------------------------------
-def make_desc(T, d, E, k, f, score="softmax", renormalize=True) -> LayerDesc:
-    return LayerDesc(T, d, E, k, f, _score(score), int(bool(renormalize)), 0)
+def make_desc(T, d, E, k, f, score="softmax", renormalize=True, temperature=1.0,
+              min_prob=0.0) -> LayerDesc:
+    return LayerDesc(T, d, E, k, f, _score(score), int(bool(renormalize)), 0, float(temperature),
+                     float(min_prob))
 
 
 def moe_workspace_size(desc: LayerDesc) -> int:
@@ -285,7 +305,7 @@ def moe_kernel_launches_per_forward(desc: LayerDesc, with_router: bool) -> int:
 
 def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=None, Wr=None,
                       Y=None, topk_idx_out=None, gates_out=None, counts_out=None, ws=None,
-                      stream=None):
+                      stream=None, temperature=1.0, min_prob=0.0):
     lib = load_library()
     T, d = X.shape
     E, f, _ = W1.shape
@@ -304,7 +324,7 @@ def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=No
         _need(gates_out, "gates_out", torch.float32, (T, k), dev)
     if counts_out is not None:
         _need(counts_out, "counts_out", torch.int32, (E,), dev)
-    desc = make_desc(T, d, E, k, f, score, renormalize)
+    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob)
     if ws is None:
         ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
     _need(ws, "ws", torch.uint8, None, dev)
@@ -327,9 +347,11 @@ def moe_device_status(clear: bool = True) -> int:
 class MoeLayer:
     """A layer's weights plus a reusable workspace (allocation stays outside the call)."""
 
-    def __init__(self, W1, W2, k, score="softmax", renormalize=True, Wr=None):
+    def __init__(self, W1, W2, k, score="softmax", renormalize=True, Wr=None, temperature=1.0,
+                 min_prob=0.0):
         self.W1, self.W2, self.Wr = W1, W2, Wr
         self.k, self.score, self.renormalize = k, score, renormalize
+        self.temperature, self.min_prob = temperature, min_prob
         self.E, self.f, self.d = W1.shape
         self._ws = None
 
@@ -346,4 +368,5 @@ class MoeLayer:
                                  logits=logits, Wr=None if logits is not None else self.Wr,
                                  Y=Y, topk_idx_out=topk_idx_out, gates_out=gates_out,
                                  counts_out=counts_out, ws=self.workspace(X.shape[0]),
-                                 stream=stream)
+                                 stream=stream, temperature=self.temperature,
+                                 min_prob=self.min_prob)

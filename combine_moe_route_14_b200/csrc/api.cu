@@ -2,6 +2,7 @@
 // per-device state, workspace layout and the fused layer forward.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <mutex>
 #include <string>
 
@@ -160,8 +161,13 @@ moe_status check_desc(const moe_layer_desc* desc) {
   if (desc->renormalize != 0 && desc->renormalize != 1)
     return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
   if (desc->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved must be 0");
+  if (!std::isfinite(desc->temperature) || desc->temperature < 0.f)
+    return fail(MOE_ERR_INVALID_ARG, "temperature must be >= 0 (0 reads as 1)");
+  if (!std::isfinite(desc->min_prob)) return fail(MOE_ERR_INVALID_ARG, "min_prob must be finite");
   return MOE_OK;
 }
+
+float desc_temperature(const moe_layer_desc& d) { return d.temperature > 0.f ? d.temperature : 1.f; }
 
 }  // namespace
 
@@ -193,21 +199,30 @@ moe_status moe_router_logits(const void* X, const void* Wr, int32_t T, int32_t d
   return MOE_OK;
 }
 
-moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
-                     int32_t renormalize, int32_t* topk_idx, float* gates, void* stream) {
+moe_status moe_route_ex(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
+                        int32_t renormalize, float temperature, float min_prob,
+                        int32_t* topk_idx, float* gates, void* stream) {
   MOE_TRY(check_ET(T, E, k));
   if (score != MOE_SCORE_SOFTMAX && score != MOE_SCORE_SIGMOID)
     return fail(MOE_ERR_INVALID_ARG, "unknown score");
   if (renormalize != 0 && renormalize != 1)
     return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
+  if (!std::isfinite(temperature) || !(temperature > 0.f))
+    return fail(MOE_ERR_INVALID_ARG, "temperature must be > 0");
+  if (!std::isfinite(min_prob)) return fail(MOE_ERR_INVALID_ARG, "min_prob must be finite");
   if (T == 0) return MOE_OK;
   MOE_TRY(check_ptr4(logits, "logits"));
   MOE_TRY(check_ptr4(topk_idx, "topk_idx"));
   MOE_TRY(check_ptr4(gates, "gates"));
-  MOE_CUDA(moe::launch_route(logits, T, E, k, score, renormalize, topk_idx, gates,
-                             as_stream(stream)),
+  MOE_CUDA(moe::launch_route(logits, T, E, k, score, renormalize, temperature, min_prob, topk_idx,
+                             gates, as_stream(stream)),
            "route");
   return MOE_OK;
+}
+
+moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
+                     int32_t renormalize, int32_t* topk_idx, float* gates, void* stream) {
+  return moe_route_ex(logits, T, E, k, score, renormalize, 1.0f, 0.0f, topk_idx, gates, stream);
 }
 
 size_t moe_layout_workspace_size(int32_t T, int32_t E, int32_t k) {
@@ -363,7 +378,9 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const void* X, const fl
   const int R = d.T * d.k;
 
   if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, s), "router_logits");
-  MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, idx, gates, s), "route");
+  MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
+                             d.min_prob, idx, gates, s),
+           "route");
   MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s), "layout");
   MOE_CUDA(moe::launch_dispatch(X, src_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
   std::string err;

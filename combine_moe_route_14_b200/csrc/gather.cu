@@ -26,7 +26,8 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
   for (int r = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); r < R; r += nwarps) {
     const int s = __ldg(src_of + r);
     if (s < 0 || s >= R) {
-      if (lane == 0) flag_error(status, MOE_DEV_BAD_ROW);
+      // -1: a row past the kept slots (dropped slots leave it unused)
+      if (s != -1 && lane == 0) flag_error(status, MOE_DEV_BAD_ROW);
       continue;
     }
     const uint4* src = X + (size_t)(s / k) * row_vecs;
@@ -47,7 +48,8 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
   }
 }
 
-// Y[t, :] = bf16( sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :] ), fp32 sum in slot order.
+// Y[t, :] = bf16( sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :] ), fp32 sum in slot order;
+// a dropped slot (row_of -1) contributes nothing.
 // kK > 0: k known at compile time; kK == 0: runtime k (<= kMaxTopK).
 template <int kK>
 __global__ void __launch_bounds__(kGatherWarps * 32)
@@ -61,25 +63,26 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
   const int nwarps = gridDim.x * kGatherWarps;
   for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
     // lanes j < k fetch slot j's row and gate; broadcast below
-    int my_row = 0;
+    int my_row = -1;
     float my_gate = 0.f;
     if (lane < k) {
       my_row = __ldg(row_of + (size_t)t * k + lane);
       my_gate = __ldg(gates + (size_t)t * k + lane);
-      if (my_row < 0 || my_row >= R) {
+      if (my_row < -1 || my_row >= R) {  // -1 is a dropped slot
         flag_error(status, MOE_DEV_BAD_ROW);
-        my_row = -1;
+        my_row = -2;
       }
     }
-    const bool bad = __any_sync(0xffffffffu, lane < k && my_row < 0);
+    const bool bad = __any_sync(0xffffffffu, lane < k && my_row == -2);
     if (bad) continue;
+    const uint32_t live = __ballot_sync(0xffffffffu, lane < k && my_row >= 0);  // kept slots
     const uint4* src[kSlots];
     float g[kSlots];
 #pragma unroll
     for (int j = 0; j < kSlots; ++j) {
       const int rj = __shfl_sync(0xffffffffu, my_row, j);
       g[j] = __shfl_sync(0xffffffffu, my_gate, j);
-      src[j] = Ye + (size_t)rj * row_vecs;
+      src[j] = Ye + (size_t)(rj < 0 ? 0 : rj) * row_vecs;
     }
     uint4* dst = Y + (size_t)t * row_vecs;
     for (int c0 = 0; c0 < row_vecs; c0 += 32 * kUnroll) {
@@ -89,7 +92,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
         const int c = c0 + u * 32 + lane;
 #pragma unroll
         for (int j = 0; j < kSlots; ++j)
-          if (j < k && c < row_vecs) v[u][j] = ld_stream_v4(src[j] + c);
+          if (j < k && ((live >> j) & 1u) && c < row_vecs) v[u][j] = ld_stream_v4(src[j] + c);
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
@@ -100,7 +103,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
         for (int q = 0; q < 8; ++q) acc[q] = 0.f;
 #pragma unroll
         for (int j = 0; j < kSlots; ++j) {
-          if (j < k) {
+          if (j < k && ((live >> j) & 1u)) {
             const uint4 w = v[u][j];
             acc[0] = fmaf(g[j], bf16_lo(w.x), acc[0]);
             acc[1] = fmaf(g[j], bf16_hi(w.x), acc[1]);

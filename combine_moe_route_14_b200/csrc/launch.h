@@ -29,7 +29,8 @@ cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, in
                                  cudaStream_t stream);
 
 cudaError_t launch_route(const float* L, int T, int E, int k, int score, int renormalize,
-                         int32_t* idx, float* gates, cudaStream_t stream);
+                         float temperature, float min_prob, int32_t* idx, float* gates,
+                         cudaStream_t stream);
 
 size_t layout_workspace_bytes(int64_t R, int E);
 // Number of kernels launch_layout issues for R slots.

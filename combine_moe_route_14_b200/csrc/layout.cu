@@ -9,6 +9,8 @@
 // With R = T*k slots, slot i = t*k + j bound for expert e_i:
 //   counts[e]  = #{i : e_i = e},  offsets = exclusive scan of counts,
 //   row_of[i]  = offsets[e_i] + #{i' < i : e_i' = e_i},  src_of[row_of[i]] = i.
+// A dropped slot (e_i = -1) takes no row: row_of[i] = -1, and the rows past
+// offsets[E] get src_of = -1.
 // This is a stable counting sort of the slots by expert id.  It is
 // deterministic: ranks come from warp match/popc over items in order, never
 // from the order in which atomics land.
@@ -36,18 +38,36 @@ constexpr uint32_t kFlagInclusive = 2u << 30;
 constexpr uint32_t kValueMask = (1u << 30) - 1u;
 
 // Copies the expert ids of slots [begin, end) into shared memory (one
-// coalesced pass, all loads in flight together), replacing ids outside
-// [0, E) by -1 and flagging them.
+// coalesced pass, all loads in flight together).  -1 marks a dropped slot
+// (no row); any other id outside [0, E) is flagged and treated as dropped.
 __device__ __forceinline__ void stage_keys(const int32_t* idx, int begin, int end, int E,
                                            int* keys, uint32_t* status) {
-  for (int i = begin + threadIdx.x; i < end; i += blockDim.x) {
-    int e = __ldg(idx + i);
-    if (e < 0 || e >= E) {
-      if (status) flag_error(status, MOE_DEV_BAD_EXPERT_ID);
-      e = -1;
+  constexpr int kBatch = 8;  // loads in flight per thread before the stores
+  for (int i0 = begin + threadIdx.x; i0 < end; i0 += blockDim.x * kBatch) {
+    int e[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * blockDim.x;
+      e[u] = i < end ? __ldg(idx + i) : -1;
     }
-    keys[i - begin] = e;
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < end) {
+        int v = e[u];
+        if (v < -1 || v >= E) {
+          if (status) flag_error(status, MOE_DEV_BAD_EXPERT_ID);
+          v = -1;
+        }
+        keys[i - begin] = v;
+      }
+    }
   }
+}
+
+// Rows past the last kept slot hold no token: src_of[total..R) = -1.
+__device__ __forceinline__ void mark_unused_rows(int32_t* src_of, int total, int R) {
+  for (int r = total + threadIdx.x; r < R; r += blockDim.x) src_of[r] = -1;
 }
 
 // Per-warp histogram of the staged slots [begin, end) (indices into `keys`)
@@ -86,9 +106,54 @@ __device__ __forceinline__ void warp_scatter(const int* keys, int first, int beg
       row_of[first + li] = row;
       src_of[row] = first + li;
     } else if (li < end) {
-      row_of[first + li] = -1;  // a bad expert id has no row
+      row_of[first + li] = -1;  // a dropped slot (or a bad expert id) has no row
     }
     __syncwarp();
+  }
+}
+
+// The same two walks for E <= 32 without shared-memory updates: per 32-slot
+// chunk one ballot per expert; lane e keeps expert e's running count in a
+// register, and a slot's rank is the popcount of its expert's ballot below
+// its lane (fetched from lane `key` with one shuffle).
+__device__ __forceinline__ void warp_histogram_small(const int* keys, int begin, int end, int E,
+                                                     int* warp_hist) {
+  const int lane = threadIdx.x & 31;
+  int count = 0;  // lane e: slots of expert e seen so far
+  for (int c = begin; c < end; c += 32) {
+    const int key = c + lane < end ? keys[c + lane] : -1;
+    for (int e = 0; e < E; ++e) {
+      const uint32_t m = __ballot_sync(0xffffffffu, key == e);
+      if (lane == e) count += __popc(m);
+    }
+  }
+  if (lane < E) warp_hist[lane] = count;
+}
+
+__device__ __forceinline__ void warp_scatter_small(const int* keys, int first, int begin, int end,
+                                                   int E, const int* warp_base, const int* base,
+                                                   int32_t* row_of, int32_t* src_of) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int run = lane < E ? warp_base[lane] : 0;  // lane e: slots of expert e before this chunk
+  for (int c = begin; c < end; c += 32) {
+    const int li = c + lane;
+    const int key = li < end ? keys[li] : -1;
+    uint32_t mine = 0;  // lane e: ballot of expert e in this chunk
+    for (int e = 0; e < E; ++e) {
+      const uint32_t m = __ballot_sync(0xffffffffu, key == e);
+      if (lane == e) mine = m;
+    }
+    const uint32_t mk = __shfl_sync(0xffffffffu, mine, key < 0 ? 0 : key);
+    const int rk = __shfl_sync(0xffffffffu, run, key < 0 ? 0 : key);
+    if (key >= 0) {
+      const int row = base[key] + rk + __popc(mk & lt_mask);
+      row_of[first + li] = row;
+      src_of[row] = first + li;
+    } else if (li < end) {
+      row_of[first + li] = -1;  // a dropped slot (or a bad expert id) has no row
+    }
+    run += __popc(mine);
   }
 }
 
@@ -165,7 +230,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int warp = threadIdx.x >> 5;
   const int per_warp = ((R + kLayoutWarps * 32 - 1) / (kLayoutWarps * 32)) * 32;
   const int begin = min(R, warp * per_warp), end = min(R, begin + per_warp);
-  warp_histogram(keys, begin, end, hist + warp * E);
+  if (E <= 32) warp_histogram_small(keys, begin, end, E, hist + warp * E);
+  else warp_histogram(keys, begin, end, hist + warp * E);
   __syncthreads();
   scan_over_warps(hist, E, base);
   __syncthreads();
@@ -174,7 +240,9 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int total = block_exclusive_scan(base, E, tmp);
   for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = base[e];
   if (threadIdx.x == 0) offsets[E] = total;
-  warp_scatter(keys, 0, begin, end, hist + warp * E, base, row_of, src_of);
+  mark_unused_rows(src_of, total, R);
+  if (E <= 32) warp_scatter_small(keys, 0, begin, end, E, hist + warp * E, base, row_of, src_of);
+  else warp_scatter(keys, 0, begin, end, hist + warp * E, base, row_of, src_of);
 }
 
 // ---------------------------------------------------------------------------
@@ -199,7 +267,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   for (int i = tile_begin + threadIdx.x; i < tile_end; i += blockDim.x) {
     const int e = __ldg(idx + i);
     if (e >= 0 && e < E) atomicAdd(&hist[e], 1);  // order of adds does not matter for a count
-    else flag_error(status, MOE_DEV_BAD_EXPERT_ID);
+    else if (e != -1) flag_error(status, MOE_DEV_BAD_EXPERT_ID);  // -1: a dropped slot
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -235,7 +303,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int per_warp = ((n + kLayoutWarps * 32 - 1) / (kLayoutWarps * 32)) * 32;
   const int begin = min(n, warp * per_warp);
   const int end = min(n, begin + per_warp);
-  warp_histogram(keys, begin, end, hist + warp * E);
+  if (E <= 32) warp_histogram_small(keys, begin, end, E, hist + warp * E);
+  else warp_histogram(keys, begin, end, hist + warp * E);
   __syncthreads();
   scan_over_warps(hist, E, agg);
   __syncthreads();
@@ -287,10 +356,14 @@ __global__ void __launch_bounds__(kLayoutThreads)
   if (tile == 0) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = base[e];
     if (threadIdx.x == 0) offsets[E] = total;
+    mark_unused_rows(src_of, total, R);
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x) base[e] += agg[e];
   __syncthreads();
-  warp_scatter(keys, tile_begin, begin, end, hist + warp * E, base, row_of, src_of);
+  if (E <= 32)
+    warp_scatter_small(keys, tile_begin, begin, end, E, hist + warp * E, base, row_of, src_of);
+  else
+    warp_scatter(keys, tile_begin, begin, end, hist + warp * E, base, row_of, src_of);
 }
 
 // ---------------------------------------------------------------------------

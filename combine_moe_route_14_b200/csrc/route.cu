@@ -25,7 +25,7 @@ namespace moe {
 // ---------------------------------------------------------------------------
 constexpr int kRouterWarps = 8;
 constexpr int kTokPerWarp = 2;
-constexpr int kRouterUnroll = 4;
+constexpr int kRouterUnroll = 8;
 constexpr int kRouterSmemMax = 96 * 1024;
 
 __device__ __forceinline__ float dot8(const uint4& a, const uint4& b, float acc) {
@@ -45,9 +45,22 @@ __global__ void __launch_bounds__(kRouterWarps * 32)
     router_logits_kernel(const uint4* __restrict__ X, const uint4* __restrict__ Wr, int T,
                          int row_vecs, int E, float* __restrict__ L) {
   extern __shared__ uint4 s_w[];
-  if (kSmemW) {
+  if (kSmemW) {  // stage the weights: 8 loads in flight per thread before the stores
     const int n = E * row_vecs;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) s_w[i] = __ldg(Wr + i);
+    constexpr int kBatch = 8;
+    for (int i0 = threadIdx.x; i0 < n; i0 += blockDim.x * kBatch) {
+      uint4 w[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n) w[u] = __ldg(Wr + i);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * blockDim.x;
+        if (i < n) s_w[i] = w[u];
+      }
+    }
     __syncthreads();
   }
   const uint4* W = kSmemW ? s_w : Wr;
@@ -134,7 +147,10 @@ cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, in
 // of a warp-wide argmax pick the experts in descending order; the comparison
 // (value greater, or equal value and lower id) breaks ties toward the lower
 // expert id, and -0 == +0 counts as a tie.  The chosen expert is marked taken
-// in its owner lane.  Gates are computed in fp32 from the chosen logits.
+// in its owner lane, and lane j keeps slot j.  Gates are computed in fp32
+// from logit / temperature ([GPT] §2.3, §4.1); with a threshold, a slot whose
+// probability is not above it is dropped (index -1, gate 0) and renormalised
+// gates divide by the kept slots' sum.
 // ---------------------------------------------------------------------------
 constexpr int kRouteWarps = 8;
 
@@ -145,7 +161,8 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
 template <int kEPL>
 __global__ void __launch_bounds__(kRouteWarps * 32)
     route_topk_kernel(const float* __restrict__ L, int T, int E, int k, int score, int renorm,
-                      int32_t* __restrict__ idx, float* __restrict__ gates) {
+                      float inv_temp, float min_prob, int32_t* __restrict__ idx,
+                      float* __restrict__ gates) {
   const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -157,13 +174,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     v[i] = (e < E) ? __ldg(row + e) : -FLT_MAX;
   }
   uint32_t taken = 0;
-  float selv[kMaxTopK];
-  int sele[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    selv[j] = 0.f;
-    sele[j] = 0;
-  }
+  float my_v = 0.f;  // lane j < k: logit of slot j
+  int my_e = 0;      // lane j < k: expert of slot j
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
     if (j < k) {
@@ -186,82 +198,67 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
           be = oe;
         }
       }
-      selv[j] = bv;
-      sele[j] = be;
+      if (lane == j) {
+        my_v = bv;
+        my_e = be;
+      }
       if ((be & 31) == lane) taken |= 1u << (be >> 5);
     }
   }
-  // gates
-  const float m = selv[0];
-  float denom = 0.f;
+  // Gates.  z = logit / temperature; the largest chosen logit is lane 0's.
+  const bool slot = lane < k;
+  const bool thr = min_prob > 0.f;
+  const float m = __shfl_sync(0xffffffffu, my_v, 0);
+  float q;  // unnormalised score of this lane's slot
   if (score == MOE_SCORE_SOFTMAX) {
-    if (renorm) {
-#pragma unroll
-      for (int j = 0; j < kMaxTopK; ++j)
-        if (j < k) denom += expf(selv[j] - m);
-    } else {
-      float part = 0.f;
-#pragma unroll
-      for (int i = 0; i < kEPL; ++i)
-        if (lane + 32 * i < E) part += expf(v[i] - m);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-      denom = part;
-    }
+    q = slot ? expf((my_v - m) * inv_temp) : 0.f;
   } else {
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < k) denom += 1.f / (1.f + expf(-selv[j]));
+    q = slot ? 1.f / (1.f + expf(-my_v * inv_temp)) : 0.f;
   }
+  float prob = q;  // softmax: q / sum over all E; sigmoid: q
+  if (score == MOE_SCORE_SOFTMAX && (thr || !renorm)) {
+    float part = 0.f;
 #pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    if (j < k && lane == j) {
-      float g;
-      if (score == MOE_SCORE_SOFTMAX) {
-        g = expf(selv[j] - m) / denom;
-      } else {
-        const float s = 1.f / (1.f + expf(-selv[j]));
-        g = renorm ? s / denom : s;
-      }
-      idx[(size_t)t * k + j] = sele[j];
-      gates[(size_t)t * k + j] = g;
-    }
+    for (int i = 0; i < kEPL; ++i)
+      if (lane + 32 * i < E) part += expf((v[i] - m) * inv_temp);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+    prob = q / part;
+  }
+  const bool keep = slot && (!thr || prob > min_prob);
+  float g;
+  if (renorm) {
+    // softmax: prob_j / sum_kept prob = q_j / sum_kept q; sigmoid: s_j / sum_kept s
+    float den = keep ? q : 0.f;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    g = (keep && den > 0.f) ? q / den : 0.f;
+  } else {
+    g = keep ? prob : 0.f;
+  }
+  if (slot) {
+    idx[(size_t)t * k + lane] = keep ? my_e : -1;
+    gates[(size_t)t * k + lane] = g;
   }
 }
 
 cudaError_t launch_route(const float* L, int T, int E, int k, int score, int renormalize,
-                         int32_t* idx, float* gates, cudaStream_t stream) {
+                         float temperature, float min_prob, int32_t* idx, float* gates,
+                         cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const int blocks = (T + kRouteWarps - 1) / kRouteWarps;
   const int epl = (E + 31) / 32;
-#define MOE_ROUTE_CASE(N)                                                                    \
-  case N:                                                                                    \
-    route_topk_kernel<N><<<blocks, kRouteWarps * 32, 0, stream>>>(L, T, E, k, score,         \
-                                                                  renormalize, idx, gates); \
-    break;
-  switch (epl) {
-    MOE_ROUTE_CASE(1)
-    MOE_ROUTE_CASE(2)
-    MOE_ROUTE_CASE(4)
-    MOE_ROUTE_CASE(8)
-    MOE_ROUTE_CASE(16)
-    MOE_ROUTE_CASE(32)
-    default:
-      if (epl <= 4) {
-        route_topk_kernel<4><<<blocks, kRouteWarps * 32, 0, stream>>>(L, T, E, k, score,
-                                                                      renormalize, idx, gates);
-      } else if (epl <= 8) {
-        route_topk_kernel<8><<<blocks, kRouteWarps * 32, 0, stream>>>(L, T, E, k, score,
-                                                                      renormalize, idx, gates);
-      } else if (epl <= 16) {
-        route_topk_kernel<16><<<blocks, kRouteWarps * 32, 0, stream>>>(L, T, E, k, score,
-                                                                       renormalize, idx, gates);
-      } else {
-        route_topk_kernel<32><<<blocks, kRouteWarps * 32, 0, stream>>>(L, T, E, k, score,
-                                                                       renormalize, idx, gates);
-      }
-  }
-#undef MOE_ROUTE_CASE
+  const float inv_temp = 1.0f / temperature;
+#define MOE_ROUTE_LAUNCH(N)                                                                    \
+  route_topk_kernel<N><<<blocks, kRouteWarps * 32, 0, stream>>>(L, T, E, k, score, renormalize, \
+                                                                inv_temp, min_prob, idx, gates)
+  if (epl <= 1) MOE_ROUTE_LAUNCH(1);
+  else if (epl <= 2) MOE_ROUTE_LAUNCH(2);
+  else if (epl <= 4) MOE_ROUTE_LAUNCH(4);
+  else if (epl <= 8) MOE_ROUTE_LAUNCH(8);
+  else if (epl <= 16) MOE_ROUTE_LAUNCH(16);
+  else MOE_ROUTE_LAUNCH(32);
+#undef MOE_ROUTE_LAUNCH
   return cudaGetLastError();
 }
 

@@ -6,8 +6,10 @@ path and the CPU oracle can consume its bytes without sharing method code.
 
 Workloads mirror the shapes the source pages discuss (a Mixtral-class layer
 with hidden size 4096 and 8 experts, top-1/top-2 routing; a DeepSeek-class
-layer with 256 experts) -- see "用消费级显卡跑 MoE" §1.2 for d=4096 and
-"DySHARP" §1 / TensorRT-LLM large-EP article for 256 experts per layer.
+layer with 256 experts) -- the ThunderEP PCIe blog §1.2 for d=4096, the
+DySHARP review §1 and the TensorRT-LLM large-EP article for 256 experts per
+layer, the GPT-4 "2%" article §2.3 and the xDeepServe blog §5.3 for router
+temperature and a minimum-probability threshold.
 Nothing here is a dataset: every tensor is drawn from a seeded generator.
 
 Draws
@@ -55,6 +57,8 @@ class LayerConfig:
     x_std: float = 1.0
     w_std: float = 0.02
     logit_std: float = 1.0
+    temperature: float = 1.0  # router temperature
+    min_prob: float = 0.0     # > 0: drop chosen slots whose probability is not above it
     extra: dict = field(default_factory=dict)
 
     @property
@@ -80,6 +84,12 @@ WORKLOADS: dict[str, LayerConfig] = {
     # Fine-grained many-expert layer: 256 experts, sigmoid top-8 renormalised.
     "fine_grained": _mk("fine_grained", 8192, 7168, 256, 8, 2048, "logits", "sigmoid", 1),
 }
+# Routing variants on the Mixtral shape: temperature 1.3 and a 0.05 minimum
+# probability (the values the pages discuss) -- some second choices are dropped.
+WORKLOADS["mixtral_threshold"] = _mk("mixtral_threshold", 4096, 4096, 8, 2, 14336, "weights",
+                                     "softmax", 1, temperature=1.3, min_prob=0.05)
+WORKLOADS["tiny_threshold"] = _mk("tiny_threshold", 256, 128, 8, 2, 256, "logits", "softmax", 1,
+                                  temperature=0.5, min_prob=0.2)
 for _T in (16, 64, 256, 1024):
     WORKLOADS[f"decode_{_T}"] = _mk(f"decode_{_T}", _T, 4096, 8, 2, 14336, "weights",
                                     "softmax", 1)

@@ -77,6 +77,8 @@ typedef struct moe_layer_desc {
   int32_t score;       /* moe_score */
   int32_t renormalize; /* 1: gates renormalised over the chosen k; 0: plain probability */
   int32_t reserved;    /* must be 0 */
+  float temperature;   /* router temperature (see moe_route_ex); 0 reads as 1 */
+  float min_prob;      /* drop chosen slots whose probability is <= min_prob; <= 0 keeps all */
 } moe_layer_desc;
 
 /* ---------------------------------------------------------------------------
@@ -108,6 +110,26 @@ moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32
                      int32_t renormalize, int32_t* topk_idx, float* gates, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_route_ex -- moe_route with a router temperature and a minimum-probability
+ * threshold (GPT-4 "2%" article §2.3: a temperature scales the logits before
+ * the softmax, and chosen experts whose probability falls under a minimum
+ * activation threshold are dropped; §4.1: probabilities not above the
+ * threshold give index -1).
+ *   Scores use z = logit / temperature (temperature > 0; the top-k order is
+ *   the same for every temperature).  A chosen slot's probability is its
+ *   softmax over all E experts, or its sigmoid.  When min_prob > 0, a slot
+ *   whose probability is <= min_prob is dropped: topk_idx = -1, gate 0.
+ *   Gates of kept slots: renormalize=1 divides by the kept slots' sum (the
+ *   softmax case equals exp(z_j - z_0) / sum_kept exp(z_i - z_0));
+ *   renormalize=0 keeps the probability.  A token with every slot dropped has
+ *   all gates 0 (its layer output is 0).  moe_route(...) ==
+ *   moe_route_ex(..., temperature = 1, min_prob = 0, ...).
+ * ------------------------------------------------------------------------- */
+moe_status moe_route_ex(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
+                        int32_t renormalize, float temperature, float min_prob,
+                        int32_t* topk_idx, float* gates, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_layout -- per-expert histogram, exclusive scan and the logical->layout
  * table (DySHARP §3.1 item 3: an AL table translates the logical i-th token to
  * its position in a dense per-expert tensor, layout blocks being allocated
@@ -118,8 +140,11 @@ moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32
  *     offsets[e]  = sum_{e' < e} counts[e'],  offsets[E] = R
  *     row_of[i]   = offsets[e_i] + #{i' < i : e_i' == e_i}   (stable by token)
  *     src_of[row_of[i]] = i
- *   topk_idx [T, k] int32 in [0, E) (others set MOE_DEV_BAD_EXPERT_ID and are
- *   skipped); counts [E], offsets [E+1], row_of [R], src_of [R] int32.
+ *   topk_idx [T, k] int32 in [0, E), or -1 for a dropped slot (see
+ *   moe_route_ex), which takes no row: row_of = -1, and offsets[E] counts the
+ *   kept slots only; rows r >= offsets[E] get src_of[r] = -1.  Any other id
+ *   sets MOE_DEV_BAD_EXPERT_ID and is treated as dropped.
+ *   counts [E], offsets [E+1], row_of [R], src_of [R] int32.
  *   ws: at least moe_layout_workspace_size(T, E, k) bytes; its contents are
  *   scratch (look-back status words for the multi-block scan).
  * ------------------------------------------------------------------------- */
@@ -157,7 +182,8 @@ moe_status moe_layout_static(const int32_t* topk_idx, int32_t T, int32_t E, int3
 /* ---------------------------------------------------------------------------
  * moe_dispatch -- copy each token to its k experts' rows (DySHARP §1: the same
  * token data goes to each of its k experts; ThunderEP §1.1).
- *   Xe[r, :] = X[src_of[r] / k, :]   for r in [0, T*k).
+ *   Xe[r, :] = X[src_of[r] / k, :]   for r in [0, T*k) with src_of[r] >= 0;
+ *   rows with src_of[r] = -1 (past the kept slots) are left untouched.
  *   X [T, d] bf16, src_of [T*k] int32, Xe [T*k, d] bf16.
  * ------------------------------------------------------------------------- */
 moe_status moe_dispatch(const void* X, const int32_t* src_of, int32_t T, int32_t d, int32_t k,
@@ -193,7 +219,8 @@ moe_status moe_expert_ffn(const void* Xe, const int32_t* offsets, const void* W1
  * (DySHARP §1: the k results are summed into one; ThunderEP §2.1: the gate
  * values weight the combine sum).
  *   Y[t, :] = bf16( sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :] ),
- *   summed in fp32 in slot order j = 0..k-1.
+ *   summed in fp32 in slot order j = 0..k-1; a dropped slot (row_of = -1)
+ *   contributes nothing (its Ye row is not read).
  *   Ye [T*k, d] bf16, row_of [T*k] int32, gates [T, k] fp32, Y [T, d] bf16.
  * ------------------------------------------------------------------------- */
 moe_status moe_combine(const void* Ye, const int32_t* row_of, const float* gates, int32_t T,

@@ -97,6 +97,35 @@ def test_route_parity(T, E, k, score, renorm, kind):
     np.testing.assert_allclose(g.cpu().numpy(), ref_g, rtol=2e-6, atol=2e-7)
 
 
+ROUTE_EX_CASES = [
+    # (T, E, k, score, renorm, temperature, min_prob)
+    (2000, 8, 2, "softmax", 1, 1.3, 0.05),
+    (2000, 16, 4, "softmax", 0, 0.3, 0.05),
+    (1000, 64, 6, "softmax", 1, 2.0, 0.02),
+    (1000, 256, 8, "sigmoid", 1, 1.0, 0.6),
+    (500, 8, 2, "sigmoid", 0, 0.5, 0.7),
+    (300, 8, 8, "softmax", 1, 1.0, 0.2),      # most slots dropped
+    (300, 1024, 16, "softmax", 1, 0.7, 0.0),  # temperature only
+]
+
+
+@pytest.mark.parametrize("T,E,k,score,renorm,temp,thr", ROUTE_EX_CASES)
+def test_route_ex_parity(T, E, k, score, renorm, temp, thr):
+    L = _logits(T, E, "normal", seed=3)
+    idx, g = moe.moe_route_ex(L.to(DEV), k, score, renorm, temp, thr)
+    ref_idx, ref_g = O.route(L.numpy(), k, score, renorm, temp, thr)
+    # the keep decision compares a probability with the threshold: slots
+    # within fp32 rounding of it may go either way on the GPU
+    sel = O.topk_order(L.numpy(), k)
+    gates_all, _ = O.gates_from_logits(L.numpy(), sel, score, 0, temp, 0.0)
+    ambiguous = (np.abs(gates_all - thr) <= 1e-6 * max(thr, 1e-30)).any(1) if thr > 0 else np.zeros(T, bool)
+    gi, gg = idx.cpu().numpy(), g.cpu().numpy()
+    ok = ~ambiguous
+    assert np.array_equal(gi[ok], ref_idx[ok])
+    np.testing.assert_allclose(gg[ok], ref_g[ok], rtol=2e-6, atol=2e-7)
+    assert ((gi == -1) == (gg == 0))[ok].all()
+
+
 # ----------------------------------------------------------------------------
 # router linear
 # ----------------------------------------------------------------------------
@@ -158,12 +187,27 @@ def test_layout_repeatable_and_stable_under_reuse():
 def test_layout_flags_bad_expert_ids():
     idx = I.random_topk(64, 8, 2, 7)
     idx[3, 1] = 8
-    idx[10, 0] = -1
+    idx[10, 0] = -5
     counts, offsets, row_of, src_of = moe.moe_layout(idx.to(DEV), 8)
     assert moe.moe_device_status(clear=True) & 1  # MOE_DEV_BAD_EXPERT_ID
     rc = row_of.cpu().numpy()
     assert rc[3 * 2 + 1] == -1 and rc[10 * 2] == -1
     assert counts.sum().item() == 64 * 2 - 2
+
+
+@pytest.mark.parametrize("T,E,k,drop", [(256, 8, 2, 0.2), (8192, 256, 8, 0.3), (9000, 7, 3, 0.5),
+                                        (40, 1024, 4, 1.0)])
+def test_layout_dropped_slots(T, E, k, drop):
+    """-1 marks a dropped slot: no row, not counted, no flag; unused rows get src_of -1."""
+    idx = I.random_topk(T, E, k, 8)
+    rng = np.random.default_rng(8)
+    idx[torch.from_numpy(rng.random((T, k)) < drop)] = -1
+    counts, offsets, row_of, src_of = moe.moe_layout(idx.to(DEV), E)
+    rc, ro, rr, rs = O.layout(idx.numpy(), E)
+    assert np.array_equal(counts.cpu().numpy(), rc)
+    assert np.array_equal(offsets.cpu().numpy(), ro)
+    assert np.array_equal(row_of.cpu().numpy(), rr)
+    assert np.array_equal(src_of.cpu().numpy(), rs)
 
 
 # ----------------------------------------------------------------------------
@@ -197,6 +241,31 @@ def test_combine_parity(T, d, E, k):
     # one bf16 rounding of an fp32 sum: |err| <= 2^-8 |ref| + fp32 slack
     slack = 1e-6 * (np.abs(g32.double().numpy()).sum(1, keepdims=True) * 8)
     assert (np.abs(out - ref) <= 2.0 ** -8 * np.abs(ref) + slack).all()
+
+
+def test_dispatch_and_combine_with_dropped_slots():
+    T, d, E, k = 500, 256, 8, 2
+    idx = I.random_topk(T, E, k, 9)
+    rng = np.random.default_rng(9)
+    idx[torch.from_numpy(rng.random((T, k)) < 0.3)] = -1
+    idx[7] = -1                                   # a token with every slot dropped
+    _, ro, rr, rs = O.layout(idx.numpy(), E)
+    kept = int(ro[-1])
+    X = I.random_bf16((T, d), 9, "X")
+    Xe = torch.full((T * k, d), 3.0, dtype=torch.bfloat16, device=DEV)
+    moe.moe_dispatch(X.to(DEV), torch.from_numpy(rs).to(DEV), k, Xe=Xe)
+    assert np.array_equal(bits(Xe[:kept]), O.dispatch(bits(X), rs, k)[:kept])
+    assert (Xe[kept:] == 3.0).all()                # unused rows untouched
+    Ye = I.random_bf16((T * k, d), 9, "Ye")
+    Ye[kept:] = float("nan")                       # never read
+    g = torch.rand((T, k), generator=torch.Generator().manual_seed(9))
+    g[idx < 0] = 0.0
+    Y = moe.moe_combine(Ye.to(DEV), torch.from_numpy(rr).to(DEV), g.to(DEV))
+    ref = O.combine(O.bf16_to_f64(bits(Ye)), rr, g.double().numpy(), k)
+    out = f64(Y)
+    assert not np.isnan(out).any()
+    assert (out[7] == 0).all()
+    assert_close(out, ref, "combine with drops")
 
 
 def test_identity_experts_return_input():
@@ -282,7 +351,7 @@ def test_expert_ffn_tiny_matches_oracle():
 def _run_layer(inp, cfg):
     dev_in = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
     layer = moe.MoeLayer(dev_in["W1"], dev_in["W2"], cfg.k, cfg.score, cfg.renormalize,
-                         Wr=dev_in["Wr"])
+                         Wr=dev_in["Wr"], temperature=cfg.temperature, min_prob=cfg.min_prob)
     T = cfg.T
     idx = torch.empty((T, cfg.k), dtype=torch.int32, device=DEV)
     g = torch.empty((T, cfg.k), dtype=torch.float32, device=DEV)
@@ -303,6 +372,28 @@ def test_layer_tiny_full_parity():
     assert np.array_equal(counts.cpu().numpy(), ref["counts"])
     np.testing.assert_allclose(g.cpu().numpy(), ref["gates"], rtol=2e-6, atol=2e-7)
     assert_close(f64(Y), ref["Y"], "Y")
+
+
+def test_layer_tiny_threshold_full_parity():
+    cfg = I.workload("tiny_threshold")
+    inp = I.make_layer_inputs(cfg, 0, device=DEV)
+    ref = O.layer_forward(bits(inp["X"]), bits(inp["W1"]), bits(inp["W2"]), cfg.k, cfg.score,
+                          cfg.renormalize, logits=inp["logits"].numpy(),
+                          temperature=cfg.temperature, min_prob=cfg.min_prob)
+    dropped = int((ref["topk_idx"] < 0).sum())
+    assert 0 < dropped < cfg.R  # the variant is exercised
+    sel = O.topk_order(inp["logits"].numpy(), cfg.k)
+    p, _ = O.gates_from_logits(inp["logits"].numpy(), sel, cfg.score, 0, cfg.temperature, 0.0)
+    assert not (np.abs(p - cfg.min_prob) <= 1e-6 * cfg.min_prob).any()  # no ambiguous slot
+    dev_in = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    layer = moe.MoeLayer(dev_in["W1"], dev_in["W2"], cfg.k, cfg.score, cfg.renormalize,
+                         temperature=cfg.temperature, min_prob=cfg.min_prob)
+    idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=DEV)
+    counts = torch.empty((cfg.E,), dtype=torch.int32, device=DEV)
+    Y = layer(dev_in["X"], logits=dev_in["logits"], topk_idx_out=idx, counts_out=counts)
+    assert np.array_equal(idx.cpu().numpy(), ref["topk_idx"])
+    assert np.array_equal(counts.cpu().numpy(), ref["counts"])
+    assert_close(f64(Y), ref["Y"], "Y (threshold)")
 
 
 def test_layer_deterministic():
@@ -330,6 +421,7 @@ def _near_ties(L, k, eps):
 @pytest.mark.slow
 @pytest.mark.parametrize("name,nsample", [("skewed_top1", 48), ("skewed_top1_harsh", 24),
                                           ("fine_grained", 12), ("mixtral", 32),
+                                          ("mixtral_threshold", 32),
                                           ("decode_16", 16), ("decode_64", 24),
                                           ("decode_256", 24), ("decode_1024", 24)])
 def test_layer_full_size_sampled(name, nsample):
@@ -348,10 +440,16 @@ def test_layer_full_size_sampled(name, nsample):
     else:
         Lref = inp["logits"].numpy()
         ties = np.zeros(cfg.T, bool)
-    ref_idx, ref_g = O.route(Lref, cfg.k, cfg.score, cfg.renormalize)
+    ref_idx, ref_g = O.route(Lref, cfg.k, cfg.score, cfg.renormalize, cfg.temperature,
+                             cfg.min_prob)
+    if cfg.min_prob > 0:  # slots within rounding of the threshold may go either way
+        sel = O.topk_order(Lref, cfg.k)
+        p, _ = O.gates_from_logits(Lref, sel, cfg.score, 0, cfg.temperature, 0.0)
+        ties |= (np.abs(p - cfg.min_prob) <= 1e-5 * cfg.min_prob).any(1)
     mism = np.any(gi != ref_idx, axis=1)
     assert not (mism & ~ties).any(), f"{int((mism & ~ties).sum())} tokens routed differently"
-    assert np.array_equal(counts.cpu().numpy()[None], np.bincount(gi.ravel(), minlength=cfg.E)[None])
+    kept = gi[gi >= 0]
+    assert np.array_equal(counts.cpu().numpy(), np.bincount(kept, minlength=cfg.E))
     toks = np.array([t for t in _sample_tokens(cfg.T, nsample) if not ties[t]])
     ref = O.layer_forward_tokens(X_bits, LazyExperts(inp["W1"]), LazyExperts(inp["W2"]), ref_idx,
                                  ref_g, toks)

@@ -341,6 +341,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         f1.record(stream)
         sync_all()
         e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+
     finally:
         if sampler:
             sampler.__exit__(None, None, None)

@@ -311,6 +311,11 @@ GEMM_CASES = [
     ([5, 3], 8, 8, False),                            # smallest dims
     ([128] * 3, 1024, 1024, True),
     ([1] * 64, 256, 256, False),                      # many one-row experts
+    # mean > 192 rows per expert: tiles of up to 512 rows in two accumulators
+    ([300, 0, 513, 1, 256, 257], 512, 192, True),
+    ([600, 520], 264, 128, False),                    # N tail with wide tiles
+    ([1030, 990, 1024], 256, 320, True),
+    ([260] * 16, 384, 64, False),                     # 16 experts just over one block
 ]
 
 
@@ -476,3 +481,30 @@ def test_gemm_gelu_is_exact_to_bf16():
     big = np.abs(ref) > 1e-3  # where bf16 resolution dominates: the rounded value itself
     ref_bits = I.f32_to_bf16_bits(ref.astype(np.float32))
     assert (bits(out)[big] == ref_bits[big]).mean() >= 0.99
+
+
+@pytest.mark.parametrize("name", ["decode_16", "tiny"])
+def test_layer_forward_replays_in_a_cuda_graph(name):
+    """Sizes stay on the device and nothing syncs the host, so one layer forward
+    captures into a CUDA graph; replays reproduce the eager output bit for bit."""
+    cfg = I.workload(name)
+    inp = I.make_layer_inputs(cfg, 2, device=DEV)
+    X = inp["X"].to(DEV)
+    L = inp["logits"].to(DEV) if inp["logits"] is not None else None
+    Wr = inp["Wr"].to(DEV) if inp["Wr"] is not None else None
+    layer = moe.MoeLayer(inp["W1"], inp["W2"], cfg.k, cfg.score, cfg.renormalize, Wr=Wr)
+    Y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=DEV)
+    s = torch.cuda.Stream(device=DEV)
+    s.wait_stream(torch.cuda.current_stream(DEV))
+    with torch.cuda.stream(s):
+        layer(X, logits=L, Y=Y)  # first call: per-device set-up happens outside the capture
+        eager = Y.clone()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            layer(X, logits=L, Y=Y)
+    torch.cuda.current_stream(DEV).wait_stream(s)
+    Y.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y.view(torch.int16), eager.view(torch.int16))

@@ -41,6 +41,15 @@ Readings where the pages are silent (each is also listed in the design notes):
   * GELU is the exact erf form 0.5*x*(1+erf(x/sqrt 2)).
   * everything is float64 from the same bf16 / fp32 input bytes; H and Ye
     are NOT rounded to bf16 here (the GPU does; the tolerance covers it).
+  * FP8 mode ([TEP] §3.3, §5.2: activations cast to FP8 with one dynamic
+    per-tensor scale before they move, cast back after): the token matrix X
+    is quantised to E4M3 with inv = 448 / amax(|X|) and codes =
+    E4M3(x * inv), both fp32 operations and round-to-nearest-even with
+    saturation, so the codes are an integer result both sides decide in the
+    same precision.  GEMM-1 then runs on the FP8 operands (the pages' FP8
+    tensor-core compute); the pages do not say how the weights get to FP8,
+    so each expert's W1 is quantised once with its own per-tensor scale.
+    GEMM-2 and combine stay bf16.
 
 Parity status: every function here is pinned by tests that do not reuse its
 code (brute force, invariants, closed forms, library special cases).
@@ -323,3 +332,120 @@ def tolerance(ref: np.ndarray, rel: float = 2e-2, abs_: float = 1e-3) -> float:
     """Float parity bound max|out - ref| <= rel * max|ref| + abs (bf16 I/O, fp32 accumulate)."""
     ref = np.asarray(ref, np.float64)
     return rel * (float(np.abs(ref).max()) if ref.size else 0.0) + abs_
+
+
+# ----------------------------------------------------------------------------
+# FP8 dispatch + FP8 GEMM-1   [TEP] §3.3 (activations cast to fp8 with a
+# per-tensor dynamic scale before the transfer; tensor cores that support
+# FP8 compute on it natively), §5.2 (cast before sending, per-tensor scale)
+# ----------------------------------------------------------------------------
+# E4M3: 1 sign, 4 exponent (bias 7), 3 mantissa bits; no infinities; the
+# largest finite value is 448 (exponent 15, mantissa 6); 0x7F / 0xFF is NaN.
+E4M3_MAX = 448.0
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """E4M3 codes (uint8) -> float64 values, from the format's definition."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * 2.0 ** (e - 7.0))
+    val = np.where((e == 15) & (m == 7), np.nan, val)
+    return sign * val
+
+
+_E4M3_POS = e4m3_decode(np.arange(0x7F, dtype=np.uint8))  # codes 0x00..0x7E, increasing
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Round finite values to E4M3: nearest representable value, ties to the
+    even code (mantissa LSB 0), magnitudes past 448 saturate to 448."""
+    a = np.asarray(x, dtype=np.float64)
+    mag = np.abs(a)
+    hi = np.searchsorted(_E4M3_POS, mag, side="left").clip(0, 0x7E)  # first value >= mag
+    lo = (hi - 1).clip(0, 0x7E)
+    d_hi = _E4M3_POS[hi] - mag
+    d_lo = mag - _E4M3_POS[lo]
+    pick_lo = (d_lo < d_hi) | ((d_lo == d_hi) & (lo % 2 == 0))
+    code = np.where(pick_lo, lo, hi)
+    code = np.where(mag >= E4M3_MAX, 0x7E, code)          # saturate
+    code = code | np.where(np.signbit(a), 0x80, 0)
+    code = np.where(np.isnan(a), 0x7F, code)
+    return code.astype(np.uint8)
+
+
+def fp8_quantize(x_f32, amax=None):
+    """Per-tensor dynamic FP8 quantisation, every step in fp32 as the kernel does.
+
+    amax = max |x| (the tensor's own unless given); inv = 448 / amax and
+    x * inv are fp32 operations (round to nearest); codes = e4m3_encode of the
+    product; the dequantisation scale is s = amax / 448 (fp32).  amax = 0
+    gives inv = s = 1.  Returns (codes uint8, s float32).
+    """
+    x = np.asarray(x_f32, dtype=np.float32)
+    if amax is None:
+        amax = np.float32(np.abs(x).max()) if x.size else np.float32(0)
+    amax = np.float32(amax)
+    if amax > 0:
+        inv = np.float32(E4M3_MAX) / amax
+        s = amax / np.float32(E4M3_MAX)
+    else:
+        inv = np.float32(1.0)
+        s = np.float32(1.0)
+    y = (x * inv).astype(np.float32)
+    return e4m3_encode(y), np.float32(s)
+
+
+def fp8_quantize_experts(W_bits):
+    """Per-expert quantisation of bf16 expert weights [E, rows, cols]:
+    one scale per expert.  Returns (codes uint8 [E, rows, cols], s [E] float32)."""
+    W = np.asarray(W_bits)
+    E = W.shape[0]
+    codes = np.empty(W.shape, dtype=np.uint8)
+    s = np.empty(E, dtype=np.float32)
+    for e in range(E):
+        w = bf16_to_f64(W[e]).astype(np.float32)  # exact: bf16 widens to fp32
+        codes[e], s[e] = fp8_quantize(w)
+    return codes, s
+
+
+def fp8_gemm1(Xq_rows, x_scale, W1q_e, w_scale_e) -> np.ndarray:
+    """H = GELU((Xq * s_x) @ (W1q[e] * s_w[e])^T) on the dequantised FP8 operands."""
+    x = e4m3_decode(Xq_rows) * float(x_scale)
+    w = e4m3_decode(W1q_e) * float(w_scale_e)
+    return gelu(x @ w.T)
+
+
+def layer_forward_fp8(X_bits, W1q, w1_scale, W2_bits, k, score=SOFTMAX, renormalize=1,
+                      logits=None, Wr_bits=None, temperature=1.0, min_prob=0.0):
+    """The layer with FP8 dispatch and FP8 GEMM-1 (GEMM-2 and combine as in bf16).
+
+    The dispatched activations are the tokens quantised with one per-tensor
+    scale over all of X; GEMM-1 runs on the dequantised FP8 operands.
+    """
+    X = bf16_to_f64(X_bits)
+    T, d = X.shape
+    E = W1q.shape[0]
+    if logits is None:
+        L = router_logits(X, bf16_to_f64(Wr_bits)).astype(np.float32)
+    else:
+        L = np.asarray(logits, dtype=np.float32)
+    idx, gates = route(L, k, score, renormalize, temperature, min_prob)
+    counts, offsets, row_of, src_of = layout(idx, E)
+    Xq, x_scale = fp8_quantize(X.astype(np.float32))
+    Xe_q = np.zeros((src_of.size, d), dtype=np.uint8)
+    ok = src_of >= 0
+    Xe_q[ok] = Xq[src_of[ok] // k]
+    R = src_of.size
+    H = np.zeros((R, W1q.shape[1]))
+    Ye = np.zeros((R, d))
+    for e in range(E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if a == b:
+            continue
+        H[a:b] = fp8_gemm1(Xe_q[a:b], x_scale, W1q[e], w1_scale[e])
+        Ye[a:b] = expert_gemm2(H[a:b], _as_f64(W2_bits[e]))
+    Y = combine(Ye, row_of, gates, k)
+    return dict(logits=L, topk_idx=idx, gates=gates, counts=counts, offsets=offsets,
+                row_of=row_of, src_of=src_of, Xq=Xq, x_scale=x_scale, Xe_q=Xe_q, H=H, Ye=Ye, Y=Y)

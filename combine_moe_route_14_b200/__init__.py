@@ -24,6 +24,8 @@ __all__ = [
     "moe_dispatch", "moe_expert_gemm", "moe_expert_ffn", "moe_combine",
     "moe_workspace_size", "moe_layer_forward", "moe_device_status",
     "moe_kernel_launches_per_forward", "MoeLayer", "SCORES",
+    "moe_quantize_experts_fp8", "moe_dispatch_fp8", "moe_expert_gemm_fp8",
+    "moe_layer_forward_fp8", "moe_kernel_launches_per_forward_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -74,6 +76,12 @@ _SIG = {
     "moe_last_error_string": ([], ctypes.c_char_p),
     "moe_device_status": ([ctypes.POINTER(ctypes.c_uint32), _I], ctypes.c_int),
     "moe_kernel_launches_per_forward": ([ctypes.POINTER(LayerDesc), _I], ctypes.c_int32),
+    "moe_quantize_experts_fp8": ([_P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
+    "moe_dispatch_fp8": ([_P, _P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
+    "moe_expert_gemm_fp8": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
+    "moe_layer_forward_fp8": ([ctypes.POINTER(LayerDesc), _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                               _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_kernel_launches_per_forward_fp8": ([ctypes.POINTER(LayerDesc), _I], ctypes.c_int32),
 }
 
 
@@ -334,6 +342,95 @@ def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=No
     return Y
 
 
+# ----------------------------------------------------------------------------
+# FP8 (E4M3) mode: codes are torch.uint8 tensors, scales fp32
+# ----------------------------------------------------------------------------
+def moe_quantize_experts_fp8(W, Wq=None, scales=None, stream=None):
+    """Per-expert E4M3 quantisation of bf16 expert weights [E, rows, cols]."""
+    lib = load_library()
+    E, rows, cols = W.shape
+    dev = W.device
+    _need(W, "W", torch.bfloat16, (E, rows, cols))
+    Wq = _out(Wq, "Wq", torch.uint8, (E, rows, cols), dev)
+    scales = _out(scales, "scales", torch.float32, (E,), dev)
+    _check(lib.moe_quantize_experts_fp8(_ptr(W), E, rows, cols, _ptr(Wq), _ptr(scales),
+                                        _stream(stream, dev)))
+    return Wq, scales
+
+
+def moe_dispatch_fp8(X, src_of, k, Xeq=None, x_scale=None, stream=None):
+    """Quantising dispatch; returns (Xeq uint8 [T*k, d], x_scale fp32 [2] = [scale, amax])."""
+    lib = load_library()
+    T, d = X.shape
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (T, d))
+    _need(src_of, "src_of", torch.int32, (T * k,), dev)
+    Xeq = _out(Xeq, "Xeq", torch.uint8, (T * k, d), dev)
+    x_scale = _out(x_scale, "x_scale", torch.float32, (2,), dev)
+    _check(lib.moe_dispatch_fp8(_ptr(X), _ptr(src_of), T, d, k, _ptr(Xeq), _ptr(x_scale),
+                                _stream(stream, dev)))
+    return Xeq, x_scale
+
+
+def moe_expert_gemm_fp8(Aq, a_scale, offsets, Wq, w_scale, gelu, out=None, stream=None):
+    lib = load_library()
+    R, K = Aq.shape
+    E, N, K2 = Wq.shape
+    dev = Aq.device
+    if K2 != K:
+        raise ValueError("Wq's last dim must equal Aq's")
+    _need(Aq, "Aq", torch.uint8, (R, K))
+    if a_scale.dtype != torch.float32 or a_scale.device != dev or a_scale.numel() < 1:
+        raise ValueError("a_scale must be a float32 device tensor")
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(Wq, "Wq", torch.uint8, (E, N, K), dev)
+    _need(w_scale, "w_scale", torch.float32, (E,), dev)
+    out = _out(out, "out", torch.bfloat16, (R, N), dev)
+    _check(lib.moe_expert_gemm_fp8(_ptr(Aq), _ptr(a_scale), _ptr(offsets), _ptr(Wq),
+                                   _ptr(w_scale), E, R, N, K, int(bool(gelu)), _ptr(out),
+                                   _stream(stream, dev)))
+    return out
+
+
+def moe_kernel_launches_per_forward_fp8(desc: LayerDesc, with_router: bool) -> int:
+    return int(load_library().moe_kernel_launches_per_forward_fp8(ctypes.byref(desc),
+                                                                  int(bool(with_router))))
+
+
+def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=True,
+                          logits=None, Wr=None, Y=None, topk_idx_out=None, gates_out=None,
+                          counts_out=None, ws=None, stream=None, temperature=1.0, min_prob=0.0):
+    """The layer with FP8 dispatch and FP8 GEMM-1 (W1q, w1_scale from moe_quantize_experts_fp8)."""
+    lib = load_library()
+    T, d = X.shape
+    E, f, _ = W1q.shape
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (T, d))
+    _need(W1q, "W1q", torch.uint8, (E, f, d), dev)
+    _need(w1_scale, "w1_scale", torch.float32, (E,), dev)
+    _need(W2, "W2", torch.bfloat16, (E, d, f), dev)
+    if logits is not None:
+        _need(logits, "logits", torch.float32, (T, E), dev)
+    if Wr is not None:
+        _need(Wr, "Wr", torch.bfloat16, (E, d), dev)
+    Y = _out(Y, "Y", torch.bfloat16, (T, d), dev)
+    if topk_idx_out is not None:
+        _need(topk_idx_out, "topk_idx_out", torch.int32, (T, k), dev)
+    if gates_out is not None:
+        _need(gates_out, "gates_out", torch.float32, (T, k), dev)
+    if counts_out is not None:
+        _need(counts_out, "counts_out", torch.int32, (E,), dev)
+    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob)
+    if ws is None:
+        ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _check(lib.moe_layer_forward_fp8(ctypes.byref(desc), _ptr(X), _ptr(logits), _ptr(Wr),
+                                     _ptr(W1q), _ptr(w1_scale), _ptr(W2), _ptr(Y),
+                                     _ptr(topk_idx_out), _ptr(gates_out), _ptr(counts_out),
+                                     _ptr(ws), ws.numel(), _stream(stream, dev)))
+    return Y
+
+
 def moe_device_status(clear: bool = True) -> int:
     """Synchronise the current device and return its sticky MOE_DEV_* bits."""
     lib = load_library()
@@ -348,8 +445,11 @@ class MoeLayer:
     """A layer's weights plus a reusable workspace (allocation stays outside the call)."""
 
     def __init__(self, W1, W2, k, score="softmax", renormalize=True, Wr=None, temperature=1.0,
-                 min_prob=0.0):
+                 min_prob=0.0, fp8=False):
         self.W1, self.W2, self.Wr = W1, W2, Wr
+        self.fp8 = bool(fp8)
+        # FP8 mode keeps W1 as E4M3 codes with per-expert scales (quantised once here)
+        self.W1q, self.w1_scale = moe_quantize_experts_fp8(W1) if self.fp8 else (None, None)
         self.k, self.score, self.renormalize = k, score, renormalize
         self.temperature, self.min_prob = temperature, min_prob
         self.E, self.f, self.d = W1.shape
@@ -364,9 +464,11 @@ class MoeLayer:
 
     def __call__(self, X, logits=None, Y=None, topk_idx_out=None, gates_out=None,
                  counts_out=None, stream=None):
-        return moe_layer_forward(X, self.W1, self.W2, self.k, self.score, self.renormalize,
-                                 logits=logits, Wr=None if logits is not None else self.Wr,
-                                 Y=Y, topk_idx_out=topk_idx_out, gates_out=gates_out,
-                                 counts_out=counts_out, ws=self.workspace(X.shape[0]),
-                                 stream=stream, temperature=self.temperature,
-                                 min_prob=self.min_prob)
+        kw = dict(logits=logits, Wr=None if logits is not None else self.Wr, Y=Y,
+                  topk_idx_out=topk_idx_out, gates_out=gates_out, counts_out=counts_out,
+                  ws=self.workspace(X.shape[0]), stream=stream, temperature=self.temperature,
+                  min_prob=self.min_prob)
+        if self.fp8:
+            return moe_layer_forward_fp8(X, self.W1q, self.w1_scale, self.W2, self.k, self.score,
+                                         self.renormalize, **kw)
+        return moe_layer_forward(X, self.W1, self.W2, self.k, self.score, self.renormalize, **kw)

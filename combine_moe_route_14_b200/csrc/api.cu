@@ -127,7 +127,7 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // Workspace of the fused forward: sub-buffers, each 256-byte aligned.
 struct LayerWs {
-  size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, total;
+  size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, scale, total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -144,9 +144,10 @@ LayerWs layer_ws(const moe_layer_desc& d) {
   w.row_of = o;  o += up256(R * sizeof(int32_t));
   w.src_of = o;  o += up256(R * sizeof(int32_t));
   w.layout = o;  o += up256(moe::layout_workspace_bytes((int64_t)R, d.E));
-  w.Xe = o;      o += up256(R * d.d * 2);
+  w.Xe = o;      o += up256(R * d.d * 2);  // bf16 rows, or E4M3 rows in the first half
   w.H = o;       o += up256(R * d.f * 2);
   w.Ye = o;      o += up256(R * d.d * 2);
+  w.scale = o;   o += up256(2 * sizeof(float));  // FP8 mode: activation scale and amax
   w.total = o;
   return w;
 }
@@ -168,6 +169,95 @@ moe_status check_desc(const moe_layer_desc* desc) {
 }
 
 float desc_temperature(const moe_layer_desc& d) { return d.temperature > 0.f ? d.temperature : 1.f; }
+
+moe_status check_fp8_dim(int32_t v, const char* name) {
+  if (v % 16) return fail(MOE_ERR_UNSUPPORTED, std::string(name) + " must be a multiple of 16 in FP8 mode");
+  return MOE_OK;
+}
+
+moe_status gemm_fail(cudaError_t e, const std::string& err, const char* where) {
+  return err.empty() ? cuda_fail(e, where) : fail(MOE_ERR_CUDA, std::string(where) + ": " + err);
+}
+
+// The layer forward of both modes: W1s == nullptr runs bf16, otherwise
+// W1 holds E4M3 codes with per-expert scales W1s (FP8 dispatch + GEMM-1).
+moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float* logits,
+                         const void* Wr, const void* W1, const float* W1s, const void* W2,
+                         void* Y, int32_t* topk_idx_out, float* gates_out, int32_t* counts_out,
+                         void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc d = *desc;
+  const bool fp8 = W1s != nullptr;
+  if ((logits == nullptr) == (Wr == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "give exactly one of logits and Wr");
+  if (fp8) MOE_TRY(check_fp8_dim(d.d, "d"));
+  if (d.T == 0) return MOE_OK;
+  if ((int64_t)d.E * d.f >= (1ll << 31) || (int64_t)d.E * d.d >= (1ll << 31))
+    return fail(MOE_ERR_UNSUPPORTED, "E*f and E*d must be < 2^31");
+  MOE_TRY(check_ptr(X, "X"));
+  if (logits) MOE_TRY(check_ptr4(logits, "logits"));
+  if (Wr) MOE_TRY(check_ptr(Wr, "Wr"));
+  MOE_TRY(check_ptr(W1, fp8 ? "W1q" : "W1"));
+  if (fp8) MOE_TRY(check_ptr4(W1s, "w1_scale"));
+  MOE_TRY(check_ptr(W2, "W2"));
+  MOE_TRY(check_ptr(Y, "Y"));
+  if (topk_idx_out) MOE_TRY(check_ptr4(topk_idx_out, "topk_idx_out"));
+  if (gates_out) MOE_TRY(check_ptr4(gates_out, "gates_out"));
+  if (counts_out) MOE_TRY(check_ptr4(counts_out, "counts_out"));
+  const LayerWs w = layer_ws(d);
+  if (ws_bytes < w.total) return fail(MOE_ERR_INVALID_ARG, "workspace too small");
+  MOE_TRY(check_ptr(ws, "ws"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  cudaStream_t s = as_stream(stream);
+  char* base = static_cast<char*>(ws);
+  float* L = logits ? const_cast<float*>(logits) : reinterpret_cast<float*>(base + w.logits);
+  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(base + w.idx);
+  float* gates = gates_out ? gates_out : reinterpret_cast<float*>(base + w.gates);
+  int32_t* counts = counts_out ? counts_out : reinterpret_cast<int32_t*>(base + w.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + w.offsets);
+  int32_t* row_of = reinterpret_cast<int32_t*>(base + w.row_of);
+  int32_t* src_of = reinterpret_cast<int32_t*>(base + w.src_of);
+  void* lws = base + w.layout;
+  void* Xe = base + w.Xe;
+  void* H = base + w.H;
+  void* Ye = base + w.Ye;
+  float* x_scale = reinterpret_cast<float*>(base + w.scale);
+  const int R = d.T * d.k;
+
+  if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, s), "router_logits");
+  MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
+                             d.min_prob, idx, gates, s),
+           "route");
+  MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s), "layout");
+  std::string err;
+  cudaError_t e;
+  if (fp8) {
+    MOE_CUDA(moe::launch_dispatch_fp8(X, src_of, d.T, d.d, d.k, Xe, x_scale, *dev, s), "dispatch_fp8");
+    e = moe::launch_grouped_gemm_fp8(Xe, x_scale, offsets, W1, W1s, d.E, R, d.f, d.d, true, H,
+                                     *dev, s, &err);
+  } else {
+    MOE_CUDA(moe::launch_dispatch(X, src_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+    e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err);
+  }
+  if (e != cudaSuccess) return gemm_fail(e, err, "gemm1");
+  e = moe::launch_grouped_gemm(H, offsets, W2, d.E, R, d.d, d.f, false, Ye, *dev, s, &err);
+  if (e != cudaSuccess) return gemm_fail(e, err, "gemm2");
+  MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
+  return MOE_OK;
+}
+
+moe_status check_gemm_shape(int32_t E, int32_t R, int32_t N, int32_t K, int32_t gelu) {
+  if (E < 1) return fail(MOE_ERR_INVALID_ARG, "E must be >= 1");
+  if (E > moe::kMaxExperts) return fail(MOE_ERR_UNSUPPORTED, "E > 1024 is not supported");
+  if (R < 0) return fail(MOE_ERR_INVALID_ARG, "R must be >= 0");
+  if (R >= (1 << 30)) return fail(MOE_ERR_UNSUPPORTED, "R must be < 2^30");
+  MOE_TRY(check_dim(N, "N"));
+  MOE_TRY(check_dim(K, "K"));
+  if ((int64_t)E * N >= (1ll << 31)) return fail(MOE_ERR_UNSUPPORTED, "E*N must be < 2^31");
+  if (gelu != 0 && gelu != 1) return fail(MOE_ERR_INVALID_ARG, "gelu must be 0 or 1");
+  return MOE_OK;
+}
 
 }  // namespace
 
@@ -276,14 +366,7 @@ moe_status moe_dispatch(const void* X, const int32_t* src_of, int32_t T, int32_t
 moe_status moe_expert_gemm(const void* A, const int32_t* offsets, const void* W, int32_t E,
                            int32_t R, int32_t N, int32_t K, int32_t gelu, void* out,
                            void* stream) {
-  if (E < 1) return fail(MOE_ERR_INVALID_ARG, "E must be >= 1");
-  if (E > moe::kMaxExperts) return fail(MOE_ERR_UNSUPPORTED, "E > 1024 is not supported");
-  if (R < 0) return fail(MOE_ERR_INVALID_ARG, "R must be >= 0");
-  if (R >= (1 << 30)) return fail(MOE_ERR_UNSUPPORTED, "R must be < 2^30");
-  MOE_TRY(check_dim(N, "N"));
-  MOE_TRY(check_dim(K, "K"));
-  if ((int64_t)E * N >= (1ll << 31)) return fail(MOE_ERR_UNSUPPORTED, "E*N must be < 2^31");
-  if (gelu != 0 && gelu != 1) return fail(MOE_ERR_INVALID_ARG, "gelu must be 0 or 1");
+  MOE_TRY(check_gemm_shape(E, R, N, K, gelu));
   if (R == 0) return MOE_OK;
   MOE_TRY(check_ptr(A, "A"));
   MOE_TRY(check_ptr4(offsets, "offsets"));
@@ -294,10 +377,66 @@ moe_status moe_expert_gemm(const void* A, const int32_t* offsets, const void* W,
   std::string err;
   cudaError_t e = moe::launch_grouped_gemm(A, offsets, W, E, R, N, K, gelu != 0, out, *dev,
                                            as_stream(stream), &err);
-  if (e != cudaSuccess) {
-    if (!err.empty()) return fail(MOE_ERR_CUDA, "expert_gemm: " + err);
-    return cuda_fail(e, "expert_gemm");
+  if (e != cudaSuccess) return gemm_fail(e, err, "expert_gemm");
+  return MOE_OK;
+}
+
+moe_status moe_expert_gemm_fp8(const void* Aq, const float* a_scale, const int32_t* offsets,
+                               const void* Wq, const float* w_scale, int32_t E, int32_t R,
+                               int32_t N, int32_t K, int32_t gelu, void* out, void* stream) {
+  MOE_TRY(check_gemm_shape(E, R, N, K, gelu));
+  MOE_TRY(check_fp8_dim(K, "K"));
+  if (R == 0) return MOE_OK;
+  MOE_TRY(check_ptr(Aq, "Aq"));
+  MOE_TRY(check_ptr4(a_scale, "a_scale"));
+  MOE_TRY(check_ptr4(offsets, "offsets"));
+  MOE_TRY(check_ptr(Wq, "Wq"));
+  MOE_TRY(check_ptr4(w_scale, "w_scale"));
+  MOE_TRY(check_ptr(out, "out"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  std::string err;
+  cudaError_t e = moe::launch_grouped_gemm_fp8(Aq, a_scale, offsets, Wq, w_scale, E, R, N, K,
+                                               gelu != 0, out, *dev, as_stream(stream), &err);
+  if (e != cudaSuccess) return gemm_fail(e, err, "expert_gemm_fp8");
+  return MOE_OK;
+}
+
+moe_status moe_quantize_experts_fp8(const void* W, int32_t E, int32_t rows, int32_t cols,
+                                    void* Wq, float* scales, void* stream) {
+  if (E < 1 || rows < 0 || cols < 1) return fail(MOE_ERR_INVALID_ARG, "need E >= 1, rows >= 0, cols >= 1");
+  if (E > 65535) return fail(MOE_ERR_UNSUPPORTED, "E > 65535 is not supported");
+  MOE_TRY(check_fp8_dim(cols, "cols"));
+  MOE_TRY(check_ptr4(scales, "scales"));
+  const int64_t per = (int64_t)rows * cols;
+  if (per > 0) {
+    MOE_TRY(check_ptr(W, "W"));
+    MOE_TRY(check_ptr(Wq, "Wq"));
   }
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(moe::launch_quantize_experts(W, E, per, Wq, scales, *dev, as_stream(stream)),
+           "quantize_experts_fp8");
+  return MOE_OK;
+}
+
+moe_status moe_dispatch_fp8(const void* X, const int32_t* src_of, int32_t T, int32_t d,
+                            int32_t k, void* Xeq, float* x_scale, void* stream) {
+  if (T < 0 || k < 1) return fail(MOE_ERR_INVALID_ARG, "need T >= 0 and k >= 1");
+  if (k > moe::kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k > 16 is not supported");
+  if ((int64_t)T * k >= (1ll << 30)) return fail(MOE_ERR_UNSUPPORTED, "T*k must be < 2^30");
+  MOE_TRY(check_dim(d, "d"));
+  MOE_TRY(check_fp8_dim(d, "d"));
+  MOE_TRY(check_ptr4(x_scale, "x_scale"));
+  if (T > 0) {
+    MOE_TRY(check_ptr(X, "X"));
+    MOE_TRY(check_ptr4(src_of, "src_of"));
+    MOE_TRY(check_ptr(Xeq, "Xeq"));
+  }
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(moe::launch_dispatch_fp8(X, src_of, T, d, k, Xeq, x_scale, *dev, as_stream(stream)),
+           "dispatch_fp8");
   return MOE_OK;
 }
 
@@ -337,59 +476,29 @@ int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with
          2 + 1;
 }
 
+int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t with_router) {
+  if (check_desc(desc) != MOE_OK || desc->T == 0) return 0;
+  // the quantising dispatch adds the absmax kernel
+  return moe_kernel_launches_per_forward(desc, with_router) - 1 +
+         moe::fp8_dispatch_kernel_count(desc->T);
+}
+
 moe_status moe_layer_forward(const moe_layer_desc* desc, const void* X, const float* logits,
                              const void* Wr, const void* W1, const void* W2, void* Y,
                              int32_t* topk_idx_out, float* gates_out, int32_t* counts_out,
                              void* ws, size_t ws_bytes, void* stream) {
-  MOE_TRY(check_desc(desc));
-  const moe_layer_desc d = *desc;
-  if ((logits == nullptr) == (Wr == nullptr))
-    return fail(MOE_ERR_INVALID_ARG, "give exactly one of logits and Wr");
-  if (d.T == 0) return MOE_OK;
-  if ((int64_t)d.E * d.f >= (1ll << 31) || (int64_t)d.E * d.d >= (1ll << 31))
-    return fail(MOE_ERR_UNSUPPORTED, "E*f and E*d must be < 2^31");
-  MOE_TRY(check_ptr(X, "X"));
-  if (logits) MOE_TRY(check_ptr4(logits, "logits"));
-  if (Wr) MOE_TRY(check_ptr(Wr, "Wr"));
-  MOE_TRY(check_ptr(W1, "W1"));
-  MOE_TRY(check_ptr(W2, "W2"));
-  MOE_TRY(check_ptr(Y, "Y"));
-  if (topk_idx_out) MOE_TRY(check_ptr4(topk_idx_out, "topk_idx_out"));
-  if (gates_out) MOE_TRY(check_ptr4(gates_out, "gates_out"));
-  if (counts_out) MOE_TRY(check_ptr4(counts_out, "counts_out"));
-  const LayerWs w = layer_ws(d);
-  if (ws_bytes < w.total) return fail(MOE_ERR_INVALID_ARG, "workspace too small");
-  MOE_TRY(check_ptr(ws, "ws"));
-  const moe::DeviceInfo* dev;
-  MOE_TRY(get_dev(&dev));
-  cudaStream_t s = as_stream(stream);
-  char* base = static_cast<char*>(ws);
-  float* L = logits ? const_cast<float*>(logits) : reinterpret_cast<float*>(base + w.logits);
-  int32_t* idx = topk_idx_out ? topk_idx_out : reinterpret_cast<int32_t*>(base + w.idx);
-  float* gates = gates_out ? gates_out : reinterpret_cast<float*>(base + w.gates);
-  int32_t* counts = counts_out ? counts_out : reinterpret_cast<int32_t*>(base + w.counts);
-  int32_t* offsets = reinterpret_cast<int32_t*>(base + w.offsets);
-  int32_t* row_of = reinterpret_cast<int32_t*>(base + w.row_of);
-  int32_t* src_of = reinterpret_cast<int32_t*>(base + w.src_of);
-  void* lws = base + w.layout;
-  void* Xe = base + w.Xe;
-  void* H = base + w.H;
-  void* Ye = base + w.Ye;
-  const int R = d.T * d.k;
+  return layer_forward(desc, X, logits, Wr, W1, nullptr, W2, Y, topk_idx_out, gates_out,
+                       counts_out, ws, ws_bytes, stream);
+}
 
-  if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, s), "router_logits");
-  MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
-                             d.min_prob, idx, gates, s),
-           "route");
-  MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s), "layout");
-  MOE_CUDA(moe::launch_dispatch(X, src_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
-  std::string err;
-  cudaError_t e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err);
-  if (e != cudaSuccess) return err.empty() ? cuda_fail(e, "gemm1") : fail(MOE_ERR_CUDA, "gemm1: " + err);
-  e = moe::launch_grouped_gemm(H, offsets, W2, d.E, R, d.d, d.f, false, Ye, *dev, s, &err);
-  if (e != cudaSuccess) return err.empty() ? cuda_fail(e, "gemm2") : fail(MOE_ERR_CUDA, "gemm2: " + err);
-  MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
-  return MOE_OK;
+moe_status moe_layer_forward_fp8(const moe_layer_desc* desc, const void* X, const float* logits,
+                                 const void* Wr, const void* W1q, const float* w1_scale,
+                                 const void* W2, void* Y, int32_t* topk_idx_out,
+                                 float* gates_out, int32_t* counts_out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  if (!w1_scale) return fail(MOE_ERR_INVALID_ARG, "w1_scale is NULL");
+  return layer_forward(desc, X, logits, Wr, W1q, w1_scale, W2, Y, topk_idx_out, gates_out,
+                       counts_out, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -6,13 +6,21 @@
 //
 //   out[r, n] = act( sum_c A[r, c] * W[e, n, c] )   for r in expert e's block
 //
+// Operands are bf16, or E4M3 FP8 codes with per-tensor scales (ThunderEP PCIe
+// blog §3.3 and §5.2: activations cast to FP8 with a per-tensor dynamic scale;
+// FP8-capable tensor cores compute on them directly):
+//   out[r, n] = act( a_scale * w_scale[e] * sum_c Aq[r, c] * Wq[e, n, c] ).
+// A stage holds 128 bytes of K per row in both cases (64 bf16 or 128 E4M3
+// values), so the ring, the swizzle and the descriptors are shared; the FP8
+// form issues kind::f8f6f4 MMAs (K = 32) and scales in the epilogue.
+//
 // Design (one persistent CTA per SM, 11 warps):
 //   * Operand roles are swapped with respect to the usual token-major GEMM:
 //     128 weight rows (output features) form the MMA's M side, and up to 256
 //     token rows of one expert form its N side.  N is chosen per tile at run
 //     time (a multiple of 16), so a ragged expert block of c rows costs
 //     ceil(c/16)*16 columns of MMA work instead of a full 128-row tile.
-//   * warps 0 and 1 (one lane each) stream K-blocks of 64 of the weight and
+//   * warps 0 and 1 (one lane each) stream 128-byte K-blocks of the weight and
 //     the token operand through a ring of 6-7 stages (as many as shared
 //     memory holds) with TMA (128-byte swizzle),
 //     warp 2 (one lane) issues tcgen05.mma into one of two TMEM
@@ -40,7 +48,9 @@ namespace gg {
 constexpr int BM = 128;                      // weight rows per CTA (UMMA M per CTA)
 constexpr int BN = 256;                      // token rows per tile, at most (UMMA N)
 constexpr int BK = 64;                       // K per stage: one 128-byte swizzled bf16 row
-constexpr int UMMA_K = 16;                   // K per tcgen05.mma (kind::f16)
+constexpr int BK_FP8 = 128;                  // the same 128 bytes as E4M3 values
+constexpr int UMMA_K = 16;                   // K per tcgen05.mma (kind::f16); 32 for kind::f8f6f4
+constexpr int UMMA_K_BYTES = UMMA_K * 2;     // 32 bytes of a row per MMA in both kinds
 constexpr int A_STAGE = BM * BK * 2;         // 16 KB of weight rows per CTA and stage
 constexpr int B_BOX_ROWS = 32;
 constexpr int B_BOX = B_BOX_ROWS * BK * 2;   // 4 KB
@@ -92,9 +102,11 @@ struct Args {
   const int32_t* offsets;  // [E+1]
   uint16_t* out;           // [R, N] bf16
   uint32_t* status;
+  const float* a_scale;    // FP8 form: dequantisation scale of A (device scalar)
+  const float* w_scale;    // FP8 form: [E] dequantisation scales of W
   int E, R, N, K;
   int n_fblocks;           // ceil(N / features per tile)
-  int num_kb;              // ceil(K / BK)
+  int num_kb;              // ceil(K / K-values per stage)
   int stages;              // ring depth (<= MAX_STAGES)
 };
 
@@ -159,12 +171,13 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
-template <bool kGelu, int kPair>
+template <bool kGelu, int kPair, bool kFp8>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_xw, const Args args) {
   using C = Cfg<kPair>;
+  constexpr int KB = kFp8 ? BK_FP8 : BK;  // K values per stage (128 bytes of a row)
   const int STAGES = args.stages;
   constexpr int B_STAGE = C::B_STAGE;
   extern __shared__ uint8_t smem_raw[];
@@ -284,12 +297,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes);
           if (is_w) {
-            tma_load_2d_cg<kPair>(sA + s * A_STAGE, &tm_w, kb * BK, wy, fb_addr, pol);
+            tma_load_2d_cg<kPair>(sA + s * A_STAGE, &tm_w, kb * KB, wy, fb_addr, pol);
           } else if (wide) {  // (nearly) a full half-tile: one large request
-            tma_load_2d_cg<kPair>(sB + s * B_STAGE, &tm_xw, kb * BK, by, fb_addr, pol);
+            tma_load_2d_cg<kPair>(sB + s * B_STAGE, &tm_xw, kb * KB, by, fb_addr, pol);
           } else {
             for (int j = 0; j < nbox; ++j)
-              tma_load_2d_cg<kPair>(sB + s * B_STAGE + j * B_BOX, &tm_x, kb * BK,
+              tma_load_2d_cg<kPair>(sB + s * B_STAGE + j * B_BOX, &tm_x, kb * KB,
                                     by + j * B_BOX_ROWS, fb_addr, pol);
           }
         }
@@ -320,7 +333,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int tile = cid; ok && tile < total_tiles; tile += ncl, ++it) {
         const Tile t = decode(tile, s_start, s_lo, s_hi, E);
         const uint32_t nmma = (uint32_t)((t.ntok + 15) & ~15);
-        const uint32_t idesc = idesc_bf16_f32((uint32_t)C::FEAT, nmma);
+        const uint32_t idesc = kFp8 ? idesc_e4m3_f32((uint32_t)C::FEAT, nmma)
+                                    : idesc_bf16_f32((uint32_t)C::FEAT, nmma);
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)((it >> 1) & 1);
         ok = warp_wait(&tempty[acc], aph ^ 1u, args.status, s_abort);
@@ -335,10 +349,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t a0 = smem_u32(sA + s * A_STAGE);
             const uint32_t b0 = smem_u32(sB + s * B_STAGE);
 #pragma unroll
-            for (int kk = 0; kk < BK / UMMA_K; ++kk)
-              tc_mma_bf16<kPair>(d_tmem, smem_desc_k128(a0 + kk * UMMA_K * 2),
-                                 smem_desc_k128(b0 + kk * UMMA_K * 2), idesc,
-                                 (kb | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 128 / UMMA_K_BYTES; ++kk) {
+              const uint64_t ad = smem_desc_k128(a0 + kk * UMMA_K_BYTES);
+              const uint64_t bd = smem_desc_k128(b0 + kk * UMMA_K_BYTES);
+              if constexpr (kFp8)
+                tc_mma_e4m3<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              else
+                tc_mma_bf16<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            }
             // the stage is free (in both CTAs) once these MMAs have read it
             tc_commit<kPair>(smem_u32(&empty[s]));
             if (kPair == 2) tc_commit<kPair>(empty_peer + (uint32_t)s * 8u);
@@ -380,6 +398,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_after_sync();
       // this lane's output feature; the warp covers 32 consecutive features
       const int f = t.fb * C::FEAT + (int)rank * BM + q * 32 + lane;
+      const float sc = kFp8 ? __ldg(args.a_scale) * __ldg(args.w_scale + t.e) : 1.0f;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int c_end = min(t.ntok, hsel * SPAN + SPAN);
       for (int c0 = hsel * SPAN; c0 < c_end; c0 += 32) {
@@ -395,6 +414,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             float x = __uint_as_float(v[j]);
+            if (kFp8) x *= sc;
             if (kGelu) x = gelu_erf(x);
             if (j < jmax) col[(size_t)j * N] = to_bf16_bits(x);
           }
@@ -439,20 +459,22 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 2-D bf16 map over a row-major [rows, cols] matrix, box = box_rows x 64
-// columns, 128-byte swizzle (the layout the MMA descriptors expect).
+// 2-D map over a row-major [rows, cols] matrix of bf16 (fp8 = false) or
+// 1-byte E4M3 codes (fp8 = true); box = box_rows x 128 bytes of columns,
+// 128-byte swizzle (the layout the MMA descriptors expect).
 static bool make_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                     uint32_t box_rows, std::string* err) {
+                     uint32_t box_rows, bool fp8, std::string* err) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) {
     *err = "cuTensorMapEncodeTiled is unavailable from the driver";
     return false;
   }
   const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)gg::BK, box_rows};
+  const cuuint64_t strides[1] = {cols * (fp8 ? 1 : 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)(fp8 ? gg::BK_FP8 : gg::BK), box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -467,15 +489,15 @@ struct KernelSlot {
   cudaError_t err = cudaSuccess;
   int max_clusters = 0;  // co-resident clusters (pairs) or CTAs of this kernel
 };
-static KernelSlot g_slots[64][4];
+static KernelSlot g_slots[64][8];
 
-template <bool kGelu, int kPair>
+template <bool kGelu, int kPair, bool kFp8>
 static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                                   const CUtensorMap& tm_xw, const gg::Args& args, long long max_tiles, const DeviceInfo& dev,
                                   cudaStream_t stream) {
-  auto kern = gg::grouped_gemm_kernel<kGelu, kPair>;
+  auto kern = gg::grouped_gemm_kernel<kGelu, kPair, kFp8>;
   const size_t smem_max = gg::kSmemBudget;  // one attribute for every E
-  const int slot = (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0);
+  const int slot = (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0) + (kFp8 ? 4 : 0);
   KernelSlot& ks = g_slots[dev.device & 63][slot];
   std::call_once(ks.once, [&] {
     ks.err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
@@ -517,36 +539,56 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, tm_xw, args);
 }
 
-cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const void* W, int E,
-                                int R, int N, int K, bool gelu, void* out,
-                                const DeviceInfo& dev, cudaStream_t stream, std::string* err) {
+template <bool kFp8>
+static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_t* offsets,
+                               const void* W, const float* w_scale, int E, int R, int N, int K,
+                               bool gelu, void* out, const DeviceInfo& dev, cudaStream_t stream,
+                               std::string* err) {
   if (R == 0 || N == 0) return cudaSuccess;
   // Paired CTAs (256 features per tile) unless the layer is too narrow to fill them.
   const int pair = N > gg::BM ? 2 : 1;
   CUtensorMap tm_w, tm_x, tm_xw;
-  if (!make_map(&tm_w, W, (uint64_t)E * (uint64_t)N, (uint64_t)K, gg::BM, err) ||
-      !make_map(&tm_x, A, (uint64_t)R, (uint64_t)K, gg::B_BOX_ROWS, err) ||
-      !make_map(&tm_xw, A, (uint64_t)R, (uint64_t)K, gg::B_WIDE_ROWS, err))
+  if (!make_map(&tm_w, W, (uint64_t)E * (uint64_t)N, (uint64_t)K, gg::BM, kFp8, err) ||
+      !make_map(&tm_x, A, (uint64_t)R, (uint64_t)K, gg::B_BOX_ROWS, kFp8, err) ||
+      !make_map(&tm_xw, A, (uint64_t)R, (uint64_t)K, gg::B_WIDE_ROWS, kFp8, err))
     return cudaErrorInvalidValue;
   gg::Args args;
   args.offsets = offsets;
   args.out = static_cast<uint16_t*>(out);
   args.status = dev.status;
+  args.a_scale = a_scale;
+  args.w_scale = w_scale;
   args.E = E;
   args.R = R;
   args.N = N;
   args.K = K;
   args.n_fblocks = (N + gg::BM * pair - 1) / (gg::BM * pair);
-  args.num_kb = (K + gg::BK - 1) / gg::BK;
+  const int kb = kFp8 ? gg::BK_FP8 : gg::BK;
+  args.num_kb = (K + kb - 1) / kb;
   args.stages = pair == 2 ? gg::stages_for<2>(E) : gg::stages_for<1>(E);
   // an upper bound on the tile count: every expert adds at most one partial token block
   const long long max_tiles =
       ((long long)(R + gg::BN - 1) / gg::BN + E) * (long long)args.n_fblocks;
   if (pair == 2)
-    return gelu ? launch_variant<true, 2>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
-                : launch_variant<false, 2>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream);
-  return gelu ? launch_variant<true, 1>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
-              : launch_variant<false, 1>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream);
+    return gelu ? launch_variant<true, 2, kFp8>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
+                : launch_variant<false, 2, kFp8>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream);
+  return gelu ? launch_variant<true, 1, kFp8>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
+              : launch_variant<false, 1, kFp8>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream);
+}
+
+cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const void* W, int E,
+                                int R, int N, int K, bool gelu, void* out,
+                                const DeviceInfo& dev, cudaStream_t stream, std::string* err) {
+  return launch_gemm<false>(A, nullptr, offsets, W, nullptr, E, R, N, K, gelu, out, dev, stream,
+                            err);
+}
+
+cudaError_t launch_grouped_gemm_fp8(const void* Aq, const float* a_scale, const int32_t* offsets,
+                                    const void* Wq, const float* w_scale, int E, int R, int N,
+                                    int K, bool gelu, void* out, const DeviceInfo& dev,
+                                    cudaStream_t stream, std::string* err) {
+  return launch_gemm<true>(Aq, a_scale, offsets, Wq, w_scale, E, R, N, K, gelu, out, dev, stream,
+                           err);
 }
 
 }  // namespace moe

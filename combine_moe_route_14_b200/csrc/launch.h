@@ -51,6 +51,19 @@ cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const voi
                                 int R, int N, int K, bool gelu, void* out,
                                 const DeviceInfo& dev, cudaStream_t stream, std::string* err);
 
+// FP8 (E4M3) mode: grouped GEMM on codes with per-tensor scales, the
+// quantising dispatch (x_scale: [scale, amax]) and per-expert weight quantisation.
+cudaError_t launch_grouped_gemm_fp8(const void* Aq, const float* a_scale, const int32_t* offsets,
+                                    const void* Wq, const float* w_scale, int E, int R, int N,
+                                    int K, bool gelu, void* out, const DeviceInfo& dev,
+                                    cudaStream_t stream, std::string* err);
+cudaError_t launch_dispatch_fp8(const void* X, const int32_t* src_of, int T, int d, int k,
+                                void* Xeq, float* x_scale, const DeviceInfo& dev,
+                                cudaStream_t stream);
+int fp8_dispatch_kernel_count(int64_t T);
+cudaError_t launch_quantize_experts(const void* W, int E, int64_t per_expert, void* Wq,
+                                    float* scales, const DeviceInfo& dev, cudaStream_t stream);
+
 // Records `msg` as this thread's moe_last_error_string() and returns `status`.
 int set_last_error(int status, const std::string& msg);
 

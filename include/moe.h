@@ -243,6 +243,61 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const void* X, const fl
                              void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * FP8 mode (ThunderEP PCIe blog §3.3 "transport-side bit reduction" and §5.2:
+ * the activations a dispatch moves are cast to FP8 with one dynamic
+ * per-tensor scale before they move and cast back after, halving the bytes;
+ * FP8-capable tensor cores consume them directly).  Here: the dispatched
+ * token rows are E4M3 codes (1 byte per value) with one scale for all of X,
+ * and GEMM-1 runs on FP8 tensor cores against per-expert-quantised W1.
+ * GEMM-2 and combine stay bf16.
+ *
+ * Quantisation of a tensor x (identical wherever the library does it):
+ *   amax  = max |x|;  inv = 448 / amax  (fp32, round to nearest; 1 if amax = 0)
+ *   code  = E4M3(x * inv)  (fp32 product; round to nearest even; magnitudes
+ *           past 448 saturate to +-448; E4M3 = 1 sign, 4 exponent bits with
+ *           bias 7, 3 mantissa bits, no infinities)
+ *   scale = amax / 448     (fp32; 1 if amax = 0);  x ~= scale * code.
+ * Inputs must be finite.  FP8 calls need d % 16 == 0 and K % 16 == 0 (rows of
+ * codes are 16-byte aligned).
+ *
+ * moe_quantize_experts_fp8 -- per-expert quantisation of expert weights (done
+ *   once, when the weights are loaded; the pages leave weight quantisation
+ *   open, and one scale per expert matrix is the plainest choice).
+ *   W [E, rows, cols] bf16 -> Wq [E, rows, cols] E4M3 codes (uint8),
+ *   scales [E] fp32 (expert e's `scale`).  cols % 16 == 0.
+ *
+ * moe_dispatch_fp8 -- moe_dispatch writing E4M3 codes:
+ *   Xeq[r, :] = E4M3(X[src_of[r] / k, :] * inv), one scale over all of X [T, d].
+ *   x_scale: device float[2]; on return x_scale[0] = scale (what GEMM-1 reads),
+ *   x_scale[1] = amax.  Rows with src_of = -1 are left untouched.
+ *
+ * moe_expert_gemm_fp8 -- moe_expert_gemm on E4M3 operands:
+ *   out[r, n] = act( a_scale[0] * w_scale[e] * sum_c Aq[r, c] * Wq[e, n, c] ),
+ *   products exact, sums in fp32 on the tensor cores, the scaled result
+ *   rounded once to bf16.  Aq [R, K] uint8, a_scale device float[1],
+ *   Wq [E, N, K] uint8, w_scale [E] fp32, out [R, N] bf16.
+ *
+ * moe_layer_forward_fp8 -- moe_layer_forward with FP8 dispatch and FP8 GEMM-1:
+ *   W1q / w1_scale from moe_quantize_experts_fp8(W1); other arguments as in
+ *   moe_layer_forward; ws: at least moe_workspace_size(desc) bytes (the same
+ *   workspace serves both modes).
+ * moe_kernel_launches_per_forward_fp8 -- its kernel count (memsets excluded).
+ * ------------------------------------------------------------------------- */
+moe_status moe_quantize_experts_fp8(const void* W, int32_t E, int32_t rows, int32_t cols,
+                                    void* Wq, float* scales, void* stream);
+moe_status moe_dispatch_fp8(const void* X, const int32_t* src_of, int32_t T, int32_t d,
+                            int32_t k, void* Xeq, float* x_scale, void* stream);
+moe_status moe_expert_gemm_fp8(const void* Aq, const float* a_scale, const int32_t* offsets,
+                               const void* Wq, const float* w_scale, int32_t E, int32_t R,
+                               int32_t N, int32_t K, int32_t gelu, void* out, void* stream);
+moe_status moe_layer_forward_fp8(const moe_layer_desc* desc, const void* X, const float* logits,
+                                 const void* Wr, const void* W1q, const float* w1_scale,
+                                 const void* W2, void* Y, int32_t* topk_idx_out,
+                                 float* gates_out, int32_t* counts_out, void* ws,
+                                 size_t ws_bytes, void* stream);
+int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t with_router);
+
+/* ---------------------------------------------------------------------------
  * Diagnostics.
  *   moe_last_error_string: a description of the last failed call on this
  *   host thread ("" if none).  The pointer stays valid until the next call.

@@ -449,3 +449,35 @@ def layer_forward_fp8(X_bits, W1q, w1_scale, W2_bits, k, score=SOFTMAX, renormal
     Y = combine(Ye, row_of, gates, k)
     return dict(logits=L, topk_idx=idx, gates=gates, counts=counts, offsets=offsets,
                 row_of=row_of, src_of=src_of, Xq=Xq, x_scale=x_scale, Xe_q=Xe_q, H=H, Ye=Ye, Y=Y)
+
+
+def layer_forward_fp8_tokens(Xq, x_scale, W1q, w1_scale, W2_bits, topk_idx, gates, tokens):
+    """The FP8 layer's Y for a subset of tokens, each computed on its own
+    (the argument of layer_forward_tokens applies unchanged: a token's output
+    depends on its own quantised row and its k experts only).
+
+    Xq: the E4M3 codes of all of X (fp8_quantize over the whole tensor) or any
+    array whose rows `tokens` index; W1q[e] / w1_scale[e]: expert e's codes and
+    scale (only the routed experts are indexed).  Returns float64 [len(tokens), d].
+    """
+    tokens = np.asarray(tokens, dtype=np.int64)
+    k = topk_idx.shape[1]
+    xq = np.asarray(Xq)[tokens]
+    idx = np.asarray(topk_idx)[tokens]
+    g = np.asarray(gates, np.float64)[tokens]
+    d = xq.shape[1]
+    ye = np.zeros((len(tokens), k, d))
+    by_e = {}
+    for n in range(len(tokens)):
+        for j in range(k):
+            if idx[n, j] >= 0:
+                by_e.setdefault(int(idx[n, j]), []).append((n, j))
+    for e, pairs in sorted(by_e.items()):
+        ns = np.array([p[0] for p in pairs])
+        js = np.array([p[1] for p in pairs])
+        h = fp8_gemm1(xq[ns], x_scale, W1q[e], w1_scale[e])
+        ye[ns, js] = expert_gemm2(h, _as_f64(W2_bits[e]))
+    Y = np.zeros((len(tokens), d))
+    for j in range(k):
+        Y += g[:, j:j + 1] * ye[:, j]
+    return Y

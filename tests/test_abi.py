@@ -113,3 +113,26 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(moe, "_LIB_PATH", str(tmp_path / "libmoe.so"))
     with pytest.raises(moe.MoeError):
         moe.load_library()
+
+
+def test_fp8_calls_check_on_the_host(lib):
+    p = ctypes.c_void_p(0x10000)
+    # FP8 rows of codes must be 16-byte aligned: d, K, cols multiples of 16
+    assert lib.moe_dispatch_fp8(p, p, 4, 72, 2, p, p, N) == UNSUPPORTED
+    assert "multiple of 16" in _err(lib)
+    assert lib.moe_expert_gemm_fp8(p, p, p, p, p, 8, 16, 64, 40, 1, p, N) == UNSUPPORTED
+    assert lib.moe_quantize_experts_fp8(p, 8, 64, 24, p, p, N) == UNSUPPORTED
+    assert lib.moe_expert_gemm_fp8(p, N, p, p, p, 8, 16, 64, 64, 1, p, N) == INVALID  # no a_scale
+    assert lib.moe_quantize_experts_fp8(p, 0, 64, 64, p, p, N) == INVALID
+    d = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 0)
+    ws = lib.moe_workspace_size(ctypes.byref(d))
+    assert lib.moe_layer_forward_fp8(ctypes.byref(d), p, p, N, p, N, p, p, N, N, N, p, ws,
+                                     N) == INVALID                        # no w1_scale
+    assert lib.moe_layer_forward_fp8(ctypes.byref(d), p, p, N, p, p, p, p, N, N, N, p, ws - 1,
+                                     N) == INVALID                        # short workspace
+    d72 = moe.LayerDesc(64, 72, 8, 2, 128, 0, 1, 0)
+    ws72 = lib.moe_workspace_size(ctypes.byref(d72))
+    assert lib.moe_layer_forward_fp8(ctypes.byref(d72), p, p, N, p, p, p, p, N, N, N, p, ws72,
+                                     N) == UNSUPPORTED
+    # the quantising dispatch adds one kernel (the absmax reduction)
+    assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(d), 1) == 8

@@ -80,3 +80,20 @@ def _encode_ties_away(x):
 def test_planted_rounding_mistake_is_caught():
     with pytest.raises(AssertionError):
         assert _encode_ties_away(np.array([1.0 + 1 / 16]))[0] == 0x38
+
+
+def test_sampled_tokens_equal_the_whole_fp8_layer():
+    T, d, E, k, f = 40, 32, 4, 2, 48
+    X = I.f32_to_bf16_bits(I.random_f32((T, d), 7, "X").numpy())
+    W1 = I.f32_to_bf16_bits(I.random_f32((E, f, d), 7, "W1", 0.1).numpy())
+    W2 = I.f32_to_bf16_bits(I.random_f32((E, d, f), 7, "W2", 0.1).numpy())
+    L = I.random_f32((T, E), 7, "L").numpy()
+    W1q, s_w = O.fp8_quantize_experts(W1)
+    full = O.layer_forward_fp8(X, W1q, s_w, W2, k, logits=L)
+    toks = np.array([0, 3, 17, 39])
+    part = O.layer_forward_fp8_tokens(full["Xq"], full["x_scale"], W1q, s_w, W2,
+                                      full["topk_idx"], full["gates"], toks)
+    np.testing.assert_allclose(part, full["Y"][toks], rtol=1e-12, atol=1e-14)
+    # the dispatched rows are the token's codes, one per (token, slot)
+    ok = full["src_of"] >= 0
+    assert np.array_equal(full["Xe_q"][ok], full["Xq"][full["src_of"][ok] // k])

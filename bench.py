@@ -2,6 +2,7 @@
 """Benchmark: MoE-layer tokens/s on B200 (route -> layout -> dispatch -> expert FFN -> combine).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
+                    [--fp8]
 
 One step = one full layer forward (every stage) over one batch of T tokens.
 Default workload: the Mixtral-shaped layer (T=4096, d=4096, E=8, top-2,
@@ -10,7 +11,9 @@ inputs.  Multi-GPU runs are replicas (one process per GPU, each with its own
 token batch and a full copy of the weights, no data-path collective): weak
 scaling, value = all ranks' tokens / the slowest rank's time.
 
-Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+``--fp8`` runs the layer's FP8 mode (E4M3 dispatch with a per-tensor scale
+and FP8 GEMM-1; GEMM-2 and combine stay bf16); W1 is quantised once before
+timing.  Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 (the only reference this method has) on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -51,7 +54,7 @@ def log(*a):
 # ----------------------------------------------------------------------------
 # bookkeeping: algorithmic bytes / flops per stage
 # ----------------------------------------------------------------------------
-def stage_model(cfg, counts=None):
+def stage_model(cfg, counts=None, fp8=False):
     """Algorithmic work of each stage for one forward (bytes moved that the math needs)."""
     T, d, E, k, f, R = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.R
     E_act = E if counts is None else int((np.asarray(counts) > 0).sum())
@@ -64,6 +67,10 @@ def stage_model(cfg, counts=None):
     m["gemm1"] = {"flops": 2 * R * d * f, "bytes": E_act * f * d * 2 + R * d * 2 + R * f * 2}
     m["gemm2"] = {"flops": 2 * R * d * f, "bytes": E_act * d * f * 2 + R * f * 2 + R * d * 2}
     m["combine"] = {"bytes": R * d * 2 + R * 8 + T * d * 2}
+    if fp8:
+        # absmax pass over X, then the gather writes one byte per value
+        m["dispatch"] = {"bytes": 2 * T * d * 2 + R * d + R * 4}
+        m["gemm1"] = {"flops": 2 * R * d * f, "bytes": E_act * f * d + R * d + R * f * 2}
     return m
 
 
@@ -234,7 +241,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     logits = inp["logits"].to(dev) if inp["logits"] is not None else None
     Wr = inp["Wr"].to(dev) if inp["Wr"] is not None else None
     layer = moe.MoeLayer(inp["W1"], inp["W2"], cfg.k, cfg.score, cfg.renormalize, Wr=Wr,
-                         temperature=cfg.temperature, min_prob=cfg.min_prob)
+                         temperature=cfg.temperature, min_prob=cfg.min_prob, fp8=args.fp8)
     Y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
     counts = torch.empty((cfg.E,), dtype=torch.int32, device=dev)
     ws = layer.workspace(cfg.T)
@@ -283,7 +290,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         src_of = torch.empty((R,), dtype=torch.int32, device=dev)
         lws = torch.empty(max(16, moe.moe_layout_workspace_size(cfg.T, cfg.E, cfg.k)),
                           dtype=torch.uint8, device=dev)
-        Xe = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=dev)
+        Xe = torch.empty((R, cfg.d), dtype=torch.uint8 if args.fp8 else torch.bfloat16, device=dev)
+        xs = torch.empty((2,), dtype=torch.float32, device=dev)
         H = torch.empty((R, cfg.f), dtype=torch.bfloat16, device=dev)
         Ye = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=dev)
         fns = {
@@ -291,8 +299,11 @@ def run_ours(args, cfg, rank, world, local_rank):
             "route": lambda: moe.moe_route_ex(L_buf, cfg.k, cfg.score, cfg.renormalize,
                                               cfg.temperature, cfg.min_prob, idx, g),
             "layout": lambda: moe.moe_layout(idx, cfg.E, counts, offs, row_of, src_of, lws),
-            "dispatch": lambda: moe.moe_dispatch(X, src_of, cfg.k, Xe),
-            "gemm1": lambda: moe.moe_expert_gemm(Xe, offs, inp["W1"], True, H),
+            "dispatch": (lambda: moe.moe_dispatch_fp8(X, src_of, cfg.k, Xe, xs)) if args.fp8 else
+                        (lambda: moe.moe_dispatch(X, src_of, cfg.k, Xe)),
+            "gemm1": (lambda: moe.moe_expert_gemm_fp8(Xe, xs, offs, layer.W1q, layer.w1_scale,
+                                                      True, H)) if args.fp8 else
+                     (lambda: moe.moe_expert_gemm(Xe, offs, inp["W1"], True, H)),
             "gemm2": lambda: moe.moe_expert_gemm(H, offs, inp["W2"], False, Ye),
             "combine": lambda: moe.moe_combine(Ye, row_of, g, Y),
         }
@@ -352,7 +363,7 @@ def run_ours(args, cfg, rank, world, local_rank):
 
     # ---- roofline of the dominant kernel
     counts_h = counts.cpu().numpy()
-    model = stage_model(cfg, counts_h)
+    model = stage_model(cfg, counts_h, args.fp8)
     dom = max(stage_ms, key=lambda n: stage_ms[n])
     peaks, peak_src = load_peaks()
     clocks = sampler.summary() if sampler else None
@@ -362,20 +373,24 @@ def run_ours(args, cfg, rank, world, local_rank):
     sustained = capped or (t_ms + staged_total_ms * args.steps) > 1000.0
     per = model[dom]
     dur_s = stage_ms[dom] / 1e3
+    # an FP8 contraction's peak: the measured bf16 peak x the nominal fp8:bf16 ratio (2)
+    tc_ratio = 2.0 if (args.fp8 and dom == "gemm1") else 1.0
     if "flops" in per and per["flops"] / max(per["bytes"], 1) > (
-            peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9):
-        peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+            tc_ratio * peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9):
+        peak = tc_ratio * (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": per["flops"] / dur_s / 1e12, "peak": peak,
                 "unit": "TFLOP/s"}
-        roof["frac_vs_burst"] = roof["achieved"] / peaks["bf16_tflops"]
+        roof["frac_vs_burst"] = roof["achieved"] / (tc_ratio * peaks["bf16_tflops"])
     else:
         roof = {"bound": "hbm", "achieved": per["bytes"] / dur_s / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = dom
     roof["peak_source"] = (f"{peak_src} ("
-                           f"{'sustained: power cap active in the timed region' if sustained and roof['bound'] == 'tensor' else 'burst'})")
-    kname = {"gemm1": "grouped_gemm_gelu", "gemm2": "grouped_gemm"}.get(dom, dom)
+                           f"{'sustained: power cap active in the timed region' if sustained and roof['bound'] == 'tensor' else 'burst'})"
+                           + (" x 2 (fp8:bf16 nominal ratio)" if tc_ratio != 1.0 else ""))
+    kname = {"gemm1": "grouped_gemm_fp8_gelu" if args.fp8 else "grouped_gemm_gelu",
+             "gemm2": "grouped_gemm"}.get(dom, dom)
     tr = ncu_traffic(kname, cfg.name)
     roof["traffic"] = tr
     roof["algorithmic_bytes"] = per["bytes"]
@@ -394,14 +409,15 @@ def run_ours(args, cfg, rank, world, local_rank):
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3 (dispatch, GEMM-1) + bf16" if args.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                   "f": cfg.f, "router": cfg.router, "score": cfg.score,
+                   "f": cfg.f, "router": cfg.router, "score": cfg.score, "fp8": bool(args.fp8),
                    "renormalize": cfg.renormalize, "temperature": cfg.temperature,
                    "min_prob": cfg.min_prob, "tokens_per_gpu": cfg.T,
                    "parallelism": f"replicas x{world} (no collective)",
                    "l2": f"inputs larger than L2: each step streams "
-                         f"{2 * cfg.E * cfg.d * cfg.f * 2 / 1e9:.2f} GB of expert weights"},
+                         f"{(3 if args.fp8 else 4) * cfg.E * cfg.d * cfg.f / 1e9:.2f} GB of expert weights"},
         "roofline": roof,
         "stages": stages,
         "expert_counts": {"max": int(counts_h.max()), "mean": float(counts_h.mean()),
@@ -409,7 +425,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                           "dropped_slots": int(cfg.R - counts_h.sum())},
         "e2e": {"value": Rp.weak_scaling_throughput(cfg.T, args.steps, world, e2e_ms), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * moe.moe_kernel_launches_per_forward(
+        "gpu_launches": args.steps * (moe.moe_kernel_launches_per_forward_fp8 if args.fp8 else
+                                      moe.moe_kernel_launches_per_forward)(
             moe.make_desc(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.score, cfg.renormalize),
             Wr is not None),
         "clocks": clocks,
@@ -428,6 +445,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8", action="store_true",
+                    help="FP8 mode: E4M3 dispatch with a per-tensor scale and FP8 GEMM-1")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -468,7 +487,11 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     try:
         res = run_ours(args, cfg, rank, world, local_rank)
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if rank == 0 and args.fp8:
+            res["cpu_baseline"] = {"skipped": "FP8 mode: the oracle's E4M3 quantisation of W1 "
+                                              "takes ~10 s per expert; the bf16 line carries "
+                                              "the oracle baseline"}
+        elif rank == 0 and world == 1 and not args.no_cpu_baseline:
             S_base, _ = ORACLE_SAMPLE.get(cfg.name, (64, 16))
             h = host_inputs(cfg, args.seed)
             v, dt = time_oracle(cfg, h, S_base)

@@ -26,6 +26,7 @@ __all__ = [
     "moe_kernel_launches_per_forward", "MoeLayer", "SCORES",
     "moe_quantize_experts_fp8", "moe_dispatch_fp8", "moe_expert_gemm_fp8",
     "moe_layer_forward_fp8", "moe_kernel_launches_per_forward_fp8",
+    "moe_quantize_fp8", "moe_expert_gemm_gather", "moe_expert_gemm_gather_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -82,6 +83,10 @@ _SIG = {
     "moe_layer_forward_fp8": ([ctypes.POINTER(LayerDesc), _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_kernel_launches_per_forward_fp8": ([ctypes.POINTER(LayerDesc), _I], ctypes.c_int32),
+    "moe_quantize_fp8": ([_P, _I, _I, _P, _P, _P], ctypes.c_int),
+    "moe_expert_gemm_gather": ([_P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P], ctypes.c_int),
+    "moe_expert_gemm_gather_fp8": ([_P, _P, _P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P],
+                                   ctypes.c_int),
 }
 
 
@@ -389,6 +394,59 @@ def moe_expert_gemm_fp8(Aq, a_scale, offsets, Wq, w_scale, gelu, out=None, strea
     _check(lib.moe_expert_gemm_fp8(_ptr(Aq), _ptr(a_scale), _ptr(offsets), _ptr(Wq),
                                    _ptr(w_scale), E, R, N, K, int(bool(gelu)), _ptr(out),
                                    _stream(stream, dev)))
+    return out
+
+
+def moe_quantize_fp8(X, Xq=None, x_scale=None, stream=None):
+    """Per-tensor E4M3 quantisation of a bf16 matrix; returns (Xq uint8, x_scale [scale, amax])."""
+    lib = load_library()
+    rows, cols = X.shape
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (rows, cols))
+    Xq = _out(Xq, "Xq", torch.uint8, (rows, cols), dev)
+    x_scale = _out(x_scale, "x_scale", torch.float32, (2,), dev)
+    _check(lib.moe_quantize_fp8(_ptr(X), rows, cols, _ptr(Xq), _ptr(x_scale),
+                                _stream(stream, dev)))
+    return Xq, x_scale
+
+
+def moe_expert_gemm_gather(X, src_of, k, offsets, W, gelu, out=None, stream=None):
+    """Grouped GEMM whose row r reads token src_of[r] // k of X directly (no dispatched copy)."""
+    lib = load_library()
+    T, K = X.shape
+    E, N, K2 = W.shape
+    dev = X.device
+    if K2 != K:
+        raise ValueError("W's last dim must equal X's")
+    _need(X, "X", torch.bfloat16, (T, K))
+    _need(src_of, "src_of", torch.int32, (T * k,), dev)
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(W, "W", torch.bfloat16, (E, N, K), dev)
+    out = _out(out, "out", torch.bfloat16, (T * k, N), dev)
+    _check(lib.moe_expert_gemm_gather(_ptr(X), _ptr(src_of), T, k, _ptr(offsets), _ptr(W), E, N,
+                                      K, int(bool(gelu)), _ptr(out), _stream(stream, dev)))
+    return out
+
+
+def moe_expert_gemm_gather_fp8(Xq, x_scale, src_of, k, offsets, Wq, w_scale, gelu, out=None,
+                               stream=None):
+    lib = load_library()
+    T, K = Xq.shape
+    E, N, K2 = Wq.shape
+    dev = Xq.device
+    if K2 != K:
+        raise ValueError("Wq's last dim must equal Xq's")
+    _need(Xq, "Xq", torch.uint8, (T, K))
+    if x_scale.dtype != torch.float32 or x_scale.device != dev or x_scale.numel() < 1:
+        raise ValueError("x_scale must be a float32 device tensor")
+    _need(src_of, "src_of", torch.int32, (T * k,), dev)
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(Wq, "Wq", torch.uint8, (E, N, K), dev)
+    _need(w_scale, "w_scale", torch.float32, (E,), dev)
+    out = _out(out, "out", torch.bfloat16, (T * k, N), dev)
+    _check(lib.moe_expert_gemm_gather_fp8(_ptr(Xq), _ptr(x_scale), _ptr(src_of), T, k,
+                                          _ptr(offsets), _ptr(Wq), _ptr(w_scale), E, N, K,
+                                          int(bool(gelu)), _ptr(out), _stream(stream, dev)))
     return out
 
 

@@ -402,6 +402,68 @@ moe_status moe_expert_gemm_fp8(const void* Aq, const float* a_scale, const int32
   return MOE_OK;
 }
 
+moe_status moe_quantize_fp8(const void* X, int32_t rows, int32_t cols, void* Xq, float* x_scale,
+                            void* stream) {
+  if (rows < 0 || cols < 1) return fail(MOE_ERR_INVALID_ARG, "need rows >= 0 and cols >= 1");
+  MOE_TRY(check_fp8_dim(cols, "cols"));
+  MOE_TRY(check_ptr4(x_scale, "x_scale"));
+  const int64_t n = (int64_t)rows * cols;
+  if (n > 0) {
+    MOE_TRY(check_ptr(X, "X"));
+    MOE_TRY(check_ptr(Xq, "Xq"));
+  }
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(moe::launch_quantize_tensor(X, n, Xq, x_scale, *dev, as_stream(stream)), "quantize_fp8");
+  return MOE_OK;
+}
+
+namespace {
+moe_status gemm_gather(const void* X, const float* x_scale, const int32_t* src_of, int32_t T,
+                       int32_t k, const int32_t* offsets, const void* W, const float* w_scale,
+                       int32_t E, int32_t N, int32_t K, int32_t gelu, void* out, void* stream,
+                       bool fp8) {
+  if (T < 0 || k < 1) return fail(MOE_ERR_INVALID_ARG, "need T >= 0 and k >= 1");
+  if (k > moe::kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k > 16 is not supported");
+  if ((int64_t)T * k >= (1ll << 30)) return fail(MOE_ERR_UNSUPPORTED, "T*k must be < 2^30");
+  MOE_TRY(check_gemm_shape(E, T * k, N, K, gelu));
+  if (fp8) MOE_TRY(check_fp8_dim(K, "K"));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr(X, "X"));
+  MOE_TRY(check_ptr4(src_of, "src_of"));
+  MOE_TRY(check_ptr4(offsets, "offsets"));
+  MOE_TRY(check_ptr(W, "W"));
+  MOE_TRY(check_ptr(out, "out"));
+  if (fp8) {
+    MOE_TRY(check_ptr4(x_scale, "x_scale"));
+    MOE_TRY(check_ptr4(w_scale, "w_scale"));
+  }
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  std::string err;
+  cudaError_t e = moe::launch_grouped_gemm_gather(X, x_scale, src_of, T, k, offsets, W, w_scale,
+                                                  E, N, K, gelu != 0, fp8, out, *dev,
+                                                  as_stream(stream), &err);
+  if (e != cudaSuccess) return gemm_fail(e, err, fp8 ? "expert_gemm_gather_fp8" : "expert_gemm_gather");
+  return MOE_OK;
+}
+}  // namespace
+
+moe_status moe_expert_gemm_gather(const void* X, const int32_t* src_of, int32_t T, int32_t k,
+                                  const int32_t* offsets, const void* W, int32_t E, int32_t N,
+                                  int32_t K, int32_t gelu, void* out, void* stream) {
+  return gemm_gather(X, nullptr, src_of, T, k, offsets, W, nullptr, E, N, K, gelu, out, stream,
+                     false);
+}
+
+moe_status moe_expert_gemm_gather_fp8(const void* Xq, const float* x_scale, const int32_t* src_of,
+                                      int32_t T, int32_t k, const int32_t* offsets,
+                                      const void* Wq, const float* w_scale, int32_t E, int32_t N,
+                                      int32_t K, int32_t gelu, void* out, void* stream) {
+  return gemm_gather(Xq, x_scale, src_of, T, k, offsets, Wq, w_scale, E, N, K, gelu, out, stream,
+                     true);
+}
+
 moe_status moe_quantize_experts_fp8(const void* W, int32_t E, int32_t rows, int32_t cols,
                                     void* Wq, float* scales, void* stream) {
   if (E < 1 || rows < 0 || cols < 1) return fail(MOE_ERR_INVALID_ARG, "need E >= 1, rows >= 0, cols >= 1");

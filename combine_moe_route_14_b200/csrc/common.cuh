@@ -202,6 +202,32 @@ __device__ __forceinline__ void tma_load_2d_cg(void* smem_dst, const CUtensorMap
   }
 }
 
+// Four rows of a 2-D map (box = one row of 128 bytes) into four consecutive
+// 128-byte rows of shared memory: rows y0..y3 of the tensor at column x.
+// The 128-byte swizzle is applied by shared-memory address, as for tiled
+// loads, so four gathered rows can fill half of a 1024-byte swizzle atom.
+template <int kPair>
+__device__ __forceinline__ void tma_gather4_cg(void* smem_dst, const CUtensorMap* map, int32_t x,
+                                               int32_t y0, int32_t y1, int32_t y2, int32_t y3,
+                                               uint32_t mbar_cluster, uint64_t cache_hint) {
+  if constexpr (kPair == 2) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        ".cta_group::2.L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y0), "r"(y1),
+        "r"(y2), "r"(y3), "l"(cache_hint)
+        : "memory");
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%3, %4, %5, %6, %7}], [%2], %8;" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar_cluster), "r"(x), "r"(y0), "r"(y1),
+        "r"(y2), "r"(y3), "l"(cache_hint)
+        : "memory");
+  }
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory (TMEM) and the 5th-generation MMA.  kPair selects
 // cta_group::1 (one CTA) or cta_group::2 (a CTA pair; the allocation and the

@@ -14,6 +14,11 @@
 // values), so the ring, the swizzle and the descriptors are shared; the FP8
 // form issues kind::f8f6f4 MMAs (K = 32) and scales in the epilogue.
 //
+// Gather-on-load form (DySHARP review §3.2: dispatch fused into the expert
+// GEMM): A's rows are fetched straight from the token matrix through the
+// layout table, A[r] = X[src_of[r] / k], with TMA gather4 loads (four rows
+// per request), so no dispatched copy of the tokens is ever written.
+//
 // Design (one persistent CTA per SM, 11 warps):
 //   * Operand roles are swapped with respect to the usual token-major GEMM:
 //     128 weight rows (output features) form the MMA's M side, and up to 256
@@ -104,6 +109,9 @@ struct Args {
   uint32_t* status;
   const float* a_scale;    // FP8 form: dequantisation scale of A (device scalar)
   const float* w_scale;    // FP8 form: [E] dequantisation scales of W
+  const int32_t* gather_src;  // gather form: src_of [R]; A row r is token src_of[r] / gather_k
+  int gather_k;
+  int a_rows;              // gather form: rows of the token matrix (T)
   int E, R, N, K;
   int n_fblocks;           // ceil(N / features per tile)
   int num_kb;              // ceil(K / K-values per stage)
@@ -171,7 +179,7 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
-template <bool kGelu, int kPair, bool kFp8>
+template <bool kGelu, int kPair, bool kFp8, bool kGather>
 __global__ void __launch_bounds__(THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x,
@@ -290,10 +298,45 @@ __global__ void __launch_bounds__(THREADS, 1)
                                   : (uint32_t)kPair * (wide ? B_WIDE_ROWS * BK * 2 : nbox * B_BOX);
       const int wy = t.e * args.N + t.fb * C::FEAT + (int)rank * BM;
       const int by = t.row0 + (int)rank * half;
+      // gather form: request q (4 rows) of this CTA's half-tile is issued
+      // by lane q % 32 (up to 64 requests: 256 rows with a single CTA); the
+      // token ids are read once per tile.  Rows past the expert's block (the
+      // MMA's padding to a multiple of 16) read token 0 and are never stored.
+      const int nreq = half / 4;
+      int g[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+      if (kGather && !is_w) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int q = lane + 32 * h;
+          if (q >= nreq) continue;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int local = (int)rank * half + q * 4 + i;
+            int row = 0;
+            if (local < t.ntok) {
+              const int src = __ldg(args.gather_src + t.row0 + local);
+              if (src >= 0 && src < args.a_rows * args.gather_k) row = src / args.gather_k;
+              else flag_error(args.status, MOE_DEV_BAD_ROW);
+            }
+            g[h][i] = row;
+          }
+        }
+      }
+      const uint32_t gbytes = (uint32_t)(kPair * half * 128);
       for (int kb = 0; kb < args.num_kb; ++kb) {
         ok = warp_wait(&empty[s], ph ^ 1u, args.status, s_abort);
         if (!ok) break;
-        if (lane == 0) {
+        if (kGather && !is_w) {
+          const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
+          if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&full[s], gbytes);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int q = lane + 32 * h;
+            if (q < nreq)
+              tma_gather4_cg<kPair>(sB + s * B_STAGE + q * 512, &tm_x, kb * KB, g[h][0], g[h][1],
+                                    g[h][2], g[h][3], fb_addr, pol);
+          }
+        } else if (lane == 0) {
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes);
           if (is_w) {
@@ -489,15 +532,15 @@ struct KernelSlot {
   cudaError_t err = cudaSuccess;
   int max_clusters = 0;  // co-resident clusters (pairs) or CTAs of this kernel
 };
-static KernelSlot g_slots[64][8];
+static KernelSlot g_slots[64][16];
 
-template <bool kGelu, int kPair, bool kFp8>
+template <bool kGelu, int kPair, bool kFp8, bool kGather>
 static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                                   const CUtensorMap& tm_xw, const gg::Args& args, long long max_tiles, const DeviceInfo& dev,
                                   cudaStream_t stream) {
-  auto kern = gg::grouped_gemm_kernel<kGelu, kPair, kFp8>;
+  auto kern = gg::grouped_gemm_kernel<kGelu, kPair, kFp8, kGather>;
   const size_t smem_max = gg::kSmemBudget;  // one attribute for every E
-  const int slot = (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0) + (kFp8 ? 4 : 0);
+  const int slot = (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0) + (kFp8 ? 4 : 0) + (kGather ? 8 : 0);
   KernelSlot& ks = g_slots[dev.device & 63][slot];
   std::call_once(ks.once, [&] {
     ks.err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
@@ -539,25 +582,38 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, tm_xw, args);
 }
 
+// Gather form: A is the token matrix [a_rows, K] and row r of the GEMM reads
+// A[gather_src[r] / gather_k]; otherwise A is [R, K] and gather_src is null.
 template <bool kFp8>
-static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_t* offsets,
-                               const void* W, const float* w_scale, int E, int R, int N, int K,
-                               bool gelu, void* out, const DeviceInfo& dev, cudaStream_t stream,
+static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_t* gather_src,
+                               int gather_k, int a_rows, const int32_t* offsets, const void* W,
+                               const float* w_scale, int E, int R, int N, int K, bool gelu,
+                               void* out, const DeviceInfo& dev, cudaStream_t stream,
                                std::string* err) {
   if (R == 0 || N == 0) return cudaSuccess;
+  const bool gather = gather_src != nullptr;
   // Paired CTAs (256 features per tile) unless the layer is too narrow to fill them.
   const int pair = N > gg::BM ? 2 : 1;
   CUtensorMap tm_w, tm_x, tm_xw;
-  if (!make_map(&tm_w, W, (uint64_t)E * (uint64_t)N, (uint64_t)K, gg::BM, kFp8, err) ||
-      !make_map(&tm_x, A, (uint64_t)R, (uint64_t)K, gg::B_BOX_ROWS, kFp8, err) ||
-      !make_map(&tm_xw, A, (uint64_t)R, (uint64_t)K, gg::B_WIDE_ROWS, kFp8, err))
+  if (!make_map(&tm_w, W, (uint64_t)E * (uint64_t)N, (uint64_t)K, gg::BM, kFp8, err))
     return cudaErrorInvalidValue;
+  if (gather) {  // one-row boxes for gather4; the wide map is unused
+    if (!make_map(&tm_x, A, (uint64_t)a_rows, (uint64_t)K, 1, kFp8, err))
+      return cudaErrorInvalidValue;
+    tm_xw = tm_x;
+  } else if (!make_map(&tm_x, A, (uint64_t)R, (uint64_t)K, gg::B_BOX_ROWS, kFp8, err) ||
+             !make_map(&tm_xw, A, (uint64_t)R, (uint64_t)K, gg::B_WIDE_ROWS, kFp8, err)) {
+    return cudaErrorInvalidValue;
+  }
   gg::Args args;
   args.offsets = offsets;
   args.out = static_cast<uint16_t*>(out);
   args.status = dev.status;
   args.a_scale = a_scale;
   args.w_scale = w_scale;
+  args.gather_src = gather_src;
+  args.gather_k = gather_k;
+  args.a_rows = a_rows;
   args.E = E;
   args.R = R;
   args.N = N;
@@ -569,26 +625,43 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
   // an upper bound on the tile count: every expert adds at most one partial token block
   const long long max_tiles =
       ((long long)(R + gg::BN - 1) / gg::BN + E) * (long long)args.n_fblocks;
-  if (pair == 2)
-    return gelu ? launch_variant<true, 2, kFp8>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
-                : launch_variant<false, 2, kFp8>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream);
-  return gelu ? launch_variant<true, 1, kFp8>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
-              : launch_variant<false, 1, kFp8>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream);
+#define MOE_GG_LAUNCH(G, P, GA) \
+  launch_variant<G, P, kFp8, GA>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
+  if (gather) {
+    if (pair == 2) return gelu ? MOE_GG_LAUNCH(true, 2, true) : MOE_GG_LAUNCH(false, 2, true);
+    return gelu ? MOE_GG_LAUNCH(true, 1, true) : MOE_GG_LAUNCH(false, 1, true);
+  }
+  if (pair == 2) return gelu ? MOE_GG_LAUNCH(true, 2, false) : MOE_GG_LAUNCH(false, 2, false);
+  return gelu ? MOE_GG_LAUNCH(true, 1, false) : MOE_GG_LAUNCH(false, 1, false);
+#undef MOE_GG_LAUNCH
 }
 
 cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const void* W, int E,
                                 int R, int N, int K, bool gelu, void* out,
                                 const DeviceInfo& dev, cudaStream_t stream, std::string* err) {
-  return launch_gemm<false>(A, nullptr, offsets, W, nullptr, E, R, N, K, gelu, out, dev, stream,
-                            err);
+  return launch_gemm<false>(A, nullptr, nullptr, 1, R, offsets, W, nullptr, E, R, N, K, gelu,
+                            out, dev, stream, err);
 }
 
 cudaError_t launch_grouped_gemm_fp8(const void* Aq, const float* a_scale, const int32_t* offsets,
                                     const void* Wq, const float* w_scale, int E, int R, int N,
                                     int K, bool gelu, void* out, const DeviceInfo& dev,
                                     cudaStream_t stream, std::string* err) {
-  return launch_gemm<true>(Aq, a_scale, offsets, Wq, w_scale, E, R, N, K, gelu, out, dev, stream,
-                           err);
+  return launch_gemm<true>(Aq, a_scale, nullptr, 1, R, offsets, Wq, w_scale, E, R, N, K, gelu,
+                           out, dev, stream, err);
+}
+
+cudaError_t launch_grouped_gemm_gather(const void* X, const float* x_scale, const int32_t* src_of,
+                                       int T, int k, const int32_t* offsets, const void* W,
+                                       const float* w_scale, int E, int N, int K, bool gelu,
+                                       bool fp8, void* out, const DeviceInfo& dev,
+                                       cudaStream_t stream, std::string* err) {
+  const int R = T * k;
+  if (fp8)
+    return launch_gemm<true>(X, x_scale, src_of, k, T, offsets, W, w_scale, E, R, N, K, gelu, out,
+                             dev, stream, err);
+  return launch_gemm<false>(X, nullptr, src_of, k, T, offsets, W, nullptr, E, R, N, K, gelu, out,
+                            dev, stream, err);
 }
 
 }  // namespace moe

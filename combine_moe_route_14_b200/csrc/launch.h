@@ -57,6 +57,16 @@ cudaError_t launch_grouped_gemm_fp8(const void* Aq, const float* a_scale, const 
                                     const void* Wq, const float* w_scale, int E, int R, int N,
                                     int K, bool gelu, void* out, const DeviceInfo& dev,
                                     cudaStream_t stream, std::string* err);
+// Gather-on-load grouped GEMM: row r of the GEMM reads X[src_of[r] / k]
+// (X: [T, K] bf16, or E4M3 codes with scale x_scale[0] when fp8).
+cudaError_t launch_grouped_gemm_gather(const void* X, const float* x_scale, const int32_t* src_of,
+                                       int T, int k, const int32_t* offsets, const void* W,
+                                       const float* w_scale, int E, int N, int K, bool gelu,
+                                       bool fp8, void* out, const DeviceInfo& dev,
+                                       cudaStream_t stream, std::string* err);
+// Per-tensor E4M3 quantisation of n bf16 values (n % 8 == 0): x_scale = [scale, amax].
+cudaError_t launch_quantize_tensor(const void* X, int64_t n, void* Xq, float* x_scale,
+                                   const DeviceInfo& dev, cudaStream_t stream);
 cudaError_t launch_dispatch_fp8(const void* X, const int32_t* src_of, int T, int d, int k,
                                 void* Xeq, float* x_scale, const DeviceInfo& dev,
                                 cudaStream_t stream);

@@ -87,11 +87,14 @@ __global__ void __launch_bounds__(kQThreads)
   }
 }
 
-// Wq[g] = E4M3(W[g] * inv(amax[g])) for each group g = blockIdx.y.
+// Wq[g] = E4M3(W[g] * inv(amax[g])) for each group g = blockIdx.y; when
+// scale_out is given (not aliasing amax), CTA (0, g) writes its scale there.
 __global__ void __launch_bounds__(kQThreads)
     quantize_kernel(const uint4* __restrict__ W, size_t vecs, const float* __restrict__ amax,
-                    uint2* __restrict__ Wq) {
+                    uint2* __restrict__ Wq, float* scale_out) {
   const float inv = inv_scale_of(amax[blockIdx.y]);
+  if (scale_out && blockIdx.x == 0 && threadIdx.x == 0)
+    scale_out[blockIdx.y] = scale_of(amax[blockIdx.y]);
   const uint4* p = W + (size_t)blockIdx.y * vecs;
   uint2* q = Wq + (size_t)blockIdx.y * vecs;
   const size_t stride = (size_t)gridDim.x * kQThreads;
@@ -175,10 +178,21 @@ cudaError_t launch_quantize_experts(const void* W, int E, int64_t per_expert, vo
   if (e != cudaSuccess) return e;
   if (vecs > 0) {
     quantize_kernel<<<dim3(stream_grid(vecs, E, dev), E), kQThreads, 0, stream>>>(
-        static_cast<const uint4*>(W), vecs, scales, static_cast<uint2*>(Wq));
+        static_cast<const uint4*>(W), vecs, scales, static_cast<uint2*>(Wq), nullptr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   scale_finalize_kernel<<<(E + 255) / 256, 256, 0, stream>>>(scales, E);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_tensor(const void* X, int64_t n, void* Xq, float* x_scale,
+                                   const DeviceInfo& dev, cudaStream_t stream) {
+  const size_t vecs = (size_t)n / 8;
+  cudaError_t e = launch_amax(X, vecs, 1, x_scale + 1, dev, stream);
+  if (e != cudaSuccess) return e;
+  // n == 0 still runs one CTA so that x_scale[0] is written
+  quantize_kernel<<<stream_grid(vecs, 1, dev), kQThreads, 0, stream>>>(
+      static_cast<const uint4*>(X), vecs, x_scale + 1, static_cast<uint2*>(Xq), x_scale);
   return cudaGetLastError();
 }
 

@@ -297,6 +297,38 @@ moe_status moe_layer_forward_fp8(const moe_layer_desc* desc, const void* X, cons
                                  size_t ws_bytes, void* stream);
 int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t with_router);
 
+/* moe_quantize_fp8 -- per-tensor E4M3 quantisation of a bf16 matrix by the
+ *   rule above: X [rows, cols] bf16 -> Xq [rows, cols] codes, x_scale device
+ *   float[2] = {scale, amax}.  cols % 16 == 0.  Feeds the gather-on-load
+ *   FP8 GEMM below (the tokens are quantised once, not once per expert slot). */
+moe_status moe_quantize_fp8(const void* X, int32_t rows, int32_t cols, void* Xq, float* x_scale,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Gather-on-load expert GEMM (DySHARP review §3.2: dispatch fused into the
+ * expert GEMM, so the dispatched copy of the tokens is never written).
+ *   moe_expert_gemm_gather: for each expert e and row r in
+ *     [offsets[e], offsets[e+1]):
+ *       out[r, n] = act( sum_c X[src_of[r] / k, c] * W[e, n, c] ),
+ *     i.e. moe_expert_gemm applied to the rows moe_dispatch would produce.
+ *     X [T, K] bf16, src_of [T*k] int32 (from moe_layout), offsets [E+1],
+ *     W [E, N, K] bf16, out [T*k, N] bf16.  Rows at or past offsets[E] are not
+ *     written.  A src_of entry inside an expert block outside [0, T*k) sets
+ *     MOE_DEV_BAD_ROW and reads token 0.
+ *   moe_expert_gemm_gather_fp8: the same on E4M3 codes (moe_quantize_fp8 of
+ *     X, moe_quantize_experts_fp8 of W):
+ *       out[r, n] = act( x_scale[0] * w_scale[e] *
+ *                        sum_c Xq[src_of[r] / k, c] * Wq[e, n, c] ).
+ *     K % 16 == 0.
+ * ------------------------------------------------------------------------- */
+moe_status moe_expert_gemm_gather(const void* X, const int32_t* src_of, int32_t T, int32_t k,
+                                  const int32_t* offsets, const void* W, int32_t E, int32_t N,
+                                  int32_t K, int32_t gelu, void* out, void* stream);
+moe_status moe_expert_gemm_gather_fp8(const void* Xq, const float* x_scale, const int32_t* src_of,
+                                      int32_t T, int32_t k, const int32_t* offsets,
+                                      const void* Wq, const float* w_scale, int32_t E, int32_t N,
+                                      int32_t K, int32_t gelu, void* out, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Diagnostics.
  *   moe_last_error_string: a description of the last failed call on this

@@ -2,7 +2,7 @@
 """Benchmark: MoE-layer tokens/s on B200 (route -> layout -> dispatch -> expert FFN -> combine).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
-                    [--fp8]
+                    [--fp8] [--gather]
 
 One step = one full layer forward (every stage) over one batch of T tokens.
 Default workload: the Mixtral-shaped layer (T=4096, d=4096, E=8, top-2,
@@ -13,7 +13,9 @@ scaling, value = all ranks' tokens / the slowest rank's time.
 
 ``--fp8`` runs the layer's FP8 mode (E4M3 dispatch with a per-tensor scale
 and FP8 GEMM-1; GEMM-2 and combine stay bf16); W1 is quantised once before
-timing.  Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+timing.  ``--gather`` fuses the dispatch into GEMM-1 (rows read through the
+layout table with TMA gather4 loads; no dispatch kernel).  Prints one JSON
+line (rank 0).  ``--impl reference`` times the CPU oracle
 (the only reference this method has) on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -54,7 +56,7 @@ def log(*a):
 # ----------------------------------------------------------------------------
 # bookkeeping: algorithmic bytes / flops per stage
 # ----------------------------------------------------------------------------
-def stage_model(cfg, counts=None, fp8=False):
+def stage_model(cfg, counts=None, fp8=False):  # gather form: same algorithmic bytes per stage
     """Algorithmic work of each stage for one forward (bytes moved that the math needs)."""
     T, d, E, k, f, R = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.R
     E_act = E if counts is None else int((np.asarray(counts) > 0).sum())
@@ -71,6 +73,7 @@ def stage_model(cfg, counts=None, fp8=False):
         # absmax pass over X, then the gather writes one byte per value
         m["dispatch"] = {"bytes": 2 * T * d * 2 + R * d + R * 4}
         m["gemm1"] = {"flops": 2 * R * d * f, "bytes": E_act * f * d + R * d + R * f * 2}
+        m["quantize"] = {"bytes": 2 * T * d * 2 + T * d}
     return m
 
 
@@ -241,7 +244,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     logits = inp["logits"].to(dev) if inp["logits"] is not None else None
     Wr = inp["Wr"].to(dev) if inp["Wr"] is not None else None
     layer = moe.MoeLayer(inp["W1"], inp["W2"], cfg.k, cfg.score, cfg.renormalize, Wr=Wr,
-                         temperature=cfg.temperature, min_prob=cfg.min_prob, fp8=args.fp8)
+                         temperature=cfg.temperature, min_prob=cfg.min_prob, fp8=args.fp8,
+                         gather_on_load=args.gather)
     Y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
     counts = torch.empty((cfg.E,), dtype=torch.int32, device=dev)
     ws = layer.workspace(cfg.T)
@@ -280,7 +284,9 @@ def run_ours(args, cfg, rank, world, local_rank):
 
         # ---- per-stage times: the same kernels, launched stage by stage with events between
         stage_names = (["router_logits"] if Wr is not None else []) + [
-            "route", "layout", "dispatch", "gemm1", "gemm2", "combine"]
+            "route", "layout"] + (["quantize"] if args.gather and args.fp8 else
+                                  [] if args.gather else ["dispatch"]) + [
+            "gemm1", "gemm2", "combine"]
         R = cfg.R
         L_buf = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev) if Wr is not None else logits
         idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
@@ -291,6 +297,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         lws = torch.empty(max(16, moe.moe_layout_workspace_size(cfg.T, cfg.E, cfg.k)),
                           dtype=torch.uint8, device=dev)
         Xe = torch.empty((R, cfg.d), dtype=torch.uint8 if args.fp8 else torch.bfloat16, device=dev)
+        Xq = torch.empty((cfg.T, cfg.d), dtype=torch.uint8, device=dev)
         xs = torch.empty((2,), dtype=torch.float32, device=dev)
         H = torch.empty((R, cfg.f), dtype=torch.bfloat16, device=dev)
         Ye = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=dev)
@@ -301,9 +308,15 @@ def run_ours(args, cfg, rank, world, local_rank):
             "layout": lambda: moe.moe_layout(idx, cfg.E, counts, offs, row_of, src_of, lws),
             "dispatch": (lambda: moe.moe_dispatch_fp8(X, src_of, cfg.k, Xe, xs)) if args.fp8 else
                         (lambda: moe.moe_dispatch(X, src_of, cfg.k, Xe)),
-            "gemm1": (lambda: moe.moe_expert_gemm_fp8(Xe, xs, offs, layer.W1q, layer.w1_scale,
-                                                      True, H)) if args.fp8 else
-                     (lambda: moe.moe_expert_gemm(Xe, offs, inp["W1"], True, H)),
+            "quantize": lambda: moe.moe_quantize_fp8(X, Xq, xs),
+            "gemm1": ((lambda: moe.moe_expert_gemm_gather_fp8(Xq, xs, src_of, cfg.k, offs,
+                                                              layer.W1q, layer.w1_scale, True, H))
+                      if args.gather else
+                      (lambda: moe.moe_expert_gemm_fp8(Xe, xs, offs, layer.W1q, layer.w1_scale,
+                                                       True, H))) if args.fp8 else
+                     ((lambda: moe.moe_expert_gemm_gather(X, src_of, cfg.k, offs, inp["W1"], True,
+                                                          H)) if args.gather else
+                      (lambda: moe.moe_expert_gemm(Xe, offs, inp["W1"], True, H))),
             "gemm2": lambda: moe.moe_expert_gemm(H, offs, inp["W2"], False, Ye),
             "combine": lambda: moe.moe_combine(Ye, row_of, g, Y),
         }
@@ -389,7 +402,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     roof["peak_source"] = (f"{peak_src} ("
                            f"{'sustained: power cap active in the timed region' if sustained and roof['bound'] == 'tensor' else 'burst'})"
                            + (" x 2 (fp8:bf16 nominal ratio)" if tc_ratio != 1.0 else ""))
-    kname = {"gemm1": "grouped_gemm_fp8_gelu" if args.fp8 else "grouped_gemm_gelu",
+    kname = {"gemm1": ("grouped_gemm_fp8_gelu" if args.fp8 else "grouped_gemm_gelu")
+                      + ("_gather" if args.gather else ""),
              "gemm2": "grouped_gemm"}.get(dom, dom)
     tr = ncu_traffic(kname, cfg.name)
     roof["traffic"] = tr
@@ -413,6 +427,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "dtype": "e4m3 (dispatch, GEMM-1) + bf16" if args.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
                    "f": cfg.f, "router": cfg.router, "score": cfg.score, "fp8": bool(args.fp8),
+                   "gather_on_load": bool(args.gather),
                    "renormalize": cfg.renormalize, "temperature": cfg.temperature,
                    "min_prob": cfg.min_prob, "tokens_per_gpu": cfg.T,
                    "parallelism": f"replicas x{world} (no collective)",
@@ -427,7 +442,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (moe.moe_kernel_launches_per_forward_fp8 if args.fp8 else
                                       moe.moe_kernel_launches_per_forward)(
-            moe.make_desc(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.score, cfg.renormalize),
+            moe.make_desc(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.score, cfg.renormalize,
+                          gather_on_load=args.gather),
             Wr is not None),
         "clocks": clocks,
     }
@@ -447,6 +463,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fp8", action="store_true",
                     help="FP8 mode: E4M3 dispatch with a per-tensor scale and FP8 GEMM-1")
+    ap.add_argument("--gather", action="store_true",
+                    help="fuse the dispatch into GEMM-1 (gather-on-load)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -35,6 +35,7 @@ _lib = None
 _lock = threading.Lock()
 
 SCORES = {"softmax": 0, "sigmoid": 1}
+LAYER_GATHER_ON_LOAD = 0x1  # moe_layer_desc.flags: dispatch fused into GEMM-1
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
           4: "MOE_ERR_DEVICE"}
 DEV_BITS = {1: "MOE_DEV_BAD_EXPERT_ID", 2: "MOE_DEV_TIMEOUT", 4: "MOE_DEV_BAD_ROW"}
@@ -49,7 +50,7 @@ class MoeError(RuntimeError):
 class LayerDesc(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("E", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("f", ctypes.c_int32), ("score", ctypes.c_int32),
-                ("renormalize", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("renormalize", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("temperature", ctypes.c_float), ("min_prob", ctypes.c_float)]
 
 
@@ -302,8 +303,9 @@ def moe_combine(Ye, row_of, gates, Y=None, stream=None):
 # whole layer
 # ----------------------------------------------------------------------------
 def make_desc(T, d, E, k, f, score="softmax", renormalize=True, temperature=1.0,
-              min_prob=0.0) -> LayerDesc:
-    return LayerDesc(T, d, E, k, f, _score(score), int(bool(renormalize)), 0, float(temperature),
+              min_prob=0.0, gather_on_load=False) -> LayerDesc:
+    return LayerDesc(T, d, E, k, f, _score(score), int(bool(renormalize)),
+                     LAYER_GATHER_ON_LOAD if gather_on_load else 0, float(temperature),
                      float(min_prob))
 
 
@@ -318,7 +320,7 @@ def moe_kernel_launches_per_forward(desc: LayerDesc, with_router: bool) -> int:
 
 def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=None, Wr=None,
                       Y=None, topk_idx_out=None, gates_out=None, counts_out=None, ws=None,
-                      stream=None, temperature=1.0, min_prob=0.0):
+                      stream=None, temperature=1.0, min_prob=0.0, gather_on_load=False):
     lib = load_library()
     T, d = X.shape
     E, f, _ = W1.shape
@@ -337,7 +339,7 @@ def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=No
         _need(gates_out, "gates_out", torch.float32, (T, k), dev)
     if counts_out is not None:
         _need(counts_out, "counts_out", torch.int32, (E,), dev)
-    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob)
+    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, gather_on_load)
     if ws is None:
         ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
     _need(ws, "ws", torch.uint8, None, dev)
@@ -457,7 +459,8 @@ def moe_kernel_launches_per_forward_fp8(desc: LayerDesc, with_router: bool) -> i
 
 def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=True,
                           logits=None, Wr=None, Y=None, topk_idx_out=None, gates_out=None,
-                          counts_out=None, ws=None, stream=None, temperature=1.0, min_prob=0.0):
+                          counts_out=None, ws=None, stream=None, temperature=1.0, min_prob=0.0,
+                          gather_on_load=False):
     """The layer with FP8 dispatch and FP8 GEMM-1 (W1q, w1_scale from moe_quantize_experts_fp8)."""
     lib = load_library()
     T, d = X.shape
@@ -478,7 +481,7 @@ def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=
         _need(gates_out, "gates_out", torch.float32, (T, k), dev)
     if counts_out is not None:
         _need(counts_out, "counts_out", torch.int32, (E,), dev)
-    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob)
+    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, gather_on_load)
     if ws is None:
         ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
     _need(ws, "ws", torch.uint8, None, dev)
@@ -503,9 +506,10 @@ class MoeLayer:
     """A layer's weights plus a reusable workspace (allocation stays outside the call)."""
 
     def __init__(self, W1, W2, k, score="softmax", renormalize=True, Wr=None, temperature=1.0,
-                 min_prob=0.0, fp8=False):
+                 min_prob=0.0, fp8=False, gather_on_load=False):
         self.W1, self.W2, self.Wr = W1, W2, Wr
         self.fp8 = bool(fp8)
+        self.gather_on_load = bool(gather_on_load)
         # FP8 mode keeps W1 as E4M3 codes with per-expert scales (quantised once here)
         self.W1q, self.w1_scale = moe_quantize_experts_fp8(W1) if self.fp8 else (None, None)
         self.k, self.score, self.renormalize = k, score, renormalize
@@ -525,7 +529,7 @@ class MoeLayer:
         kw = dict(logits=logits, Wr=None if logits is not None else self.Wr, Y=Y,
                   topk_idx_out=topk_idx_out, gates_out=gates_out, counts_out=counts_out,
                   ws=self.workspace(X.shape[0]), stream=stream, temperature=self.temperature,
-                  min_prob=self.min_prob)
+                  min_prob=self.min_prob, gather_on_load=self.gather_on_load)
         if self.fp8:
             return moe_layer_forward_fp8(X, self.W1q, self.w1_scale, self.W2, self.k, self.score,
                                          self.renormalize, **kw)

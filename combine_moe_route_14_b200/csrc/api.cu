@@ -161,7 +161,7 @@ moe_status check_desc(const moe_layer_desc* desc) {
     return fail(MOE_ERR_INVALID_ARG, "unknown score");
   if (desc->renormalize != 0 && desc->renormalize != 1)
     return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
-  if (desc->reserved != 0) return fail(MOE_ERR_INVALID_ARG, "reserved must be 0");
+  if (desc->flags & ~MOE_LAYER_GATHER_ON_LOAD) return fail(MOE_ERR_INVALID_ARG, "unknown flags");
   if (!std::isfinite(desc->temperature) || desc->temperature < 0.f)
     return fail(MOE_ERR_INVALID_ARG, "temperature must be >= 0 (0 reads as 1)");
   if (!std::isfinite(desc->min_prob)) return fail(MOE_ERR_INVALID_ARG, "min_prob must be finite");
@@ -232,7 +232,17 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s), "layout");
   std::string err;
   cudaError_t e;
-  if (fp8) {
+  const bool gather = (d.flags & MOE_LAYER_GATHER_ON_LOAD) != 0;
+  if (gather) {  // dispatch fused into GEMM-1: its rows are read through src_of
+    const void* A = X;
+    if (fp8) {   // the tokens are quantised once (T rows), into the Xe slot
+      MOE_CUDA(moe::launch_quantize_tensor(X, (int64_t)d.T * d.d, Xe, x_scale, *dev, s),
+               "quantize_fp8");
+      A = Xe;
+    }
+    e = moe::launch_grouped_gemm_gather(A, x_scale, src_of, d.T, d.k, offsets, W1, W1s, d.E, d.f,
+                                        d.d, true, fp8, H, *dev, s, &err);
+  } else if (fp8) {
     MOE_CUDA(moe::launch_dispatch_fp8(X, src_of, d.T, d.d, d.k, Xe, x_scale, *dev, s), "dispatch_fp8");
     e = moe::launch_grouped_gemm_fp8(Xe, x_scale, offsets, W1, W1s, d.E, R, d.f, d.d, true, H,
                                      *dev, s, &err);
@@ -533,15 +543,18 @@ size_t moe_workspace_size(const moe_layer_desc* desc) {
 
 int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with_router) {
   if (check_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  // [router linear] + route + layout + dispatch + 2 GEMMs + combine
-  return (with_router ? 1 : 0) + 1 + moe::layout_kernel_count((int64_t)desc->T * desc->k) + 1 +
-         2 + 1;
+  // [router linear] + route + layout + [dispatch] + 2 GEMMs + combine
+  const int dispatch = (desc->flags & MOE_LAYER_GATHER_ON_LOAD) ? 0 : 1;
+  return (with_router ? 1 : 0) + 1 + moe::layout_kernel_count((int64_t)desc->T * desc->k) +
+         dispatch + 2 + 1;
 }
 
 int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t with_router) {
   if (check_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  // the quantising dispatch adds the absmax kernel
-  return moe_kernel_launches_per_forward(desc, with_router) - 1 +
+  // the quantising dispatch (or, gathering, the quantisation of X) is the
+  // absmax kernel plus one
+  const int dispatch = (desc->flags & MOE_LAYER_GATHER_ON_LOAD) ? 0 : 1;
+  return moe_kernel_launches_per_forward(desc, with_router) - dispatch +
          moe::fp8_dispatch_kernel_count(desc->T);
 }
 

@@ -67,8 +67,20 @@ constexpr int B_BOX = B_BOX_ROWS * BK * 2;   // 4 KB
 constexpr int B_WIDE_ROWS = 128;
 constexpr int kWideMin = 96;
 constexpr int EPI_WARPS = 8;                 // two per SM sub-partition
-constexpr int EPI_WARP0 = 3;                 // warps 0-1 load, warp 2 issues MMAs
-constexpr int THREADS = (EPI_WARP0 + EPI_WARPS) * 32;
+#ifndef MOE_GATHER_WARPS
+#define MOE_GATHER_WARPS 8
+#endif
+// Gather form: gather4 requests are issued one lane at a time, about one per
+// ~90 cycles per issuing warp, so the token rows are fetched by several warps.
+constexpr int kGatherWarps = MOE_GATHER_WARPS;
+// Warp roles: warp 0 streams weights, warps 1..NTOK stream token rows, warp
+// MMA issues the MMAs (leader CTA), warps EPI0.. drain the accumulators.
+template <bool kGather> struct Roles {
+  static constexpr int NTOK = kGather ? kGatherWarps : 1;
+  static constexpr int MMA = 1 + NTOK;
+  static constexpr int EPI0 = MMA + 1;
+  static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
+};
 constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int MAX_STAGES = 8;                // barrier slots; the ring uses Args::stages of them
 constexpr size_t kSmemBudget = 232448;       // B200 opt-in shared memory per block
@@ -180,11 +192,12 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
 }
 
 template <bool kGelu, int kPair, bool kFp8, bool kGather>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_xw, const Args args) {
   using C = Cfg<kPair>;
+  using Ro = Roles<kGather>;
   constexpr int KB = kFp8 ? BK_FP8 : BK;  // K values per stage (128 bytes of a row)
   const int STAGES = args.stages;
   constexpr int B_STAGE = C::B_STAGE;
@@ -230,7 +243,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_xw);
   }
-  if (warp == 2) {
+  if (warp == Ro::MMA) {
     tmem_alloc<kPair>(s_tmem, TMEM_COLS);
     tmem_relinquish<kPair>();
   }
@@ -274,13 +287,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t full_lead = kPair == 2 ? cluster_map(smem_u32(full), 0) : smem_u32(full);
   const uint32_t tempty_lead = kPair == 2 ? cluster_map(smem_u32(tempty), 0) : smem_u32(tempty);
 
-  if (warp <= 1) {
+  if (warp <= Ro::NTOK) {
     // ------------------------------------------------------------ producers (both CTAs)
-    // Warp 0 streams the weight rows, warp 1 the token rows, each into the
-    // same ring of stages: two issuing threads keep twice as many TMA
-    // requests in flight as one.  In the leader CTA each arms the stage's
-    // barrier with the bytes of its operand in both CTAs of the pair.
+    // Warp 0 streams the weight rows, warp 1 (and in the gather form warps
+    // 2..NTOK) the token rows, each into the same ring of stages: separate
+    // issuing threads keep more TMA requests in flight than one.  In the
+    // leader CTA warps 0 and 1 arm the stage's barrier with the bytes of
+    // their operand in both CTAs of the pair.
     const bool is_w = warp == 0;
+    const int tw = warp - 1;  // token warp index
     const uint64_t pol = is_w ? l2_policy_evict_normal()  // shared by the CTAs of a feature block
                               : l2_policy_evict_last();   // re-read by every feature block
     int s = 0;
@@ -299,15 +314,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int wy = t.e * args.N + t.fb * C::FEAT + (int)rank * BM;
       const int by = t.row0 + (int)rank * half;
       // gather form: request q (4 rows) of this CTA's half-tile is issued
-      // by lane q % 32 (up to 64 requests: 256 rows with a single CTA); the
-      // token ids are read once per tile.  Rows past the expert's block (the
-      // MMA's padding to a multiple of 16) read token 0 and are never stored.
+      // by token warp q % NTOK, lane q / NTOK % 32 (up to 64 requests: 256
+      // rows with a single CTA); the token ids are read once per tile.  Rows
+      // past the expert's block (the MMA's padding to a multiple of 16) read
+      // token 0 and are never stored.
       const int nreq = half / 4;
       int g[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
       if (kGather && !is_w) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int q = lane + 32 * h;
+          const int q = (lane + 32 * h) * Ro::NTOK + tw;
           if (q >= nreq) continue;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -328,10 +344,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!ok) break;
         if (kGather && !is_w) {
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
-          if (lane == 0 && rank == 0) mbar_arrive_expect_tx(&full[s], gbytes);
+          if (tw == 0 && lane == 0 && rank == 0) mbar_arrive_expect_tx(&full[s], gbytes);
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int q = lane + 32 * h;
+            const int q = (lane + 32 * h) * Ro::NTOK + tw;
             if (q < nreq)
               tma_gather4_cg<kPair>(sB + s * B_STAGE + q * 512, &tm_x, kb * KB, g[h][0], g[h][1],
                                     g[h][2], g[h][3], fb_addr, pol);
@@ -364,7 +380,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if ((issued >> q) & 1u)
           mbar_wait(&full[q], (last_ph >> q) & 1u, nullptr, (volatile int*)&dummy, kDrainLimitNs);
     }
-  } else if (warp == 2) {
+  } else if (warp == Ro::MMA) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (rank == 0) {
       const uint32_t empty_peer = kPair == 2 ? cluster_map(smem_u32(empty), 1) : 0u;
@@ -429,7 +445,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int q = warp & 3;              // TMEM lane quarter this warp may access
     // which span of the tile's 256 token columns (EPI_WARPS / 4 spans)
     constexpr int SPAN = BN / (EPI_WARPS / 4);
-    const int hsel = (warp - EPI_WARP0) >> 2;
+    const int hsel = (warp - Ro::EPI0) >> 2;
     uint16_t* out = args.out;
     const int N = args.N;
     int it = 0;
@@ -472,7 +488,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_before_sync();
   __syncthreads();
   if (kPair == 2) cluster_sync();  // no CTA leaves while its peer may still signal it
-  if (warp == 2) {
+  if (warp == Ro::MMA) {
     tc_fence_after_sync();
     tmem_dealloc<kPair>(tmem_base, TMEM_COLS);
   }
@@ -553,7 +569,7 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(2 * dev.sm_count, 1, 1);
-      cfg.blockDim = dim3(gg::THREADS, 1, 1);
+      cfg.blockDim = dim3(gg::Roles<kGather>::THREADS, 1, 1);
       cfg.dynamicSmemBytes = smem_max;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
@@ -574,7 +590,7 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3((unsigned)(units * kPair), 1, 1);
-  cfg.blockDim = dim3(gg::THREADS, 1, 1);
+  cfg.blockDim = dim3(gg::Roles<kGather>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = gg::smem_bytes<kPair>(args.E, args.stages);
   cfg.stream = stream;
   cfg.attrs = attr;

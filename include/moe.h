@@ -67,6 +67,11 @@ typedef enum moe_score {
 #define MOE_DEV_TIMEOUT       0x2u /* a bounded device-side wait gave up; outputs are invalid */
 #define MOE_DEV_BAD_ROW       0x4u /* a row index outside [0, T*k) reached dispatch / combine */
 
+/* moe_layer_desc.flags */
+#define MOE_LAYER_GATHER_ON_LOAD 0x1 /* GEMM-1 reads token rows through src_of (TMA gather4)
+                                        instead of a dispatched copy; see
+                                        moe_expert_gemm_gather.  Same results, bit for bit. */
+
 /* Shape and routing recipe of one layer. */
 typedef struct moe_layer_desc {
   int32_t T;           /* tokens */
@@ -76,7 +81,7 @@ typedef struct moe_layer_desc {
   int32_t f;           /* FFN hidden dim */
   int32_t score;       /* moe_score */
   int32_t renormalize; /* 1: gates renormalised over the chosen k; 0: plain probability */
-  int32_t reserved;    /* must be 0 */
+  int32_t flags;       /* MOE_LAYER_* bits; 0 = the default path */
   float temperature;   /* router temperature (see moe_route_ex); 0 reads as 1 */
   float min_prob;      /* drop chosen slots whose probability is <= min_prob; <= 0 keeps all */
 } moe_layer_desc;
@@ -235,6 +240,11 @@ moe_status moe_combine(const void* Ye, const int32_t* row_of, const float* gates
  *   topk_idx_out [T, k], gates_out [T, k], counts_out [E]: optional copies
  *   of the routing (NULL to skip).
  *   ws: at least moe_workspace_size(desc) bytes.
+ *   desc->flags & MOE_LAYER_GATHER_ON_LOAD fuses the dispatch into GEMM-1
+ *   (no dispatch kernel, no dispatched copy of X); the output is identical.
+ *   On a B200 it is slower than the default for every shape measured (the
+ *   gathered loads cost more tensor-memory-access time than the dispatch
+ *   saves), so it is off by default.
  * ------------------------------------------------------------------------- */
 size_t moe_workspace_size(const moe_layer_desc* desc);
 moe_status moe_layer_forward(const moe_layer_desc* desc, const void* X, const float* logits,

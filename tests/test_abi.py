@@ -89,7 +89,7 @@ def test_layer_workspace_and_desc_checks(lib):
     ws = lib.moe_workspace_size(ctypes.byref(d))
     R = 4096 * 2
     assert ws >= R * 4096 * 2 * 2 + R * 14336 * 2  # Xe + Ye + H at least
-    bad = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 7)
+    bad = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 6)  # unknown flag bits
     assert lib.moe_workspace_size(ctypes.byref(bad)) == 0
     p = ctypes.c_void_p(0x10000)
     # both logits and Wr given
@@ -106,6 +106,9 @@ def test_launch_count(lib):
     assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 0) == 6
     d4 = moe.LayerDesc(8192, 7168, 256, 8, 2048, 1, 1, 0)
     assert lib.moe_kernel_launches_per_forward(ctypes.byref(d4), 0) == 7  # two-kernel layout
+    dg = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, moe.LAYER_GATHER_ON_LOAD)
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(dg), 1) == 6   # no dispatch kernel
+    assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(dg), 1) == 8  # absmax + quantise
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -137,3 +137,26 @@ def test_expert_gemm_gather_fp8_parity(T, E, k, N, K, gelu, drop):
                           (O.e4m3_decode(xe[lo:hi]) * float(x_s))
                           @ (O.e4m3_decode(Wq[e]) * float(w_s[e])).T)
     assert_close(f64(out[:used]), ref, "gather gemm fp8")
+
+
+@pytest.mark.parametrize("name,fp8", [("tiny", False), ("tiny", True), ("tiny_threshold", False),
+                                      ("tiny_threshold", True), ("decode_64", False)])
+def test_layer_gather_on_load_is_bitwise_the_default_layer(name, fp8):
+    """The MOE_LAYER_GATHER_ON_LOAD layer gives the default layer's bytes, which
+    the oracle checks (tests/test_gpu_parity.py, tests/test_gpu_fp8.py); the
+    tiny case is also checked against the oracle here directly."""
+    cfg = I.workload(name)
+    inp = I.make_layer_inputs(cfg, 4, device=DEV)
+    dev_in = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+    outs = []
+    for gather in (False, True):
+        layer = moe.MoeLayer(dev_in["W1"], dev_in["W2"], cfg.k, cfg.score, cfg.renormalize,
+                             Wr=dev_in["Wr"], temperature=cfg.temperature,
+                             min_prob=cfg.min_prob, fp8=fp8, gather_on_load=gather)
+        outs.append(layer(dev_in["X"], logits=dev_in["logits"]).clone())
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0].view(torch.int16), outs[1].view(torch.int16))
+    if name == "tiny" and not fp8:
+        ref = O.layer_forward(bits(inp["X"]), bits(inp["W1"]), bits(inp["W2"]), cfg.k, cfg.score,
+                              cfg.renormalize, logits=inp["logits"].numpy())
+        assert_close(f64(outs[1]), ref["Y"], "Y (gather on load)", rel=2e-2)

@@ -2,7 +2,7 @@
 """Benchmark: MoE-layer tokens/s on B200 (route -> layout -> dispatch -> expert FFN -> combine).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
-                    [--fp8] [--gather]
+                    [--fp8] [--gather] [--fused]
 
 One step = one full layer forward (every stage) over one batch of T tokens.
 Default workload: the Mixtral-shaped layer (T=4096, d=4096, E=8, top-2,
@@ -14,8 +14,9 @@ scaling, value = all ranks' tokens / the slowest rank's time.
 ``--fp8`` runs the layer's FP8 mode (E4M3 dispatch with a per-tensor scale
 and FP8 GEMM-1; GEMM-2 and combine stay bf16); W1 is quantised once before
 timing.  ``--gather`` fuses the dispatch into GEMM-1 (rows read through the
-layout table with TMA gather4 loads; no dispatch kernel).  Prints one JSON
-line (rank 0).  ``--impl reference`` times the CPU oracle
+layout table with TMA gather4 loads; no dispatch kernel).  ``--fused`` runs
+both expert GEMMs as one persistent kernel (GEMM-2 starts per token block as
+soon as GEMM-1 has produced it).  Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 (the only reference this method has) on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -74,6 +75,8 @@ def stage_model(cfg, counts=None, fp8=False):  # gather form: same algorithmic b
         m["dispatch"] = {"bytes": 2 * T * d * 2 + R * d + R * 4}
         m["gemm1"] = {"flops": 2 * R * d * f, "bytes": E_act * f * d + R * d + R * f * 2}
         m["quantize"] = {"bytes": 2 * T * d * 2 + T * d}
+    m["ffn"] = {"flops": m["gemm1"]["flops"] + m["gemm2"]["flops"],
+                "bytes": m["gemm1"]["bytes"] + m["gemm2"]["bytes"]}
     return m
 
 
@@ -245,7 +248,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     Wr = inp["Wr"].to(dev) if inp["Wr"] is not None else None
     layer = moe.MoeLayer(inp["W1"], inp["W2"], cfg.k, cfg.score, cfg.renormalize, Wr=Wr,
                          temperature=cfg.temperature, min_prob=cfg.min_prob, fp8=args.fp8,
-                         gather_on_load=args.gather)
+                         gather_on_load=args.gather, fused_ffn=args.fused)
     Y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
     counts = torch.empty((cfg.E,), dtype=torch.int32, device=dev)
     ws = layer.workspace(cfg.T)
@@ -285,8 +288,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         # ---- per-stage times: the same kernels, launched stage by stage with events between
         stage_names = (["router_logits"] if Wr is not None else []) + [
             "route", "layout"] + (["quantize"] if args.gather and args.fp8 else
-                                  [] if args.gather else ["dispatch"]) + [
-            "gemm1", "gemm2", "combine"]
+                                  [] if args.gather else ["dispatch"]) + (
+            ["ffn"] if args.fused else ["gemm1", "gemm2"]) + ["combine"]
         R = cfg.R
         L_buf = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev) if Wr is not None else logits
         idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
@@ -298,6 +301,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                           dtype=torch.uint8, device=dev)
         Xe = torch.empty((R, cfg.d), dtype=torch.uint8 if args.fp8 else torch.bfloat16, device=dev)
         Xq = torch.empty((cfg.T, cfg.d), dtype=torch.uint8, device=dev)
+        ffn_ws = torch.empty(max(16, moe.moe_expert_ffn_fused_workspace_size(cfg.E, R)),
+                             dtype=torch.uint8, device=dev)
         xs = torch.empty((2,), dtype=torch.float32, device=dev)
         H = torch.empty((R, cfg.f), dtype=torch.bfloat16, device=dev)
         Ye = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=dev)
@@ -318,6 +323,10 @@ def run_ours(args, cfg, rank, world, local_rank):
                                                           H)) if args.gather else
                       (lambda: moe.moe_expert_gemm(Xe, offs, inp["W1"], True, H))),
             "gemm2": lambda: moe.moe_expert_gemm(H, offs, inp["W2"], False, Ye),
+            "ffn": (lambda: moe.moe_expert_ffn_fused_fp8(Xe, xs, offs, layer.W1q, layer.w1_scale,
+                                                         inp["W2"], H, Ye, ffn_ws)) if args.fp8 else
+                   (lambda: moe.moe_expert_ffn_fused(Xe, offs, inp["W1"], inp["W2"], H, Ye,
+                                                     ffn_ws)),
             "combine": lambda: moe.moe_combine(Ye, row_of, g, Y),
         }
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stage_names) + 1)]
@@ -386,8 +395,10 @@ def run_ours(args, cfg, rank, world, local_rank):
     sustained = capped or (t_ms + staged_total_ms * args.steps) > 1000.0
     per = model[dom]
     dur_s = stage_ms[dom] / 1e3
-    # an FP8 contraction's peak: the measured bf16 peak x the nominal fp8:bf16 ratio (2)
-    tc_ratio = 2.0 if (args.fp8 and dom == "gemm1") else 1.0
+    # an FP8 contraction's peak: the measured bf16 peak x the nominal fp8:bf16 ratio (2);
+    # the fused FFN in FP8 mode does half its FLOPs at each rate (harmonic mean)
+    tc_ratio = 2.0 if (args.fp8 and dom == "gemm1") else (
+        4.0 / 3.0 if (args.fp8 and dom == "ffn") else 1.0)
     if "flops" in per and per["flops"] / max(per["bytes"], 1) > (
             tc_ratio * peaks["bf16_tflops"] * 1e12) / (peaks["hbm_gbs"] * 1e9):
         peak = tc_ratio * (peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"])
@@ -401,10 +412,13 @@ def run_ours(args, cfg, rank, world, local_rank):
     roof["kernel"] = dom
     roof["peak_source"] = (f"{peak_src} ("
                            f"{'sustained: power cap active in the timed region' if sustained and roof['bound'] == 'tensor' else 'burst'})"
-                           + (" x 2 (fp8:bf16 nominal ratio)" if tc_ratio != 1.0 else ""))
+                           + ("" if tc_ratio == 1.0 else
+                              " x 2 (fp8:bf16 nominal ratio)" if tc_ratio == 2.0 else
+                              " x 4/3 (half the FLOPs at the fp8 rate, half at bf16)"))
     kname = {"gemm1": ("grouped_gemm_fp8_gelu" if args.fp8 else "grouped_gemm_gelu")
                       + ("_gather" if args.gather else ""),
-             "gemm2": "grouped_gemm"}.get(dom, dom)
+             "gemm2": "grouped_gemm",
+             "ffn": "fused_ffn_fp8" if args.fp8 else "fused_ffn"}.get(dom, dom)
     tr = ncu_traffic(kname, cfg.name)
     roof["traffic"] = tr
     roof["algorithmic_bytes"] = per["bytes"]
@@ -427,7 +441,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "dtype": "e4m3 (dispatch, GEMM-1) + bf16" if args.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
                    "f": cfg.f, "router": cfg.router, "score": cfg.score, "fp8": bool(args.fp8),
-                   "gather_on_load": bool(args.gather),
+                   "gather_on_load": bool(args.gather), "fused_ffn": bool(args.fused),
                    "renormalize": cfg.renormalize, "temperature": cfg.temperature,
                    "min_prob": cfg.min_prob, "tokens_per_gpu": cfg.T,
                    "parallelism": f"replicas x{world} (no collective)",
@@ -443,7 +457,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "gpu_launches": args.steps * (moe.moe_kernel_launches_per_forward_fp8 if args.fp8 else
                                       moe.moe_kernel_launches_per_forward)(
             moe.make_desc(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.score, cfg.renormalize,
-                          gather_on_load=args.gather),
+                          gather_on_load=args.gather, fused_ffn=args.fused),
             Wr is not None),
         "clocks": clocks,
     }
@@ -465,7 +479,11 @@ def main():
                     help="FP8 mode: E4M3 dispatch with a per-tensor scale and FP8 GEMM-1")
     ap.add_argument("--gather", action="store_true",
                     help="fuse the dispatch into GEMM-1 (gather-on-load)")
+    ap.add_argument("--fused", action="store_true",
+                    help="both expert GEMMs in one persistent kernel")
     args = ap.parse_args()
+    if args.gather and args.fused:
+        ap.error("--gather and --fused cannot be combined")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

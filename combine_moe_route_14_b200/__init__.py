@@ -27,6 +27,7 @@ __all__ = [
     "moe_quantize_experts_fp8", "moe_dispatch_fp8", "moe_expert_gemm_fp8",
     "moe_layer_forward_fp8", "moe_kernel_launches_per_forward_fp8",
     "moe_quantize_fp8", "moe_expert_gemm_gather", "moe_expert_gemm_gather_fp8",
+    "moe_expert_ffn_fused_workspace_size", "moe_expert_ffn_fused", "moe_expert_ffn_fused_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +37,7 @@ _lock = threading.Lock()
 
 SCORES = {"softmax": 0, "sigmoid": 1}
 LAYER_GATHER_ON_LOAD = 0x1  # moe_layer_desc.flags: dispatch fused into GEMM-1
+LAYER_FUSED_FFN = 0x2       # moe_layer_desc.flags: both expert GEMMs in one persistent launch
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
           4: "MOE_ERR_DEVICE"}
 DEV_BITS = {1: "MOE_DEV_BAD_EXPERT_ID", 2: "MOE_DEV_TIMEOUT", 4: "MOE_DEV_BAD_ROW"}
@@ -85,6 +87,11 @@ _SIG = {
                                _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_kernel_launches_per_forward_fp8": ([ctypes.POINTER(LayerDesc), _I], ctypes.c_int32),
     "moe_quantize_fp8": ([_P, _I, _I, _P, _P, _P], ctypes.c_int),
+    "moe_expert_ffn_fused_workspace_size": ([_I, _I], ctypes.c_size_t),
+    "moe_expert_ffn_fused": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P],
+                             ctypes.c_int),
+    "moe_expert_ffn_fused_fp8": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P,
+                                  ctypes.c_size_t, _P], ctypes.c_int),
     "moe_expert_gemm_gather": ([_P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P], ctypes.c_int),
     "moe_expert_gemm_gather_fp8": ([_P, _P, _P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P],
                                    ctypes.c_int),
@@ -283,6 +290,56 @@ def moe_expert_ffn(Xe, offsets, W1, W2, H=None, Ye=None, stream=None):
     return H, Ye
 
 
+def moe_expert_ffn_fused_workspace_size(E, R) -> int:
+    return int(load_library().moe_expert_ffn_fused_workspace_size(E, R))
+
+
+def moe_expert_ffn_fused(Xe, offsets, W1, W2, H=None, Ye=None, ws=None, stream=None):
+    """moe_expert_ffn as one persistent kernel (GEMM-2 starts per token block)."""
+    lib = load_library()
+    R, d = Xe.shape
+    E, f, _ = W1.shape
+    dev = Xe.device
+    _need(Xe, "Xe", torch.bfloat16, (R, d))
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(W1, "W1", torch.bfloat16, (E, f, d), dev)
+    _need(W2, "W2", torch.bfloat16, (E, d, f), dev)
+    H = _out(H, "H", torch.bfloat16, (R, f), dev)
+    Ye = _out(Ye, "Ye", torch.bfloat16, (R, d), dev)
+    if ws is None:
+        ws = torch.empty(max(moe_expert_ffn_fused_workspace_size(E, R), 16), dtype=torch.uint8,
+                         device=dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _check(lib.moe_expert_ffn_fused(_ptr(Xe), _ptr(offsets), _ptr(W1), _ptr(W2), E, R, d, f,
+                                    _ptr(H), _ptr(Ye), _ptr(ws), ws.numel(), _stream(stream, dev)))
+    return H, Ye
+
+
+def moe_expert_ffn_fused_fp8(Xeq, x_scale, offsets, W1q, w1_scale, W2, H=None, Ye=None, ws=None,
+                             stream=None):
+    lib = load_library()
+    R, d = Xeq.shape
+    E, f, _ = W1q.shape
+    dev = Xeq.device
+    _need(Xeq, "Xeq", torch.uint8, (R, d))
+    if x_scale.dtype != torch.float32 or x_scale.device != dev or x_scale.numel() < 1:
+        raise ValueError("x_scale must be a float32 device tensor")
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(W1q, "W1q", torch.uint8, (E, f, d), dev)
+    _need(w1_scale, "w1_scale", torch.float32, (E,), dev)
+    _need(W2, "W2", torch.bfloat16, (E, d, f), dev)
+    H = _out(H, "H", torch.bfloat16, (R, f), dev)
+    Ye = _out(Ye, "Ye", torch.bfloat16, (R, d), dev)
+    if ws is None:
+        ws = torch.empty(max(moe_expert_ffn_fused_workspace_size(E, R), 16), dtype=torch.uint8,
+                         device=dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _check(lib.moe_expert_ffn_fused_fp8(_ptr(Xeq), _ptr(x_scale), _ptr(offsets), _ptr(W1q),
+                                        _ptr(w1_scale), _ptr(W2), E, R, d, f, _ptr(H), _ptr(Ye),
+                                        _ptr(ws), ws.numel(), _stream(stream, dev)))
+    return H, Ye
+
+
 def moe_combine(Ye, row_of, gates, Y=None, stream=None):
     lib = load_library()
     T, k = gates.shape
@@ -303,10 +360,10 @@ def moe_combine(Ye, row_of, gates, Y=None, stream=None):
 # whole layer
 # ----------------------------------------------------------------------------
 def make_desc(T, d, E, k, f, score="softmax", renormalize=True, temperature=1.0,
-              min_prob=0.0, gather_on_load=False) -> LayerDesc:
-    return LayerDesc(T, d, E, k, f, _score(score), int(bool(renormalize)),
-                     LAYER_GATHER_ON_LOAD if gather_on_load else 0, float(temperature),
-                     float(min_prob))
+              min_prob=0.0, gather_on_load=False, fused_ffn=False) -> LayerDesc:
+    flags = (LAYER_GATHER_ON_LOAD if gather_on_load else 0) | (LAYER_FUSED_FFN if fused_ffn else 0)
+    return LayerDesc(T, d, E, k, f, _score(score), int(bool(renormalize)), flags,
+                     float(temperature), float(min_prob))
 
 
 def moe_workspace_size(desc: LayerDesc) -> int:
@@ -320,7 +377,8 @@ def moe_kernel_launches_per_forward(desc: LayerDesc, with_router: bool) -> int:
 
 def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=None, Wr=None,
                       Y=None, topk_idx_out=None, gates_out=None, counts_out=None, ws=None,
-                      stream=None, temperature=1.0, min_prob=0.0, gather_on_load=False):
+                      stream=None, temperature=1.0, min_prob=0.0, gather_on_load=False,
+                      fused_ffn=False):
     lib = load_library()
     T, d = X.shape
     E, f, _ = W1.shape
@@ -339,7 +397,8 @@ def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=No
         _need(gates_out, "gates_out", torch.float32, (T, k), dev)
     if counts_out is not None:
         _need(counts_out, "counts_out", torch.int32, (E,), dev)
-    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, gather_on_load)
+    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, gather_on_load,
+                     fused_ffn)
     if ws is None:
         ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
     _need(ws, "ws", torch.uint8, None, dev)
@@ -460,7 +519,7 @@ def moe_kernel_launches_per_forward_fp8(desc: LayerDesc, with_router: bool) -> i
 def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=True,
                           logits=None, Wr=None, Y=None, topk_idx_out=None, gates_out=None,
                           counts_out=None, ws=None, stream=None, temperature=1.0, min_prob=0.0,
-                          gather_on_load=False):
+                          gather_on_load=False, fused_ffn=False):
     """The layer with FP8 dispatch and FP8 GEMM-1 (W1q, w1_scale from moe_quantize_experts_fp8)."""
     lib = load_library()
     T, d = X.shape
@@ -481,7 +540,8 @@ def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=
         _need(gates_out, "gates_out", torch.float32, (T, k), dev)
     if counts_out is not None:
         _need(counts_out, "counts_out", torch.int32, (E,), dev)
-    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, gather_on_load)
+    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, gather_on_load,
+                     fused_ffn)
     if ws is None:
         ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
     _need(ws, "ws", torch.uint8, None, dev)
@@ -506,10 +566,11 @@ class MoeLayer:
     """A layer's weights plus a reusable workspace (allocation stays outside the call)."""
 
     def __init__(self, W1, W2, k, score="softmax", renormalize=True, Wr=None, temperature=1.0,
-                 min_prob=0.0, fp8=False, gather_on_load=False):
+                 min_prob=0.0, fp8=False, gather_on_load=False, fused_ffn=False):
         self.W1, self.W2, self.Wr = W1, W2, Wr
         self.fp8 = bool(fp8)
         self.gather_on_load = bool(gather_on_load)
+        self.fused_ffn = bool(fused_ffn)
         # FP8 mode keeps W1 as E4M3 codes with per-expert scales (quantised once here)
         self.W1q, self.w1_scale = moe_quantize_experts_fp8(W1) if self.fp8 else (None, None)
         self.k, self.score, self.renormalize = k, score, renormalize
@@ -529,7 +590,8 @@ class MoeLayer:
         kw = dict(logits=logits, Wr=None if logits is not None else self.Wr, Y=Y,
                   topk_idx_out=topk_idx_out, gates_out=gates_out, counts_out=counts_out,
                   ws=self.workspace(X.shape[0]), stream=stream, temperature=self.temperature,
-                  min_prob=self.min_prob, gather_on_load=self.gather_on_load)
+                  min_prob=self.min_prob, gather_on_load=self.gather_on_load,
+                  fused_ffn=self.fused_ffn)
         if self.fp8:
             return moe_layer_forward_fp8(X, self.W1q, self.w1_scale, self.W2, self.k, self.score,
                                          self.renormalize, **kw)

@@ -127,7 +127,8 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // Workspace of the fused forward: sub-buffers, each 256-byte aligned.
 struct LayerWs {
-  size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, scale, total;
+  size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, scale, ready,
+      total;
 };
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -148,6 +149,7 @@ LayerWs layer_ws(const moe_layer_desc& d) {
   w.H = o;       o += up256(R * d.f * 2);
   w.Ye = o;      o += up256(R * d.d * 2);
   w.scale = o;   o += up256(2 * sizeof(float));  // FP8 mode: activation scale and amax
+  w.ready = o;   o += up256((size_t)moe::ffn_ready_count((int)R, d.E) * sizeof(uint32_t));
   w.total = o;
   return w;
 }
@@ -161,7 +163,10 @@ moe_status check_desc(const moe_layer_desc* desc) {
     return fail(MOE_ERR_INVALID_ARG, "unknown score");
   if (desc->renormalize != 0 && desc->renormalize != 1)
     return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
-  if (desc->flags & ~MOE_LAYER_GATHER_ON_LOAD) return fail(MOE_ERR_INVALID_ARG, "unknown flags");
+  if (desc->flags & ~(MOE_LAYER_GATHER_ON_LOAD | MOE_LAYER_FUSED_FFN))
+    return fail(MOE_ERR_INVALID_ARG, "unknown flags");
+  if ((desc->flags & MOE_LAYER_GATHER_ON_LOAD) && (desc->flags & MOE_LAYER_FUSED_FFN))
+    return fail(MOE_ERR_UNSUPPORTED, "MOE_LAYER_GATHER_ON_LOAD with MOE_LAYER_FUSED_FFN");
   if (!std::isfinite(desc->temperature) || desc->temperature < 0.f)
     return fail(MOE_ERR_INVALID_ARG, "temperature must be >= 0 (0 reads as 1)");
   if (!std::isfinite(desc->min_prob)) return fail(MOE_ERR_INVALID_ARG, "min_prob must be finite");
@@ -223,6 +228,7 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   void* H = base + w.H;
   void* Ye = base + w.Ye;
   float* x_scale = reinterpret_cast<float*>(base + w.scale);
+  uint32_t* ready = reinterpret_cast<uint32_t*>(base + w.ready);
   const int R = d.T * d.k;
 
   if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, s), "router_logits");
@@ -233,6 +239,18 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   std::string err;
   cudaError_t e;
   const bool gather = (d.flags & MOE_LAYER_GATHER_ON_LOAD) != 0;
+  if (d.flags & MOE_LAYER_FUSED_FFN) {  // both GEMMs in one persistent launch
+    if (fp8)
+      MOE_CUDA(moe::launch_dispatch_fp8(X, src_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
+               "dispatch_fp8");
+    else
+      MOE_CUDA(moe::launch_dispatch(X, src_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+    e = moe::launch_fused_ffn(Xe, x_scale, offsets, W1, W1s, W2, d.E, R, d.d, d.f, fp8, H, Ye,
+                              ready, *dev, s, &err);
+    if (e != cudaSuccess) return gemm_fail(e, err, "fused_ffn");
+    MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
+    return MOE_OK;
+  }
   if (gather) {  // dispatch fused into GEMM-1: its rows are read through src_of
     const void* A = X;
     if (fp8) {   // the tokens are quantised once (T rows), into the Xe slot
@@ -519,6 +537,60 @@ moe_status moe_expert_ffn(const void* Xe, const int32_t* offsets, const void* W1
   return moe_expert_gemm(H, offsets, W2, E, R, d, f, 0, Ye, stream);
 }
 
+size_t moe_expert_ffn_fused_workspace_size(int32_t E, int32_t R) {
+  if (E < 1 || R < 0) return 0;
+  return up256((size_t)moe::ffn_ready_count(R, E) * sizeof(uint32_t));
+}
+
+namespace {
+moe_status ffn_fused(const void* A, const float* a_scale, const int32_t* offsets, const void* W1,
+                     const float* w1_scale, const void* W2, int32_t E, int32_t R, int32_t d,
+                     int32_t f, void* H, void* Ye, void* ws, size_t ws_bytes, void* stream,
+                     bool fp8) {
+  MOE_TRY(check_gemm_shape(E, R, f, d, 1));
+  MOE_TRY(check_gemm_shape(E, R, d, f, 0));
+  if (fp8) MOE_TRY(check_fp8_dim(d, "d"));
+  if (R == 0) return MOE_OK;
+  MOE_TRY(check_ptr(A, fp8 ? "Xeq" : "Xe"));
+  MOE_TRY(check_ptr4(offsets, "offsets"));
+  MOE_TRY(check_ptr(W1, fp8 ? "W1q" : "W1"));
+  MOE_TRY(check_ptr(W2, "W2"));
+  MOE_TRY(check_ptr(H, "H"));
+  MOE_TRY(check_ptr(Ye, "Ye"));
+  if (fp8) {
+    MOE_TRY(check_ptr4(a_scale, "x_scale"));
+    MOE_TRY(check_ptr4(w1_scale, "w1_scale"));
+  }
+  if (ws_bytes < moe_expert_ffn_fused_workspace_size(E, R))
+    return fail(MOE_ERR_INVALID_ARG, "workspace too small");
+  MOE_TRY(check_ptr(ws, "ws"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  std::string err;
+  cudaError_t e = moe::launch_fused_ffn(A, a_scale, offsets, W1, w1_scale, W2, E, R, d, f, fp8,
+                                        H, Ye, static_cast<uint32_t*>(ws), *dev,
+                                        as_stream(stream), &err);
+  if (e != cudaSuccess) return gemm_fail(e, err, "expert_ffn_fused");
+  return MOE_OK;
+}
+}  // namespace
+
+moe_status moe_expert_ffn_fused(const void* Xe, const int32_t* offsets, const void* W1,
+                                const void* W2, int32_t E, int32_t R, int32_t d, int32_t f,
+                                void* H, void* Ye, void* ws, size_t ws_bytes, void* stream) {
+  return ffn_fused(Xe, nullptr, offsets, W1, nullptr, W2, E, R, d, f, H, Ye, ws, ws_bytes,
+                   stream, false);
+}
+
+moe_status moe_expert_ffn_fused_fp8(const void* Xeq, const float* x_scale,
+                                    const int32_t* offsets, const void* W1q,
+                                    const float* w1_scale, const void* W2, int32_t E, int32_t R,
+                                    int32_t d, int32_t f, void* H, void* Ye, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  return ffn_fused(Xeq, x_scale, offsets, W1q, w1_scale, W2, E, R, d, f, H, Ye, ws, ws_bytes,
+                   stream, true);
+}
+
 moe_status moe_combine(const void* Ye, const int32_t* row_of, const float* gates, int32_t T,
                        int32_t d, int32_t k, void* Y, void* stream) {
   if (T < 0 || k < 1) return fail(MOE_ERR_INVALID_ARG, "need T >= 0 and k >= 1");
@@ -543,10 +615,11 @@ size_t moe_workspace_size(const moe_layer_desc* desc) {
 
 int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with_router) {
   if (check_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  // [router linear] + route + layout + [dispatch] + 2 GEMMs + combine
+  // [router linear] + route + layout + [dispatch] + 2 GEMMs (1 fused) + combine
   const int dispatch = (desc->flags & MOE_LAYER_GATHER_ON_LOAD) ? 0 : 1;
+  const int gemms = (desc->flags & MOE_LAYER_FUSED_FFN) ? 1 : 2;
   return (with_router ? 1 : 0) + 1 + moe::layout_kernel_count((int64_t)desc->T * desc->k) +
-         dispatch + 2 + 1;
+         dispatch + gemms + 1;
 }
 
 int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t with_router) {

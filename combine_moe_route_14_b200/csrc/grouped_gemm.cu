@@ -40,6 +40,16 @@
 //     host synchronisation.  Tiles are ordered (expert, feature block, token
 //     block) with the token block fastest, so CTAs running at the same time
 //     share one weight block through L2.
+//   * Fused FFN form (kFused): GEMM-1 and GEMM-2 in one persistent launch
+//     (the GEMM half of the token-centric pipeline of the DySHARP review
+//     §3.2).  The tile list is GEMM-1's tiles followed by GEMM-2's; a GEMM-2
+//     tile of token block b starts once every GEMM-1 tile of b has stored
+//     its part of H: each GEMM-1 epilogue warp publishes its stores (fence,
+//     then an atomic add on b's counter) and GEMM-2's token producer waits,
+//     bounded, for the count (acquire), then fences the async proxy before
+//     its TMA reads of H.  GEMM-1 tiles wait on nothing and every CTA is
+//     resident, so the waits always end; the GEMM-1 tail, the second launch
+//     and its prologue disappear.
 //   * Every wait is bounded (see mbar_wait); on a timeout the CTA raises a
 //     status bit, drains what it issued and frees its TMEM.
 #include <mutex>
@@ -101,7 +111,7 @@ template <int kPair> struct Cfg {
 // Shared memory: the stage ring, barriers, and the per-expert tile table.
 template <int kPair>
 __host__ __device__ constexpr size_t fixed_smem(int E) {
-  return 1024 /* alignment slack */ + Cfg<kPair>::NUM_BARS * 8 + 16 + (size_t)3 * (E + 1) * sizeof(int);
+  return 1024 /* alignment slack */ + Cfg<kPair>::NUM_BARS * 8 + 16 + (size_t)4 * (E + 1) * sizeof(int);
 }
 template <int kPair>
 __host__ __device__ constexpr size_t smem_bytes(int E, int stages) {
@@ -128,6 +138,11 @@ struct Args {
   int n_fblocks;           // ceil(N / features per tile)
   int num_kb;              // ceil(K / K-values per stage)
   int stages;              // ring depth (<= MAX_STAGES)
+  // fused FFN form: phase 1 = GEMM-2 over phase 0's output (A = out)
+  uint16_t* out2;          // [R, N2] bf16
+  int N2, n_fblocks2, num_kb2;
+  uint32_t* ready;         // [token blocks]: GEMM-1 epilogue warps done, per token block
+  uint32_t ready_target;   // arrivals that complete a token block
 };
 
 struct Tile {
@@ -191,11 +206,14 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
-template <bool kGelu, int kPair, bool kFp8, bool kGather>
+template <bool kGelu, int kPair, bool kFp8, bool kGather, bool kFused>
 __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x,
-                        const __grid_constant__ CUtensorMap tm_xw, const Args args) {
+                        const __grid_constant__ CUtensorMap tm_xw,
+                        const __grid_constant__ CUtensorMap tm_w2,
+                        const __grid_constant__ CUtensorMap tm_x2,
+                        const __grid_constant__ CUtensorMap tm_xw2, const Args args) {
   using C = Cfg<kPair>;
   using Ro = Roles<kGather>;
   constexpr int KB = kFp8 ? BK_FP8 : BK;  // K values per stage (128 bytes of a row)
@@ -218,6 +236,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
   int* s_lo = reinterpret_cast<int*>(s_tmem + 4);
   int* s_hi = s_lo + (E + 1);
   int* s_start = s_hi + (E + 1);
+  int* s_start2 = s_start + (E + 1);  // fused form: GEMM-2's per-expert first tile
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -242,6 +261,11 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_xw);
+    if (kFused) {
+      tma_prefetch_desc(&tm_w2);
+      tma_prefetch_desc(&tm_x2);
+      tma_prefetch_desc(&tm_xw2);
+    }
   }
   if (warp == Ro::MMA) {
     tmem_alloc<kPair>(s_tmem, TMEM_COLS);
@@ -276,13 +300,35 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
       run += token_blocks(s_hi[e] - s_lo[e]) * args.n_fblocks;
     }
     if (lane == 31) s_start[E] = incl;
+    if (kFused) {  // GEMM-2's tiles: same token blocks, n_fblocks2 feature blocks each
+      run = (incl - sum) / args.n_fblocks * args.n_fblocks2;
+      for (int e = e0; e < e1; ++e) {
+        s_start2[e] = run;
+        run += token_blocks(s_hi[e] - s_lo[e]) * args.n_fblocks2;
+      }
+      if (lane == 31) s_start2[E] = incl / args.n_fblocks * args.n_fblocks2;
+    }
   }
   tc_fence_before_sync();
   if (kPair == 2) cluster_sync();  // the peer's barriers are initialised before any remote use
   else __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
-  const int total_tiles = s_start[E];
+  const int tiles0 = s_start[E];
+  const int total_tiles = tiles0 + (kFused ? s_start2[E] : 0);
+  // tile -> (tile, phase); phase 1 only in the fused form
+  auto tile_at = [&](int tile, int& phase) -> Tile {
+    if (kFused && tile >= tiles0) {
+      phase = 1;
+      return decode(tile - tiles0, s_start2, s_lo, s_hi, E);
+    }
+    phase = 0;
+    return decode(tile, s_start, s_lo, s_hi, E);
+  };
+  // fused form: index of the token block holding a tile's rows
+  auto block_of = [&](const Tile& t) -> int {
+    return s_start[t.e] / args.n_fblocks + (t.row0 - s_lo[t.e]) / BN;
+  };
   // the leader's barriers as cluster addresses (the CTA's own when kPair == 1)
   const uint32_t full_lead = kPair == 2 ? cluster_map(smem_u32(full), 0) : smem_u32(full);
   const uint32_t tempty_lead = kPair == 2 ? cluster_map(smem_u32(tempty), 0) : smem_u32(tempty);
@@ -304,14 +350,33 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     uint32_t last_ph = 0; // bit s: parity of the last load issued on stage s
     bool ok = true;
     for (int tile = cid; ok && tile < total_tiles; tile += ncl) {
-      const Tile t = decode(tile, s_start, s_lo, s_hi, E);
+      int phase;
+      const Tile t = tile_at(tile, phase);
+      const bool p1 = kFused && phase == 1;
+      const CUtensorMap* map_w = p1 ? &tm_w2 : &tm_w;
+      const CUtensorMap* map_x = p1 ? &tm_x2 : &tm_x;
+      const CUtensorMap* map_xw = p1 ? &tm_xw2 : &tm_xw;
+      const int kbv = (kFp8 && !p1) ? BK_FP8 : BK;  // K values per stage in this phase
+      const int nkb = p1 ? args.num_kb2 : args.num_kb;
+      const int Np = p1 ? args.N2 : args.N;
+      if (p1 && !is_w) {  // GEMM-2 reads H rows that GEMM-1 tiles of other CTAs store
+        bool rdy = true;
+        if (lane == 0) {
+          rdy = wait_count_geq(args.ready + block_of(t), args.ready_target, args.status, s_abort);
+          if (rdy) fence_proxy_async_global();
+        }
+        if (!__shfl_sync(0xffffffffu, rdy, 0)) {
+          ok = false;
+          break;
+        }
+      }
       const int nmma = (t.ntok + 15) & ~15;
       const int half = nmma / kPair;  // token rows staged by this CTA (a multiple of 8)
       const bool wide = half >= kWideMin;
       const int nbox = (half + B_BOX_ROWS - 1) / B_BOX_ROWS;
       const uint32_t bytes = is_w ? (uint32_t)(kPair * A_STAGE)
                                   : (uint32_t)kPair * (wide ? B_WIDE_ROWS * BK * 2 : nbox * B_BOX);
-      const int wy = t.e * args.N + t.fb * C::FEAT + (int)rank * BM;
+      const int wy = t.e * Np + t.fb * C::FEAT + (int)rank * BM;
       const int by = t.row0 + (int)rank * half;
       // gather form: request q (4 rows) of this CTA's half-tile is issued
       // by token warp q % NTOK, lane q / NTOK % 32 (up to 64 requests: 256
@@ -339,7 +404,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
         }
       }
       const uint32_t gbytes = (uint32_t)(kPair * half * 128);
-      for (int kb = 0; kb < args.num_kb; ++kb) {
+      for (int kb = 0; kb < nkb; ++kb) {
         ok = warp_wait(&empty[s], ph ^ 1u, args.status, s_abort);
         if (!ok) break;
         if (kGather && !is_w) {
@@ -356,12 +421,12 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes);
           if (is_w) {
-            tma_load_2d_cg<kPair>(sA + s * A_STAGE, &tm_w, kb * KB, wy, fb_addr, pol);
+            tma_load_2d_cg<kPair>(sA + s * A_STAGE, map_w, kb * kbv, wy, fb_addr, pol);
           } else if (wide) {  // (nearly) a full half-tile: one large request
-            tma_load_2d_cg<kPair>(sB + s * B_STAGE, &tm_xw, kb * KB, by, fb_addr, pol);
+            tma_load_2d_cg<kPair>(sB + s * B_STAGE, map_xw, kb * kbv, by, fb_addr, pol);
           } else {
             for (int j = 0; j < nbox; ++j)
-              tma_load_2d_cg<kPair>(sB + s * B_STAGE + j * B_BOX, &tm_x, kb * KB,
+              tma_load_2d_cg<kPair>(sB + s * B_STAGE + j * B_BOX, map_x, kb * kbv,
                                     by + j * B_BOX_ROWS, fb_addr, pol);
           }
         }
@@ -390,17 +455,21 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int tile = cid; ok && tile < total_tiles; tile += ncl, ++it) {
-        const Tile t = decode(tile, s_start, s_lo, s_hi, E);
+        int phase;
+        const Tile t = tile_at(tile, phase);
+        const bool p1 = kFused && phase == 1;
+        const bool f8 = kFp8 && !p1;  // GEMM-2 of the fused form is bf16
+        const int nkb = p1 ? args.num_kb2 : args.num_kb;
         const uint32_t nmma = (uint32_t)((t.ntok + 15) & ~15);
-        const uint32_t idesc = kFp8 ? idesc_e4m3_f32((uint32_t)C::FEAT, nmma)
-                                    : idesc_bf16_f32((uint32_t)C::FEAT, nmma);
+        const uint32_t idesc = f8 ? idesc_e4m3_f32((uint32_t)C::FEAT, nmma)
+                                  : idesc_bf16_f32((uint32_t)C::FEAT, nmma);
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)((it >> 1) & 1);
         ok = warp_wait(&tempty[acc], aph ^ 1u, args.status, s_abort);
         if (!ok) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < args.num_kb; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           ok = warp_wait(&full[s], ph, args.status, s_abort);
           if (!ok) break;
           tc_fence_after_sync();
@@ -411,7 +480,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
             for (int kk = 0; kk < 128 / UMMA_K_BYTES; ++kk) {
               const uint64_t ad = smem_desc_k128(a0 + kk * UMMA_K_BYTES);
               const uint64_t bd = smem_desc_k128(b0 + kk * UMMA_K_BYTES);
-              if constexpr (kFp8)
+              if (f8)
                 tc_mma_e4m3<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
               else
                 tc_mma_bf16<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
@@ -446,18 +515,22 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     // which span of the tile's 256 token columns (EPI_WARPS / 4 spans)
     constexpr int SPAN = BN / (EPI_WARPS / 4);
     const int hsel = (warp - Ro::EPI0) >> 2;
-    uint16_t* out = args.out;
-    const int N = args.N;
     int it = 0;
     for (int tile = cid; tile < total_tiles; tile += ncl, ++it) {
-      const Tile t = decode(tile, s_start, s_lo, s_hi, E);
+      int phase;
+      const Tile t = tile_at(tile, phase);
+      const bool p1 = kFused && phase == 1;
+      const bool f8 = kFp8 && !p1;
+      const bool gelu = kGelu && !p1;  // the fused form's GEMM-2 has no activation
+      uint16_t* out = p1 ? args.out2 : args.out;
+      const int N = p1 ? args.N2 : args.N;
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       if (!warp_wait(&tfull[acc], aph, args.status, s_abort)) break;
       tc_fence_after_sync();
       // this lane's output feature; the warp covers 32 consecutive features
       const int f = t.fb * C::FEAT + (int)rank * BM + q * 32 + lane;
-      const float sc = kFp8 ? __ldg(args.a_scale) * __ldg(args.w_scale + t.e) : 1.0f;
+      const float sc = f8 ? __ldg(args.a_scale) * __ldg(args.w_scale + t.e) : 1.0f;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int c_end = min(t.ntok, hsel * SPAN + SPAN);
       for (int c0 = hsel * SPAN; c0 < c_end; c0 += 32) {
@@ -473,11 +546,16 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             float x = __uint_as_float(v[j]);
-            if (kFp8) x *= sc;
-            if (kGelu) x = gelu_erf(x);
+            if (f8) x *= sc;
+            if (gelu) x = gelu_erf(x);
             if (j < jmax) col[(size_t)j * N] = to_bf16_bits(x);
           }
         }
+      }
+      if (kFused && !p1) {  // publish this warp's part of H for GEMM-2's tiles
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(args.ready + block_of(t), 1u);
       }
       tc_fence_before_sync();
       __syncwarp();
@@ -548,15 +626,16 @@ struct KernelSlot {
   cudaError_t err = cudaSuccess;
   int max_clusters = 0;  // co-resident clusters (pairs) or CTAs of this kernel
 };
-static KernelSlot g_slots[64][16];
+static KernelSlot g_slots[64][32];
 
-template <bool kGelu, int kPair, bool kFp8, bool kGather>
+template <bool kGelu, int kPair, bool kFp8, bool kGather, bool kFused = false>
 static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                                   const CUtensorMap& tm_xw, const gg::Args& args, long long max_tiles, const DeviceInfo& dev,
-                                  cudaStream_t stream) {
-  auto kern = gg::grouped_gemm_kernel<kGelu, kPair, kFp8, kGather>;
+                                  cudaStream_t stream, const CUtensorMap* tm2 = nullptr) {
+  auto kern = gg::grouped_gemm_kernel<kGelu, kPair, kFp8, kGather, kFused>;
   const size_t smem_max = gg::kSmemBudget;  // one attribute for every E
-  const int slot = (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0) + (kFp8 ? 4 : 0) + (kGather ? 8 : 0);
+  const int slot =
+      (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0) + (kFp8 ? 4 : 0) + (kGather ? 8 : 0) + (kFused ? 16 : 0);
   KernelSlot& ks = g_slots[dev.device & 63][slot];
   std::call_once(ks.once, [&] {
     ks.err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
@@ -595,7 +674,11 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, tm_xw, args);
+  // the fused form's GEMM-2 maps; the other forms pass copies they never read
+  const CUtensorMap& w2 = tm2 ? tm2[0] : tm_w;
+  const CUtensorMap& x2 = tm2 ? tm2[1] : tm_x;
+  const CUtensorMap& xw2 = tm2 ? tm2[2] : tm_xw;
+  return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, tm_xw, w2, x2, xw2, args);
 }
 
 // Gather form: A is the token matrix [a_rows, K] and row r of the GEMM reads
@@ -621,7 +704,7 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
              !make_map(&tm_xw, A, (uint64_t)R, (uint64_t)K, gg::B_WIDE_ROWS, kFp8, err)) {
     return cudaErrorInvalidValue;
   }
-  gg::Args args;
+  gg::Args args = {};
   args.offsets = offsets;
   args.out = static_cast<uint16_t*>(out);
   args.status = dev.status;
@@ -665,6 +748,64 @@ cudaError_t launch_grouped_gemm_fp8(const void* Aq, const float* a_scale, const 
                                     cudaStream_t stream, std::string* err) {
   return launch_gemm<true>(Aq, a_scale, nullptr, 1, R, offsets, Wq, w_scale, E, R, N, K, gelu,
                            out, dev, stream, err);
+}
+
+// Fused FFN: H = act(A W1[e]^T) (A = Xe, bf16 or E4M3 codes), then
+// Ye = H W2[e]^T, in one persistent launch.  `ready` holds one counter per
+// token block (ffn_ready_count) and is zeroed here before the launch.
+int ffn_ready_count(int R, int E) { return (R + gg::BN - 1) / gg::BN + E; }
+
+cudaError_t launch_fused_ffn(const void* A, const float* a_scale, const int32_t* offsets,
+                             const void* W1, const float* w1_scale, const void* W2, int E, int R,
+                             int d, int f, bool fp8, void* H, void* Ye, uint32_t* ready,
+                             const DeviceInfo& dev, cudaStream_t stream, std::string* err) {
+  if (R == 0) return cudaSuccess;
+  cudaError_t e = cudaMemsetAsync(ready, 0, (size_t)ffn_ready_count(R, E) * sizeof(uint32_t),
+                                  stream);
+  if (e != cudaSuccess) return e;
+  // one pair setting for both phases: paired CTAs when both GEMMs are wide enough
+  const int pair = (f > gg::BM && d > gg::BM) ? 2 : 1;
+  CUtensorMap tm_w, tm_x, tm_xw, tm2[3];
+  if (!make_map(&tm_w, W1, (uint64_t)E * (uint64_t)f, (uint64_t)d, gg::BM, fp8, err) ||
+      !make_map(&tm_x, A, (uint64_t)R, (uint64_t)d, gg::B_BOX_ROWS, fp8, err) ||
+      !make_map(&tm_xw, A, (uint64_t)R, (uint64_t)d, gg::B_WIDE_ROWS, fp8, err) ||
+      !make_map(&tm2[0], W2, (uint64_t)E * (uint64_t)d, (uint64_t)f, gg::BM, false, err) ||
+      !make_map(&tm2[1], H, (uint64_t)R, (uint64_t)f, gg::B_BOX_ROWS, false, err) ||
+      !make_map(&tm2[2], H, (uint64_t)R, (uint64_t)f, gg::B_WIDE_ROWS, false, err))
+    return cudaErrorInvalidValue;
+  gg::Args args = {};
+  args.offsets = offsets;
+  args.out = static_cast<uint16_t*>(H);
+  args.status = dev.status;
+  args.a_scale = a_scale;
+  args.w_scale = w1_scale;
+  args.gather_k = 1;
+  args.a_rows = R;
+  args.E = E;
+  args.R = R;
+  args.N = f;
+  args.K = d;
+  args.n_fblocks = (f + gg::BM * pair - 1) / (gg::BM * pair);
+  const int kb1 = fp8 ? gg::BK_FP8 : gg::BK;
+  args.num_kb = (d + kb1 - 1) / kb1;
+  args.out2 = static_cast<uint16_t*>(Ye);
+  args.N2 = d;
+  args.n_fblocks2 = (d + gg::BM * pair - 1) / (gg::BM * pair);
+  args.num_kb2 = (f + gg::BK - 1) / gg::BK;
+  args.ready = ready;
+  args.ready_target = (uint32_t)(args.n_fblocks * pair * gg::EPI_WARPS);
+  args.stages = pair == 2 ? gg::stages_for<2>(E) : gg::stages_for<1>(E);
+  const long long max_tiles = ((long long)(R + gg::BN - 1) / gg::BN + E) *
+                              (long long)(args.n_fblocks + args.n_fblocks2);
+  if (fp8)
+    return pair == 2 ? launch_variant<true, 2, true, false, true>(tm_w, tm_x, tm_xw, args, max_tiles,
+                                                                  dev, stream, tm2)
+                     : launch_variant<true, 1, true, false, true>(tm_w, tm_x, tm_xw, args, max_tiles,
+                                                                  dev, stream, tm2);
+  return pair == 2 ? launch_variant<true, 2, false, false, true>(tm_w, tm_x, tm_xw, args, max_tiles,
+                                                                 dev, stream, tm2)
+                   : launch_variant<true, 1, false, false, true>(tm_w, tm_x, tm_xw, args, max_tiles,
+                                                                 dev, stream, tm2);
 }
 
 cudaError_t launch_grouped_gemm_gather(const void* X, const float* x_scale, const int32_t* src_of,

@@ -64,6 +64,14 @@ cudaError_t launch_grouped_gemm_gather(const void* X, const float* x_scale, cons
                                        const float* w_scale, int E, int N, int K, bool gelu,
                                        bool fp8, void* out, const DeviceInfo& dev,
                                        cudaStream_t stream, std::string* err);
+// Fused FFN (GEMM-1 + GELU, then GEMM-2) in one persistent launch; A is Xe
+// (bf16) or E4M3 codes with scale a_scale[0] and per-expert w1_scale (fp8).
+// `ready`: ffn_ready_count(R, E) counters of scratch, zeroed by the launcher.
+int ffn_ready_count(int R, int E);
+cudaError_t launch_fused_ffn(const void* A, const float* a_scale, const int32_t* offsets,
+                             const void* W1, const float* w1_scale, const void* W2, int E, int R,
+                             int d, int f, bool fp8, void* H, void* Ye, uint32_t* ready,
+                             const DeviceInfo& dev, cudaStream_t stream, std::string* err);
 // Per-tensor E4M3 quantisation of n bf16 values (n % 8 == 0): x_scale = [scale, amax].
 cudaError_t launch_quantize_tensor(const void* X, int64_t n, void* Xq, float* x_scale,
                                    const DeviceInfo& dev, cudaStream_t stream);

@@ -71,6 +71,9 @@ typedef enum moe_score {
 #define MOE_LAYER_GATHER_ON_LOAD 0x1 /* GEMM-1 reads token rows through src_of (TMA gather4)
                                         instead of a dispatched copy; see
                                         moe_expert_gemm_gather.  Same results, bit for bit. */
+#define MOE_LAYER_FUSED_FFN 0x2      /* GEMM-1 and GEMM-2 in one persistent launch; see
+                                        moe_expert_ffn_fused.  Same results, bit for bit.
+                                        Not combinable with MOE_LAYER_GATHER_ON_LOAD. */
 
 /* Shape and routing recipe of one layer. */
 typedef struct moe_layer_desc {
@@ -220,6 +223,29 @@ moe_status moe_expert_ffn(const void* Xe, const int32_t* offsets, const void* W1
                           void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_expert_ffn_fused -- moe_expert_ffn as ONE persistent kernel (the GEMM
+ * part of the token-centric pipeline in the DySHARP review §3.2: GEMM-2
+ * work on a block of tokens starts as soon as GEMM-1 has produced that
+ * block's H, with no kernel boundary in between).
+ *   Same arguments and results as moe_expert_ffn (bitwise), plus scratch:
+ *   ws of at least moe_expert_ffn_fused_workspace_size(E, R) bytes holding
+ *   one readiness counter per 256-row token block (zeroed by the call).
+ *   Every device wait is bounded; a timeout sets MOE_DEV_TIMEOUT.
+ * moe_expert_ffn_fused_fp8 -- the same with GEMM-1 on E4M3 operands
+ *   (Xeq, x_scale from moe_dispatch_fp8; W1q, w1_scale from
+ *   moe_quantize_experts_fp8); GEMM-2 stays bf16.  d % 16 == 0.
+ * ------------------------------------------------------------------------- */
+size_t moe_expert_ffn_fused_workspace_size(int32_t E, int32_t R);
+moe_status moe_expert_ffn_fused(const void* Xe, const int32_t* offsets, const void* W1,
+                                const void* W2, int32_t E, int32_t R, int32_t d, int32_t f,
+                                void* H, void* Ye, void* ws, size_t ws_bytes, void* stream);
+moe_status moe_expert_ffn_fused_fp8(const void* Xeq, const float* x_scale,
+                                    const int32_t* offsets, const void* W1q,
+                                    const float* w1_scale, const void* W2, int32_t E, int32_t R,
+                                    int32_t d, int32_t f, void* H, void* Ye, void* ws,
+                                    size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_combine -- gate-weighted reduction of each token's k expert outputs
  * (DySHARP §1: the k results are summed into one; ThunderEP §2.1: the gate
  * values weight the combine sum).
@@ -240,6 +266,8 @@ moe_status moe_combine(const void* Ye, const int32_t* row_of, const float* gates
  *   topk_idx_out [T, k], gates_out [T, k], counts_out [E]: optional copies
  *   of the routing (NULL to skip).
  *   ws: at least moe_workspace_size(desc) bytes.
+ *   desc->flags & MOE_LAYER_FUSED_FFN runs both expert GEMMs as one persistent
+ *   kernel (moe_expert_ffn_fused); the output is identical.
  *   desc->flags & MOE_LAYER_GATHER_ON_LOAD fuses the dispatch into GEMM-1
  *   (no dispatch kernel, no dispatched copy of X); the output is identical.
  *   On a B200 it is slower than the default for every shape measured (the

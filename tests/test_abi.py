@@ -139,3 +139,22 @@ def test_fp8_calls_check_on_the_host(lib):
                                      N) == UNSUPPORTED
     # the quantising dispatch adds one kernel (the absmax reduction)
     assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(d), 1) == 8
+
+
+def test_fused_ffn_checks_on_the_host(lib):
+    p = ctypes.c_void_p(0x10000)
+    need = lib.moe_expert_ffn_fused_workspace_size(8, 8192)
+    assert need >= (8192 // 256 + 8) * 4
+    assert lib.moe_expert_ffn_fused(p, p, p, p, 8, 8192, 4096, 14336, p, p, p, need - 1,
+                                    N) == INVALID
+    assert "workspace" in _err(lib)
+    assert lib.moe_expert_ffn_fused_fp8(p, p, p, p, p, p, 8, 64, 72, 256, p, p, p, need,
+                                        N) == UNSUPPORTED                 # d % 16 for FP8
+    both = moe.LayerDesc(64, 128, 8, 2, 256, 0, 1,
+                         moe.LAYER_GATHER_ON_LOAD | moe.LAYER_FUSED_FFN)
+    ws = lib.moe_workspace_size(ctypes.byref(moe.LayerDesc(64, 128, 8, 2, 256, 0, 1, 0)))
+    assert lib.moe_layer_forward(ctypes.byref(both), p, p, N, p, p, p, N, N, N, p, ws,
+                                 N) == UNSUPPORTED
+    fused = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, moe.LAYER_FUSED_FFN)
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(fused), 1) == 6  # one GEMM launch
+    assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(fused), 1) == 7

@@ -307,6 +307,16 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                      bar) : "memory");
 }
 
+// One commit whose arrival lands on the mbarrier at the same shared-memory
+// offset in both CTAs of a pair (CTA mask 0b11): half the commits of one per
+// CTA.  Each tcgen05.commit costs MMA issue throughput (measured: two extra
+// commits per 128-byte K-block slow the grouped GEMM by 5-17%).
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar_local) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+      "[%0], %1;" ::"r"(bar_local), "h"((uint16_t)3) : "memory");
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate (kind::f16).
 // With kPair == 2 the instruction (issued by the leader CTA) reads A and B
 // from both CTAs' shared memory at the same offsets and writes both CTAs'

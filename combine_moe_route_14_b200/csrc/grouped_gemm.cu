@@ -26,8 +26,12 @@
 //     time (a multiple of 16), so a ragged expert block of c rows costs
 //     ceil(c/16)*16 columns of MMA work instead of a full 128-row tile.
 //   * warps 0 and 1 (one lane each) stream 128-byte K-blocks of the weight and
-//     the token operand through a ring of 6-7 stages (as many as shared
-//     memory holds) with TMA (128-byte swizzle),
+//     the token operand with TMA (128-byte swizzle) through a ring of 3
+//     slots of KPS = 2 K-blocks each (paired CTAs; as many as shared memory
+//     holds; one K-block per slot in 4 slots with a single CTA): one
+//     barrier round trip and one MMA commit per two K-blocks (each commit
+//     costs MMA issue throughput; measured 8% faster than one K-block per
+//     slot in 7 slots, despite one K-block less in flight),
 //     warp 2 (one lane) issues tcgen05.mma into one of two TMEM
 //     accumulators (2 x 256 fp32 columns), warps 3-10 drain the
 //     other accumulator (tcgen05.ld), apply GELU, round to bf16 and store
@@ -103,7 +107,10 @@ constexpr uint64_t kDrainLimitNs = 20ull * 1000ull * 1000ull;  // 20 ms
 //   and L2 reads per FLOP are a third lower, and 6 stages fit.
 template <int kPair> struct Cfg {
   static constexpr int B_STAGE = (BN / kPair) * BK * 2;  // token rows this CTA stages
-  static constexpr int STAGE = A_STAGE + B_STAGE;
+  // K-blocks per ring slot: two with paired CTAs (3 slots of 64 KB), one with
+  // a single CTA (its 48 KB K-block already leaves only 4 slots)
+  static constexpr int KPS = kPair == 2 ? 2 : 1;
+  static constexpr int STAGE = KPS * (A_STAGE + B_STAGE);  // one ring slot
   static constexpr int NUM_BARS = 2 * MAX_STAGES + 4 + 1;
   static constexpr int FEAT = BM * kPair;                // output features per tile
 };
@@ -137,7 +144,7 @@ struct Args {
   int E, R, N, K;
   int n_fblocks;           // ceil(N / features per tile)
   int num_kb;              // ceil(K / K-values per stage)
-  int stages;              // ring depth (<= MAX_STAGES)
+  int stages;              // ring slots of KPS K-blocks (<= MAX_STAGES)
   // fused FFN form: phase 1 = GEMM-2 over phase 0's output (A = out)
   uint16_t* out2;          // [R, N2] bf16
   int N2, n_fblocks2, num_kb2;
@@ -216,6 +223,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
                         const __grid_constant__ CUtensorMap tm_xw2, const Args args) {
   using C = Cfg<kPair>;
   using Ro = Roles<kGather>;
+  constexpr int KPS = C::KPS;
   constexpr int KB = kFp8 ? BK_FP8 : BK;  // K values per stage (128 bytes of a row)
   const int STAGES = args.stages;
   constexpr int B_STAGE = C::B_STAGE;
@@ -223,8 +231,8 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = sA + STAGES * A_STAGE;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  uint8_t* sB = sA + STAGES * KPS * A_STAGE;  // slot s, K-block h: sA + (s*KPS + h)*A_STAGE
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * KPS * B_STAGE);
   uint64_t* full = bars;                   // used in the leader CTA: both CTAs' bytes land here
   uint64_t* empty = bars + MAX_STAGES;     // per CTA: the MMAs have read this stage
   uint64_t* tfull = bars + 2 * MAX_STAGES; // per CTA: accumulator ready
@@ -404,30 +412,41 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
         }
       }
       const uint32_t gbytes = (uint32_t)(kPair * half * 128);
-      for (int kb = 0; kb < nkb; ++kb) {
+      for (int ks = 0; ks * KPS < nkb; ++ks) {  // ring slot of K-blocks ks*KPS ..
+        const int nsub = min(KPS, nkb - ks * KPS);
         ok = warp_wait(&empty[s], ph ^ 1u, args.status, s_abort);
         if (!ok) break;
         if (kGather && !is_w) {
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
-          if (tw == 0 && lane == 0 && rank == 0) mbar_arrive_expect_tx(&full[s], gbytes);
+          if (tw == 0 && lane == 0 && rank == 0)
+            mbar_arrive_expect_tx(&full[s], gbytes * (uint32_t)nsub);
+          for (int hh = 0; hh < nsub; ++hh) {
+            const int kb = ks * KPS + hh;
+            uint8_t* dst = sB + (s * KPS + hh) * B_STAGE;
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int q = (lane + 32 * h) * Ro::NTOK + tw;
-            if (q < nreq)
-              tma_gather4_cg<kPair>(sB + s * B_STAGE + q * 512, &tm_x, kb * KB, g[h][0], g[h][1],
-                                    g[h][2], g[h][3], fb_addr, pol);
+            for (int h = 0; h < 2; ++h) {
+              const int q = (lane + 32 * h) * Ro::NTOK + tw;
+              if (q < nreq)
+                tma_gather4_cg<kPair>(dst + q * 512, &tm_x, kb * KB, g[h][0], g[h][1], g[h][2],
+                                      g[h][3], fb_addr, pol);
+            }
           }
         } else if (lane == 0) {
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
-          if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes);
-          if (is_w) {
-            tma_load_2d_cg<kPair>(sA + s * A_STAGE, map_w, kb * kbv, wy, fb_addr, pol);
-          } else if (wide) {  // (nearly) a full half-tile: one large request
-            tma_load_2d_cg<kPair>(sB + s * B_STAGE, map_xw, kb * kbv, by, fb_addr, pol);
-          } else {
-            for (int j = 0; j < nbox; ++j)
-              tma_load_2d_cg<kPair>(sB + s * B_STAGE + j * B_BOX, map_x, kb * kbv,
-                                    by + j * B_BOX_ROWS, fb_addr, pol);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)nsub);
+          for (int hh = 0; hh < nsub; ++hh) {
+            const int kb = ks * KPS + hh;
+            if (is_w) {
+              tma_load_2d_cg<kPair>(sA + (s * KPS + hh) * A_STAGE, map_w, kb * kbv, wy, fb_addr,
+                                    pol);
+            } else if (wide) {  // (nearly) a full half-tile: one large request
+              tma_load_2d_cg<kPair>(sB + (s * KPS + hh) * B_STAGE, map_xw, kb * kbv, by, fb_addr,
+                                    pol);
+            } else {
+              for (int j = 0; j < nbox; ++j)
+                tma_load_2d_cg<kPair>(sB + (s * KPS + hh) * B_STAGE + j * B_BOX, map_x, kb * kbv,
+                                      by + j * B_BOX_ROWS, fb_addr, pol);
+            }
           }
         }
         __syncwarp();
@@ -448,8 +467,6 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
   } else if (warp == Ro::MMA) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (rank == 0) {
-      const uint32_t empty_peer = kPair == 2 ? cluster_map(smem_u32(empty), 1) : 0u;
-      const uint32_t tfull_peer = kPair == 2 ? cluster_map(smem_u32(tfull), 1) : 0u;
       int s = 0;
       uint32_t ph = 0;
       int it = 0;
@@ -469,25 +486,29 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
         if (!ok) break;
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int ks = 0; ks * KPS < nkb; ++ks) {
+          const int nsub = min(KPS, nkb - ks * KPS);
           ok = warp_wait(&full[s], ph, args.status, s_abort);
           if (!ok) break;
           tc_fence_after_sync();
           if (lane == 0) {
-            const uint32_t a0 = smem_u32(sA + s * A_STAGE);
-            const uint32_t b0 = smem_u32(sB + s * B_STAGE);
+            for (int hh = 0; hh < nsub; ++hh) {
+              const int kb = ks * KPS + hh;
+              const uint32_t a0 = smem_u32(sA + (s * KPS + hh) * A_STAGE);
+              const uint32_t b0 = smem_u32(sB + (s * KPS + hh) * B_STAGE);
 #pragma unroll
-            for (int kk = 0; kk < 128 / UMMA_K_BYTES; ++kk) {
-              const uint64_t ad = smem_desc_k128(a0 + kk * UMMA_K_BYTES);
-              const uint64_t bd = smem_desc_k128(b0 + kk * UMMA_K_BYTES);
-              if (f8)
-                tc_mma_e4m3<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-              else
-                tc_mma_bf16<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              for (int kk = 0; kk < 128 / UMMA_K_BYTES; ++kk) {
+                const uint64_t ad = smem_desc_k128(a0 + kk * UMMA_K_BYTES);
+                const uint64_t bd = smem_desc_k128(b0 + kk * UMMA_K_BYTES);
+                if (f8)
+                  tc_mma_e4m3<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                else
+                  tc_mma_bf16<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+              }
             }
             // the stage is free (in both CTAs) once these MMAs have read it
-            tc_commit<kPair>(smem_u32(&empty[s]));
-            if (kPair == 2) tc_commit<kPair>(empty_peer + (uint32_t)s * 8u);
+            if (kPair == 2) tc_commit_pair(smem_u32(&empty[s]));
+            else tc_commit<kPair>(smem_u32(&empty[s]));
           }
           __syncwarp();
           if (++s == STAGES) {
@@ -497,8 +518,8 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
         }
         if (!ok) break;
         if (lane == 0) {  // accumulator complete, in both CTAs
-          tc_commit<kPair>(smem_u32(&tfull[acc]));
-          if (kPair == 2) tc_commit<kPair>(tfull_peer + (uint32_t)acc * 8u);
+          if (kPair == 2) tc_commit_pair(smem_u32(&tfull[acc]));
+          else tc_commit<kPair>(smem_u32(&tfull[acc]));
         }
         __syncwarp();
       }

@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   const uint32_t rank = kPair == 2 ? cluster_ctarank() : 0u;  // 0 = MMA leader
   const int cid = blockIdx.x / kPair;                          // tile-scheduling unit
-  const int ncl = gridDim.x / kPair;
+  const int ncl_launched = gridDim.x / kPair;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -324,6 +324,15 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
   const uint32_t tmem_base = *s_tmem;
   const int tiles0 = s_start[E];
   const int total_tiles = tiles0 + (kFused ? s_start2[E] : 0);
+  // Balanced grid: the fewest clusters that still need the same number of
+  // rounds of the static schedule (the tile count is known only here, from
+  // the routing).  A last round with a few busy clusters would otherwise set
+  // the kernel's time while most SMs idle; e.g. 448 tiles over 74 clusters
+  // run 6 full rounds and a seventh of 4 tiles, over 64 clusters 7 full
+  // rounds.  Surplus clusters take no tile.
+  const int rounds = (total_tiles + ncl_launched - 1) / max(ncl_launched, 1);
+  const int ncl = rounds > 0 ? (total_tiles + rounds - 1) / rounds : ncl_launched;
+  const int first_tile = cid < ncl ? cid : total_tiles;
   // tile -> (tile, phase); phase 1 only in the fused form
   auto tile_at = [&](int tile, int& phase) -> Tile {
     if (kFused && tile >= tiles0) {
@@ -357,10 +366,20 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     uint32_t issued = 0;  // bit s: stage s has a load in flight or landed
     uint32_t last_ph = 0; // bit s: parity of the last load issued on stage s
     bool ok = true;
-    for (int tile = cid; ok && tile < total_tiles; tile += ncl) {
+    // fused form: the readiness count of this producer's next GEMM-2 tile,
+    // loaded (acquire) one tile ahead so that its L2 round trip overlaps the
+    // current tile's loads; counts only grow, so a count seen as complete stays so
+    uint32_t next_count = 0;
+    for (int tile = first_tile; ok && tile < total_tiles; tile += ncl) {
       int phase;
       const Tile t = tile_at(tile, phase);
       const bool p1 = kFused && phase == 1;
+      const uint32_t this_count = next_count;
+      if (kFused && !is_w && lane == 0 && tile + ncl < total_tiles) {
+        int nphase;
+        const Tile nt = tile_at(tile + ncl, nphase);
+        if (nphase == 1) next_count = ld_acquire_gpu(args.ready + block_of(nt));
+      }
       const CUtensorMap* map_w = p1 ? &tm_w2 : &tm_w;
       const CUtensorMap* map_x = p1 ? &tm_x2 : &tm_x;
       const CUtensorMap* map_xw = p1 ? &tm_xw2 : &tm_xw;
@@ -370,7 +389,8 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
       if (p1 && !is_w) {  // GEMM-2 reads H rows that GEMM-1 tiles of other CTAs store
         bool rdy = true;
         if (lane == 0) {
-          rdy = wait_count_geq(args.ready + block_of(t), args.ready_target, args.status, s_abort);
+          rdy = this_count >= args.ready_target ||
+                wait_count_geq(args.ready + block_of(t), args.ready_target, args.status, s_abort);
           if (rdy) fence_proxy_async_global();
         }
         if (!__shfl_sync(0xffffffffu, rdy, 0)) {
@@ -471,7 +491,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
       uint32_t ph = 0;
       int it = 0;
       bool ok = true;
-      for (int tile = cid; ok && tile < total_tiles; tile += ncl, ++it) {
+      for (int tile = first_tile; ok && tile < total_tiles; tile += ncl, ++it) {
         int phase;
         const Tile t = tile_at(tile, phase);
         const bool p1 = kFused && phase == 1;
@@ -537,7 +557,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     constexpr int SPAN = BN / (EPI_WARPS / 4);
     const int hsel = (warp - Ro::EPI0) >> 2;
     int it = 0;
-    for (int tile = cid; tile < total_tiles; tile += ncl, ++it) {
+    for (int tile = first_tile; tile < total_tiles; tile += ncl, ++it) {
       int phase;
       const Tile t = tile_at(tile, phase);
       const bool p1 = kFused && phase == 1;

@@ -16,127 +16,130 @@ namespace moe {
 // ---------------------------------------------------------------------------
 // router linear: L[t, e] = sum_c X[t, c] * Wr[e, c]   (fp32 accumulate)
 //
-// HBM-bound on X (T*d*2 bytes).  A CTA of 8 warps takes 16 tokens, two per
-// warp; each lane owns 16-byte slices (8 bf16) of the row and keeps
-// kUnroll slices of both tokens in flight before the FMAs.  Router weights
-// (E*d*2 bytes) are staged once per CTA in shared memory when they fit,
-// else read through L1.  Experts are processed in groups of 8 (one partial
-// sum per token and expert per lane), then reduced across the warp.
+// A GEMM with N = E (8 for the Mixtral shape): tensor-core mma.sync tiles of
+// 16 tokens x 8 experts x 16 K (bf16 in, fp32 accumulate) fit it exactly,
+// and it is bound by streaming X (T*d*2 bytes) from HBM.  A CTA of 8 warps
+// takes 16 tokens; the warps split K into 64-column chunks (warp w takes
+// chunks w, w+8, ...) and their partial 16 x E tiles are summed in shared
+// memory in warp order (deterministic).
+//
+// Operand loads use a K permutation shared by both operands: in a 64-column
+// chunk, the thread with q = lane % 4 loads columns [16q, 16q+16) of its two
+// token rows (lane / 4 and lane / 4 + 8) and of expert row lane / 4, as two
+// 16-byte vectors each (the four threads of a row read 128 contiguous
+// bytes).  MMA m of the chunk takes words 2m, 2m+1 of each: logical k-pair
+// (2q, 2q+1) is column 16q + 4m + {0, 1} and (2q+8, 2q+9) is 16q + 4m + {2, 3}
+// for A and B alike, so the 4 MMAs cover the chunk's 64 columns exactly once.
+// More than 64 experts are processed in groups of 8 n-tiles, re-reading X.
+// The X vectors of a warp's next chunk are loaded while the current chunk's
+// MMAs run (a warp walks nchunks / 8 chunks; for a handful of tokens, e.g.
+// decode, those loads would otherwise be serial round trips).
 // ---------------------------------------------------------------------------
 constexpr int kRouterWarps = 8;
-constexpr int kTokPerWarp = 2;
-constexpr int kRouterUnroll = 8;
-constexpr int kRouterSmemMax = 96 * 1024;
+constexpr int kRouterTok = 16;     // tokens per CTA (the MMA's M)
+constexpr int kRouterGroup = 8;    // n-tiles of 8 experts per pass
 
-__device__ __forceinline__ float dot8(const uint4& a, const uint4& b, float acc) {
-  acc = fmaf(bf16_lo(a.x), bf16_lo(b.x), acc);
-  acc = fmaf(bf16_hi(a.x), bf16_hi(b.x), acc);
-  acc = fmaf(bf16_lo(a.y), bf16_lo(b.y), acc);
-  acc = fmaf(bf16_hi(a.y), bf16_hi(b.y), acc);
-  acc = fmaf(bf16_lo(a.z), bf16_lo(b.z), acc);
-  acc = fmaf(bf16_hi(a.z), bf16_hi(b.z), acc);
-  acc = fmaf(bf16_lo(a.w), bf16_lo(b.w), acc);
-  acc = fmaf(bf16_hi(a.w), bf16_hi(b.w), acc);
-  return acc;
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <bool kSmemW>
+// 16 bytes at p (8 bf16) when the 8 values at column `col` exist, else zeros
+__device__ __forceinline__ uint4 ld_row_v4(const uint4* p, bool ok) {
+  return ok ? ld_stream_v4(p) : make_uint4(0u, 0u, 0u, 0u);
+}
+
 __global__ void __launch_bounds__(kRouterWarps * 32)
     router_logits_kernel(const uint4* __restrict__ X, const uint4* __restrict__ Wr, int T,
                          int row_vecs, int E, float* __restrict__ L) {
-  extern __shared__ uint4 s_w[];
-  if (kSmemW) {  // stage the weights: 8 loads in flight per thread before the stores
-    const int n = E * row_vecs;
-    constexpr int kBatch = 8;
-    for (int i0 = threadIdx.x; i0 < n; i0 += blockDim.x * kBatch) {
-      uint4 w[kBatch];
+  __shared__ float s_part[kRouterWarps][kRouterGroup][kRouterTok * 8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = lane >> 2, q = lane & 3;
+  const int t0 = blockIdx.x * kRouterTok;
+  const bool okA0 = t0 + r0 < T, okA1 = t0 + r0 + 8 < T;
+  const uint4* xa0 = X + (size_t)(okA0 ? t0 + r0 : 0) * row_vecs;
+  const uint4* xa1 = X + (size_t)(okA1 ? t0 + r0 + 8 : 0) * row_vecs;
+  const int nchunks = (row_vecs + 7) / 8;  // 64 columns = 8 vectors per chunk
+  const int ntiles = (E + 7) / 8;
+  for (int g0 = 0; g0 < ntiles; g0 += kRouterGroup) {
+    const int G = min(kRouterGroup, ntiles - g0);
+    float acc[kRouterGroup][4];
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int i = i0 + u * blockDim.x;
-        if (i < n) w[u] = __ldg(Wr + i);
+    for (int j = 0; j < kRouterGroup; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+    uint4 n00, n01, n10, n11;  // the next chunk's X vectors
+    {
+      const int v = warp * 8 + 2 * q;
+      const bool ok0 = warp < nchunks && v < row_vecs, ok1 = warp < nchunks && v + 1 < row_vecs;
+      n00 = ld_row_v4(xa0 + v, okA0 && ok0);
+      n01 = ld_row_v4(xa0 + v + 1, okA0 && ok1);
+      n10 = ld_row_v4(xa1 + v, okA1 && ok0);
+      n11 = ld_row_v4(xa1 + v + 1, okA1 && ok1);
+    }
+    for (int c = warp; c < nchunks; c += kRouterWarps) {
+      const int v = c * 8 + 2 * q;  // this thread's first vector of the chunk
+      const bool ok0 = v < row_vecs, ok1 = v + 1 < row_vecs;
+      const uint4 x00 = n00, x01 = n01, x10 = n10, x11 = n11;
+      {
+        const int cn = c + kRouterWarps, vn = cn * 8 + 2 * q;
+        const bool m0 = cn < nchunks && vn < row_vecs, m1 = cn < nchunks && vn + 1 < row_vecs;
+        n00 = ld_row_v4(xa0 + vn, okA0 && m0);
+        n01 = ld_row_v4(xa0 + vn + 1, okA0 && m1);
+        n10 = ld_row_v4(xa1 + vn, okA1 && m0);
+        n11 = ld_row_v4(xa1 + vn + 1, okA1 && m1);
       }
+      const uint32_t A0[8] = {x00.x, x00.y, x00.z, x00.w, x01.x, x01.y, x01.z, x01.w};
+      const uint32_t A1[8] = {x10.x, x10.y, x10.z, x10.w, x11.x, x11.y, x11.z, x11.w};
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int i = i0 + u * blockDim.x;
-        if (i < n) s_w[i] = w[u];
+      for (int j = 0; j < kRouterGroup; ++j) {
+        if (j < G) {
+          const int e = (g0 + j) * 8 + r0;
+          const bool okB = e < E;
+          const uint4* wr = Wr + (size_t)(okB ? e : 0) * row_vecs;
+          const uint4 w0 = okB && ok0 ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 w1 = okB && ok1 ? __ldg(wr + v + 1) : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t B[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+            mma_bf16_16816(acc[j], A0[2 * m], A1[2 * m], A0[2 * m + 1], A1[2 * m + 1], B[2 * m],
+                           B[2 * m + 1]);
+        }
+      }
+    }
+    // partial tile of this warp: c0,c1 = (row r0, experts 2q, 2q+1), c2,c3 = row r0 + 8
+#pragma unroll
+    for (int j = 0; j < kRouterGroup; ++j) {
+      if (j < G) {
+        float* p = s_part[warp][j];
+        p[r0 * 8 + 2 * q] = acc[j][0];
+        p[r0 * 8 + 2 * q + 1] = acc[j][1];
+        p[(r0 + 8) * 8 + 2 * q] = acc[j][2];
+        p[(r0 + 8) * 8 + 2 * q + 1] = acc[j][3];
       }
     }
     __syncthreads();
-  }
-  const uint4* W = kSmemW ? s_w : Wr;
-  const int lane = threadIdx.x & 31;
-  const int t0 = (blockIdx.x * kRouterWarps + (threadIdx.x >> 5)) * kTokPerWarp;
-  if (t0 >= T) return;
-  const bool two = t0 + 1 < T;
-  const uint4* x0 = X + (size_t)t0 * row_vecs;
-  const uint4* x1 = X + (size_t)(two ? t0 + 1 : t0) * row_vecs;
-  for (int e0 = 0; e0 < E; e0 += 8) {
-    const int ne = min(8, E - e0);
-    float acc0[8], acc1[8];
+    for (int i = threadIdx.x; i < G * kRouterTok * 8; i += blockDim.x) {
+      const int j = i / (kRouterTok * 8), rc = i % (kRouterTok * 8);
+      const int r = rc / 8, e = (g0 + j) * 8 + rc % 8;
+      float sum = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc0[j] = acc1[j] = 0.f;
-    for (int c0 = lane; c0 < row_vecs; c0 += 32 * kRouterUnroll) {
-      uint4 a[kRouterUnroll], b[kRouterUnroll];
-#pragma unroll
-      for (int u = 0; u < kRouterUnroll; ++u) {
-        const int c = c0 + u * 32;
-        if (c < row_vecs) {
-          a[u] = ld_stream_v4(x0 + c);
-          b[u] = ld_stream_v4(x1 + c);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < kRouterUnroll; ++u) {
-        const int c = c0 + u * 32;
-        if (c < row_vecs) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (j < ne) {
-              const uint4 w = kSmemW ? W[(size_t)(e0 + j) * row_vecs + c]
-                                     : __ldg(W + (size_t)(e0 + j) * row_vecs + c);
-              acc0[j] = dot8(a[u], w, acc0[j]);
-              acc1[j] = dot8(b[u], w, acc1[j]);
-            }
-          }
-        }
-      }
+      for (int w = 0; w < kRouterWarps; ++w) sum += s_part[w][j][rc];
+      if (t0 + r < T && e < E) L[(size_t)(t0 + r) * E + e] = sum;
     }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        acc0[j] += __shfl_xor_sync(0xffffffffu, acc0[j], off);
-        acc1[j] += __shfl_xor_sync(0xffffffffu, acc1[j], off);
-      }
-    }
-    // lane j < ne writes expert e0+j of token t0, lane 8+j of token t0+1
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (lane == j && j < ne) L[(size_t)t0 * E + e0 + j] = acc0[j];
-      if (two && lane == 8 + j && j < ne) L[(size_t)(t0 + 1) * E + e0 + j] = acc1[j];
-    }
+    __syncthreads();
   }
 }
 
 cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, int E, float* L,
                                  cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const int per_cta = kRouterWarps * kTokPerWarp;
-  const int blocks = (T + per_cta - 1) / per_cta;
-  const size_t wbytes = (size_t)E * d * 2;
-  const uint4* x = static_cast<const uint4*>(X);
-  const uint4* w = static_cast<const uint4*>(Wr);
-  if (wbytes <= (size_t)kRouterSmemMax) {
-    if (wbytes > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<true>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           kRouterSmemMax);
-      if (e != cudaSuccess) return e;
-    }
-    router_logits_kernel<true><<<blocks, kRouterWarps * 32, wbytes, stream>>>(x, w, T, d / 8, E, L);
-  } else {
-    router_logits_kernel<false><<<blocks, kRouterWarps * 32, 0, stream>>>(x, w, T, d / 8, E, L);
-  }
+  const int blocks = (T + kRouterTok - 1) / kRouterTok;
+  router_logits_kernel<<<blocks, kRouterWarps * 32, 0, stream>>>(
+      static_cast<const uint4*>(X), static_cast<const uint4*>(Wr), T, d / 8, E, L);
   return cudaGetLastError();
 }
 

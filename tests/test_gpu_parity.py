@@ -130,7 +130,8 @@ def test_route_ex_parity(T, E, k, score, renorm, temp, thr):
 # router linear
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("T,d,E", [(4096, 4096, 8), (16, 4096, 8), (300, 136, 3), (77, 512, 40),
-                                   (1, 8, 1)])
+                                   (1, 8, 1), (100, 256, 72), (33, 4104, 130), (8, 64, 1024),
+                                   (17, 72, 8)])
 def test_router_logits_parity(T, d, E):
     X = I.random_bf16((T, d), 1, "X")
     Wr = I.random_bf16((E, d), 1, "Wr", 0.02)

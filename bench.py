@@ -2,7 +2,7 @@
 """Benchmark: MoE-layer tokens/s on B200 (route -> layout -> dispatch -> expert FFN -> combine).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
-                    [--fp8] [--gather] [--fused]
+                    [--fp8] [--gather] [--fused] [--graph]
 
 One step = one full layer forward (every stage) over one batch of T tokens.
 Default workload: the Mixtral-shaped layer (T=4096, d=4096, E=8, top-2,
@@ -16,7 +16,9 @@ and FP8 GEMM-1; GEMM-2 and combine stay bf16); W1 is quantised once before
 timing.  ``--gather`` fuses the dispatch into GEMM-1 (rows read through the
 layout table with TMA gather4 loads; no dispatch kernel).  ``--fused`` runs
 both expert GEMMs as one persistent kernel (GEMM-2 starts per token block as
-soon as GEMM-1 has produced it).  Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+soon as GEMM-1 has produced it).  ``--graph`` also times the same forward
+captured once into a CUDA graph and replayed (launch overhead removed; the
+decode configurations' second figure).  Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 (the only reference this method has) on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -271,19 +273,55 @@ def run_ours(args, cfg, rank, world, local_rank):
     if bits:
         raise RuntimeError(f"device status bits {bits} after warm-up")
 
+    def step_percentiles(durs_ms):
+        a = np.asarray(durs_ms) * 1e3
+        return {"p10": float(np.percentile(a, 10)), "p50": float(np.percentile(a, 50)),
+                "p90": float(np.percentile(a, 90))}
+
+    graph_res = None
+    if args.graph:
+        # one forward captured on a side stream (per-device set-up already done
+        # by the warm-up), replayed W times untimed, then K times with events
+        gs = torch.cuda.Stream(device=dev)
+        gs.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gs):
+            with torch.cuda.graph(graph, stream=gs):
+                step()
+            for _ in range(args.warmup):
+                graph.replay()
+        gs.synchronize()
+        gev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        sync_all()
+        with torch.cuda.stream(gs):
+            gev[0].record(gs)
+            for i in range(args.steps):
+                graph.replay()
+                gev[i + 1].record(gs)
+        gs.synchronize()
+        sync_all()
+        g_ms = max_over_ranks(gev[0].elapsed_time(gev[-1]))
+        graph_res = {"value": Rp.weak_scaling_throughput(cfg.T, args.steps, world, g_ms),
+                     "ms_per_step": g_ms / args.steps,
+                     "step_us": step_percentiles([gev[i].elapsed_time(gev[i + 1])
+                                                  for i in range(args.steps)])}
+        del graph
+        torch.cuda.synchronize(dev)
+
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if sampler:
         sampler.__enter__()
     try:
         # ---- value: K whole-layer forwards, inputs resident in HBM
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        vev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
         sync_all()
-        e0.record(stream)
-        for _ in range(args.steps):
+        vev[0].record(stream)
+        for i in range(args.steps):
             step()
-        e1.record(stream)
+            vev[i + 1].record(stream)
         sync_all()
-        t_ms = max_over_ranks(e0.elapsed_time(e1))
+        t_ms = max_over_ranks(vev[0].elapsed_time(vev[-1]))
+        step_us = step_percentiles([vev[i].elapsed_time(vev[i + 1]) for i in range(args.steps)])
 
         # ---- per-stage times: the same kernels, launched stage by stage with events between
         stage_names = (["router_logits"] if Wr is not None else []) + [
@@ -436,7 +474,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     value = Rp.weak_scaling_throughput(cfg.T, args.steps, world, t_ms)
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
+        "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "step_us": step_us,
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 (dispatch, GEMM-1) + bf16" if args.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
@@ -461,6 +500,8 @@ def run_ours(args, cfg, rank, world, local_rank):
             Wr is not None),
         "clocks": clocks,
     }
+    if graph_res is not None:
+        res["graph"] = graph_res
     del X, logits, Wr, layer, inp, ws, Xe, H, Ye
     torch.cuda.empty_cache()
     return res
@@ -481,6 +522,8 @@ def main():
                     help="fuse the dispatch into GEMM-1 (gather-on-load)")
     ap.add_argument("--fused", action="store_true",
                     help="both expert GEMMs in one persistent kernel")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the forward replayed from a CUDA graph")
     args = ap.parse_args()
     if args.gather and args.fused:
         ap.error("--gather and --fused cannot be combined")

@@ -596,3 +596,8 @@ class MoeLayer:
             return moe_layer_forward_fp8(X, self.W1q, self.w1_scale, self.W2, self.k, self.score,
                                          self.renormalize, **kw)
         return moe_layer_forward(X, self.W1, self.W2, self.k, self.score, self.renormalize, **kw)
+
+
+from .pipeline import HostPipeline  # noqa: E402  (stream plumbing for host-buffer batches)
+
+__all__.append("HostPipeline")

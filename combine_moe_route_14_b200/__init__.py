@@ -28,6 +28,7 @@ __all__ = [
     "moe_layer_forward_fp8", "moe_kernel_launches_per_forward_fp8",
     "moe_quantize_fp8", "moe_expert_gemm_gather", "moe_expert_gemm_gather_fp8",
     "moe_expert_ffn_fused_workspace_size", "moe_expert_ffn_fused", "moe_expert_ffn_fused_fp8",
+    "moe_selftest_bounded_wait",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -87,6 +88,7 @@ _SIG = {
                                _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_kernel_launches_per_forward_fp8": ([ctypes.POINTER(LayerDesc), _I], ctypes.c_int32),
     "moe_quantize_fp8": ([_P, _I, _I, _P, _P, _P], ctypes.c_int),
+    "moe_selftest_bounded_wait": ([_I, ctypes.c_uint32, _P, _P], ctypes.c_int),
     "moe_expert_ffn_fused_workspace_size": ([_I, _I], ctypes.c_size_t),
     "moe_expert_ffn_fused": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, ctypes.c_size_t, _P],
                              ctypes.c_int),
@@ -550,6 +552,16 @@ def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=
                                      _ptr(topk_idx_out), _ptr(gates_out), _ptr(counts_out),
                                      _ptr(ws), ws.numel(), _stream(stream, dev)))
     return Y
+
+
+def moe_selftest_bounded_wait(which: int, limit_us: int, counter=None, stream=None):
+    """Run one bounded device wait that times out (0: global counter, 1: mbarrier)."""
+    lib = load_library()
+    dev = counter.device if counter is not None else torch.device("cuda", torch.cuda.current_device())
+    if counter is not None:
+        _need(counter, "counter", torch.int32, (1,), dev)
+    _check(lib.moe_selftest_bounded_wait(int(which), int(limit_us), _ptr(counter),
+                                         _stream(stream, dev)))
 
 
 def moe_device_status(clear: bool = True) -> int:

@@ -82,6 +82,10 @@ int fp8_dispatch_kernel_count(int64_t T);
 cudaError_t launch_quantize_experts(const void* W, int E, int64_t per_expert, void* Wq,
                                     float* scales, const DeviceInfo& dev, cudaStream_t stream);
 
+// Diagnostics: one bounded wait on a condition nothing satisfies (see selftest.cu).
+cudaError_t launch_selftest_wait(int which, uint64_t limit_ns, uint32_t* counter,
+                                 const DeviceInfo& dev, cudaStream_t stream);
+
 // Records `msg` as this thread's moe_last_error_string() and returns `status`.
 int set_last_error(int status, const std::string& msg);
 

@@ -379,6 +379,19 @@ moe_status moe_expert_gemm_gather_fp8(const void* Xq, const float* x_scale, cons
  *   linear (for launch accounting; memsets excluded).
  * ------------------------------------------------------------------------- */
 const char* moe_last_error_string(void);
+
+/* moe_selftest_bounded_wait -- runs one of the library's bounded device waits
+ * on a condition that nothing ever satisfies, so that a caller (or a test)
+ * can check the failure path without faulting or hanging the GPU: the wait
+ * gives up after limit_us microseconds, the kernel sets MOE_DEV_TIMEOUT in
+ * the status word and returns; read it with moe_device_status().
+ *   which = 0: the global-counter wait of the fused FFN (counter: a device
+ *              uint32 holding 0, which nothing increments; caller-owned);
+ *   which = 1: the shared-memory mbarrier wait of the grouped GEMM (counter
+ *              unused, may be NULL).
+ *   1 <= limit_us <= 10^7. */
+moe_status moe_selftest_bounded_wait(int32_t which, uint32_t limit_us, uint32_t* counter,
+                                     void* stream);
 moe_status moe_device_status(uint32_t* bits, int32_t clear);
 int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with_router);
 

@@ -350,8 +350,9 @@ def run_ours(args, cfg, rank, world, local_rank):
             "route": lambda: moe.moe_route_ex(L_buf, cfg.k, cfg.score, cfg.renormalize,
                                               cfg.temperature, cfg.min_prob, idx, g),
             "layout": lambda: moe.moe_layout(idx, cfg.E, counts, offs, row_of, src_of, lws),
-            "dispatch": (lambda: moe.moe_dispatch_fp8(X, src_of, cfg.k, Xe, xs)) if args.fp8 else
-                        (lambda: moe.moe_dispatch(X, src_of, cfg.k, Xe)),
+            # the layer's form: walked by token through row_of
+            "dispatch": (lambda: moe.moe_dispatch_fp8_by_token(X, row_of, cfg.k, Xe, xs))
+                        if args.fp8 else (lambda: moe.moe_dispatch_by_token(X, row_of, cfg.k, Xe)),
             "quantize": lambda: moe.moe_quantize_fp8(X, Xq, xs),
             "gemm1": ((lambda: moe.moe_expert_gemm_gather_fp8(Xq, xs, src_of, cfg.k, offs,
                                                               layer.W1q, layer.w1_scale, True, H))

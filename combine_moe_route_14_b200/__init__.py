@@ -28,7 +28,7 @@ __all__ = [
     "moe_layer_forward_fp8", "moe_kernel_launches_per_forward_fp8",
     "moe_quantize_fp8", "moe_expert_gemm_gather", "moe_expert_gemm_gather_fp8",
     "moe_expert_ffn_fused_workspace_size", "moe_expert_ffn_fused", "moe_expert_ffn_fused_fp8",
-    "moe_selftest_bounded_wait",
+    "moe_selftest_bounded_wait", "moe_dispatch_by_token", "moe_dispatch_fp8_by_token",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -72,6 +72,8 @@ _SIG = {
     "moe_layout": ([_P, _I, _I, _I, _P, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_layout_static": ([_P, _I, _I, _I, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_dispatch": ([_P, _P, _I, _I, _I, _P, _P], ctypes.c_int),
+    "moe_dispatch_by_token": ([_P, _P, _I, _I, _I, _P, _P], ctypes.c_int),
+    "moe_dispatch_fp8_by_token": ([_P, _P, _I, _I, _I, _P, _P, _P], ctypes.c_int),
     "moe_expert_gemm": ([_P, _P, _P, _I, _I, _I, _I, _I, _P, _P], ctypes.c_int),
     "moe_expert_ffn": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P], ctypes.c_int),
     "moe_combine": ([_P, _P, _P, _I, _I, _I, _P, _P], ctypes.c_int),
@@ -258,6 +260,32 @@ def moe_dispatch(X, src_of, k, Xe=None, stream=None):
     Xe = _out(Xe, "Xe", torch.bfloat16, (T * k, d), dev)
     _check(lib.moe_dispatch(_ptr(X), _ptr(src_of), T, d, k, _ptr(Xe), _stream(stream, dev)))
     return Xe
+
+
+def moe_dispatch_by_token(X, row_of, k, Xe=None, stream=None):
+    """moe_dispatch walked by token: Xe[row_of[t*k+j]] = X[t] (each token read once)."""
+    lib = load_library()
+    T, d = X.shape
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (T, d))
+    _need(row_of, "row_of", torch.int32, (T * k,), dev)
+    Xe = _out(Xe, "Xe", torch.bfloat16, (T * k, d), dev)
+    _check(lib.moe_dispatch_by_token(_ptr(X), _ptr(row_of), T, d, k, _ptr(Xe),
+                                     _stream(stream, dev)))
+    return Xe
+
+
+def moe_dispatch_fp8_by_token(X, row_of, k, Xeq=None, x_scale=None, stream=None):
+    lib = load_library()
+    T, d = X.shape
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (T, d))
+    _need(row_of, "row_of", torch.int32, (T * k,), dev)
+    Xeq = _out(Xeq, "Xeq", torch.uint8, (T * k, d), dev)
+    x_scale = _out(x_scale, "x_scale", torch.float32, (2,), dev)
+    _check(lib.moe_dispatch_fp8_by_token(_ptr(X), _ptr(row_of), T, d, k, _ptr(Xeq),
+                                         _ptr(x_scale), _stream(stream, dev)))
+    return Xeq, x_scale
 
 
 def moe_expert_gemm(A, offsets, W, gelu, out=None, stream=None):

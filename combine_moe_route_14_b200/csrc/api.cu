@@ -241,10 +241,10 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   const bool gather = (d.flags & MOE_LAYER_GATHER_ON_LOAD) != 0;
   if (d.flags & MOE_LAYER_FUSED_FFN) {  // both GEMMs in one persistent launch
     if (fp8)
-      MOE_CUDA(moe::launch_dispatch_fp8(X, src_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
+      MOE_CUDA(moe::launch_dispatch_fp8_rows(X, row_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
                "dispatch_fp8");
     else
-      MOE_CUDA(moe::launch_dispatch(X, src_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+      MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
     e = moe::launch_fused_ffn(Xe, x_scale, offsets, W1, W1s, W2, d.E, R, d.d, d.f, fp8, H, Ye,
                               ready, *dev, s, &err);
     if (e != cudaSuccess) return gemm_fail(e, err, "fused_ffn");
@@ -261,11 +261,12 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
     e = moe::launch_grouped_gemm_gather(A, x_scale, src_of, d.T, d.k, offsets, W1, W1s, d.E, d.f,
                                         d.d, true, fp8, H, *dev, s, &err);
   } else if (fp8) {
-    MOE_CUDA(moe::launch_dispatch_fp8(X, src_of, d.T, d.d, d.k, Xe, x_scale, *dev, s), "dispatch_fp8");
+    MOE_CUDA(moe::launch_dispatch_fp8_rows(X, row_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
+             "dispatch_fp8");
     e = moe::launch_grouped_gemm_fp8(Xe, x_scale, offsets, W1, W1s, d.E, R, d.f, d.d, true, H,
                                      *dev, s, &err);
   } else {
-    MOE_CUDA(moe::launch_dispatch(X, src_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+    MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
     e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err);
   }
   if (e != cudaSuccess) return gemm_fail(e, err, "gemm1");
@@ -402,6 +403,44 @@ moe_status moe_dispatch(const void* X, const int32_t* src_of, int32_t T, int32_t
   const moe::DeviceInfo* dev;
   MOE_TRY(get_dev(&dev));
   MOE_CUDA(moe::launch_dispatch(X, src_of, T, d, k, Xe, *dev, as_stream(stream)), "dispatch");
+  return MOE_OK;
+}
+
+moe_status moe_dispatch_by_token(const void* X, const int32_t* row_of, int32_t T, int32_t d,
+                                 int32_t k, void* Xe, void* stream) {
+  if (T < 0 || k < 1) return fail(MOE_ERR_INVALID_ARG, "need T >= 0 and k >= 1");
+  if (k > moe::kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k > 16 is not supported");
+  if ((int64_t)T * k >= (1ll << 30)) return fail(MOE_ERR_UNSUPPORTED, "T*k must be < 2^30");
+  MOE_TRY(check_dim(d, "d"));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr(X, "X"));
+  MOE_TRY(check_ptr4(row_of, "row_of"));
+  MOE_TRY(check_ptr(Xe, "Xe"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(moe::launch_dispatch_rows(X, row_of, T, d, k, Xe, *dev, as_stream(stream)),
+           "dispatch_by_token");
+  return MOE_OK;
+}
+
+moe_status moe_dispatch_fp8_by_token(const void* X, const int32_t* row_of, int32_t T, int32_t d,
+                                     int32_t k, void* Xeq, float* x_scale, void* stream) {
+  if (T < 0 || k < 1) return fail(MOE_ERR_INVALID_ARG, "need T >= 0 and k >= 1");
+  if (k > moe::kMaxTopK) return fail(MOE_ERR_UNSUPPORTED, "k > 16 is not supported");
+  if ((int64_t)T * k >= (1ll << 30)) return fail(MOE_ERR_UNSUPPORTED, "T*k must be < 2^30");
+  MOE_TRY(check_dim(d, "d"));
+  MOE_TRY(check_fp8_dim(d, "d"));
+  MOE_TRY(check_ptr4(x_scale, "x_scale"));
+  if (T > 0) {
+    MOE_TRY(check_ptr(X, "X"));
+    MOE_TRY(check_ptr4(row_of, "row_of"));
+    MOE_TRY(check_ptr(Xeq, "Xeq"));
+  }
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(moe::launch_dispatch_fp8_rows(X, row_of, T, d, k, Xeq, x_scale, *dev,
+                                         as_stream(stream)),
+           "dispatch_fp8_by_token");
   return MOE_OK;
 }
 

@@ -48,6 +48,48 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
   }
 }
 
+// Token-ordered dispatch: Xe[row_of[t*k + j], :] = X[t, :] for each kept slot j.
+// Each token row is read from HBM once and written to its k rows; the
+// row-ordered form above reads X[t] once per slot, which goes back to HBM
+// k times when X does not stay in L2 (8192 x 7168 bf16 tokens with k = 8:
+// 117 MB read 8 times beside a 940 MB write stream).
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    dispatch_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ row_of, int T,
+                         int k, int R, int row_vecs, uint4* __restrict__ Xe, uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * kGatherWarps;
+  for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
+    int my_row = -1;  // lane j < k: the row of slot j (-1: dropped)
+    if (lane < k) {
+      my_row = __ldg(row_of + (size_t)t * k + lane);
+      if (my_row < -1 || my_row >= R) {
+        flag_error(status, MOE_DEV_BAD_ROW);
+        my_row = -1;
+      }
+    }
+    const uint32_t live = __ballot_sync(0xffffffffu, lane < k && my_row >= 0);
+    if (!live) continue;
+    const uint4* src = X + (size_t)t * row_vecs;
+    for (int c0 = 0; c0 < row_vecs; c0 += 32 * kCopyUnroll) {
+      uint4 v[kCopyUnroll];
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_vecs) v[u] = ld_stream_v4(src + c);
+      }
+      for (uint32_t m = live; m; m &= m - 1) {
+        const int r = __shfl_sync(0xffffffffu, my_row, __ffs(m) - 1);
+        uint4* dst = Xe + (size_t)r * row_vecs;
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+          const int c = c0 + u * 32 + lane;
+          if (c < row_vecs) dst[c] = v[u];
+        }
+      }
+    }
+  }
+}
+
 // Y[t, :] = bf16( sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :] ), fp32 sum in slot order;
 // a dropped slot (row_of -1) contributes nothing.
 // kK > 0: k known at compile time; kK == 0: runtime k (<= kMaxTopK).
@@ -139,6 +181,15 @@ cudaError_t launch_dispatch(const void* X, const int32_t* src_of, int T, int d, 
   if (R == 0) return cudaSuccess;
   dispatch_kernel<<<gather_grid(R, dev), kGatherWarps * 32, 0, stream>>>(
       static_cast<const uint4*>(X), src_of, R, k, d / 8, static_cast<uint4*>(Xe), dev.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_rows(const void* X, const int32_t* row_of, int T, int d, int k,
+                                 void* Xe, const DeviceInfo& dev, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  dispatch_rows_kernel<<<gather_grid(T, dev), kGatherWarps * 32, 0, stream>>>(
+      static_cast<const uint4*>(X), row_of, T, k, T * k, d / 8, static_cast<uint4*>(Xe),
+      dev.status);
   return cudaGetLastError();
 }
 

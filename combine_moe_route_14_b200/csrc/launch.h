@@ -42,6 +42,13 @@ cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int
 cudaError_t launch_dispatch(const void* X, const int32_t* src_of, int T, int d, int k, void* Xe,
                             const DeviceInfo& dev, cudaStream_t stream);
 
+// Token-ordered dispatch through row_of (each token row read once).
+cudaError_t launch_dispatch_rows(const void* X, const int32_t* row_of, int T, int d, int k,
+                                 void* Xe, const DeviceInfo& dev, cudaStream_t stream);
+cudaError_t launch_dispatch_fp8_rows(const void* X, const int32_t* row_of, int T, int d, int k,
+                                     void* Xeq, float* x_scale, const DeviceInfo& dev,
+                                     cudaStream_t stream);
+
 cudaError_t launch_combine(const void* Ye, const int32_t* row_of, const float* gates, int T,
                            int d, int k, void* Y, const DeviceInfo& dev, cudaStream_t stream);
 

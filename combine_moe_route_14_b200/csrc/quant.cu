@@ -154,6 +154,50 @@ __global__ void __launch_bounds__(kDispWarps * 32)
   }
 }
 
+// Token-ordered form: Xeq[row_of[t*k + j], :] = E4M3(X[t, :] * inv(amax)) for
+// each kept slot j (each token read and quantised once, written k times).
+__global__ void __launch_bounds__(kDispWarps * 32)
+    dispatch_fp8_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ row_of,
+                             int T, int k, int row_vecs, float* x_scale, uint2* __restrict__ Xeq,
+                             uint32_t* status) {
+  const float amax = x_scale[1];
+  const float inv = inv_scale_of(amax);
+  if (blockIdx.x == 0 && threadIdx.x == 0) x_scale[0] = scale_of(amax);
+  const int R = T * k;
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * kDispWarps;
+  for (int t = blockIdx.x * kDispWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
+    int my_row = -1;
+    if (lane < k) {
+      my_row = __ldg(row_of + (size_t)t * k + lane);
+      if (my_row < -1 || my_row >= R) {
+        flag_error(status, MOE_DEV_BAD_ROW);
+        my_row = -1;
+      }
+    }
+    const uint32_t live = __ballot_sync(0xffffffffu, lane < k && my_row >= 0);
+    if (!live) continue;
+    const uint4* src = X + (size_t)t * row_vecs;
+    for (int c0 = 0; c0 < row_vecs; c0 += 32 * kDispUnroll) {
+      uint2 q[kDispUnroll];
+#pragma unroll
+      for (int u = 0; u < kDispUnroll; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_vecs) q[u] = quant8(ld_stream_v4(src + c), inv);
+      }
+      for (uint32_t m = live; m; m &= m - 1) {
+        const int r = __shfl_sync(0xffffffffu, my_row, __ffs(m) - 1);
+        uint2* dst = Xeq + (size_t)r * row_vecs;
+#pragma unroll
+        for (int u = 0; u < kDispUnroll; ++u) {
+          const int c = c0 + u * 32 + lane;
+          if (c < row_vecs) dst[c] = q[u];
+        }
+      }
+    }
+  }
+}
+
 static int stream_grid(size_t vecs, int groups, const DeviceInfo& dev) {
   const size_t need = (vecs + (size_t)kQThreads * kQUnroll - 1) / ((size_t)kQThreads * kQUnroll);
   const int cap = (dev.sm_count * 8 + groups - 1) / groups;  // ~8 CTAs of 256 threads per SM
@@ -208,6 +252,21 @@ cudaError_t launch_dispatch_fp8(const void* X, const int32_t* src_of, int T, int
   // R == 0 still runs one CTA so that x_scale[0] is written
   dispatch_fp8_kernel<<<grid, kDispWarps * 32, 0, stream>>>(
       static_cast<const uint4*>(X), src_of, R, k, d / 8, x_scale, static_cast<uint2*>(Xeq),
+      dev.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_fp8_rows(const void* X, const int32_t* row_of, int T, int d, int k,
+                                     void* Xeq, float* x_scale, const DeviceInfo& dev,
+                                     cudaStream_t stream) {
+  cudaError_t e = launch_amax(X, (size_t)T * d / 8, 1, x_scale + 1, dev, stream);
+  if (e != cudaSuccess) return e;
+  const int need = (T + kDispWarps - 1) / kDispWarps;
+  const int cap = dev.sm_count * 8;
+  const int grid = need < 1 ? 1 : (need < cap ? need : cap);
+  // T == 0 still runs one CTA so that x_scale[0] is written
+  dispatch_fp8_rows_kernel<<<grid, kDispWarps * 32, 0, stream>>>(
+      static_cast<const uint4*>(X), row_of, T, k, d / 8, x_scale, static_cast<uint2*>(Xeq),
       dev.status);
   return cudaGetLastError();
 }

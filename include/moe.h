@@ -198,6 +198,19 @@ moe_status moe_dispatch(const void* X, const int32_t* src_of, int32_t T, int32_t
                         void* Xe, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_dispatch_by_token -- the same copy as moe_dispatch, walked by token:
+ *   Xe[row_of[t*k + j], :] = X[t, :]   for every slot with row_of >= 0.
+ *   Each token row is read once and written to its k rows.  moe_dispatch walks
+ *   the rows instead and reads a token once per slot, which goes back to HBM
+ *   when X does not stay in L2 (many tokens, large k).  Rows no slot maps to
+ *   are left untouched; a row_of entry outside [-1, T*k) sets MOE_DEV_BAD_ROW
+ *   and is skipped.  moe_layer_forward uses this form.
+ *   X [T, d] bf16, row_of [T*k] int32 (from moe_layout), Xe [T*k, d] bf16.
+ * ------------------------------------------------------------------------- */
+moe_status moe_dispatch_by_token(const void* X, const int32_t* row_of, int32_t T, int32_t d,
+                                 int32_t k, void* Xe, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_expert_gemm -- one grouped expert linear layer over variable-size row
  * blocks (GPT-4 "2%" article §3.1 table: each expert is Linear -> GELU ->
  * Linear; DySHARP §3.2: GEMM-1 then GEMM-2 per expert).
@@ -325,6 +338,10 @@ moe_status moe_quantize_experts_fp8(const void* W, int32_t E, int32_t rows, int3
                                     void* Wq, float* scales, void* stream);
 moe_status moe_dispatch_fp8(const void* X, const int32_t* src_of, int32_t T, int32_t d,
                             int32_t k, void* Xeq, float* x_scale, void* stream);
+/* moe_dispatch_fp8_by_token: moe_dispatch_fp8 walked by token through row_of
+ * (see moe_dispatch_by_token); the same codes and x_scale. */
+moe_status moe_dispatch_fp8_by_token(const void* X, const int32_t* row_of, int32_t T, int32_t d,
+                                     int32_t k, void* Xeq, float* x_scale, void* stream);
 moe_status moe_expert_gemm_fp8(const void* Aq, const float* a_scale, const int32_t* offsets,
                                const void* Wq, const float* w_scale, int32_t E, int32_t R,
                                int32_t N, int32_t K, int32_t gelu, void* out, void* stream);

@@ -27,7 +27,8 @@ def declared_functions():
 
 def test_header_declares_the_layer_calls():
     names = declared_functions()
-    for n in ("moe_route", "moe_layout", "moe_dispatch", "moe_expert_ffn", "moe_combine",
+    for n in ("moe_route", "moe_layout", "moe_dispatch", "moe_dispatch_by_token",
+              "moe_expert_ffn", "moe_combine",
               "moe_layer_forward", "moe_router_logits", "moe_expert_gemm"):
         assert n in names
 

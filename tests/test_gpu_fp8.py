@@ -111,6 +111,15 @@ def test_dispatch_fp8_bit_exact(case):
     ok = src_of >= 0
     assert np.array_equal(got[ok], xq[src_of[ok] // k])
     assert (got[~ok] == 0xAB).all()  # unused rows untouched
+    # walked by token through row_of: the same codes and scale
+    _, _, row_of, _ = O.layout(idx, E)
+    Xt = torch.full((T * k, d), 0xAB, dtype=torch.uint8, device=DEV)
+    xs_t = torch.full((2,), -1.0, dtype=torch.float32, device=DEV)
+    moe.moe_dispatch_fp8_by_token(X, torch.from_numpy(row_of.astype(np.int32)).to(DEV), k,
+                                  Xeq=Xt, x_scale=xs_t)
+    torch.cuda.synchronize()
+    assert np.array_equal(Xt.cpu().numpy(), got)
+    assert np.array_equal(xs_t.cpu().numpy(), got_s)
     if case == "crafted":
         # codes fixed by the format itself: 1.0625 -> 1.0 (0x38), 1.1875 -> 1.25 (0x3A),
         # 2^-10 -> +0, 3*2^-10 -> 2^-8 (0x02), 448 -> 0x7E, -0 -> 0x80

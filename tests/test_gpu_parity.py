@@ -219,10 +219,13 @@ def test_layout_dropped_slots(T, E, k, drop):
 def test_dispatch_bit_exact(T, d, E, k):
     X = I.random_bf16((T, d), 2, "X")
     idx = I.random_topk(T, E, k, 2)
-    _, _, _, rs = O.layout(idx.numpy(), E)
+    _, _, rr, rs = O.layout(idx.numpy(), E)
     Xe = moe.moe_dispatch(X.to(DEV), torch.from_numpy(rs).to(DEV), k)
     ref = O.dispatch(bits(X), rs, k)
     assert np.array_equal(bits(Xe), ref)
+    # walked by token through row_of: the same bytes
+    Xt = moe.moe_dispatch_by_token(X.to(DEV), torch.from_numpy(rr).to(DEV), k)
+    assert np.array_equal(bits(Xt), ref)
 
 
 @pytest.mark.parametrize("T,d,E,k", [(256, 128, 8, 2), (4096, 4096, 8, 2), (8192, 7168, 256, 8),
@@ -257,6 +260,10 @@ def test_dispatch_and_combine_with_dropped_slots():
     moe.moe_dispatch(X.to(DEV), torch.from_numpy(rs).to(DEV), k, Xe=Xe)
     assert np.array_equal(bits(Xe[:kept]), O.dispatch(bits(X), rs, k)[:kept])
     assert (Xe[kept:] == 3.0).all()                # unused rows untouched
+    Xt = torch.full((T * k, d), 3.0, dtype=torch.bfloat16, device=DEV)
+    moe.moe_dispatch_by_token(X.to(DEV), torch.from_numpy(rr).to(DEV), k, Xe=Xt)
+    assert np.array_equal(bits(Xt[:kept]), O.dispatch(bits(X), rs, k)[:kept])
+    assert (Xt[kept:] == 3.0).all()
     Ye = I.random_bf16((T * k, d), 9, "Ye")
     Ye[kept:] = float("nan")                       # never read
     g = torch.rand((T, k), generator=torch.Generator().manual_seed(9))

@@ -73,11 +73,11 @@ constexpr int UMMA_K_BYTES = UMMA_K * 2;     // 32 bytes of a row per MMA in bot
 constexpr int A_STAGE = BM * BK * 2;         // 16 KB of weight rows per CTA and stage
 constexpr int B_BOX_ROWS = 32;
 constexpr int B_BOX = B_BOX_ROWS * BK * 2;   // 4 KB
-// Token rows a CTA stages for a full tile (256 tokens split over a pair, or
-// 128 with one CTA) are loaded with one 16 KB request instead of four 4 KB
-// ones, since TMA throughput grows with the request size; a half-tile of at
-// least kWideMin rows also takes the single request (over-fetching at most
-// 32 rows into the stage buffer, which holds 128).
+// Token rows a CTA stages for a tile (up to 128 per CTA with a pair, up to 256
+// with one CTA) are loaded in 128-row boxes of 16 KB instead of 4 KB ones,
+// since TMA throughput grows with the request size; a half-tile of at least
+// kWideMin rows takes ceil(rows / 128) such boxes (over-fetching at most 32
+// rows past the last one, inside the stage buffer).
 constexpr int B_WIDE_ROWS = 128;
 constexpr int kWideMin = 96;
 constexpr int EPI_WARPS = 8;                 // two per SM sub-partition
@@ -402,8 +402,12 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
       const int half = nmma / kPair;  // token rows staged by this CTA (a multiple of 8)
       const bool wide = half >= kWideMin;
       const int nbox = (half + B_BOX_ROWS - 1) / B_BOX_ROWS;
+      // wide boxes of 128 rows: one with paired CTAs (half <= 128), up to two
+      // with a single CTA (half <= 256); the stage holds BN / kPair rows
+      const int nwide = (half + B_WIDE_ROWS - 1) / B_WIDE_ROWS;
       const uint32_t bytes = is_w ? (uint32_t)(kPair * A_STAGE)
-                                  : (uint32_t)kPair * (wide ? B_WIDE_ROWS * BK * 2 : nbox * B_BOX);
+                                  : (uint32_t)kPair * (wide ? nwide * B_WIDE_ROWS * BK * 2
+                                                            : nbox * B_BOX);
       const int wy = t.e * Np + t.fb * C::FEAT + (int)rank * BM;
       const int by = t.row0 + (int)rank * half;
       // gather form: request q (4 rows) of this CTA's half-tile is issued
@@ -454,14 +458,15 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
         } else if (lane == 0) {
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
           if (rank == 0) mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)nsub);
-          for (int hh = 0; hh < nsub; ++hh) {
+          for (int hh = 0; hh < nsub; ++hh) {  // one request per operand and K-block
             const int kb = ks * KPS + hh;
             if (is_w) {
               tma_load_2d_cg<kPair>(sA + (s * KPS + hh) * A_STAGE, map_w, kb * kbv, wy, fb_addr,
                                     pol);
-            } else if (wide) {  // (nearly) a full half-tile: one large request
-              tma_load_2d_cg<kPair>(sB + (s * KPS + hh) * B_STAGE, map_xw, kb * kbv, by, fb_addr,
-                                    pol);
+            } else if (wide) {  // (nearly) full 128-row boxes: large requests
+              for (int j = 0; j < nwide; ++j)
+                tma_load_2d_cg<kPair>(sB + (s * KPS + hh) * B_STAGE + j * B_WIDE_ROWS * 128,
+                                      map_xw, kb * kbv, by + j * B_WIDE_ROWS, fb_addr, pol);
             } else {
               for (int j = 0; j < nbox; ++j)
                 tma_load_2d_cg<kPair>(sB + (s * KPS + hh) * B_STAGE + j * B_BOX, map_x, kb * kbv,

@@ -46,6 +46,7 @@ FFN_CASES = [
     ([1030, 990, 1024], 256, 320),
     ([1] * 64, 256, 256),                                   # many one-row experts
     ([2048, 0, 2048, 4096], 512, 1024),                     # more token blocks than clusters
+    ([500, 300, 129], 128, 256),                            # one CTA per tile, > 128 rows per tile
 ]
 
 

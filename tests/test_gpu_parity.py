@@ -324,6 +324,10 @@ GEMM_CASES = [
     ([600, 520], 264, 128, False),                    # N tail with wide tiles
     ([1030, 990, 1024], 256, 320, True),
     ([260] * 16, 384, 64, False),                     # 16 experts just over one block
+    # one CTA per tile (N <= 128) with more than 128 rows per tile: two 128-row boxes
+    ([300, 0, 129, 256, 97, 128], 128, 64, True),
+    ([700], 64, 200, False),
+    ([1000, 3], 96, 136, True),
 ]
 
 
@@ -407,6 +411,20 @@ def test_layer_tiny_threshold_full_parity():
     assert np.array_equal(idx.cpu().numpy(), ref["topk_idx"])
     assert np.array_equal(counts.cpu().numpy(), ref["counts"])
     assert_close(f64(Y), ref["Y"], "Y (threshold)")
+
+
+def test_layer_narrow_model_dim_full_tiles():
+    """d = 128: GEMM-2 (N = d) runs one CTA per tile with full 256-row tiles
+    (about 512 rows per expert), the case that needs two 128-row token boxes."""
+    T, d, E, k, f = 1024, 128, 4, 2, 256
+    X = I.random_bf16((T, d), 13, "X")
+    W1 = I.random_bf16((E, f, d), 13, "W1", 0.05)
+    W2 = I.random_bf16((E, d, f), 13, "W2", 0.05)
+    L = I.random_f32((T, E), 13, "L")
+    Y = moe.moe_layer_forward(X.to(DEV), W1.to(DEV), W2.to(DEV), k, logits=L.to(DEV))
+    ref = O.layer_forward(bits(X), bits(W1), bits(W2), k, logits=L.numpy())
+    assert int(ref["counts"].max()) > 256
+    assert_close(f64(Y), ref["Y"], "Y (d = 128)")
 
 
 def test_layer_deterministic():

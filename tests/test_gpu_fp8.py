@@ -164,6 +164,7 @@ FP8_GEMM_CASES = [
     ([128] * 3, 1024, 1024, True),
     ([1] * 64, 256, 256, False),                       # many one-row experts
     ([1030, 990, 1024], 256, 320, True),
+    ([300, 129, 97], 128, 256, True),                  # one CTA per tile, > 128 rows per tile
 ]
 
 

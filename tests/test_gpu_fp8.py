@@ -165,6 +165,7 @@ FP8_GEMM_CASES = [
     ([1] * 64, 256, 256, False),                       # many one-row experts
     ([1030, 990, 1024], 256, 320, True),
     ([300, 129, 97], 128, 256, True),                  # one CTA per tile, > 128 rows per tile
+    ([320, 321, 272, 576], 256, 256, True),            # short last token blocks (64, 65, 16 rows)
 ]
 
 

@@ -47,6 +47,7 @@ FFN_CASES = [
     ([1] * 64, 256, 256),                                   # many one-row experts
     ([2048, 0, 2048, 4096], 512, 1024),                     # more token blocks than clusters
     ([500, 300, 129], 128, 256),                            # one CTA per tile, > 128 rows per tile
+    ([320, 321, 272, 576], 256, 512),                       # short last token blocks (64, 65, 16 rows)
 ]
 
 

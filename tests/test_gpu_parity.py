@@ -319,8 +319,10 @@ GEMM_CASES = [
     ([5, 3], 8, 8, False),                            # smallest dims
     ([128] * 3, 1024, 1024, True),
     ([1] * 64, 256, 256, False),                      # many one-row experts
-    # mean > 192 rows per expert: tiles of up to 512 rows in two accumulators
+    # short last token blocks (1, 16, 44, 64, 65 rows) after full ones
     ([300, 0, 513, 1, 256, 257], 512, 192, True),
+    ([320, 321, 272, 576, 64], 256, 256, True),
+    ([1] * 700 + [300], 256, 64, False),              # 701 experts: a large tile table in smem
     ([600, 520], 264, 128, False),                    # N tail with wide tiles
     ([1030, 990, 1024], 256, 320, True),
     ([260] * 16, 384, 64, False),                     # 16 experts just over one block

@@ -231,7 +231,7 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   uint32_t* ready = reinterpret_cast<uint32_t*>(base + w.ready);
   const int R = d.T * d.k;
 
-  if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, s), "router_logits");
+  if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, *dev, s), "router_logits");
   MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
                              d.min_prob, idx, gates, s),
            "route");
@@ -328,7 +328,10 @@ moe_status moe_router_logits(const void* X, const void* Wr, int32_t T, int32_t d
   MOE_TRY(check_ptr(X, "X"));
   MOE_TRY(check_ptr(Wr, "Wr"));
   MOE_TRY(check_ptr4(logits, "logits"));
-  MOE_CUDA(moe::launch_router_logits(X, Wr, T, d, E, logits, as_stream(stream)), "router_logits");
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  MOE_CUDA(moe::launch_router_logits(X, Wr, T, d, E, logits, *dev, as_stream(stream)),
+           "router_logits");
   return MOE_OK;
 }
 

@@ -93,6 +93,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Plain arrive (count 1) on a barrier of this CTA, release order.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
 // Wait until the phase with the given parity has completed.  Gives up after
 // kWaitLimitNs (setting MOE_DEV_TIMEOUT and the CTA's abort flag) or as soon
 // as another role of the CTA has raised the abort flag.  Returns true when
@@ -149,6 +155,17 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 1-D bulk copy (TMA, no tensor map) of `bytes` from global memory into this
+// CTA's shared memory; completion is counted on `bar` as transaction bytes.
+// dst and src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // L2 eviction-priority policies for TMA cache hints.

@@ -26,7 +26,7 @@ struct DeviceInfo {
 const DeviceInfo* current_device_info(std::string* err);
 
 cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, int E, float* L,
-                                 cudaStream_t stream);
+                                 const DeviceInfo& dev, cudaStream_t stream);
 
 cudaError_t launch_route(const float* L, int T, int E, int k, int score, int renormalize,
                          float temperature, float min_prob, int32_t* idx, float* gates,

@@ -7,6 +7,7 @@
 // Both kernels are bandwidth / latency bound: the router linear streams X
 // once (T*d*2 bytes) and the top-k reads T*E*4 bytes of logits.
 #include <cfloat>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -18,26 +19,58 @@ namespace moe {
 //
 // A GEMM with N = E (8 for the Mixtral shape): tensor-core mma.sync tiles of
 // 16 tokens x 8 experts x 16 K (bf16 in, fp32 accumulate) fit it exactly,
-// and it is bound by streaming X (T*d*2 bytes) from HBM.  A CTA of 8 warps
-// takes 16 tokens; the warps split K into 64-column chunks (warp w takes
-// chunks w, w+8, ...) and their partial 16 x E tiles are summed in shared
-// memory in warp order (deterministic).
+// and it is bound by streaming X (T*d*2 bytes) from HBM once.
 //
-// Operand loads use a K permutation shared by both operands: in a 64-column
-// chunk, the thread with q = lane % 4 loads columns [16q, 16q+16) of its two
-// token rows (lane / 4 and lane / 4 + 8) and of expert row lane / 4, as two
-// 16-byte vectors each (the four threads of a row read 128 contiguous
-// bytes).  MMA m of the chunk takes words 2m, 2m+1 of each: logical k-pair
-// (2q, 2q+1) is column 16q + 4m + {0, 1} and (2q+8, 2q+9) is 16q + 4m + {2, 3}
-// for A and B alike, so the 4 MMAs cover the chunk's 64 columns exactly once.
-// More than 64 experts are processed in groups of 8 n-tiles, re-reading X.
-// The X vectors of a warp's next chunk are loaded while the current chunk's
-// MMAs run (a warp walks nchunks / 8 chunks; for a handful of tokens, e.g.
-// decode, those loads would otherwise be serial round trips).
+// Streaming.  A CTA takes tiles of 16 tokens (CTA i: tiles i, i + grid, ...)
+// and walks each tile's rows in slices of kRouterSlice columns.  One producer
+// thread copies a slice (16 row pieces of up to 2 KB) into a ring of
+// kRouterStages shared-memory stages with 1-D bulk copies, all signalled on
+// the stage's mbarrier, so up to three slices per CTA (and two CTAs per SM)
+// are in flight while the MMA warps work on earlier ones.  The grid is at
+// most what is co-resident, so every CTA keeps its ring busy from start to
+// end; with a handful of tokens (decode) one CTA still has its whole tile in
+// flight at once.
+//
+// MMA warps.  8 warps split a slice into 64-column chunks (warp w takes
+// chunks w, w+8, ...), accumulate their 16 x 8 tiles over all slices of the
+// token tile in registers, and the partial tiles are summed in shared memory
+// in warp order (deterministic).  Operands use a K permutation shared by
+// both: in a 64-column chunk the thread with q = lane % 4 reads columns
+// [16q, 16q+16) of its two token rows (lane / 4 and lane / 4 + 8) and of
+// expert row lane / 4, as two 16-byte vectors each; MMA m of the chunk takes
+// words 2m, 2m+1 of each, so logical k-pair (2q, 2q+1) is column 16q + 4m +
+// {0, 1} and (2q+8, 2q+9) is 16q + 4m + {2, 3} for A and B alike, and the 4
+// MMAs cover the chunk's 64 columns exactly once.  Shared-memory rows are
+// padded by 16 bytes, so the 8 rows a quarter-warp reads fall in distinct
+// banks.  X comes from shared memory.  Wr (E x d) is re-read by every tile:
+// with at most 8 experts (one n-tile) and d up to kRouterWsMaxD the producer
+// copies it into shared memory once per CTA, next to the ring; otherwise it
+// is read through the read-only cache.  More than 64 experts are processed
+// in groups of 8 n-tiles, streaming the tile's X once per group.
 // ---------------------------------------------------------------------------
-constexpr int kRouterWarps = 8;
-constexpr int kRouterTok = 16;     // tokens per CTA (the MMA's M)
-constexpr int kRouterGroup = 8;    // n-tiles of 8 experts per pass
+constexpr int kRouterWarps = 8;                            // MMA warps; warp 8 copies
+constexpr int kRouterThreads = (kRouterWarps + 1) * 32;
+constexpr int kRouterTok = 16;                             // tokens per tile (the MMA's M)
+constexpr int kRouterGroup = 8;                            // n-tiles of 8 experts per pass
+constexpr int kRouterSlice = 1024;                         // columns per ring stage
+constexpr int kRouterStages = 3;
+constexpr int kRouterPitch = kRouterSlice * 2 + 16;        // bytes per staged row
+constexpr int kRouterStageBytes = kRouterTok * kRouterPitch;
+constexpr int kRouterRingBytes = kRouterStages * kRouterStageBytes;
+
+// Dynamic shared memory: ring | full[S] | empty[S] | Wr barrier | abort flag
+// | partial tiles | (staged Wr: 8 rows of d*2 + 16 bytes).
+__host__ __device__ constexpr size_t router_part_offset() {
+  return (size_t)kRouterRingBytes + (2 * kRouterStages + 1) * 8 + 8;
+}
+__host__ __device__ constexpr size_t router_smem_bytes(int groups_in_pass) {
+  return router_part_offset() + (size_t)kRouterWarps * groups_in_pass * kRouterTok * 8 * 4;
+}
+__host__ __device__ constexpr int router_w_pitch(int d) { return d * 2 + 16; }
+constexpr size_t kRouterSmemMax = 232448;  // opt-in shared memory per block
+// The largest d whose 8 staged Wr rows fit beside the ring (one n-tile per pass).
+constexpr int kRouterWsMaxD =
+    (int)(((kRouterSmemMax - router_smem_bytes(1)) / 8 - 16) / 2) / 8 * 8;
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
@@ -49,97 +82,238 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// 16 bytes at p (8 bf16) when the 8 values at column `col` exist, else zeros
-__device__ __forceinline__ uint4 ld_row_v4(const uint4* p, bool ok) {
-  return ok ? ld_stream_v4(p) : make_uint4(0u, 0u, 0u, 0u);
+// Barrier `id` over the first `threads` threads of the CTA (the MMA warps).
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-__global__ void __launch_bounds__(kRouterWarps * 32)
-    router_logits_kernel(const uint4* __restrict__ X, const uint4* __restrict__ Wr, int T,
-                         int row_vecs, int E, float* __restrict__ L) {
-  __shared__ float s_part[kRouterWarps][kRouterGroup][kRouterTok * 8];
+__device__ __forceinline__ uint4 lds_v4(const uint8_t* p, bool ok) {
+  return ok ? *reinterpret_cast<const uint4*>(p) : make_uint4(0u, 0u, 0u, 0u);
+}
+
+__device__ __forceinline__ bool router_warp_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                                 volatile int* abort_flag) {
+  const bool ok = mbar_wait(bar, parity, status, abort_flag);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// kG: n-tiles per pass at most (1 when E <= 8: fewer registers).  kWs: Wr
+// staged in shared memory (kG == 1 only).
+template <int kG, bool kWs>
+__global__ void __launch_bounds__(kRouterThreads, kG == 1 ? 2 : 1)
+    router_logits_kernel(const uint8_t* __restrict__ X, const uint4* __restrict__ Wr, int T,
+                         int d, int E, float* __restrict__ L, uint32_t* status) {
+  static_assert(!kWs || kG == 1, "Wr is staged for one n-tile only");
+  extern __shared__ __align__(128) uint8_t smem_r[];
+  uint8_t* ring = smem_r;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_r + kRouterRingBytes);
+  uint64_t* empty = full + kRouterStages;
+  uint64_t* wbar = empty + kRouterStages;  // staged Wr landed
+  volatile int* s_abort = reinterpret_cast<volatile int*>(wbar + 1);
+  float* s_part = reinterpret_cast<float*>(smem_r + router_part_offset());
+  uint8_t* s_w = smem_r + router_smem_bytes(kG);  // staged Wr (kWs)
+  const int wpitch = router_w_pitch(d);
+
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = lane >> 2, q = lane & 3;
-  const int t0 = blockIdx.x * kRouterTok;
-  const bool okA0 = t0 + r0 < T, okA1 = t0 + r0 + 8 < T;
-  const uint4* xa0 = X + (size_t)(okA0 ? t0 + r0 : 0) * row_vecs;
-  const uint4* xa1 = X + (size_t)(okA1 ? t0 + r0 + 8 : 0) * row_vecs;
-  const int nchunks = (row_vecs + 7) / 8;  // 64 columns = 8 vectors per chunk
-  const int ntiles = (E + 7) / 8;
-  for (int g0 = 0; g0 < ntiles; g0 += kRouterGroup) {
-    const int G = min(kRouterGroup, ntiles - g0);
-    float acc[kRouterGroup][4];
-#pragma unroll
-    for (int j = 0; j < kRouterGroup; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    uint4 n00, n01, n10, n11;  // the next chunk's X vectors
-    {
-      const int v = warp * 8 + 2 * q;
-      const bool ok0 = warp < nchunks && v < row_vecs, ok1 = warp < nchunks && v + 1 < row_vecs;
-      n00 = ld_row_v4(xa0 + v, okA0 && ok0);
-      n01 = ld_row_v4(xa0 + v + 1, okA0 && ok1);
-      n10 = ld_row_v4(xa1 + v, okA1 && ok0);
-      n11 = ld_row_v4(xa1 + v + 1, okA1 && ok1);
+  const int ntok_tiles = (T + kRouterTok - 1) / kRouterTok;
+  const int ntiles = (E + 7) / 8;  // n-tiles of 8 experts
+  const int ngroups = (ntiles + kG - 1) / kG;
+  const int nslices = (d + kRouterSlice - 1) / kRouterSlice;
+  const int row_vecs = d / 8;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRouterStages; ++s) {
+      mbar_init(&full[s], 1);              // the producer's expect_tx arrive
+      mbar_init(&empty[s], kRouterWarps);  // one arrive per MMA warp
     }
-    for (int c = warp; c < nchunks; c += kRouterWarps) {
-      const int v = c * 8 + 2 * q;  // this thread's first vector of the chunk
-      const bool ok0 = v < row_vecs, ok1 = v + 1 < row_vecs;
-      const uint4 x00 = n00, x01 = n01, x10 = n10, x11 = n11;
-      {
-        const int cn = c + kRouterWarps, vn = cn * 8 + 2 * q;
-        const bool m0 = cn < nchunks && vn < row_vecs, m1 = cn < nchunks && vn + 1 < row_vecs;
-        n00 = ld_row_v4(xa0 + vn, okA0 && m0);
-        n01 = ld_row_v4(xa0 + vn + 1, okA0 && m1);
-        n10 = ld_row_v4(xa1 + vn, okA1 && m0);
-        n11 = ld_row_v4(xa1 + vn + 1, okA1 && m1);
-      }
-      const uint32_t A0[8] = {x00.x, x00.y, x00.z, x00.w, x01.x, x01.y, x01.z, x01.w};
-      const uint32_t A1[8] = {x10.x, x10.y, x10.z, x10.w, x11.x, x11.y, x11.z, x11.w};
-#pragma unroll
-      for (int j = 0; j < kRouterGroup; ++j) {
-        if (j < G) {
-          const int e = (g0 + j) * 8 + r0;
-          const bool okB = e < E;
-          const uint4* wr = Wr + (size_t)(okB ? e : 0) * row_vecs;
-          const uint4 w0 = okB && ok0 ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
-          const uint4 w1 = okB && ok1 ? __ldg(wr + v + 1) : make_uint4(0u, 0u, 0u, 0u);
-          const uint32_t B[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-          for (int m = 0; m < 4; ++m)
-            mma_bf16_16816(acc[j], A0[2 * m], A1[2 * m], A0[2 * m + 1], A1[2 * m + 1], B[2 * m],
-                           B[2 * m + 1]);
+    mbar_init(wbar, 1);
+    *s_abort = 0;
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kRouterWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane != 0) return;
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t pending = 0;  // bit s: a copy into stage s may still be in flight
+    uint32_t pend_ph = 0;  // bit s: the parity that copy completes
+    bool ok = true;
+    if (kWs) {  // Wr once per CTA: E rows of d*2 bytes, padded pitch
+      const uint32_t wbytes = (uint32_t)d * 2u;
+      mbar_arrive_expect_tx(wbar, wbytes * (uint32_t)E);
+      for (int e = 0; e < E; ++e)
+        bulk_load_g2s(s_w + e * wpitch, reinterpret_cast<const uint8_t*>(Wr) + (size_t)e * wbytes,
+                      wbytes, wbar);
+    }
+    for (int tt = blockIdx.x; ok && tt < ntok_tiles; tt += gridDim.x) {
+      const int t0 = tt * kRouterTok;
+      const int nrows = min(kRouterTok, T - t0);
+      for (int g = 0; ok && g < ngroups; ++g) {
+        for (int sl = 0; sl < nslices; ++sl) {
+          if (!mbar_wait(&empty[s], ph ^ 1u, status, s_abort)) {
+            ok = false;
+            break;
+          }
+          const int c0 = sl * kRouterSlice;
+          const uint32_t bytes = (uint32_t)min(kRouterSlice, d - c0) * 2u;
+          mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)nrows);
+          uint8_t* dst = ring + s * kRouterStageBytes;
+          for (int r = 0; r < nrows; ++r)
+            bulk_load_g2s(dst + r * kRouterPitch, X + ((size_t)(t0 + r) * d + c0) * 2, bytes,
+                          &full[s]);
+          pending |= 1u << s;
+          pend_ph = (pend_ph & ~(1u << s)) | (ph << s);
+          if (++s == kRouterStages) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
     }
-    // partial tile of this warp: c0,c1 = (row r0, experts 2q, 2q+1), c2,c3 = row r0 + 8
+    if (!ok) {  // an MMA warp gave up: let issued copies land before the CTA leaves
+      int dummy = 0;
+      if (kWs) mbar_wait(wbar, 0, nullptr, (volatile int*)&dummy, 20ull * 1000ull * 1000ull);
+      for (int q = 0; q < kRouterStages; ++q)
+        if ((pending >> q) & 1u)
+          mbar_wait(&full[q], (pend_ph >> q) & 1u, nullptr, (volatile int*)&dummy,
+                    20ull * 1000ull * 1000ull);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- MMA warps
+  const int r0 = lane >> 2, q = lane & 3;
+  if (kWs && !router_warp_wait(wbar, 0, status, s_abort)) return;
+  int s = 0;
+  uint32_t ph = 0;
+  for (int tt = blockIdx.x; tt < ntok_tiles; tt += gridDim.x) {
+    const int t0 = tt * kRouterTok;
+    for (int g = 0; g < ngroups; ++g) {
+      const int G = min(kG, ntiles - g * kG);
+      float acc[kG][4];
 #pragma unroll
-    for (int j = 0; j < kRouterGroup; ++j) {
-      if (j < G) {
-        float* p = s_part[warp][j];
-        p[r0 * 8 + 2 * q] = acc[j][0];
-        p[r0 * 8 + 2 * q + 1] = acc[j][1];
-        p[(r0 + 8) * 8 + 2 * q] = acc[j][2];
-        p[(r0 + 8) * 8 + 2 * q + 1] = acc[j][3];
+      for (int j = 0; j < kG; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      for (int sl = 0; sl < nslices; ++sl) {
+        if (!router_warp_wait(&full[s], ph, status, s_abort)) return;
+        const uint8_t* st = ring + s * kRouterStageBytes;
+        const int c0 = sl * kRouterSlice;
+        const int w = min(kRouterSlice, d - c0);  // valid columns of this slice
+        const int nch = (w + 63) / 64;
+        for (int c = warp; c < nch; c += kRouterWarps) {
+          const int col = c * 64 + 16 * q;  // this thread's first column in the slice
+          const bool ok0 = col < w, ok1 = col + 8 < w;
+          const uint8_t* ra = st + r0 * kRouterPitch + col * 2;
+          const uint8_t* rb = ra + 8 * kRouterPitch;
+          const uint4 x00 = lds_v4(ra, ok0), x01 = lds_v4(ra + 16, ok1);
+          const uint4 x10 = lds_v4(rb, ok0), x11 = lds_v4(rb + 16, ok1);
+          const uint32_t A0[8] = {x00.x, x00.y, x00.z, x00.w, x01.x, x01.y, x01.z, x01.w};
+          const uint32_t A1[8] = {x10.x, x10.y, x10.z, x10.w, x11.x, x11.y, x11.z, x11.w};
+          const int v = (c0 + col) / 8;  // vector index of the column in a row of Wr
+#pragma unroll
+          for (int j = 0; j < kG; ++j) {
+            if (j < G) {
+              const int e = (g * kG + j) * 8 + r0;
+              const bool okB = e < E;
+              uint4 w0, w1;
+              if (kWs) {
+                const uint8_t* ws = s_w + (okB ? e : 0) * wpitch + (size_t)v * 16;
+                w0 = lds_v4(ws, okB && ok0);
+                w1 = lds_v4(ws + 16, okB && ok1);
+              } else {
+                const uint4* wr = Wr + (size_t)(okB ? e : 0) * row_vecs;
+                w0 = okB && ok0 ? __ldg(wr + v) : make_uint4(0u, 0u, 0u, 0u);
+                w1 = okB && ok1 ? __ldg(wr + v + 1) : make_uint4(0u, 0u, 0u, 0u);
+              }
+              const uint32_t B[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+              for (int m = 0; m < 4; ++m)
+                mma_bf16_16816(acc[j], A0[2 * m], A1[2 * m], A0[2 * m + 1], A1[2 * m + 1],
+                               B[2 * m], B[2 * m + 1]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with the stage
+        if (++s == kRouterStages) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < G * kRouterTok * 8; i += blockDim.x) {
-      const int j = i / (kRouterTok * 8), rc = i % (kRouterTok * 8);
-      const int r = rc / 8, e = (g0 + j) * 8 + rc % 8;
-      float sum = 0.f;
+      // partial tile of this warp: c0,c1 = (row r0, experts 2q, 2q+1), c2,c3 = row r0 + 8
 #pragma unroll
-      for (int w = 0; w < kRouterWarps; ++w) sum += s_part[w][j][rc];
-      if (t0 + r < T && e < E) L[(size_t)(t0 + r) * E + e] = sum;
+      for (int j = 0; j < kG; ++j) {
+        if (j < G) {
+          float* p = s_part + (size_t)(warp * G + j) * (kRouterTok * 8);
+          p[r0 * 8 + 2 * q] = acc[j][0];
+          p[r0 * 8 + 2 * q + 1] = acc[j][1];
+          p[(r0 + 8) * 8 + 2 * q] = acc[j][2];
+          p[(r0 + 8) * 8 + 2 * q + 1] = acc[j][3];
+        }
+      }
+      named_barrier_sync(1, kRouterWarps * 32);
+      for (int i = threadIdx.x; i < G * kRouterTok * 8; i += kRouterWarps * 32) {
+        const int j = i / (kRouterTok * 8), rc = i % (kRouterTok * 8);
+        const int r = rc / 8, e = (g * kG + j) * 8 + rc % 8;
+        float sum = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < kRouterWarps; ++ww)
+          sum += s_part[(size_t)(ww * G + j) * (kRouterTok * 8) + rc];
+        if (t0 + r < T && e < E) L[(size_t)(t0 + r) * E + e] = sum;
+      }
+      named_barrier_sync(1, kRouterWarps * 32);
     }
-    __syncthreads();
   }
 }
 
+struct RouterSlot {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+};
+static RouterSlot g_router[64];
+
 cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, int E, float* L,
-                                 cudaStream_t stream) {
+                                 const DeviceInfo& dev, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const int blocks = (T + kRouterTok - 1) / kRouterTok;
-  router_logits_kernel<<<blocks, kRouterWarps * 32, 0, stream>>>(
-      static_cast<const uint4*>(X), static_cast<const uint4*>(Wr), T, d / 8, E, L);
+  const int ntiles = (E + 7) / 8;
+  const int gmax = ntiles < kRouterGroup ? ntiles : kRouterGroup;  // n-tiles per pass
+  RouterSlot& rs = g_router[dev.device & 63];
+  std::call_once(rs.once, [&] {
+    rs.err = cudaFuncSetAttribute(router_logits_kernel<1, true>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRouterSmemMax);
+    if (rs.err == cudaSuccess)
+      rs.err = cudaFuncSetAttribute(router_logits_kernel<1, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kRouterSmemMax);
+    if (rs.err == cudaSuccess)
+      rs.err = cudaFuncSetAttribute(router_logits_kernel<kRouterGroup, false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)kRouterSmemMax);
+  });
+  if (rs.err != cudaSuccess) return rs.err;
+  const bool ws = gmax == 1 && d <= kRouterWsMaxD;
+  const size_t smem = router_smem_bytes(gmax) + (ws ? (size_t)8 * router_w_pitch(d) : 0);
+  // CTAs co-resident on an SM: by registers two with one n-tile per pass (72
+  // per thread), one with eight (128); by shared memory, 228 KB per SM with
+  // 1 KB reserved per CTA.  A larger grid would only run in waves.
+  int per_sm = gmax > 1 ? 1 : 2;
+  const int by_smem = (int)(233472 / (smem + 1024));
+  if (by_smem < per_sm) per_sm = by_smem > 0 ? by_smem : 1;
+  const int tiles = (T + kRouterTok - 1) / kRouterTok;
+  const int resident = per_sm * dev.sm_count;
+  const int blocks = tiles < resident ? tiles : resident;
+  const uint8_t* x = static_cast<const uint8_t*>(X);
+  const uint4* w = static_cast<const uint4*>(Wr);
+  if (ws)
+    router_logits_kernel<1, true><<<blocks, kRouterThreads, smem, stream>>>(x, w, T, d, E, L,
+                                                                            dev.status);
+  else if (gmax == 1)
+    router_logits_kernel<1, false><<<blocks, kRouterThreads, smem, stream>>>(x, w, T, d, E, L,
+                                                                             dev.status);
+  else
+    router_logits_kernel<kRouterGroup, false><<<blocks, kRouterThreads, smem, stream>>>(
+        x, w, T, d, E, L, dev.status);
   return cudaGetLastError();
 }
 

@@ -131,7 +131,13 @@ def test_route_ex_parity(T, E, k, score, renorm, temp, thr):
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("T,d,E", [(4096, 4096, 8), (16, 4096, 8), (300, 136, 3), (77, 512, 40),
                                    (1, 8, 1), (100, 256, 72), (33, 4104, 130), (8, 64, 1024),
-                                   (17, 72, 8)])
+                                   (17, 72, 8),
+                                   # more token tiles than resident CTAs: each CTA walks
+                                   # several tiles through its ring (and, at E = 72, two
+                                   # passes of expert groups per tile)
+                                   (20000, 1024, 8), (5000, 2048, 72),
+                                   # d too large to stage Wr in shared memory beside the ring
+                                   (40, 8192, 8)])
 def test_router_logits_parity(T, d, E):
     X = I.random_bf16((T, d), 1, "X")
     Wr = I.random_bf16((E, d), 1, "Wr", 0.02)

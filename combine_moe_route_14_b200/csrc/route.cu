@@ -22,11 +22,13 @@ namespace moe {
 // and it is bound by streaming X (T*d*2 bytes) from HBM once.
 //
 // Streaming.  A CTA takes tiles of 16 tokens (CTA i: tiles i, i + grid, ...)
-// and walks each tile's rows in slices of kRouterSlice columns.  One producer
-// thread copies a slice (16 row pieces of up to 2 KB) into a ring of
-// kRouterStages shared-memory stages with 1-D bulk copies, all signalled on
-// the stage's mbarrier, so up to three slices per CTA (and two CTAs per SM)
-// are in flight while the MMA warps work on earlier ones.  The grid is at
+// and walks each tile's rows in slices of kRouterSlice columns.  A producer
+// warp copies a slice (16 row pieces of up to 2 KB) into a ring of
+// kRouterStages shared-memory stages with 1-D bulk copies, one row per lane
+// (requests from one thread are issued one after another, so a single
+// issuing thread would cap the rate), all signalled on the stage's mbarrier;
+// up to three slices per CTA are in flight while the MMA warps work on
+// earlier ones.  The grid is at
 // most what is co-resident, so every CTA keeps its ring busy from start to
 // end; with a handful of tokens (decode) one CTA still has its whole tile in
 // flight at once.
@@ -133,8 +135,8 @@ __global__ void __launch_bounds__(kRouterThreads, kG == 1 ? 2 : 1)
   __syncthreads();
 
   if (warp == kRouterWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane != 0) return;
+    // ------------------------------------------------------------ producer warp
+    // Lane 0 posts a stage's byte count; then lane r issues row r's copy.
     int s = 0;
     uint32_t ph = 0;
     uint32_t pending = 0;  // bit s: a copy into stage s may still be in flight
@@ -142,8 +144,9 @@ __global__ void __launch_bounds__(kRouterThreads, kG == 1 ? 2 : 1)
     bool ok = true;
     if (kWs) {  // Wr once per CTA: E rows of d*2 bytes, padded pitch
       const uint32_t wbytes = (uint32_t)d * 2u;
-      mbar_arrive_expect_tx(wbar, wbytes * (uint32_t)E);
-      for (int e = 0; e < E; ++e)
+      if (lane == 0) mbar_arrive_expect_tx(wbar, wbytes * (uint32_t)E);
+      __syncwarp();
+      for (int e = lane; e < E; e += 32)
         bulk_load_g2s(s_w + e * wpitch, reinterpret_cast<const uint8_t*>(Wr) + (size_t)e * wbytes,
                       wbytes, wbar);
     }
@@ -152,17 +155,17 @@ __global__ void __launch_bounds__(kRouterThreads, kG == 1 ? 2 : 1)
       const int nrows = min(kRouterTok, T - t0);
       for (int g = 0; ok && g < ngroups; ++g) {
         for (int sl = 0; sl < nslices; ++sl) {
-          if (!mbar_wait(&empty[s], ph ^ 1u, status, s_abort)) {
+          if (!router_warp_wait(&empty[s], ph ^ 1u, status, s_abort)) {
             ok = false;
             break;
           }
           const int c0 = sl * kRouterSlice;
           const uint32_t bytes = (uint32_t)min(kRouterSlice, d - c0) * 2u;
-          mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)nrows);
-          uint8_t* dst = ring + s * kRouterStageBytes;
-          for (int r = 0; r < nrows; ++r)
-            bulk_load_g2s(dst + r * kRouterPitch, X + ((size_t)(t0 + r) * d + c0) * 2, bytes,
-                          &full[s]);
+          if (lane == 0) mbar_arrive_expect_tx(&full[s], bytes * (uint32_t)nrows);
+          __syncwarp();
+          if (lane < nrows)
+            bulk_load_g2s(ring + s * kRouterStageBytes + lane * kRouterPitch,
+                          X + ((size_t)(t0 + lane) * d + c0) * 2, bytes, &full[s]);
           pending |= 1u << s;
           pend_ph = (pend_ph & ~(1u << s)) | (ph << s);
           if (++s == kRouterStages) {
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(kRouterThreads, kG == 1 ? 2 : 1)
         }
       }
     }
-    if (!ok) {  // an MMA warp gave up: let issued copies land before the CTA leaves
+    if (!ok && lane == 0) {  // an MMA warp gave up: let issued copies land before the CTA leaves
       int dummy = 0;
       if (kWs) mbar_wait(wbar, 0, nullptr, (volatile int*)&dummy, 20ull * 1000ull * 1000ull);
       for (int q = 0; q < kRouterStages; ++q)

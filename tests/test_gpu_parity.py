@@ -166,6 +166,9 @@ LAYOUT_CASES = [
     (50, 1024, 2, 0.0),
     (1, 1, 1, 0.0),
     (999, 1, 1, 0.0),
+    (5461, 16, 3, 0.0),       # 16383 slots, E = 16: one-block path near its limit
+    (4096, 12, 4, 1.5),       # 16384 slots exactly (the one-block limit), skewed
+    (3000, 17, 2, 0.0),       # E = 17
 ]
 
 
@@ -203,7 +206,7 @@ def test_layout_flags_bad_expert_ids():
 
 
 @pytest.mark.parametrize("T,E,k,drop", [(256, 8, 2, 0.2), (8192, 256, 8, 0.3), (9000, 7, 3, 0.5),
-                                        (40, 1024, 4, 1.0)])
+                                        (40, 1024, 4, 1.0), (5000, 16, 3, 0.4)])
 def test_layout_dropped_slots(T, E, k, drop):
     """-1 marks a dropped slot: no row, not counted, no flag; unused rows get src_of -1."""
     idx = I.random_topk(T, E, k, 8)

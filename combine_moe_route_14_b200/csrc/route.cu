@@ -28,10 +28,9 @@ namespace moe {
 // (requests from one thread are issued one after another, so a single
 // issuing thread would cap the rate), all signalled on the stage's mbarrier;
 // up to three slices per CTA are in flight while the MMA warps work on
-// earlier ones.  The grid is at
-// most what is co-resident, so every CTA keeps its ring busy from start to
-// end; with a handful of tokens (decode) one CTA still has its whole tile in
-// flight at once.
+// earlier ones.  The grid is at most what is co-resident, so every CTA keeps
+// its ring busy from start to end; with a handful of tokens (decode) one CTA
+// still has most of its tile in flight at once.
 //
 // MMA warps.  8 warps split a slice into 64-column chunks (warp w takes
 // chunks w, w+8, ...), accumulate their 16 x 8 tiles over all slices of the

@@ -47,10 +47,11 @@ METRIC = "MoE-layer tokens/s on 1 B200; HBM GB/s (dispatch/combine), TC util (GE
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# sampled tokens per oracle call: cpu_baseline leg / reference arm
-ORACLE_SAMPLE = {"mixtral": (4096, 32), "mixtral_threshold": (4096, 32), "tiny_threshold": (256, 256), "skewed_top1": (4096, 32), "skewed_top1_harsh": (4096, 32),
-                 "fine_grained": (32, 8), "tiny": (256, 256), "decode_16": (16, 16),
-                 "decode_64": (64, 32), "decode_256": (256, 32), "decode_1024": (256, 32)}
+# tokens per oracle step (the first S of the batch, all stages): the
+# cpu_baseline leg and the reference arm time the same sample
+ORACLE_SAMPLE = {"mixtral": 4096, "mixtral_threshold": 4096, "tiny_threshold": 256,
+                 "skewed_top1": 4096, "skewed_top1_harsh": 4096, "fine_grained": 32, "tiny": 256,
+                 "decode_16": 16, "decode_64": 64, "decode_256": 256, "decode_1024": 256}
 
 
 def log(*a):
@@ -225,6 +226,43 @@ def time_oracle(cfg, h, S, reps=1):
         oracle_step(O, cfg, h, S)
     dt = time.perf_counter() - t0
     return S * reps / dt, dt
+
+
+def arm_config(cfg, args, world):
+    """The `config` object of the JSON line; both arms print the same one."""
+    return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
+            "f": cfg.f, "router": cfg.router, "score": cfg.score, "fp8": bool(args.fp8),
+            "gather_on_load": bool(args.gather), "fused_ffn": bool(args.fused),
+            "renormalize": cfg.renormalize, "temperature": cfg.temperature,
+            "min_prob": cfg.min_prob, "tokens_per_gpu": cfg.T,
+            "parallelism": f"replicas x{world} (no collective)",
+            "l2": f"inputs larger than L2: each step streams "
+                  f"{(3 if args.fp8 else 4) * cfg.E * cfg.d * cfg.f / 1e9:.2f} GB of expert weights"}
+
+
+def sustained_peak_applies(loop_ms: float) -> bool:
+    """Which measured GEMM peak a tensor-bound kernel is held to.
+
+    The burst peak holds a kernel timed alone or in a short loop; the
+    sustained one (cuBLAS after seconds under the 1 kW power cap) only a
+    kernel timed inside a loop of a second or more.  A stray sw_power_cap
+    sample in a short loop is a note, not a reason to switch peaks."""
+    return loop_ms >= 1000.0
+
+
+def host_cpu():
+    """nproc and the CPU model name of this host (lscpu, else /proc/cpuinfo)."""
+    model = None
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        m = re.search(r"^Model name:\s*(.+)$", out, re.M)
+        model = m.group(1).strip() if m else None
+    except (OSError, subprocess.SubprocessError):
+        pass
+    if model is None and os.path.exists("/proc/cpuinfo"):
+        m = re.search(r"^model name\s*:\s*(.+)$", open("/proc/cpuinfo").read(), re.M)
+        model = m.group(1).strip() if m else None
+    return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
 # ----------------------------------------------------------------------------
@@ -429,10 +467,7 @@ def run_ours(args, cfg, rank, world, local_rank):
     dom = max(stage_ms, key=lambda n: stage_ms[n])
     peaks, peak_src = load_peaks()
     clocks = sampler.summary() if sampler else None
-    capped = bool(clocks and "sw_power_cap" in clocks.get("reasons", []))
-    # The sustained peak is cuBLAS under the 1 kW power cap; a kernel timed
-    # inside a continuous step loop that ran under that cap is held to it.
-    sustained = capped or (t_ms + staged_total_ms * args.steps) > 1000.0
+    sustained = sustained_peak_applies(max(t_ms, staged_total_ms * args.steps))
     per = model[dom]
     dur_s = stage_ms[dom] / 1e3
     # an FP8 contraction's peak: the measured bf16 peak x the nominal fp8:bf16 ratio (2);
@@ -445,13 +480,14 @@ def run_ours(args, cfg, rank, world, local_rank):
         roof = {"bound": "tensor", "achieved": per["flops"] / dur_s / 1e12, "peak": peak,
                 "unit": "TFLOP/s"}
         roof["frac_vs_burst"] = roof["achieved"] / (tc_ratio * peaks["bf16_tflops"])
+        roof["frac_vs_sustained"] = roof["achieved"] / (tc_ratio * peaks["bf16_tflops_sustained"])
     else:
         roof = {"bound": "hbm", "achieved": per["bytes"] / dur_s / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = dom
     roof["peak_source"] = (f"{peak_src} ("
-                           f"{'sustained: power cap active in the timed region' if sustained and roof['bound'] == 'tensor' else 'burst'})"
+                           f"{'sustained: timed loop of 1 s or more' if sustained and roof['bound'] == 'tensor' else 'burst: timed loop under 1 s'})"
                            + ("" if tc_ratio == 1.0 else
                               " x 2 (fp8:bf16 nominal ratio)" if tc_ratio == 2.0 else
                               " x 4/3 (half the FLOPs at the fp8 rate, half at bf16)"))
@@ -480,14 +516,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3 (dispatch, GEMM-1) + bf16" if args.fp8 else "bf16", "data": "synthetic",
-        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                   "f": cfg.f, "router": cfg.router, "score": cfg.score, "fp8": bool(args.fp8),
-                   "gather_on_load": bool(args.gather), "fused_ffn": bool(args.fused),
-                   "renormalize": cfg.renormalize, "temperature": cfg.temperature,
-                   "min_prob": cfg.min_prob, "tokens_per_gpu": cfg.T,
-                   "parallelism": f"replicas x{world} (no collective)",
-                   "l2": f"inputs larger than L2: each step streams "
-                         f"{(3 if args.fp8 else 4) * cfg.E * cfg.d * cfg.f / 1e9:.2f} GB of expert weights"},
+        "config": arm_config(cfg, args, world),
         "roofline": roof,
         "stages": stages,
         "expert_counts": {"max": int(counts_h.max()), "mean": float(counts_h.mean()),
@@ -542,7 +571,9 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return 0
-        S_base, S = ORACLE_SAMPLE.get(cfg.name, (64, 16))
+        # the same sample per step as the cpu_baseline leg (the first S tokens,
+        # all stages), so that the two CPU figures measure the same work
+        S = ORACLE_SAMPLE.get(cfg.name, 64)
         h = host_inputs(cfg, args.seed)
         for _ in range(args.warmup):
             time_oracle(cfg, h, S)
@@ -553,10 +584,9 @@ def main():
                "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                "impl": "reference",
-               "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
-                          "f": cfg.f, "router": cfg.router, "score": cfg.score,
-                          "renormalize": cfg.renormalize},
+               "config": arm_config(cfg, args, args.gpus),
                "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                **host_cpu(),
                                 "sample": f"first {S} of the {cfg.T} tokens per step, all stages"},
                "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
                        "d2h_bytes_per_step": 0}}
@@ -575,7 +605,7 @@ def main():
                                               "takes ~10 s per expert; the bf16 line carries "
                                               "the oracle baseline"}
         elif rank == 0 and world == 1 and not args.no_cpu_baseline:
-            S_base, _ = ORACLE_SAMPLE.get(cfg.name, (64, 16))
+            S_base = ORACLE_SAMPLE.get(cfg.name, 64)
             h = host_inputs(cfg, args.seed)
             runs, tot = 0, 0.0
             while runs == 0 or tot < 10.0:  # about 10 s of oracle work
@@ -583,7 +613,7 @@ def main():
                 runs, tot = runs + 1, tot + dt
             v = S_base * runs / tot
             res["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(),
-                                   "kind": "oracle",
+                                   "kind": "oracle", **host_cpu(),
                                    "sample": f"first {S_base} of the {cfg.T} tokens, all stages, "
                                              f"{runs} run(s), {tot:.1f} s"}
             try:  # the same oracle on one core (BLAS limited to one thread)

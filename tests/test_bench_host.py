@@ -90,3 +90,25 @@ def test_clock_summary_flags_thermal_and_hardware_slowdown():
 def test_clock_summary_without_samples():
     out = _sampler(["garbage", "0, [N/A], 1965, 1, 0x0, a, b, c, d"])
     assert out["sm_mhz"] is None and out["samples"] == 0
+
+
+def test_peak_choice_follows_the_length_of_the_timed_loop():
+    assert not bench.sustained_peak_applies(30.0)     # 20 steps of 1.5 ms: burst
+    assert not bench.sustained_peak_applies(999.0)
+    assert bench.sustained_peak_applies(1000.0)       # a second or more: sustained
+
+
+def test_both_arms_print_the_same_config():
+    import argparse
+    cfg = I.workload("mixtral")
+    a = argparse.Namespace(fp8=False, gather=False, fused=False)
+    c = bench.arm_config(cfg, a, 1)
+    for key in ("workload", "T", "d", "E", "k", "f", "fp8", "gather_on_load", "fused_ffn",
+                "temperature", "min_prob", "renormalize", "score", "router"):
+        assert key in c
+    assert c == bench.arm_config(cfg, a, 1)
+
+
+def test_host_cpu_reports_nproc():
+    info = bench.host_cpu()
+    assert info["nproc"] >= 1 and "cpu_model" in info

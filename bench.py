@@ -2,7 +2,7 @@
 """Benchmark: MoE-layer tokens/s on B200 (route -> layout -> dispatch -> expert FFN -> combine).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl ours|reference]
-                    [--fp8] [--gather] [--fused] [--graph]
+                    [--fp8] [--gather] [--fused] [--pipeline] [--graph]
 
 One step = one full layer forward (every stage) over one batch of T tokens.
 Default workload: the Mixtral-shaped layer (T=4096, d=4096, E=8, top-2,
@@ -11,6 +11,9 @@ inputs.  Multi-GPU runs are replicas (one process per GPU, each with its own
 token batch and a full copy of the weights, no data-path collective): weak
 scaling, value = all ranks' tokens / the slowest rank's time.
 
+``--pipeline`` runs the token-centric pipeline: after route and layout, one
+persistent kernel takes dispatch chunks, GEMM-1 and GEMM-2 tiles from an
+atomic ticket and (top-2 or top-1) combines in GEMM-2's epilogue.
 ``--fp8`` runs the layer's FP8 mode (E4M3 dispatch with a per-tensor scale
 and FP8 GEMM-1; GEMM-2 and combine stay bf16); W1 is quantised once before
 timing.  ``--gather`` fuses the dispatch into GEMM-1 (rows read through the
@@ -81,6 +84,14 @@ def stage_model(cfg, counts=None, fp8=False):  # gather form: same algorithmic b
         m["quantize"] = {"bytes": 2 * T * d * 2 + T * d}
     m["ffn"] = {"flops": m["gemm1"]["flops"] + m["gemm2"]["flops"],
                 "bytes": m["gemm1"]["bytes"] + m["gemm2"]["bytes"]}
+    # token-centric pipeline (dispatch chunks + both GEMMs + combine in one
+    # launch, k <= 2): X read, dispatched rows written and read, weights, H
+    # written and read, Y written; no Ye rows
+    w = E_act * f * d * 2 * 2
+    m["pipeline"] = {"flops": m["ffn"]["flops"],
+                     "bytes": w + T * d * 2 + 2 * R * d * 2 + 2 * R * f * 2 + T * d * 2
+                     if k <= 2 else w + T * d * 2 + 2 * R * d * 2 + 2 * R * f * 2
+                     + m["combine"]["bytes"] + R * d * 2}
     return m
 
 
@@ -233,6 +244,7 @@ def arm_config(cfg, args, world):
     return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k,
             "f": cfg.f, "router": cfg.router, "score": cfg.score, "fp8": bool(args.fp8),
             "gather_on_load": bool(args.gather), "fused_ffn": bool(args.fused),
+            "pipeline": bool(args.pipeline),
             "renormalize": cfg.renormalize, "temperature": cfg.temperature,
             "min_prob": cfg.min_prob, "tokens_per_gpu": cfg.T,
             "parallelism": f"replicas x{world} (no collective)",
@@ -289,7 +301,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     Wr = inp["Wr"].to(dev) if inp["Wr"] is not None else None
     layer = moe.MoeLayer(inp["W1"], inp["W2"], cfg.k, cfg.score, cfg.renormalize, Wr=Wr,
                          temperature=cfg.temperature, min_prob=cfg.min_prob, fp8=args.fp8,
-                         gather_on_load=args.gather, fused_ffn=args.fused)
+                         gather_on_load=args.gather, fused_ffn=args.fused,
+                         pipeline=args.pipeline)
     Y = torch.empty((cfg.T, cfg.d), dtype=torch.bfloat16, device=dev)
     counts = torch.empty((cfg.E,), dtype=torch.int32, device=dev)
     ws = layer.workspace(cfg.T)
@@ -363,10 +376,10 @@ def run_ours(args, cfg, rank, world, local_rank):
         step_us = step_percentiles([vev[i].elapsed_time(vev[i + 1]) for i in range(args.steps)])
 
         # ---- per-stage times: the same kernels, launched stage by stage with events between
-        stage_names = (["router_logits"] if Wr is not None else []) + [
-            "route", "layout"] + (["quantize"] if args.gather and args.fp8 else
-                                  [] if args.gather else ["dispatch"]) + (
-            ["ffn"] if args.fused else ["gemm1", "gemm2"]) + ["combine"]
+        stage_names = (["router_logits"] if Wr is not None else []) + ["route", "layout"] + (
+            ["pipeline"] if args.pipeline else
+            (["quantize"] if args.gather and args.fp8 else [] if args.gather else ["dispatch"]) +
+            (["ffn"] if args.fused else ["gemm1", "gemm2"]) + ["combine"])
         R = cfg.R
         L_buf = torch.empty((cfg.T, cfg.E), dtype=torch.float32, device=dev) if Wr is not None else logits
         idx = torch.empty((cfg.T, cfg.k), dtype=torch.int32, device=dev)
@@ -381,6 +394,9 @@ def run_ours(args, cfg, rank, world, local_rank):
         ffn_ws = torch.empty(max(16, moe.moe_expert_ffn_fused_workspace_size(cfg.E, R)),
                              dtype=torch.uint8, device=dev)
         xs = torch.empty((2,), dtype=torch.float32, device=dev)
+        pws = torch.empty(max(16, moe.moe_ffn_pipeline_workspace_size(cfg.T, cfg.d, cfg.E, cfg.k,
+                                                                       cfg.f)),
+                          dtype=torch.uint8, device=dev) if args.pipeline else None
         H = torch.empty((R, cfg.f), dtype=torch.bfloat16, device=dev)
         Ye = torch.empty((R, cfg.d), dtype=torch.bfloat16, device=dev)
         fns = {
@@ -406,6 +422,8 @@ def run_ours(args, cfg, rank, world, local_rank):
                    (lambda: moe.moe_expert_ffn_fused(Xe, offs, inp["W1"], inp["W2"], H, Ye,
                                                      ffn_ws)),
             "combine": lambda: moe.moe_combine(Ye, row_of, g, Y),
+            "pipeline": lambda: moe.moe_ffn_pipeline(X, src_of, row_of, g, offs, inp["W1"],
+                                                     inp["W2"], Y=Y, ws=pws),
         }
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stage_names) + 1)]
                for _ in range(args.steps)]
@@ -418,7 +436,7 @@ def run_ours(args, cfg, rank, world, local_rank):
         # host enqueues every staged call below, so the events between stages
         # measure device time, not the binding's per-call host overhead.
         for _ in range(max(2, (args.steps * len(stage_names) * 40) // max(1, int(stage_ms_hint(cfg))))):
-            fns["gemm1"]()
+            fns["pipeline" if args.pipeline else "gemm1"]()
         for s in range(args.steps):
             evs[s][0].record(stream)
             for i, n in enumerate(stage_names):
@@ -494,7 +512,8 @@ def run_ours(args, cfg, rank, world, local_rank):
     kname = {"gemm1": ("grouped_gemm_fp8_gelu" if args.fp8 else "grouped_gemm_gelu")
                       + ("_gather" if args.gather else ""),
              "gemm2": "grouped_gemm",
-             "ffn": "fused_ffn_fp8" if args.fp8 else "fused_ffn"}.get(dom, dom)
+             "ffn": "fused_ffn_fp8" if args.fp8 else "fused_ffn",
+             "pipeline": "ffn_pipeline"}.get(dom, dom)
     tr = ncu_traffic(kname, cfg.name)
     roof["traffic"] = tr
     roof["algorithmic_bytes"] = per["bytes"]
@@ -529,7 +548,8 @@ def run_ours(args, cfg, rank, world, local_rank):
         "gpu_launches": args.steps * (moe.moe_kernel_launches_per_forward_fp8 if args.fp8 else
                                       moe.moe_kernel_launches_per_forward)(
             moe.make_desc(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.score, cfg.renormalize,
-                          gather_on_load=args.gather, fused_ffn=args.fused),
+                          gather_on_load=args.gather, fused_ffn=args.fused,
+                          pipeline=args.pipeline),
             Wr is not None),
         "clocks": clocks,
     }
@@ -555,11 +575,16 @@ def main():
                     help="fuse the dispatch into GEMM-1 (gather-on-load)")
     ap.add_argument("--fused", action="store_true",
                     help="both expert GEMMs in one persistent kernel")
+    ap.add_argument("--pipeline", action="store_true",
+                    help="token-centric pipeline: dispatch, both GEMMs and the combine in one "
+                         "persistent kernel after route and layout")
     ap.add_argument("--graph", action="store_true",
                     help="also time the forward replayed from a CUDA graph")
     args = ap.parse_args()
-    if args.gather and args.fused:
-        ap.error("--gather and --fused cannot be combined")
+    if args.gather and (args.fused or args.pipeline):
+        ap.error("--gather cannot be combined with --fused or --pipeline")
+    if args.pipeline and (args.fp8 or args.fused):
+        ap.error("--pipeline is a bf16 path of its own (no --fp8, no --fused)")
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

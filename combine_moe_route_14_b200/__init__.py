@@ -29,6 +29,9 @@ __all__ = [
     "moe_quantize_fp8", "moe_expert_gemm_gather", "moe_expert_gemm_gather_fp8",
     "moe_expert_ffn_fused_workspace_size", "moe_expert_ffn_fused", "moe_expert_ffn_fused_fp8",
     "moe_selftest_bounded_wait", "moe_dispatch_by_token", "moe_dispatch_fp8_by_token",
+    "moe_ffn_pipeline_workspace_size", "moe_ffn_pipeline", "make_desc",
+    "LAYER_GATHER_ON_LOAD", "LAYER_FUSED_FFN", "LAYER_FUSED_COMBINE", "LAYER_FUSED_DISPATCH",
+    "LAYER_PIPELINE",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -39,6 +42,9 @@ _lock = threading.Lock()
 SCORES = {"softmax": 0, "sigmoid": 1}
 LAYER_GATHER_ON_LOAD = 0x1  # moe_layer_desc.flags: dispatch fused into GEMM-1
 LAYER_FUSED_FFN = 0x2       # moe_layer_desc.flags: both expert GEMMs in one persistent launch
+LAYER_FUSED_COMBINE = 0x4   # moe_layer_desc.flags: combine in GEMM-2's epilogue (k <= 2)
+LAYER_FUSED_DISPATCH = 0x8  # moe_layer_desc.flags: dispatch chunks inside the fused FFN launch
+LAYER_PIPELINE = LAYER_FUSED_FFN | LAYER_FUSED_COMBINE | LAYER_FUSED_DISPATCH
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
           4: "MOE_ERR_DEVICE"}
 DEV_BITS = {1: "MOE_DEV_BAD_EXPERT_ID", 2: "MOE_DEV_TIMEOUT", 4: "MOE_DEV_BAD_ROW"}
@@ -96,6 +102,9 @@ _SIG = {
                              ctypes.c_int),
     "moe_expert_ffn_fused_fp8": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P,
                                   ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_ffn_pipeline_workspace_size": ([_I, _I, _I, _I, _I], ctypes.c_size_t),
+    "moe_ffn_pipeline": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
+                          ctypes.c_size_t, _P], ctypes.c_int),
     "moe_expert_gemm_gather": ([_P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _P, _P], ctypes.c_int),
     "moe_expert_gemm_gather_fp8": ([_P, _P, _P, _I, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P],
                                    ctypes.c_int),
@@ -386,12 +395,47 @@ def moe_combine(Ye, row_of, gates, Y=None, stream=None):
     return Y
 
 
+def moe_ffn_pipeline_workspace_size(T, d, E, k, f) -> int:
+    return int(load_library().moe_ffn_pipeline_workspace_size(T, d, E, k, f))
+
+
+def moe_ffn_pipeline(X, src_of, row_of, gates, offsets, W1, W2, Y=None, ws=None, stream=None):
+    """Dispatch, GEMM-1 + GELU, GEMM-2 and (k <= 2) the combine in one persistent launch."""
+    lib = load_library()
+    T, d = X.shape
+    E, f, _ = W1.shape
+    k = gates.shape[1]
+    dev = X.device
+    _need(X, "X", torch.bfloat16, (T, d))
+    _need(src_of, "src_of", torch.int32, (T * k,), dev)
+    _need(row_of, "row_of", torch.int32, (T * k,), dev)
+    _need(gates, "gates", torch.float32, (T, k), dev)
+    _need(offsets, "offsets", torch.int32, (E + 1,), dev)
+    _need(W1, "W1", torch.bfloat16, (E, f, d), dev)
+    _need(W2, "W2", torch.bfloat16, (E, d, f), dev)
+    Y = _out(Y, "Y", torch.bfloat16, (T, d), dev)
+    if ws is None:
+        ws = torch.empty(max(moe_ffn_pipeline_workspace_size(T, d, E, k, f), 16),
+                         dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    _check(lib.moe_ffn_pipeline(_ptr(X), _ptr(src_of), _ptr(row_of), _ptr(gates), _ptr(offsets),
+                                _ptr(W1), _ptr(W2), T, d, E, k, f, _ptr(Y), _ptr(ws), ws.numel(),
+                                _stream(stream, dev)))
+    return Y
+
+
 # ----------------------------------------------------------------------------
 # whole layer
 # ----------------------------------------------------------------------------
 def make_desc(T, d, E, k, f, score="softmax", renormalize=True, temperature=1.0,
-              min_prob=0.0, gather_on_load=False, fused_ffn=False) -> LayerDesc:
-    flags = (LAYER_GATHER_ON_LOAD if gather_on_load else 0) | (LAYER_FUSED_FFN if fused_ffn else 0)
+              min_prob=0.0, gather_on_load=False, fused_ffn=False, fused_combine=False,
+              fused_dispatch=False, pipeline=False) -> LayerDesc:
+    """pipeline=True sets fused_ffn, fused_combine and fused_dispatch together."""
+    flags = ((LAYER_GATHER_ON_LOAD if gather_on_load else 0) |
+             (LAYER_FUSED_FFN if fused_ffn else 0) |
+             (LAYER_FUSED_COMBINE if fused_combine else 0) |
+             (LAYER_FUSED_DISPATCH if fused_dispatch else 0) |
+             (LAYER_PIPELINE if pipeline else 0))
     return LayerDesc(T, d, E, k, f, _score(score), int(bool(renormalize)), flags,
                      float(temperature), float(min_prob))
 
@@ -408,7 +452,8 @@ def moe_kernel_launches_per_forward(desc: LayerDesc, with_router: bool) -> int:
 def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=None, Wr=None,
                       Y=None, topk_idx_out=None, gates_out=None, counts_out=None, ws=None,
                       stream=None, temperature=1.0, min_prob=0.0, gather_on_load=False,
-                      fused_ffn=False):
+                      fused_ffn=False, fused_combine=False, fused_dispatch=False,
+                      pipeline=False):
     lib = load_library()
     T, d = X.shape
     E, f, _ = W1.shape
@@ -428,7 +473,7 @@ def moe_layer_forward(X, W1, W2, k, score="softmax", renormalize=True, logits=No
     if counts_out is not None:
         _need(counts_out, "counts_out", torch.int32, (E,), dev)
     desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, gather_on_load,
-                     fused_ffn)
+                     fused_ffn, fused_combine, fused_dispatch, pipeline)
     if ws is None:
         ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
     _need(ws, "ws", torch.uint8, None, dev)
@@ -549,7 +594,8 @@ def moe_kernel_launches_per_forward_fp8(desc: LayerDesc, with_router: bool) -> i
 def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=True,
                           logits=None, Wr=None, Y=None, topk_idx_out=None, gates_out=None,
                           counts_out=None, ws=None, stream=None, temperature=1.0, min_prob=0.0,
-                          gather_on_load=False, fused_ffn=False):
+                          gather_on_load=False, fused_ffn=False, fused_combine=False,
+                          fused_dispatch=False, pipeline=False):
     """The layer with FP8 dispatch and FP8 GEMM-1 (W1q, w1_scale from moe_quantize_experts_fp8)."""
     lib = load_library()
     T, d = X.shape
@@ -571,7 +617,7 @@ def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=
     if counts_out is not None:
         _need(counts_out, "counts_out", torch.int32, (E,), dev)
     desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, gather_on_load,
-                     fused_ffn)
+                     fused_ffn, fused_combine, fused_dispatch, pipeline)
     if ws is None:
         ws = torch.empty(max(moe_workspace_size(desc), 16), dtype=torch.uint8, device=dev)
     _need(ws, "ws", torch.uint8, None, dev)
@@ -606,11 +652,13 @@ class MoeLayer:
     """A layer's weights plus a reusable workspace (allocation stays outside the call)."""
 
     def __init__(self, W1, W2, k, score="softmax", renormalize=True, Wr=None, temperature=1.0,
-                 min_prob=0.0, fp8=False, gather_on_load=False, fused_ffn=False):
+                 min_prob=0.0, fp8=False, gather_on_load=False, fused_ffn=False,
+                 fused_combine=False, fused_dispatch=False, pipeline=False):
         self.W1, self.W2, self.Wr = W1, W2, Wr
         self.fp8 = bool(fp8)
-        self.gather_on_load = bool(gather_on_load)
-        self.fused_ffn = bool(fused_ffn)
+        self.flags = dict(gather_on_load=bool(gather_on_load), fused_ffn=bool(fused_ffn),
+                          fused_combine=bool(fused_combine), fused_dispatch=bool(fused_dispatch),
+                          pipeline=bool(pipeline))
         # FP8 mode keeps W1 as E4M3 codes with per-expert scales (quantised once here)
         self.W1q, self.w1_scale = moe_quantize_experts_fp8(W1) if self.fp8 else (None, None)
         self.k, self.score, self.renormalize = k, score, renormalize
@@ -630,8 +678,7 @@ class MoeLayer:
         kw = dict(logits=logits, Wr=None if logits is not None else self.Wr, Y=Y,
                   topk_idx_out=topk_idx_out, gates_out=gates_out, counts_out=counts_out,
                   ws=self.workspace(X.shape[0]), stream=stream, temperature=self.temperature,
-                  min_prob=self.min_prob, gather_on_load=self.gather_on_load,
-                  fused_ffn=self.fused_ffn)
+                  min_prob=self.min_prob, **self.flags)
         if self.fp8:
             return moe_layer_forward_fp8(X, self.W1q, self.w1_scale, self.W2, self.k, self.score,
                                          self.renormalize, **kw)

@@ -127,9 +127,30 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
 // Workspace of the fused forward: sub-buffers, each 256-byte aligned.
 struct LayerWs {
-  size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, scale, ready,
+  size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, scale, ctr, part,
       total;
 };
+
+// Counter words of the layer workspace (all zeroed by one memset per forward):
+// the fused FFN's ticket and readiness counters (or GEMM-1's ticket), GEMM-2's
+// ticket, the dispatch chunks' counters, the fused combine's arrival words.
+struct LayerCtr {
+  int ffn, g2, disp, comb, used;
+};
+
+LayerCtr layer_ctr(const moe_layer_desc& d) {
+  const int R = d.T * d.k;
+  LayerCtr c;
+  c.ffn = 0;
+  c.g2 = moe::ffn_counter_words(R, d.E);
+  c.disp = c.g2 + 1;
+  c.comb = c.disp + moe::dispatch_counter_words(R);
+  const bool fused = (d.flags & MOE_LAYER_FUSED_FFN) != 0;
+  const bool comb = (d.flags & MOE_LAYER_FUSED_COMBINE) && d.k <= 2;
+  c.used = comb ? c.comb + moe::combine_counter_words(d.T, d.d)
+                : (fused && (d.flags & MOE_LAYER_FUSED_DISPATCH)) ? c.comb : c.disp;
+  return c;
+}
 
 size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
@@ -149,7 +170,10 @@ LayerWs layer_ws(const moe_layer_desc& d) {
   w.H = o;       o += up256(R * d.f * 2);
   w.Ye = o;      o += up256(R * d.d * 2);
   w.scale = o;   o += up256(2 * sizeof(float));  // FP8 mode: activation scale and amax
-  w.ready = o;   o += up256((size_t)moe::ffn_ready_count((int)R, d.E) * sizeof(uint32_t));
+  w.ctr = o;     o += up256((size_t)(moe::ffn_counter_words((int)R, d.E) + 1 +
+                                     moe::dispatch_counter_words((int)R) +
+                                     moe::combine_counter_words(d.T, d.d)) * sizeof(uint32_t));
+  w.part = o;    o += up256(T * d.d * sizeof(float));  // fused combine: fp32 partial rows
   w.total = o;
   return w;
 }
@@ -163,10 +187,13 @@ moe_status check_desc(const moe_layer_desc* desc) {
     return fail(MOE_ERR_INVALID_ARG, "unknown score");
   if (desc->renormalize != 0 && desc->renormalize != 1)
     return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
-  if (desc->flags & ~(MOE_LAYER_GATHER_ON_LOAD | MOE_LAYER_FUSED_FFN))
+  if (desc->flags & ~(MOE_LAYER_GATHER_ON_LOAD | MOE_LAYER_FUSED_FFN | MOE_LAYER_FUSED_COMBINE |
+                      MOE_LAYER_FUSED_DISPATCH))
     return fail(MOE_ERR_INVALID_ARG, "unknown flags");
   if ((desc->flags & MOE_LAYER_GATHER_ON_LOAD) && (desc->flags & MOE_LAYER_FUSED_FFN))
     return fail(MOE_ERR_UNSUPPORTED, "MOE_LAYER_GATHER_ON_LOAD with MOE_LAYER_FUSED_FFN");
+  if ((desc->flags & MOE_LAYER_FUSED_DISPATCH) && !(desc->flags & MOE_LAYER_FUSED_FFN))
+    return fail(MOE_ERR_INVALID_ARG, "MOE_LAYER_FUSED_DISPATCH needs MOE_LAYER_FUSED_FFN");
   if (!std::isfinite(desc->temperature) || desc->temperature < 0.f)
     return fail(MOE_ERR_INVALID_ARG, "temperature must be >= 0 (0 reads as 1)");
   if (!std::isfinite(desc->min_prob)) return fail(MOE_ERR_INVALID_ARG, "min_prob must be finite");
@@ -228,27 +255,58 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   void* H = base + w.H;
   void* Ye = base + w.Ye;
   float* x_scale = reinterpret_cast<float*>(base + w.scale);
-  uint32_t* ready = reinterpret_cast<uint32_t*>(base + w.ready);
+  uint32_t* ctr = reinterpret_cast<uint32_t*>(base + w.ctr);
+  const LayerCtr lc = layer_ctr(d);
   const int R = d.T * d.k;
+  const bool fused = (d.flags & MOE_LAYER_FUSED_FFN) != 0;
+  const bool gather = (d.flags & MOE_LAYER_GATHER_ON_LOAD) != 0;
+  const bool comb = (d.flags & MOE_LAYER_FUSED_COMBINE) && d.k <= 2;
+  const bool fdisp = fused && (d.flags & MOE_LAYER_FUSED_DISPATCH) && !fp8;
 
   if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, *dev, s), "router_logits");
+  // The routing kernel also clears the tickets, readiness and combine
+  // counters (they start at zero in every forward) and, with the combine in
+  // GEMM-2's epilogue, writes the zero outputs of tokens whose slots were all
+  // dropped (no expert row reaches them).
+  const bool drops = d.min_prob > 0.f;
   MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
-                             d.min_prob, idx, gates, s),
+                             d.min_prob, idx, gates, s, (comb && drops) ? Y : nullptr, d.d, ctr,
+                             lc.used),
            "route");
   MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s), "layout");
+  // The two-launch path keeps the static balanced schedule (measured faster
+  // than tickets on uniform tiles); the fused launch always takes tickets.
+  moe::GemmExtras ex1, ex2;
+  if (comb) {
+    ex2.comb_Y = Y;
+    ex2.comb_src = src_of;
+    ex2.comb_row_of = row_of;
+    ex2.comb_gates = gates;
+    ex2.comb_part = reinterpret_cast<float*>(base + w.part);
+    ex2.comb_cnt = ctr + lc.comb;
+    ex2.comb_k = d.k;
+    ex2.comb_T = d.T;
+  }
   std::string err;
   cudaError_t e;
-  const bool gather = (d.flags & MOE_LAYER_GATHER_ON_LOAD) != 0;
-  if (d.flags & MOE_LAYER_FUSED_FFN) {  // both GEMMs in one persistent launch
-    if (fp8)
+  if (fused) {  // both GEMMs in one persistent launch
+    if (fdisp) {  // dispatch chunks run inside it
+      ex2.disp_X = X;
+      ex2.disp_src = src_of;
+      ex2.disp_k = d.k;
+      ex2.disp_T = d.T;
+      ex2.dready = ctr + lc.disp;
+    } else if (fp8) {
       MOE_CUDA(moe::launch_dispatch_fp8_rows(X, row_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
                "dispatch_fp8");
-    else
+    } else {
       MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+    }
     e = moe::launch_fused_ffn(Xe, x_scale, offsets, W1, W1s, W2, d.E, R, d.d, d.f, fp8, H, Ye,
-                              ready, *dev, s, &err);
+                              ctr + lc.ffn, true, *dev, s, &err, &ex2);
     if (e != cudaSuccess) return gemm_fail(e, err, "fused_ffn");
-    MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
+    if (!comb)
+      MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
     return MOE_OK;
   }
   if (gather) {  // dispatch fused into GEMM-1: its rows are read through src_of
@@ -264,15 +322,16 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
     MOE_CUDA(moe::launch_dispatch_fp8_rows(X, row_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
              "dispatch_fp8");
     e = moe::launch_grouped_gemm_fp8(Xe, x_scale, offsets, W1, W1s, d.E, R, d.f, d.d, true, H,
-                                     *dev, s, &err);
+                                     *dev, s, &err, &ex1);
   } else {
     MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
-    e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err);
+    e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err, &ex1);
   }
   if (e != cudaSuccess) return gemm_fail(e, err, "gemm1");
-  e = moe::launch_grouped_gemm(H, offsets, W2, d.E, R, d.d, d.f, false, Ye, *dev, s, &err);
+  e = moe::launch_grouped_gemm(H, offsets, W2, d.E, R, d.d, d.f, false, Ye, *dev, s, &err, &ex2);
   if (e != cudaSuccess) return gemm_fail(e, err, "gemm2");
-  MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
+  if (!comb)
+    MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
   return MOE_OK;
 }
 
@@ -595,7 +654,7 @@ moe_status moe_expert_ffn(const void* Xe, const int32_t* offsets, const void* W1
 
 size_t moe_expert_ffn_fused_workspace_size(int32_t E, int32_t R) {
   if (E < 1 || R < 0) return 0;
-  return up256((size_t)moe::ffn_ready_count(R, E) * sizeof(uint32_t));
+  return up256((size_t)moe::ffn_counter_words(R, E) * sizeof(uint32_t));
 }
 
 namespace {
@@ -624,7 +683,7 @@ moe_status ffn_fused(const void* A, const float* a_scale, const int32_t* offsets
   MOE_TRY(get_dev(&dev));
   std::string err;
   cudaError_t e = moe::launch_fused_ffn(A, a_scale, offsets, W1, w1_scale, W2, E, R, d, f, fp8,
-                                        H, Ye, static_cast<uint32_t*>(ws), *dev,
+                                        H, Ye, static_cast<uint32_t*>(ws), false, *dev,
                                         as_stream(stream), &err);
   if (e != cudaSuccess) return gemm_fail(e, err, "expert_ffn_fused");
   return MOE_OK;
@@ -645,6 +704,89 @@ moe_status moe_expert_ffn_fused_fp8(const void* Xeq, const float* x_scale,
                                     size_t ws_bytes, void* stream) {
   return ffn_fused(Xeq, x_scale, offsets, W1q, w1_scale, W2, E, R, d, f, H, Ye, ws, ws_bytes,
                    stream, true);
+}
+
+namespace {
+// Workspace of moe_ffn_pipeline: Xe, H, (k > 2) Ye, fp32 partial rows, counters.
+struct PipeWs {
+  size_t Xe, H, Ye, part, ctr, total;
+  int ctr_words;
+};
+PipeWs pipe_ws(int32_t T, int32_t d, int32_t E, int32_t k, int32_t f) {
+  PipeWs w;
+  const size_t R = (size_t)T * k;
+  size_t o = 0;
+  w.Xe = o;   o += up256(R * d * 2);
+  w.H = o;    o += up256(R * f * 2);
+  w.Ye = o;   o += k > 2 ? up256(R * d * 2) : 0;
+  w.part = o; o += k <= 2 ? up256((size_t)T * d * sizeof(float)) : 0;
+  w.ctr_words = moe::ffn_counter_words((int)R, E) + moe::dispatch_counter_words((int)R) +
+                (k <= 2 ? moe::combine_counter_words(T, d) : 0);
+  w.ctr = o;  o += up256((size_t)w.ctr_words * sizeof(uint32_t));
+  w.total = o;
+  return w;
+}
+}  // namespace
+
+size_t moe_ffn_pipeline_workspace_size(int32_t T, int32_t d, int32_t E, int32_t k, int32_t f) {
+  if (T < 0 || d < 1 || E < 1 || k < 1 || f < 1) return 0;
+  return pipe_ws(T, d, E, k, f).total;
+}
+
+moe_status moe_ffn_pipeline(const void* X, const int32_t* src_of, const int32_t* row_of,
+                            const float* gates, const int32_t* offsets, const void* W1,
+                            const void* W2, int32_t T, int32_t d, int32_t E, int32_t k,
+                            int32_t f, void* Y, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check_ET(T, E, k));
+  MOE_TRY(check_dim(d, "d"));
+  MOE_TRY(check_dim(f, "f"));
+  const int R = T * k;
+  MOE_TRY(check_gemm_shape(E, R, f, d, 1));
+  MOE_TRY(check_gemm_shape(E, R, d, f, 0));
+  if (T == 0) return MOE_OK;
+  MOE_TRY(check_ptr(X, "X"));
+  MOE_TRY(check_ptr4(src_of, "src_of"));
+  MOE_TRY(check_ptr4(row_of, "row_of"));
+  MOE_TRY(check_ptr4(gates, "gates"));
+  MOE_TRY(check_ptr4(offsets, "offsets"));
+  MOE_TRY(check_ptr(W1, "W1"));
+  MOE_TRY(check_ptr(W2, "W2"));
+  MOE_TRY(check_ptr(Y, "Y"));
+  const PipeWs w = pipe_ws(T, d, E, k, f);
+  if (ws_bytes < w.total) return fail(MOE_ERR_INVALID_ARG, "workspace too small");
+  MOE_TRY(check_ptr(ws, "ws"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  cudaStream_t s = as_stream(stream);
+  char* base = static_cast<char*>(ws);
+  uint32_t* ctr = reinterpret_cast<uint32_t*>(base + w.ctr);
+  MOE_CUDA(cudaMemsetAsync(ctr, 0, (size_t)w.ctr_words * sizeof(uint32_t), s), "memset counters");
+  const int nffn = moe::ffn_counter_words(R, E);
+  moe::GemmExtras ex;
+  ex.disp_X = X;
+  ex.disp_src = src_of;
+  ex.disp_k = k;
+  ex.disp_T = T;
+  ex.dready = ctr + nffn;
+  const bool comb = k <= 2;
+  if (comb) {
+    ex.comb_Y = Y;
+    ex.comb_src = src_of;
+    ex.comb_row_of = row_of;
+    ex.comb_gates = gates;
+    ex.comb_part = reinterpret_cast<float*>(base + w.part);
+    ex.comb_cnt = ctr + nffn + moe::dispatch_counter_words(R);
+    ex.comb_k = k;
+    ex.comb_T = T;
+  }
+  void* Ye = comb ? nullptr : base + w.Ye;
+  std::string err;
+  cudaError_t e = moe::launch_fused_ffn(base + w.Xe, nullptr, offsets, W1, nullptr, W2, E, R, d,
+                                        f, false, base + w.H, Ye, ctr, true, *dev, s, &err, &ex);
+  if (e != cudaSuccess) return gemm_fail(e, err, "ffn_pipeline");
+  if (!comb)
+    MOE_CUDA(moe::launch_combine(Ye, row_of, gates, T, d, k, Y, *dev, s), "combine");
+  return MOE_OK;
 }
 
 moe_status moe_combine(const void* Ye, const int32_t* row_of, const float* gates, int32_t T,
@@ -671,19 +813,25 @@ size_t moe_workspace_size(const moe_layer_desc* desc) {
 
 int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with_router) {
   if (check_desc(desc) != MOE_OK || desc->T == 0) return 0;
-  // [router linear] + route + layout + [dispatch] + 2 GEMMs (1 fused) + combine
-  const int dispatch = (desc->flags & MOE_LAYER_GATHER_ON_LOAD) ? 0 : 1;
-  const int gemms = (desc->flags & MOE_LAYER_FUSED_FFN) ? 1 : 2;
+  // [router linear] + route + layout + [dispatch] + 2 GEMMs (1 fused) + [combine]
+  const int f = desc->flags;
+  const bool fused = (f & MOE_LAYER_FUSED_FFN) != 0;
+  const int dispatch =
+      ((f & MOE_LAYER_GATHER_ON_LOAD) || (fused && (f & MOE_LAYER_FUSED_DISPATCH))) ? 0 : 1;
+  const int gemms = fused ? 1 : 2;
+  const int combine = ((f & MOE_LAYER_FUSED_COMBINE) && desc->k <= 2) ? 0 : 1;
   return (with_router ? 1 : 0) + 1 + moe::layout_kernel_count((int64_t)desc->T * desc->k) +
-         dispatch + gemms + 1;
+         dispatch + gemms + combine;
 }
 
 int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t with_router) {
   if (check_desc(desc) != MOE_OK || desc->T == 0) return 0;
   // the quantising dispatch (or, gathering, the quantisation of X) is the
-  // absmax kernel plus one
-  const int dispatch = (desc->flags & MOE_LAYER_GATHER_ON_LOAD) ? 0 : 1;
-  return moe_kernel_launches_per_forward(desc, with_router) - dispatch +
+  // absmax kernel plus one; FP8 mode has no dispatch items
+  moe_layer_desc d = *desc;
+  d.flags &= ~MOE_LAYER_FUSED_DISPATCH;
+  const int dispatch = (d.flags & MOE_LAYER_GATHER_ON_LOAD) ? 0 : 1;
+  return moe_kernel_launches_per_forward(&d, with_router) - dispatch +
          moe::fp8_dispatch_kernel_count(desc->T);
 }
 

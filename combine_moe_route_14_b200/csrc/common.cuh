@@ -41,6 +41,18 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
+// Relaxed (strong, unordered) load: several can be in flight at once; follow
+// them with fence_acq_rel_gpu() to acquire what they observed.
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 __device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -93,6 +105,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with cluster-scope acquire: for barriers that a peer CTA of the
+// cluster arrives on after writing this CTA's shared memory (st.shared::cluster).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait as mbar_wait, with cluster-scope acquire (see above).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  uint32_t* status, volatile int* abort_flag,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        flag_error(status, MOE_DEV_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// 32-bit store into the shared memory of a CTA of the cluster (own or peer),
+// given the shared::cluster address.
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
 // Plain arrive (count 1) on a barrier of this CTA, release order.
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
@@ -133,6 +184,60 @@ __device__ __forceinline__ bool wait_count_geq(const uint32_t* p, uint32_t targe
   for (uint32_t it = 1;; ++it) {
     __nanosleep(128);
     if (ld_acquire_gpu(p) >= target) return true;
+    if ((it & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        flag_error(status, MOE_DEV_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// True when every counter p[0..n) has reached target (relaxed loads, all in
+// flight together; no ordering).
+__device__ __forceinline__ bool counts_reached(const uint32_t* p, int n, uint32_t target) {
+  bool ok = true;
+  for (int i = 0; i < n; ++i) ok &= ld_relaxed_gpu(p + i) >= target;
+  return ok;
+}
+
+// Bounded wait until every counter p[0..n) reaches target, then an acquire
+// fence (the writers' data published before their counts is visible).  As
+// wait_count_geq otherwise.
+__device__ __forceinline__ bool wait_counts_geq(const uint32_t* p, int n, uint32_t target,
+                                                uint32_t* status, volatile int* abort_flag,
+                                                uint64_t limit_ns = kWaitLimitNs) {
+  if (!counts_reached(p, n, target)) {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+      __nanosleep(128);
+      if (counts_reached(p, n, target)) break;
+      if ((it & 15u) == 0) {
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+          flag_error(status, MOE_DEV_TIMEOUT);
+          *abort_flag = 1;
+          return false;
+        }
+      }
+    }
+  }
+  fence_acq_rel_gpu();
+  return true;
+}
+
+// Bounded wait until (word at p) & mask is non-zero, acquire order; as
+// wait_count_geq otherwise.
+__device__ __forceinline__ bool wait_bits_set(const uint32_t* p, uint32_t mask, uint32_t* status,
+                                              volatile int* abort_flag,
+                                              uint64_t limit_ns = kWaitLimitNs) {
+  if (ld_acquire_gpu(p) & mask) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(p) & mask) return true;
     if ((it & 15u) == 0) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {

@@ -87,18 +87,33 @@ constexpr int EPI_WARPS = 8;                 // two per SM sub-partition
 // Gather form: gather4 requests are issued one lane at a time, about one per
 // ~90 cycles per issuing warp, so the token rows are fetched by several warps.
 constexpr int kGatherWarps = MOE_GATHER_WARPS;
-// Warp roles: warp 0 streams weights, warps 1..NTOK stream token rows, warp
-// MMA issues the MMAs (leader CTA), warps EPI0.. drain the accumulators.
-template <bool kGather> struct Roles {
+// Warp roles: warp 0 streams weights, the next NTOK warps token rows, warp
+// MMA issues the MMAs (leader CTA), warp SCHED (leader CTA, dynamic
+// schedule) publishes the work items, warps EPI0.. drain the accumulators.
+template <bool kGather, int kPair> struct Roles {
+  static constexpr int NW = 1;
   static constexpr int NTOK = kGather ? kGatherWarps : 1;
-  static constexpr int MMA = 1 + NTOK;
-  static constexpr int EPI0 = MMA + 1;
+  static constexpr int NPROD = NW + NTOK;
+  static constexpr int MMA = NPROD;
+  static constexpr int SCHED = MMA + 1;
+  static constexpr int EPI0 = SCHED + 1;
   static constexpr int THREADS = (EPI0 + EPI_WARPS) * 32;
+  // arrivals on a stage's full barrier (leader CTA): one per issuing warp,
+  // one for all the gather warps together
+  static constexpr int FULL_ARRIVALS = NW + (kGather ? 1 : NTOK);
 };
 constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
 constexpr int MAX_STAGES = 8;                // barrier slots; the ring uses Args::stages of them
 constexpr size_t kSmemBudget = 232448;       // B200 opt-in shared memory per block
 constexpr uint64_t kDrainLimitNs = 20ull * 1000ull * 1000ull;  // 20 ms
+// Work items reach every role of a cluster through a queue of this depth in
+// shared memory, filled by the leader CTA's weight producer (the role that
+// runs furthest ahead); a slot is reused once every other role has read it.
+constexpr int kQueue = 4;
+// Dispatch items of the fused FFN: layout rows per item, and 16-byte vectors
+// in flight per lane while copying them.
+constexpr int kDispRows = 64;
+constexpr int kDispUnroll = 8;
 
 // kPair = 1: one CTA computes a 128-feature x N-token tile (cta_group::1).
 // kPair = 2: a cluster of two CTAs computes a 256-feature x N-token tile with
@@ -111,14 +126,15 @@ template <int kPair> struct Cfg {
   // a single CTA (its 48 KB K-block already leaves only 4 slots)
   static constexpr int KPS = kPair == 2 ? 2 : 1;
   static constexpr int STAGE = KPS * (A_STAGE + B_STAGE);  // one ring slot
-  static constexpr int NUM_BARS = 2 * MAX_STAGES + 4 + 1;
+  static constexpr int NUM_BARS = 2 * MAX_STAGES + 4 + 1 + 2 * kQueue + 1;
   static constexpr int FEAT = BM * kPair;                // output features per tile
 };
 
 // Shared memory: the stage ring, barriers, and the per-expert tile table.
 template <int kPair>
 __host__ __device__ constexpr size_t fixed_smem(int E) {
-  return 1024 /* alignment slack */ + Cfg<kPair>::NUM_BARS * 8 + 16 + (size_t)4 * (E + 1) * sizeof(int);
+  return 1024 /* alignment slack */ + Cfg<kPair>::NUM_BARS * 8 + 16 + kQueue * sizeof(int) +
+         (size_t)4 * (E + 1) * sizeof(int);
 }
 template <int kPair>
 __host__ __device__ constexpr size_t smem_bytes(int E, int stages) {
@@ -150,6 +166,29 @@ struct Args {
   int N2, n_fblocks2, num_kb2;
   uint32_t* ready;         // [token blocks]: GEMM-1 epilogue warps done, per token block
   uint32_t ready_target;   // arrivals that complete a token block
+  // Dynamic schedule: non-null -> clusters take items from this counter, in
+  // item order (zeroed before the launch); null -> static round-robin.
+  uint32_t* ticket;
+  // Dispatch items (fused form with a ticket): the epilogue warps gather the
+  // token operand's rows A[r] = disp_X[disp_src[r] / disp_k] in chunks of
+  // kDispRows rows; GEMM-1 tiles wait for the chunks under their rows.
+  const uint4* disp_X;     // [disp_T, K] bf16 (null: no dispatch items)
+  uint4* disp_A;           // the token operand A [R, K], written here
+  const int32_t* disp_src; // src_of [R]
+  int disp_k, disp_T, disp_vecs;  // disp_vecs = K / 8
+  uint32_t* dready;        // [ceil(R / kDispRows)] arrivals per chunk
+  // Combine in the epilogue of the GEMM without GELU (GEMM-2), k <= 2:
+  // Y[t] = bf16(sum_j gates[t, j] * acc(row_of[t*k + j])).  A token with one
+  // kept slot is written at once; with two, the first slot to arrive stores
+  // its gate-weighted fp32 row in comb_part and raises a flag, and the second
+  // adds it to its own and writes Y.  Rows of `out` are not stored.
+  uint16_t* comb_Y;            // [comb_T, N] bf16 (null: store `out` as usual)
+  const int32_t* comb_src;     // src_of [R]
+  const int32_t* comb_row_of;  // row_of [comb_T * comb_k]
+  const float* comb_gates;     // [comb_T, comb_k]
+  float* comb_part;            // [comb_T, N] fp32
+  uint32_t* comb_cnt;          // [comb_T * ceil(N / 32)] arrival words, zeroed before the launch
+  int comb_k, comb_T;
 };
 
 struct Tile {
@@ -214,7 +253,7 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
 }
 
 template <bool kGelu, int kPair, bool kFp8, bool kGather, bool kFused>
-__global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
+__global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x,
                         const __grid_constant__ CUtensorMap tm_xw,
@@ -222,11 +261,14 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
                         const __grid_constant__ CUtensorMap tm_x2,
                         const __grid_constant__ CUtensorMap tm_xw2, const Args args) {
   using C = Cfg<kPair>;
-  using Ro = Roles<kGather>;
+  using Ro = Roles<kGather, kPair>;
   constexpr int KPS = C::KPS;
   constexpr int KB = kFp8 ? BK_FP8 : BK;  // K values per stage (128 bytes of a row)
   const int STAGES = args.stages;
   constexpr int B_STAGE = C::B_STAGE;
+  // queue readers: the producers and epilogue warps of both CTAs and the
+  // leader's MMA warp
+  constexpr uint32_t kQReaders = kPair * Ro::NPROD + 1 + kPair * EPI_WARPS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -238,10 +280,14 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
   uint64_t* tfull = bars + 2 * MAX_STAGES; // per CTA: accumulator ready
   uint64_t* tempty = tfull + 2;        // leader CTA: both CTAs' epilogues drained it
   uint64_t* drain = tempty + 2;
+  uint64_t* qfull = drain + 1;         // per CTA: queue slot holds the next item
+  uint64_t* qempty = qfull + kQueue;   // leader CTA: every reader has taken the slot
+  uint64_t* qprod = qempty + kQueue;   // leader CTA: its weight producer has taken an item
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+  volatile int* s_queue = reinterpret_cast<volatile int*>(s_tmem + 4);
   const int E = args.E;
-  int* s_lo = reinterpret_cast<int*>(s_tmem + 4);
+  int* s_lo = reinterpret_cast<int*>(s_tmem + 4 + kQueue);
   int* s_hi = s_lo + (E + 1);
   int* s_start = s_hi + (E + 1);
   int* s_start2 = s_start + (E + 1);  // fused form: GEMM-2's per-expert first tile
@@ -254,7 +300,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 2);  // the two producers of the leader CTA
+      mbar_init(&full[s], Ro::FULL_ARRIVALS);  // the issuing warps of the leader CTA
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -262,6 +308,11 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
       mbar_init(&tempty[a], kPair * EPI_WARPS);
     }
     mbar_init(drain, 1);
+    for (int q = 0; q < kQueue; ++q) {
+      mbar_init(&qfull[q], 1);
+      mbar_init(&qempty[q], kQReaders);
+    }
+    mbar_init(qprod, 1);
     *s_abort = 0;
     fence_mbarrier_init();
   }
@@ -323,24 +374,37 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
   tc_fence_after_sync();
   const uint32_t tmem_base = *s_tmem;
   const int tiles0 = s_start[E];
-  const int total_tiles = tiles0 + (kFused ? s_start2[E] : 0);
-  // Balanced grid: the fewest clusters that still need the same number of
-  // rounds of the static schedule (the tile count is known only here, from
-  // the routing).  A last round with a few busy clusters would otherwise set
-  // the kernel's time while most SMs idle; e.g. 448 tiles over 74 clusters
-  // run 6 full rounds and a seventh of 4 tiles, over 64 clusters 7 full
-  // rounds.  Surplus clusters take no tile.
-  const int rounds = (total_tiles + ncl_launched - 1) / max(ncl_launched, 1);
-  const int ncl = rounds > 0 ? (total_tiles + rounds - 1) / rounds : ncl_launched;
-  const int first_tile = cid < ncl ? cid : total_tiles;
-  // tile -> (tile, phase); phase 1 only in the fused form
-  auto tile_at = [&](int tile, int& phase) -> Tile {
-    if (kFused && tile >= tiles0) {
+  // Items, in the order clusters take them: dispatch chunks (fused form with
+  // dispatch), then GEMM-1's tiles, then (fused form) GEMM-2's.  An item only
+  // ever waits on items before it, so with tickets taken in this order every
+  // wait ends, however many clusters are resident.
+  const int kept = s_hi[E - 1];  // rows of kept slots: offsets[E], clamped
+  const bool disp = kFused && !kGather && args.disp_X != nullptr && args.ticket != nullptr;
+  const int n_disp = disp ? (kept + kDispRows - 1) / kDispRows : 0;
+  const int total_items = n_disp + tiles0 + (kFused ? s_start2[E] : 0);
+  // Static schedule (no ticket): balanced grid, the fewest clusters that
+  // still need the same number of rounds (the tile count is known only here,
+  // from the routing).  A last round with a few busy clusters would otherwise
+  // set the kernel's time while most SMs idle; e.g. 448 tiles over 74
+  // clusters run 6 full rounds and a seventh of 4 tiles, over 64 clusters 7
+  // full rounds.  Surplus clusters take no tile.
+  const int rounds = (total_items + ncl_launched - 1) / max(ncl_launched, 1);
+  const int ncl = rounds > 0 ? (total_items + rounds - 1) / rounds : ncl_launched;
+  // item -> (tile, phase); phase -1: dispatch chunk `chunk`; 1: GEMM-2 of the fused form
+  auto item_at = [&](int x, int& phase, int& chunk) -> Tile {
+    chunk = -1;
+    if (x < n_disp) {
+      phase = -1;
+      chunk = x;
+      return Tile{0, 0, 0, 0};
+    }
+    x -= n_disp;
+    if (kFused && x >= tiles0) {
       phase = 1;
-      return decode(tile - tiles0, s_start2, s_lo, s_hi, E);
+      return decode(x - tiles0, s_start2, s_lo, s_hi, E);
     }
     phase = 0;
-    return decode(tile, s_start, s_lo, s_hi, E);
+    return decode(x, s_start, s_lo, s_hi, E);
   };
   // fused form: index of the token block holding a tile's rows
   auto block_of = [&](const Tile& t) -> int {
@@ -349,16 +413,96 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
   // the leader's barriers as cluster addresses (the CTA's own when kPair == 1)
   const uint32_t full_lead = kPair == 2 ? cluster_map(smem_u32(full), 0) : smem_u32(full);
   const uint32_t tempty_lead = kPair == 2 ? cluster_map(smem_u32(tempty), 0) : smem_u32(tempty);
+  const uint32_t qempty_lead = kPair == 2 ? cluster_map(smem_u32(qempty), 0) : smem_u32(qempty);
 
-  if (warp <= Ro::NTOK) {
+  // Static schedule: every role computes this cluster's i-th item itself.
+  // Dynamic schedule (a ticket): queue slot i % kQueue carries this
+  // cluster's i-th item (-1: no more).  fill(): the leader's scheduler warp
+  // takes the next ticket and publishes the item in both CTAs; take(): every
+  // role reads it.  Both are called by a whole warp; false = aborted.  The
+  // scheduler claims item i + 1 once the weight producer has taken item i:
+  // one item ahead, so the ticket's round trip to L2 is hidden behind a
+  // tile, and a cluster never holds tiles it has not started while others
+  // run dry at the end (claiming further ahead measured slower on uniform
+  // tiles: up to a whole extra round).  kQueue slots cover the lag of the
+  // slowest role (the epilogue).
+  auto fill = [&](int i, int& item) -> bool {
+    const int q = i % kQueue;
+    const uint32_t ph = (uint32_t)(i / kQueue) & 1u;
+    int v = -1;
+    bool ok = true;
+    if (lane == 0) {
+      ok = mbar_wait_cluster(&qempty[q], ph ^ 1u, args.status, s_abort);
+      if (ok) {
+        if (args.ticket) {
+          const uint32_t x = atomicAdd(args.ticket, 1u);
+          v = x < (uint32_t)total_items ? (int)x : -1;
+        } else {
+          const long long x = (long long)cid + (long long)i * ncl;
+          v = (cid < ncl && x < total_items) ? (int)x : -1;
+        }
+        s_queue[q] = v;
+        if (kPair == 2) {
+          st_shared_cluster_u32(cluster_map(smem_u32((const void*)(s_queue + q)), 1), (uint32_t)v);
+          mbar_arrive_cluster(cluster_map(smem_u32(&qfull[q]), 1));
+        }
+        mbar_arrive(&qfull[q]);
+      }
+    }
+    item = __shfl_sync(0xffffffffu, v, 0);
+    return __shfl_sync(0xffffffffu, ok, 0);
+  };
+  const bool dyn = args.ticket != nullptr;
+  auto static_item = [&](int i) -> int {
+    const long long x = (long long)cid + (long long)i * ncl;
+    return (cid < ncl && x < total_items) ? (int)x : -1;
+  };
+  auto take = [&](int i, int& item) -> bool {
+    const int q = i % kQueue;
+    const uint32_t ph = (uint32_t)(i / kQueue) & 1u;
+    const bool got = mbar_wait_cluster(&qfull[q], ph, args.status, s_abort);
+    if (!__all_sync(0xffffffffu, got)) {
+      item = -1;
+      return false;
+    }
+    item = s_queue[q];
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(qempty_lead + (uint32_t)q * 8u);
+    return true;
+  };
+  auto next_item = [&](int i, int& item) -> bool {
+    if (!dyn) {
+      item = static_item(i);
+      return true;
+    }
+    return take(i, item);
+  };
+  // The counters that gate a tile's token rows: GEMM-2 tiles wait for their
+  // token block's H (GEMM-1 epilogue arrivals), GEMM-1 tiles of the fused
+  // form with dispatch items for the chunks under their rows.
+  auto gate = [&](const Tile& tt, bool ph1, const uint32_t*& cp, int& cn, uint32_t& tgt) {
+    if (ph1) {
+      cp = args.ready + block_of(tt);
+      cn = 1;
+      tgt = args.ready_target;
+    } else {
+      const int c0 = tt.row0 / kDispRows;
+      cp = args.dready + c0;
+      cn = (tt.row0 + tt.ntok - 1) / kDispRows - c0 + 1;  // <= BN / kDispRows + 1
+      tgt = (uint32_t)(kPair * EPI_WARPS);
+    }
+  };
+  constexpr int kMaxGate = BN / kDispRows + 1;
+
+  if (warp < Ro::NPROD) {
     // ------------------------------------------------------------ producers (both CTAs)
     // Warp 0 streams the weight rows, warp 1 (and in the gather form warps
     // 2..NTOK) the token rows, each into the same ring of stages: separate
     // issuing threads keep more TMA requests in flight than one.  In the
     // leader CTA warps 0 and 1 arm the stage's barrier with the bytes of
     // their operand in both CTAs of the pair.
-    const bool is_w = warp == 0;
-    const int tw = warp - 1;  // token warp index
+    const bool is_w = warp < Ro::NW;
+    const int tw = warp - Ro::NW;  // token warp index
     const uint64_t pol = is_w ? l2_policy_evict_normal()  // shared by the CTAs of a feature block
                               : l2_policy_evict_last();   // re-read by every feature block
     int s = 0;
@@ -366,31 +510,43 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     uint32_t issued = 0;  // bit s: stage s has a load in flight or landed
     uint32_t last_ph = 0; // bit s: parity of the last load issued on stage s
     bool ok = true;
-    // fused form: the readiness count of this producer's next GEMM-2 tile,
-    // loaded (acquire) one tile ahead so that its L2 round trip overlaps the
-    // current tile's loads; counts only grow, so a count seen as complete stays so
-    uint32_t next_count = 0;
-    for (int tile = first_tile; ok && tile < total_tiles; tile += ncl) {
-      int phase;
-      const Tile t = tile_at(tile, phase);
+    // token producers, dynamic schedule: the gate counters of the next item,
+    // loaded while this item's loads are issued (counts only grow, so a
+    // complete count seen early stays complete)
+    int peek_x = -1, peek_n = 0;
+    uint32_t peek_v[kMaxGate], peek_tgt = 0;
+    for (int qi = 0; ok; ++qi) {
+      int x;
+      ok = next_item(qi, x);
+      if (!ok || x < 0) break;
+      if (dyn && warp == 0 && rank == 0 && lane == 0) mbar_arrive(qprod);  // claim the next
+      int phase, chunk;
+      const Tile t = item_at(x, phase, chunk);
+      if (phase < 0) continue;  // a dispatch chunk: the epilogue warps copy it
       const bool p1 = kFused && phase == 1;
-      const uint32_t this_count = next_count;
-      if (kFused && !is_w && lane == 0 && tile + ncl < total_tiles) {
-        int nphase;
-        const Tile nt = tile_at(tile + ncl, nphase);
-        if (nphase == 1) next_count = ld_acquire_gpu(args.ready + block_of(nt));
-      }
       const CUtensorMap* map_w = p1 ? &tm_w2 : &tm_w;
       const CUtensorMap* map_x = p1 ? &tm_x2 : &tm_x;
       const CUtensorMap* map_xw = p1 ? &tm_xw2 : &tm_xw;
       const int kbv = (kFp8 && !p1) ? BK_FP8 : BK;  // K values per stage in this phase
       const int nkb = p1 ? args.num_kb2 : args.num_kb;
       const int Np = p1 ? args.N2 : args.N;
-      if (p1 && !is_w) {  // GEMM-2 reads H rows that GEMM-1 tiles of other CTAs store
+      if (!is_w && (p1 || disp)) {
+        // Token rows written by other CTAs in this launch: GEMM-2 reads H rows
+        // that GEMM-1 tiles store, GEMM-1 (with dispatch items) reads rows
+        // that dispatch chunks copy.  Wait (bounded) for their counts, acquire,
+        // then order those generic-proxy stores before our TMA reads.
         bool rdy = true;
         if (lane == 0) {
-          rdy = this_count >= args.ready_target ||
-                wait_count_geq(args.ready + block_of(t), args.ready_target, args.status, s_abort);
+          const uint32_t* cp;
+          int cn;
+          uint32_t tgt;
+          gate(t, p1, cp, cn, tgt);
+          bool early = x == peek_x;  // counts read one item ahead, all complete?
+#pragma unroll
+          for (int i = 0; i < kMaxGate; ++i)
+            if (i < peek_n) early &= peek_v[i] >= peek_tgt;
+          if (early) fence_acq_rel_gpu();
+          else rdy = wait_counts_geq(cp, cn, tgt, args.status, s_abort);
           if (rdy) fence_proxy_async_global();
         }
         if (!__shfl_sync(0xffffffffu, rdy, 0)) {
@@ -436,8 +592,33 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
         }
       }
       const uint32_t gbytes = (uint32_t)(kPair * half * 128);
+      // dynamic schedule: look for the next item while this one streams (it
+      // is published about one ticket round trip after this one was taken)
+      bool peeking = dyn && !is_w && lane == 0;
+      if (peeking) {
+        peek_x = -1;
+        peek_n = 0;
+      }
       for (int ks = 0; ks * KPS < nkb; ++ks) {  // ring slot of K-blocks ks*KPS ..
         const int nsub = min(KPS, nkb - ks * KPS);
+        if (peeking) {
+          const int q1 = (qi + 1) % kQueue;
+          if (mbar_try_wait_cluster(&qfull[q1], (uint32_t)((qi + 1) / kQueue) & 1u)) {
+            peeking = false;
+            const int xn = s_queue[q1];
+            int phn = -1, chn;
+            const Tile tn = xn >= 0 ? item_at(xn, phn, chn) : Tile{0, 0, 0, 0};
+            const bool p1n = kFused && phn == 1;
+            if (phn >= 0 && (p1n || disp)) {  // its gate counts, loaded while we stream
+              const uint32_t* cpn;
+              gate(tn, p1n, cpn, peek_n, peek_tgt);
+#pragma unroll
+              for (int i = 0; i < kMaxGate; ++i)
+                if (i < peek_n) peek_v[i] = ld_relaxed_gpu(cpn + i);
+              peek_x = xn;
+            }
+          }
+        }
         ok = warp_wait(&empty[s], ph ^ 1u, args.status, s_abort);
         if (!ok) break;
         if (kGather && !is_w) {
@@ -483,22 +664,36 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
         }
       }
     }
-    if (!ok && rank == 0 && is_w) {  // let issued copies land before the CTA leaves
+    if (!ok && rank == 0 && warp == 0) {  // let issued copies land before the CTA leaves
       int dummy = 0;
       for (int q = 0; q < STAGES; ++q)
         if ((issued >> q) & 1u)
           mbar_wait(&full[q], (last_ph >> q) & 1u, nullptr, (volatile int*)&dummy, kDrainLimitNs);
+    }
+  } else if (warp == Ro::SCHED) {
+    // ------------------------------------------------------------ scheduler (leader, tickets)
+    if (rank == 0 && dyn) {
+      for (int qi = 0;; ++qi) {
+        // item qi - 1 taken by the weight producer (bounded wait)
+        if (qi > 0 && !warp_wait(qprod, (uint32_t)(qi - 1) & 1u, args.status, s_abort)) break;
+        int x;
+        if (!fill(qi, x) || x < 0) break;
+      }
     }
   } else if (warp == Ro::MMA) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (rank == 0) {
       int s = 0;
       uint32_t ph = 0;
-      int it = 0;
+      int it = 0;  // GEMM tiles so far (selects the accumulator)
       bool ok = true;
-      for (int tile = first_tile; ok && tile < total_tiles; tile += ncl, ++it) {
-        int phase;
-        const Tile t = tile_at(tile, phase);
+      for (int qi = 0; ok; ++qi) {
+        int x;
+        ok = next_item(qi, x);
+        if (!ok || x < 0) break;
+        int phase, chunk;
+        const Tile t = item_at(x, phase, chunk);
+        if (phase < 0) continue;
         const bool p1 = kFused && phase == 1;
         const bool f8 = kFp8 && !p1;  // GEMM-2 of the fused form is bf16
         const int nkb = p1 ? args.num_kb2 : args.num_kb;
@@ -507,6 +702,7 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
                                   : idesc_bf16_f32((uint32_t)C::FEAT, nmma);
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)((it >> 1) & 1);
+        ++it;
         ok = warp_wait(&tempty[acc], aph ^ 1u, args.status, s_abort);
         if (!ok) break;
         tc_fence_after_sync();
@@ -561,21 +757,61 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
     // which span of the tile's 256 token columns (EPI_WARPS / 4 spans)
     constexpr int SPAN = BN / (EPI_WARPS / 4);
     const int hsel = (warp - Ro::EPI0) >> 2;
-    int it = 0;
-    for (int tile = first_tile; tile < total_tiles; tile += ncl, ++it) {
-      int phase;
-      const Tile t = tile_at(tile, phase);
+    int it = 0;  // GEMM tiles so far
+    for (int qi = 0;; ++qi) {
+      int x;
+      if (!next_item(qi, x) || x < 0) break;
+      int phase, chunk;
+      const Tile t = item_at(x, phase, chunk);
+      if (phase < 0) {
+        // ---- dispatch chunk: A[r] = X[src_of[r] / k] for rows [r0, r1), by
+        // the epilogue warps of both CTAs, then one arrival per warp
+        const int w = (int)rank * EPI_WARPS + (warp - Ro::EPI0);
+        const int r0 = chunk * kDispRows, r1 = min(r0 + kDispRows, kept);
+        const int vecs = args.disp_vecs;
+        const int nslots = args.disp_T * args.disp_k;
+        for (int r = r0 + w; r < r1; r += kPair * EPI_WARPS) {
+          const int src = __ldg(args.disp_src + r);
+          if (src < 0 || src >= nslots) {
+            if (lane == 0) flag_error(args.status, MOE_DEV_BAD_ROW);
+            continue;
+          }
+          const uint4* from = args.disp_X + (size_t)(src / args.disp_k) * vecs;
+          uint4* to = args.disp_A + (size_t)r * vecs;
+          for (int c0 = 0; c0 < vecs; c0 += 32 * kDispUnroll) {
+            uint4 v[kDispUnroll];
+#pragma unroll
+            for (int u = 0; u < kDispUnroll; ++u) {
+              const int c = c0 + u * 32 + lane;
+              if (c < vecs) v[u] = ld_stream_v4(from + c);
+            }
+#pragma unroll
+            for (int u = 0; u < kDispUnroll; ++u) {
+              const int c = c0 + u * 32 + lane;
+              if (c < vecs) to[c] = v[u];
+            }
+          }
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(args.dready + chunk, 1u);
+        continue;
+      }
       const bool p1 = kFused && phase == 1;
       const bool f8 = kFp8 && !p1;
       const bool gelu = kGelu && !p1;  // the fused form's GEMM-2 has no activation
+      // gate-weighted combine in this epilogue (GEMM-2: no activation)
+      const bool comb = args.comb_Y != nullptr && !gelu;
       uint16_t* out = p1 ? args.out2 : args.out;
       const int N = p1 ? args.N2 : args.N;
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
+      ++it;
       if (!warp_wait(&tfull[acc], aph, args.status, s_abort)) break;
       tc_fence_after_sync();
       // this lane's output feature; the warp covers 32 consecutive features
-      const int f = t.fb * C::FEAT + (int)rank * BM + q * 32 + lane;
+      const int f0 = t.fb * C::FEAT + (int)rank * BM + q * 32;
+      const int f = f0 + lane;
       const float sc = f8 ? __ldg(args.a_scale) * __ldg(args.w_scale + t.e) : 1.0f;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
       const int c_end = min(t.ntok, hsel * SPAN + SPAN);
@@ -587,14 +823,82 @@ __global__ void __launch_bounds__(Roles<kGather>::THREADS, 1)
         // warp writes 32 consecutive features of one token row: 64 contiguous
         // bytes per store instruction, no shared-memory transpose needed.
         const int jmax = min(32, t.ntok - c0);
-        uint16_t* col = out + (size_t)(t.row0 + c0) * N + f;
-        if (f < N) {
+        if (!comb) {
+          uint16_t* col = out + (size_t)(t.row0 + c0) * N + f;
+          if (f < N) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float x = __uint_as_float(v[j]);
-            if (f8) x *= sc;
-            if (gelu) x = gelu_erf(x);
-            if (j < jmax) col[(size_t)j * N] = to_bf16_bits(x);
+            for (int j = 0; j < 32; ++j) {
+              float x = __uint_as_float(v[j]);
+              if (f8) x *= sc;
+              if (gelu) x = gelu_erf(x);
+              if (j < jmax) col[(size_t)j * N] = to_bf16_bits(x);
+            }
+          }
+          continue;
+        }
+        // ---- combine: lane j describes token column j of this chunk.  A warp
+        // whose 32 features all lie past N (last feature block) has nothing
+        // to write, and its counter index would name the next token's word.
+        if (f0 >= N) continue;
+        int tok = 0, mode = 0;  // mode 1: the token's only kept slot; 2: one of two
+        float g = 0.f;
+        if (lane < jmax) {
+          const int sl = __ldg(args.comb_src + t.row0 + c0 + lane);
+          if (sl >= 0 && sl < args.comb_T * args.comb_k) {
+            tok = sl / args.comb_k;
+            g = __ldg(args.comb_gates + sl);
+            // k == 2: the token's slots are 2t and 2t + 1
+            mode = (args.comb_k == 2 && __ldg(args.comb_row_of + (sl ^ 1)) >= 0) ? 2 : 1;
+          } else {
+            flag_error(args.status, MOE_DEV_BAD_ROW);
+          }
+        }
+        uint32_t* cw = args.comb_cnt + (size_t)tok * (uint32_t)((N + 31) >> 5) + (f0 >> 5);
+        const uint32_t old = mode == 2 ? atomicAdd(cw, 1u) : 0u;
+        const uint32_t sole = __ballot_sync(0xffffffffu, mode == 1);
+        const uint32_t first = __ballot_sync(0xffffffffu, mode == 2 && old == 0u);
+        const uint32_t second = __ballot_sync(0xffffffffu, mode == 2 && old != 0u);
+        // Products and the sum are rounded explicitly (no fused multiply-add),
+        // so a token's two results give the same bits whichever arrives second.
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int tj = __shfl_sync(0xffffffffu, tok, j);
+          const float gj = __shfl_sync(0xffffffffu, g, j);
+          const float y = __fmul_rn(gj, __uint_as_float(v[j]));
+          if (f < N) {
+            if ((sole >> j) & 1u) args.comb_Y[(size_t)tj * N + f] = to_bf16_bits(y);
+            else if ((first >> j) & 1u) args.comb_part[(size_t)tj * N + f] = y;
+          }
+        }
+        if (first) {  // publish the partials, then one flag per token
+          __threadfence();
+          __syncwarp();
+          if ((first >> lane) & 1u) atomicOr(cw, 0x100u);
+        }
+        if (second) {  // the partner slot's flag, then its partial
+          bool got = true;
+          if ((second >> lane) & 1u) got = wait_bits_set(cw, 0x100u, args.status, s_abort);
+          if (!__all_sync(0xffffffffu, got)) continue;
+          __threadfence();
+          // the partners' partial rows, 8 loads in flight at a time
+#pragma unroll
+          for (int j0 = 0; j0 < 32; j0 += 8) {
+            float p[8];
+#pragma unroll
+            for (int j = j0; j < j0 + 8; ++j) {
+              const int tj = __shfl_sync(0xffffffffu, tok, j);
+              p[j - j0] = (((second >> j) & 1u) && f < N)
+                              ? __ldcg(args.comb_part + (size_t)tj * N + f) : 0.f;
+            }
+#pragma unroll
+            for (int j = j0; j < j0 + 8; ++j) {
+              const int tj = __shfl_sync(0xffffffffu, tok, j);
+              const float gj = __shfl_sync(0xffffffffu, g, j);
+              if (((second >> j) & 1u) && f < N) {
+                const float y = __fmul_rn(gj, __uint_as_float(v[j]));
+                args.comb_Y[(size_t)tj * N + f] = to_bf16_bits(__fadd_rn(p[j - j0], y));
+              }
+            }
           }
         }
       }
@@ -694,7 +998,7 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(2 * dev.sm_count, 1, 1);
-      cfg.blockDim = dim3(gg::Roles<kGather>::THREADS, 1, 1);
+      cfg.blockDim = dim3(gg::Roles<kGather, kPair>::THREADS, 1, 1);
       cfg.dynamicSmemBytes = smem_max;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
@@ -715,7 +1019,7 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3((unsigned)(units * kPair), 1, 1);
-  cfg.blockDim = dim3(gg::Roles<kGather>::THREADS, 1, 1);
+  cfg.blockDim = dim3(gg::Roles<kGather, kPair>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = gg::smem_bytes<kPair>(args.E, args.stages);
   cfg.stream = stream;
   cfg.attrs = attr;
@@ -727,6 +1031,23 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   return cudaLaunchKernelEx(&cfg, kern, tm_w, tm_x, tm_xw, w2, x2, xw2, args);
 }
 
+int combine_counter_words(int T, int N) { return T * ((N + 31) / 32); }
+int dispatch_counter_words(int R) { return (R + gg::kDispRows - 1) / gg::kDispRows; }
+
+// Copies the optional parts of a launch into the kernel arguments.
+static void apply_extras(gg::Args& args, const GemmExtras* ex) {
+  if (!ex) return;
+  args.ticket = ex->ticket;
+  args.comb_Y = static_cast<uint16_t*>(ex->comb_Y);
+  args.comb_src = ex->comb_src;
+  args.comb_row_of = ex->comb_row_of;
+  args.comb_gates = ex->comb_gates;
+  args.comb_part = ex->comb_part;
+  args.comb_cnt = ex->comb_cnt;
+  args.comb_k = ex->comb_k;
+  args.comb_T = ex->comb_T;
+}
+
 // Gather form: A is the token matrix [a_rows, K] and row r of the GEMM reads
 // A[gather_src[r] / gather_k]; otherwise A is [R, K] and gather_src is null.
 template <bool kFp8>
@@ -734,7 +1055,7 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
                                int gather_k, int a_rows, const int32_t* offsets, const void* W,
                                const float* w_scale, int E, int R, int N, int K, bool gelu,
                                void* out, const DeviceInfo& dev, cudaStream_t stream,
-                               std::string* err) {
+                               std::string* err, const GemmExtras* ex = nullptr) {
   if (R == 0 || N == 0) return cudaSuccess;
   const bool gather = gather_src != nullptr;
   // Paired CTAs (256 features per tile) unless the layer is too narrow to fill them.
@@ -767,6 +1088,8 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
   const int kb = kFp8 ? gg::BK_FP8 : gg::BK;
   args.num_kb = (K + kb - 1) / kb;
   args.stages = pair == 2 ? gg::stages_for<2>(E) : gg::stages_for<1>(E);
+  apply_extras(args, ex);
+  if (gelu) args.comb_Y = nullptr;  // the combine belongs to the GEMM without activation
   // an upper bound on the tile count: every expert adds at most one partial token block
   const long long max_tiles =
       ((long long)(R + gg::BN - 1) / gg::BN + E) * (long long)args.n_fblocks;
@@ -783,32 +1106,37 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
 
 cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const void* W, int E,
                                 int R, int N, int K, bool gelu, void* out,
-                                const DeviceInfo& dev, cudaStream_t stream, std::string* err) {
+                                const DeviceInfo& dev, cudaStream_t stream, std::string* err,
+                                const GemmExtras* ex) {
   return launch_gemm<false>(A, nullptr, nullptr, 1, R, offsets, W, nullptr, E, R, N, K, gelu,
-                            out, dev, stream, err);
+                            out, dev, stream, err, ex);
 }
 
 cudaError_t launch_grouped_gemm_fp8(const void* Aq, const float* a_scale, const int32_t* offsets,
                                     const void* Wq, const float* w_scale, int E, int R, int N,
                                     int K, bool gelu, void* out, const DeviceInfo& dev,
-                                    cudaStream_t stream, std::string* err) {
+                                    cudaStream_t stream, std::string* err, const GemmExtras* ex) {
   return launch_gemm<true>(Aq, a_scale, nullptr, 1, R, offsets, Wq, w_scale, E, R, N, K, gelu,
-                           out, dev, stream, err);
+                           out, dev, stream, err, ex);
 }
 
 // Fused FFN: H = act(A W1[e]^T) (A = Xe, bf16 or E4M3 codes), then
-// Ye = H W2[e]^T, in one persistent launch.  `ready` holds one counter per
-// token block (ffn_ready_count) and is zeroed here before the launch.
+// Ye = H W2[e]^T, in one persistent launch.  `ctr` holds the ticket (word 0)
+// and one readiness counter per token block (ffn_ready_count).
 int ffn_ready_count(int R, int E) { return (R + gg::BN - 1) / gg::BN + E; }
+int ffn_counter_words(int R, int E) { return 1 + ffn_ready_count(R, E); }
 
 cudaError_t launch_fused_ffn(const void* A, const float* a_scale, const int32_t* offsets,
                              const void* W1, const float* w1_scale, const void* W2, int E, int R,
-                             int d, int f, bool fp8, void* H, void* Ye, uint32_t* ready,
-                             const DeviceInfo& dev, cudaStream_t stream, std::string* err) {
+                             int d, int f, bool fp8, void* H, void* Ye, uint32_t* ctr,
+                             bool zeroed, const DeviceInfo& dev, cudaStream_t stream,
+                             std::string* err, const GemmExtras* ex) {
   if (R == 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(ready, 0, (size_t)ffn_ready_count(R, E) * sizeof(uint32_t),
-                                  stream);
-  if (e != cudaSuccess) return e;
+  if (!zeroed) {
+    cudaError_t e = cudaMemsetAsync(ctr, 0, (size_t)ffn_counter_words(R, E) * sizeof(uint32_t),
+                                    stream);
+    if (e != cudaSuccess) return e;
+  }
   // one pair setting for both phases: paired CTAs when both GEMMs are wide enough
   const int pair = (f > gg::BM && d > gg::BM) ? 2 : 1;
   CUtensorMap tm_w, tm_x, tm_xw, tm2[3];
@@ -838,11 +1166,26 @@ cudaError_t launch_fused_ffn(const void* A, const float* a_scale, const int32_t*
   args.N2 = d;
   args.n_fblocks2 = (d + gg::BM * pair - 1) / (gg::BM * pair);
   args.num_kb2 = (f + gg::BK - 1) / gg::BK;
-  args.ready = ready;
+  apply_extras(args, ex);
+  // Always the dynamic schedule: tickets are taken in item order, so a tile
+  // only ever waits on tiles that running clusters hold (any residency).
+  args.ticket = ctr;
+  args.ready = ctr + 1;
   args.ready_target = (uint32_t)(args.n_fblocks * pair * gg::EPI_WARPS);
+  long long items = 0;
+  if (ex && ex->disp_X && !fp8) {
+    args.disp_X = static_cast<const uint4*>(ex->disp_X);
+    args.disp_A = static_cast<uint4*>(const_cast<void*>(A));
+    args.disp_src = ex->disp_src;
+    args.disp_k = ex->disp_k;
+    args.disp_T = ex->disp_T;
+    args.disp_vecs = d / 8;
+    args.dready = ex->dready;
+    items = dispatch_counter_words(R);
+  }
   args.stages = pair == 2 ? gg::stages_for<2>(E) : gg::stages_for<1>(E);
-  const long long max_tiles = ((long long)(R + gg::BN - 1) / gg::BN + E) *
-                              (long long)(args.n_fblocks + args.n_fblocks2);
+  const long long max_tiles = items + ((long long)(R + gg::BN - 1) / gg::BN + E) *
+                                          (long long)(args.n_fblocks + args.n_fblocks2);
   if (fp8)
     return pair == 2 ? launch_variant<true, 2, true, false, true>(tm_w, tm_x, tm_xw, args, max_tiles,
                                                                   dev, stream, tm2)

@@ -28,9 +28,12 @@ const DeviceInfo* current_device_info(std::string* err);
 cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, int E, float* L,
                                  const DeviceInfo& dev, cudaStream_t stream);
 
+// zero_rows (optional): [T, zero_d] bf16 rows zeroed for tokens with no kept slot.
+// zero_words (optional): n_zero_words counter words cleared by the same launch.
 cudaError_t launch_route(const float* L, int T, int E, int k, int score, int renormalize,
                          float temperature, float min_prob, int32_t* idx, float* gates,
-                         cudaStream_t stream);
+                         cudaStream_t stream, void* zero_rows = nullptr, int zero_d = 0,
+                         uint32_t* zero_words = nullptr, int n_zero_words = 0);
 
 size_t layout_workspace_bytes(int64_t R, int E);
 // Number of kernels launch_layout issues for R slots.
@@ -52,18 +55,45 @@ cudaError_t launch_dispatch_fp8_rows(const void* X, const int32_t* row_of, int T
 cudaError_t launch_combine(const void* Ye, const int32_t* row_of, const float* gates, int T,
                            int d, int k, void* Y, const DeviceInfo& dev, cudaStream_t stream);
 
+// Optional parts of a grouped GEMM launch.
+struct GemmExtras {
+  // Dynamic schedule: clusters take work items from this counter in order
+  // (the caller zeroes it before the launch); null: static round-robin.
+  uint32_t* ticket = nullptr;
+  // Gate-weighted combine in the epilogue of the GEMM without GELU (k <= 2):
+  // Y [T, N] bf16 written instead of `out`; part [T, N] fp32 scratch; cnt
+  // [T * ceil(N / 32)] words zeroed by the caller (combine_counter_words).
+  void* comb_Y = nullptr;
+  const int32_t* comb_src = nullptr;     // src_of [R]
+  const int32_t* comb_row_of = nullptr;  // row_of [T*k]
+  const float* comb_gates = nullptr;     // [T, k]
+  float* comb_part = nullptr;
+  uint32_t* comb_cnt = nullptr;
+  int comb_k = 0, comb_T = 0;
+  // Dispatch items (fused FFN with a ticket): A[r] = disp_X[disp_src[r] / disp_k]
+  // copied inside the launch; dready: dispatch_counter_words(R) words, zeroed.
+  const void* disp_X = nullptr;
+  const int32_t* disp_src = nullptr;
+  int disp_k = 0, disp_T = 0;
+  uint32_t* dready = nullptr;
+};
+int combine_counter_words(int T, int N);
+int dispatch_counter_words(int R);
+
 // Grouped GEMM over per-expert row blocks (tcgen05 + TMA).  On a failure to
 // build the TMA descriptors, returns cudaErrorInvalidValue with *err set.
 cudaError_t launch_grouped_gemm(const void* A, const int32_t* offsets, const void* W, int E,
                                 int R, int N, int K, bool gelu, void* out,
-                                const DeviceInfo& dev, cudaStream_t stream, std::string* err);
+                                const DeviceInfo& dev, cudaStream_t stream, std::string* err,
+                                const GemmExtras* ex = nullptr);
 
 // FP8 (E4M3) mode: grouped GEMM on codes with per-tensor scales, the
 // quantising dispatch (x_scale: [scale, amax]) and per-expert weight quantisation.
 cudaError_t launch_grouped_gemm_fp8(const void* Aq, const float* a_scale, const int32_t* offsets,
                                     const void* Wq, const float* w_scale, int E, int R, int N,
                                     int K, bool gelu, void* out, const DeviceInfo& dev,
-                                    cudaStream_t stream, std::string* err);
+                                    cudaStream_t stream, std::string* err,
+                                    const GemmExtras* ex = nullptr);
 // Gather-on-load grouped GEMM: row r of the GEMM reads X[src_of[r] / k]
 // (X: [T, K] bf16, or E4M3 codes with scale x_scale[0] when fp8).
 cudaError_t launch_grouped_gemm_gather(const void* X, const float* x_scale, const int32_t* src_of,
@@ -73,12 +103,16 @@ cudaError_t launch_grouped_gemm_gather(const void* X, const float* x_scale, cons
                                        cudaStream_t stream, std::string* err);
 // Fused FFN (GEMM-1 + GELU, then GEMM-2) in one persistent launch; A is Xe
 // (bf16) or E4M3 codes with scale a_scale[0] and per-expert w1_scale (fp8).
-// `ready`: ffn_ready_count(R, E) counters of scratch, zeroed by the launcher.
+// `ctr`: ffn_counter_words(R, E) words of scratch (a ticket and one readiness
+// counter per token block), zeroed by the launcher unless `zeroed`.  `ex`
+// may add dispatch items and the combine epilogue (its ticket is ignored).
 int ffn_ready_count(int R, int E);
+int ffn_counter_words(int R, int E);
 cudaError_t launch_fused_ffn(const void* A, const float* a_scale, const int32_t* offsets,
                              const void* W1, const float* w1_scale, const void* W2, int E, int R,
-                             int d, int f, bool fp8, void* H, void* Ye, uint32_t* ready,
-                             const DeviceInfo& dev, cudaStream_t stream, std::string* err);
+                             int d, int f, bool fp8, void* H, void* Ye, uint32_t* ctr,
+                             bool zeroed, const DeviceInfo& dev, cudaStream_t stream,
+                             std::string* err, const GemmExtras* ex = nullptr);
 // Per-tensor E4M3 quantisation of n bf16 values (n % 8 == 0): x_scale = [scale, amax].
 cudaError_t launch_quantize_tensor(const void* X, int64_t n, void* Xq, float* x_scale,
                                    const DeviceInfo& dev, cudaStream_t stream);

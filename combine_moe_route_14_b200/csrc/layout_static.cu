@@ -12,11 +12,12 @@
 // holds kStaticScratchBytes of it until the process exits.  In host code its
 // name is only a host-side stand-in, so the kernels get its device address,
 // looked up once per device with cudaGetSymbolAddress.  The lookup happens on
-// the first call on each device; make that first call before any stream
-// capture.  All calls on a device share the one array, so calls whose
-// kernels could overlap on the GPU (different streams, or several host
-// threads) race on it; the kernels re-arm what must start at zero on every
-// call (look-back words, ticket), and the last call's contents stay behind.
+// the first call on each device (and again after a failed one); make that
+// first call before any stream capture.  All calls on a device share the one
+// array, so calls whose kernels could overlap on the GPU (different streams,
+// or several host threads) race on it; the kernels re-arm what must start at
+// zero on every call (look-back words, ticket), and the last call's contents
+// stay behind.
 #include <mutex>
 #include <string>
 
@@ -31,24 +32,27 @@ constexpr size_t kStaticScratchBytes = size_t(1) << 20;  // 1 MiB per device
 static __device__ __align__(256) uint8_t g_layout_scratch[kStaticScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_mu;
+void* g_scratch_ptr[kMaxDevices];  // non-null once this device's lookup succeeded
 
-// Device address of this device's scratch array, looked up on first use
-// (with the device current).  nullptr on failure, with the message set.
+// Device address of this device's scratch array, looked up with the device
+// current.  Only a successful lookup is kept: a failed one (say, a first
+// call made during a stream capture) is retried on the next call, and its
+// error is cleared from the runtime's last-error state so that no later call
+// reports it as its own.  nullptr on failure, with the message set.
 void* static_scratch(int dev) {
-  std::call_once(g_once[dev], [dev] {
-    void* p = nullptr;
-    g_scratch_err[dev] = cudaGetSymbolAddress(&p, g_layout_scratch);
-    g_scratch_ptr[dev] = (g_scratch_err[dev] == cudaSuccess) ? p : nullptr;
-  });
-  if (g_scratch_err[dev] != cudaSuccess) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_scratch_ptr[dev]) return g_scratch_ptr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_layout_scratch);
+  if (e != cudaSuccess || !p) {
+    (void)cudaGetLastError();
     set_last_error(MOE_ERR_CUDA, std::string("moe_layout_static: cudaGetSymbolAddress: ") +
-                                     cudaGetErrorString(g_scratch_err[dev]));
+                                     cudaGetErrorString(e));
     return nullptr;
   }
-  return g_scratch_ptr[dev];
+  g_scratch_ptr[dev] = p;
+  return p;
 }
 
 }  // namespace

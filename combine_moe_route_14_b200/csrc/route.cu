@@ -329,9 +329,12 @@ cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, in
 // in its owner lane, and lane j keeps slot j.  Gates are computed in fp32
 // from logit / temperature ([GPT] §2.3, §4.1); with a threshold, a slot whose
 // probability is not above it is dropped (index -1, gate 0) and renormalised
-// gates divide by the kept slots' sum.
+// gates divide by the kept slots' sum.  A -inf or NaN logit is never chosen
+// (it is not above the -FLT_MAX start value); a slot left with no candidate
+// is dropped like a thresholded one, so every index written is in [0, E) or -1.
 // ---------------------------------------------------------------------------
 constexpr int kRouteWarps = 8;
+constexpr int kNoPick = 0x7fffffff;  // larger than every expert id
 
 __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
   return v > bv || (v == bv && e < be);
@@ -341,7 +344,15 @@ template <int kEPL>
 __global__ void __launch_bounds__(kRouteWarps * 32)
     route_topk_kernel(const float* __restrict__ L, int T, int E, int k, int score, int renorm,
                       float inv_temp, float min_prob, int32_t* __restrict__ idx,
-                      float* __restrict__ gates) {
+                      float* __restrict__ gates, uint4* __restrict__ zero_rows, int zero_vecs,
+                      uint32_t* __restrict__ zero_words, int n_zero_words) {
+  // side job: clear the caller's counter words (grid-stride; the layer's
+  // later kernels run after this one on the same stream)
+  if (zero_words) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero_words;
+         i += gridDim.x * blockDim.x)
+      zero_words[i] = 0u;
+  }
   const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= T) return;
@@ -359,7 +370,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   for (int j = 0; j < kMaxTopK; ++j) {
     if (j < k) {
       float bv = -FLT_MAX;
-      int be = 0x7fffffff;
+      int be = kNoPick;
 #pragma unroll
       for (int i = 0; i < kEPL; ++i) {
         const int e = lane + 32 * i;
@@ -377,11 +388,13 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
           be = oe;
         }
       }
+      // be stays kNoPick when no candidate is left (every remaining logit
+      // is -inf or NaN): the slot is dropped below
       if (lane == j) {
         my_v = bv;
         my_e = be;
       }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      if (be < E && (be & 31) == lane) taken |= 1u << (be >> 5);
     }
   }
   // Gates.  z = logit / temperature; the largest chosen logit is lane 0's.
@@ -404,7 +417,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
     prob = q / part;
   }
-  const bool keep = slot && (!thr || prob > min_prob);
+  const bool keep = slot && my_e != kNoPick && (!thr || prob > min_prob);
   float g;
   if (renorm) {
     // softmax: prob_j / sum_kept prob = q_j / sum_kept q; sigmoid: s_j / sum_kept s
@@ -419,18 +432,27 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     idx[(size_t)t * k + lane] = keep ? my_e : -1;
     gates[(size_t)t * k + lane] = g;
   }
+  // A token with no kept slot gets no expert row, so no later stage writes
+  // its output; when asked, its output row is zeroed here.
+  if (zero_rows && __ballot_sync(0xffffffffu, keep) == 0u) {
+    uint4* row = zero_rows + (size_t)t * zero_vecs;
+    for (int c = lane; c < zero_vecs; c += 32) row[c] = make_uint4(0u, 0u, 0u, 0u);
+  }
 }
 
 cudaError_t launch_route(const float* L, int T, int E, int k, int score, int renormalize,
                          float temperature, float min_prob, int32_t* idx, float* gates,
-                         cudaStream_t stream) {
+                         cudaStream_t stream, void* zero_rows, int zero_d, uint32_t* zero_words,
+                         int n_zero_words) {
   if (T == 0) return cudaSuccess;
   const int blocks = (T + kRouteWarps - 1) / kRouteWarps;
   const int epl = (E + 31) / 32;
   const float inv_temp = 1.0f / temperature;
 #define MOE_ROUTE_LAUNCH(N)                                                                    \
   route_topk_kernel<N><<<blocks, kRouteWarps * 32, 0, stream>>>(L, T, E, k, score, renormalize, \
-                                                                inv_temp, min_prob, idx, gates)
+                                                                inv_temp, min_prob, idx, gates, \
+                                                                static_cast<uint4*>(zero_rows), \
+                                                                zero_d / 8, zero_words, n_zero_words)
   if (epl <= 1) MOE_ROUTE_LAUNCH(1);
   else if (epl <= 2) MOE_ROUTE_LAUNCH(2);
   else if (epl <= 4) MOE_ROUTE_LAUNCH(4);

@@ -90,6 +90,11 @@ WORKLOADS["mixtral_threshold"] = _mk("mixtral_threshold", 4096, 4096, 8, 2, 1433
                                      "softmax", 1, temperature=1.3, min_prob=0.05)
 WORKLOADS["tiny_threshold"] = _mk("tiny_threshold", 256, 128, 8, 2, 256, "logits", "softmax", 1,
                                   temperature=0.5, min_prob=0.2)
+# The fine-grained layer's per-expert shape (d=7168, f=2048, top-8, ~256 rows
+# per expert, sigmoid) over 32 experts: a case of a few GB for profiling the
+# expert GEMMs (inputs still larger than L2: 1.9 GB of weights per step).
+WORKLOADS["fine_grained_e32"] = _mk("fine_grained_e32", 1024, 7168, 32, 8, 2048, "logits",
+                                    "sigmoid", 1)
 for _T in (16, 64, 256, 1024):
     WORKLOADS[f"decode_{_T}"] = _mk(f"decode_{_T}", _T, 4096, 8, 2, 14336, "weights",
                                     "softmax", 1)

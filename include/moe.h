@@ -74,6 +74,23 @@ typedef enum moe_score {
 #define MOE_LAYER_FUSED_FFN 0x2      /* GEMM-1 and GEMM-2 in one persistent launch; see
                                         moe_expert_ffn_fused.  Same results, bit for bit.
                                         Not combinable with MOE_LAYER_GATHER_ON_LOAD. */
+#define MOE_LAYER_FUSED_COMBINE 0x4  /* k <= 2: the gate-weighted combine runs in GEMM-2's
+                                        epilogue (DySHARP review §3.2, kernel fusion): no Ye
+                                        rows and no combine kernel.  A token's k slot results
+                                        are weighted in fp32 from the unrounded accumulators
+                                        and summed once (a + b, so the order of the two
+                                        arrivals does not matter: deterministic).  Within the
+                                        float tolerance of the default path, not bitwise.
+                                        Ignored for k > 2 (the combine kernel runs). */
+#define MOE_LAYER_FUSED_DISPATCH 0x8 /* with MOE_LAYER_FUSED_FFN (bf16 only): the dispatch
+                                        copies run as work items of the fused FFN kernel, in
+                                        chunks of 64 expert rows, and each GEMM-1 tile starts
+                                        once the chunks under its rows are copied.  Same
+                                        results as the default path, bit for bit. */
+/* The token-centric pipeline of the DySHARP review §3.2 as one persistent kernel
+ * after the routing: dispatch chunks, GEMM-1 + GELU and GEMM-2 tiles with the
+ * combine in its epilogue, each item starting as soon as its inputs are ready. */
+#define MOE_LAYER_PIPELINE (MOE_LAYER_FUSED_FFN | MOE_LAYER_FUSED_COMBINE | MOE_LAYER_FUSED_DISPATCH)
 
 /* Shape and routing recipe of one layer. */
 typedef struct moe_layer_desc {
@@ -111,7 +128,11 @@ moe_status moe_router_logits(const void* X, const void* Wr, int32_t T, int32_t d
  *     SOFTMAX, renormalize=0: exp(L_j - L_0) / sum_{e<E} exp(L_e - L_0)
  *     SIGMOID, renormalize=1: s_j / sum_{i<k} s_i,  s = 1/(1+exp(-L))
  *     SIGMOID, renormalize=0: s_j
- *   logits [T, E] fp32 (finite; NaN/inf give unspecified choices);
+ *   logits [T, E] fp32, finite for the results above.  A -inf or NaN logit
+ *   is never chosen; a slot with no candidate left (fewer than k logits that
+ *   are finite or +inf) is dropped: topk_idx = -1, gate 0, as for
+ *   moe_route_ex's threshold.  Gates of a token with a NaN logit are
+ *   unspecified; its indices are still in [0, E) or -1.
  *   topk_idx [T, k] int32, gates [T, k] fp32.
  * ------------------------------------------------------------------------- */
 moe_status moe_route(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
@@ -257,6 +278,36 @@ moe_status moe_expert_ffn_fused_fp8(const void* Xeq, const float* x_scale,
                                     const float* w1_scale, const void* W2, int32_t E, int32_t R,
                                     int32_t d, int32_t f, void* H, void* Ye, void* ws,
                                     size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_ffn_pipeline -- dispatch, both expert layers and the combine as ONE
+ * persistent kernel: the token-centric pipeline of the DySHARP review §3.2
+ * (work on a group of tokens starts as soon as the data it needs is ready,
+ * with no kernel boundary between the stages), after route and layout.
+ *   Work items, taken by the SM pairs in this order from an atomic ticket:
+ *   dispatch chunks of 64 expert rows (Xe[r] = X[src_of[r] / k]), GEMM-1 +
+ *   GELU tiles (each waits for the chunks under its rows), GEMM-2 tiles (each
+ *   waits for its token block's H).  An item only waits on items before it,
+ *   so every wait ends, whatever share of the GPU the launch gets.  For
+ *   k <= 2 the combine runs in GEMM-2's epilogue (see MOE_LAYER_FUSED_COMBINE:
+ *   a token's output is written by the second of its two slot results to
+ *   arrive, or at once when it has one kept slot); for k > 2 the kernel
+ *   writes Ye and moe_combine's kernel follows.
+ *   Results: Y within the float tolerance of moe_dispatch + moe_expert_ffn +
+ *   moe_combine (bitwise for k > 2).  Rows of Y for tokens with no kept slot
+ *   (every row_of entry -1) are not written.
+ *   X [T, d] bf16; src_of [T*k], row_of [T*k], offsets [E+1] from moe_layout;
+ *   gates [T, k] fp32; W1 [E, f, d], W2 [E, d, f] bf16; Y [T, d] bf16.
+ *   ws: at least moe_ffn_pipeline_workspace_size(T, d, E, k, f) bytes
+ *   (dispatched rows, H, partial rows, readiness counters; zeroed counters
+ *   are set up by the call).  Every device wait is bounded; a timeout sets
+ *   MOE_DEV_TIMEOUT.
+ * ------------------------------------------------------------------------- */
+size_t moe_ffn_pipeline_workspace_size(int32_t T, int32_t d, int32_t E, int32_t k, int32_t f);
+moe_status moe_ffn_pipeline(const void* X, const int32_t* src_of, const int32_t* row_of,
+                            const float* gates, const int32_t* offsets, const void* W1,
+                            const void* W2, int32_t T, int32_t d, int32_t E, int32_t k,
+                            int32_t f, void* Y, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * moe_combine -- gate-weighted reduction of each token's k expert outputs

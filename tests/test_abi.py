@@ -90,8 +90,15 @@ def test_layer_workspace_and_desc_checks(lib):
     ws = lib.moe_workspace_size(ctypes.byref(d))
     R = 4096 * 2
     assert ws >= R * 4096 * 2 * 2 + R * 14336 * 2  # Xe + Ye + H at least
-    bad = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 6)  # unknown flag bits
+    bad = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 0x10)  # unknown flag bits
     assert lib.moe_workspace_size(ctypes.byref(bad)) == 0
+    # dispatch chunks live inside the fused FFN launch only
+    lone = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, moe.LAYER_FUSED_DISPATCH)
+    assert lib.moe_workspace_size(ctypes.byref(lone)) == 0
+    for ok in (moe.LAYER_PIPELINE, moe.LAYER_FUSED_COMBINE,
+               moe.LAYER_FUSED_FFN | moe.LAYER_FUSED_COMBINE):
+        good = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, ok)
+        assert lib.moe_workspace_size(ctypes.byref(good)) == ws  # one workspace serves all
     p = ctypes.c_void_p(0x10000)
     # both logits and Wr given
     assert lib.moe_layer_forward(ctypes.byref(d), p, p, p, p, p, p, N, N, N, p, ws, N) == INVALID

@@ -101,7 +101,7 @@ def test_peak_choice_follows_the_length_of_the_timed_loop():
 def test_both_arms_print_the_same_config():
     import argparse
     cfg = I.workload("mixtral")
-    a = argparse.Namespace(fp8=False, gather=False, fused=False)
+    a = argparse.Namespace(fp8=False, gather=False, fused=False, pipeline=False)
     c = bench.arm_config(cfg, a, 1)
     for key in ("workload", "T", "d", "E", "k", "f", "fp8", "gather_on_load", "fused_ffn",
                 "temperature", "min_prob", "renormalize", "score", "router"):

@@ -126,6 +126,36 @@ def test_route_ex_parity(T, E, k, score, renorm, temp, thr):
     assert ((gi == -1) == (gg == 0))[ok].all()
 
 
+def test_route_masked_experts_are_never_chosen():
+    """-inf logits (masked experts) are never picked; a token with fewer than k
+    other experts gets its remaining slots dropped (-1, gate 0), and the kept
+    gates are the softmax over the kept logits.  NaN logits only ever yield
+    indices in [-1, E)."""
+    T, E, k = 600, 16, 4
+    L = _logits(T, E, "normal", seed=5).numpy().copy()
+    rng = np.random.default_rng(5)
+    n_masked = rng.integers(0, E + 1, size=T)       # 0 .. all experts masked
+    for t in range(T):
+        L[t, rng.permutation(E)[:n_masked[t]]] = -np.inf
+    idx, g = moe.moe_route(torch.from_numpy(L).to(DEV), k, "softmax", 1)
+    gi, gg = idx.cpu().numpy(), g.cpu().numpy()
+    for t in range(T):
+        fin = [e for e in range(E) if np.isfinite(L[t, e])]
+        order = sorted(fin, key=lambda e: (-L[t, e], e))[:k]
+        exp_idx = order + [-1] * (k - len(order))
+        assert gi[t].tolist() == exp_idx, (t, gi[t], exp_idx)
+        if order:
+            z = np.exp(L[t, order].astype(np.float64) - L[t, order[0]])
+            np.testing.assert_allclose(gg[t, :len(order)], z / z.sum(), rtol=2e-6, atol=2e-7)
+        assert (gg[t, len(order):] == 0).all()
+    Ln = L.copy()
+    Ln[rng.random(Ln.shape) < 0.2] = np.nan
+    idx, _ = moe.moe_route(torch.from_numpy(Ln).to(DEV), k, "softmax", 1)
+    gi = idx.cpu().numpy()
+    assert ((gi >= -1) & (gi < E)).all()
+    assert not np.isnan(Ln[np.arange(T)[:, None].repeat(k, 1)[gi >= 0], gi[gi >= 0]]).any()
+
+
 # ----------------------------------------------------------------------------
 # router linear
 # ----------------------------------------------------------------------------

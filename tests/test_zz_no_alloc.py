@@ -5,9 +5,10 @@ inside another framework's callback that is handed only the tensors it works
 on, or code that must not allocate after start-up).  moe_layout_static keeps
 the layout's scratch in a fixed 1 MiB array inside the library instead.  These
 tests call it through the C ABI and check that it returns exactly what
-moe_layout returns with a caller workspace, twice in a row (the shared array
-keeps the previous call's contents, so the second call checks that the kernels
-re-arm it).  The file is named to be collected last.
+moe_layout returns with a caller workspace, and what the oracle's layout
+returns, twice in a row (the shared array keeps the previous call's contents,
+so the second call checks that the kernels re-arm it).  The file is named to
+be collected last.
 """
 import ctypes
 
@@ -17,6 +18,7 @@ import torch
 
 import combine_moe_route_14_b200 as moe
 from combine_moe_route_14_b200 import inputs as I
+from oracle import moe_oracle as O
 
 DEV = "cuda:0"
 
@@ -49,6 +51,10 @@ def test_static_layout_matches_workspace_layout_twice(cuda_lib, T, E, k, skew):
         torch.cuda.synchronize()
         for name, a, b in zip(("counts", "offsets", "row_of", "src_of"), outs, ref):
             assert torch.equal(a, b), f"call {call}: {name} differs"
+        # and the oracle's layout of the same routing, bit for bit
+        for name, a, b in zip(("counts", "offsets", "row_of", "src_of"), outs,
+                              O.layout(idx.cpu().numpy(), E)):
+            assert np.array_equal(a.cpu().numpy(), b), f"call {call}: {name} differs from the oracle"
     assert moe.moe_device_status(clear=True) == 0
 
 

@@ -113,6 +113,19 @@ constexpr int kQueue = 4;
 // Dispatch items of the fused FFN: layout rows per item, and 16-byte vectors
 // in flight per lane while copying them.
 constexpr int kDispRows = 64;
+// Weight K-blocks prefetched into L2 ahead of their TMA loads by the weight
+// producer's idle lanes, for launches whose expert blocks are small (few
+// rows per expert: the weight stream is the whole cost and DRAM latency
+// bounds it).  Measured on a B200: decode-sized layers -5 %; with 256 or
+// more rows per expert it costs 4-6 %, so it is off there.
+constexpr int kWPrefetchSmall = 4;
+#ifndef MOE_W_EVICT_FIRST
+#define MOE_W_EVICT_FIRST 0  // L2 policy of the weight stream: evict_first instead of normal
+#endif
+#ifndef MOE_KPS_PAIR
+#define MOE_KPS_PAIR 2       // K-blocks per ring slot with paired CTAs
+#endif
+constexpr int kWPrefetchMaxRows = 64;  // mean rows per expert at or below which it is on
 constexpr int kDispUnroll = 8;
 
 // kPair = 1: one CTA computes a 128-feature x N-token tile (cta_group::1).
@@ -124,7 +137,7 @@ template <int kPair> struct Cfg {
   static constexpr int B_STAGE = (BN / kPair) * BK * 2;  // token rows this CTA stages
   // K-blocks per ring slot: two with paired CTAs (3 slots of 64 KB), one with
   // a single CTA (its 48 KB K-block already leaves only 4 slots)
-  static constexpr int KPS = kPair == 2 ? 2 : 1;
+  static constexpr int KPS = kPair == 2 ? MOE_KPS_PAIR : 1;
   static constexpr int STAGE = KPS * (A_STAGE + B_STAGE);  // one ring slot
   static constexpr int NUM_BARS = 2 * MAX_STAGES + 4 + 1 + 2 * kQueue + 1;
   static constexpr int FEAT = BM * kPair;                // output features per tile
@@ -166,6 +179,10 @@ struct Args {
   int N2, n_fblocks2, num_kb2;
   uint32_t* ready;         // [token blocks]: GEMM-1 epilogue warps done, per token block
   uint32_t ready_target;   // arrivals that complete a token block
+  const uint8_t* w_ptr;    // W as bytes (phase 0), row pitch w_pitch; W2 for phase 1
+  const uint8_t* w2_ptr;
+  int w_pitch, w2_pitch;
+  int w_prefetch;          // weight K-blocks prefetched into L2 ahead (0: none)
   // Dynamic schedule: non-null -> clusters take items from this counter, in
   // item order (zeroed before the launch); null -> static round-robin.
   uint32_t* ticket;
@@ -503,7 +520,7 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     // their operand in both CTAs of the pair.
     const bool is_w = warp < Ro::NW;
     const int tw = warp - Ro::NW;  // token warp index
-    const uint64_t pol = is_w ? l2_policy_evict_normal()  // shared by the CTAs of a feature block
+    const uint64_t pol = is_w ? (MOE_W_EVICT_FIRST ? l2_policy_evict_first() : l2_policy_evict_normal())
                               : l2_policy_evict_last();   // re-read by every feature block
     int s = 0;
     uint32_t ph = 0;
@@ -565,6 +582,18 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
                                   : (uint32_t)kPair * (wide ? nwide * B_WIDE_ROWS * BK * 2
                                                             : nbox * B_BOX);
       const int wy = t.e * Np + t.fb * C::FEAT + (int)rank * BM;
+      // weight prefetch: this CTA's 128 weight rows, 4 per lane
+      const uint8_t* wrow = (p1 ? args.w2_ptr : args.w_ptr) +
+                            (size_t)(wy + lane) * (size_t)(p1 ? args.w2_pitch : args.w_pitch);
+      const size_t wstep = (size_t)32 * (size_t)(p1 ? args.w2_pitch : args.w_pitch);
+      const int wpf = args.w_prefetch;
+      if (wpf > 0 && is_w) {
+        const int nrow = min(BM, Np - (wy - t.e * Np));
+        for (int kb = 0; kb < min(wpf, nkb); ++kb)
+#pragma unroll
+          for (int r4 = 0; r4 < 4; ++r4)
+            if (lane + 32 * r4 < nrow) prefetch_l2(wrow + r4 * wstep + (size_t)kb * 128);
+      }
       const int by = t.row0 + (int)rank * half;
       // gather form: request q (4 rows) of this CTA's half-tile is issued
       // by token warp q % NTOK, lane q / NTOK % 32 (up to 64 requests: 256
@@ -621,6 +650,17 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
         }
         ok = warp_wait(&empty[s], ph ^ 1u, args.status, s_abort);
         if (!ok) break;
+        if (wpf > 0 && is_w) {  // K-blocks wpf ahead
+          const int nrow = min(BM, Np - (wy - t.e * Np));
+          for (int hh = 0; hh < nsub; ++hh) {
+            const int kb = ks * KPS + hh + wpf;
+            if (kb < nkb) {
+#pragma unroll
+              for (int r4 = 0; r4 < 4; ++r4)
+                if (lane + 32 * r4 < nrow) prefetch_l2(wrow + r4 * wstep + (size_t)kb * 128);
+            }
+          }
+        }
         if (kGather && !is_w) {
           const uint32_t fb_addr = full_lead + (uint32_t)s * 8u;
           if (tw == 0 && lane == 0 && rank == 0)
@@ -1077,6 +1117,9 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
   args.status = dev.status;
   args.a_scale = a_scale;
   args.w_scale = w_scale;
+  args.w_ptr = static_cast<const uint8_t*>(W);
+  args.w_pitch = K * (kFp8 ? 1 : 2);
+  args.w_prefetch = R <= gg::kWPrefetchMaxRows * E ? gg::kWPrefetchSmall : 0;
   args.gather_src = gather_src;
   args.gather_k = gather_k;
   args.a_rows = a_rows;
@@ -1153,6 +1196,11 @@ cudaError_t launch_fused_ffn(const void* A, const float* a_scale, const int32_t*
   args.status = dev.status;
   args.a_scale = a_scale;
   args.w_scale = w1_scale;
+  args.w_ptr = static_cast<const uint8_t*>(W1);
+  args.w_pitch = d * (fp8 ? 1 : 2);
+  args.w2_ptr = static_cast<const uint8_t*>(W2);
+  args.w2_pitch = f * 2;
+  args.w_prefetch = R <= gg::kWPrefetchMaxRows * E ? gg::kWPrefetchSmall : 0;
   args.gather_k = 1;
   args.a_rows = R;
   args.E = E;

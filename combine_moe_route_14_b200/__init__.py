@@ -30,6 +30,7 @@ __all__ = [
     "moe_expert_ffn_fused_workspace_size", "moe_expert_ffn_fused", "moe_expert_ffn_fused_fp8",
     "moe_selftest_bounded_wait", "moe_dispatch_by_token", "moe_dispatch_fp8_by_token",
     "moe_ffn_pipeline_workspace_size", "moe_ffn_pipeline", "make_desc",
+    "moe_host_workspace_size", "moe_layer_forward_host",
     "LAYER_GATHER_ON_LOAD", "LAYER_FUSED_FFN", "LAYER_FUSED_COMBINE", "LAYER_FUSED_DISPATCH",
     "LAYER_PIPELINE",
 ]
@@ -102,6 +103,9 @@ _SIG = {
                              ctypes.c_int),
     "moe_expert_ffn_fused_fp8": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P,
                                   ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_host_workspace_size": ([ctypes.POINTER(LayerDesc), _I], ctypes.c_size_t),
+    "moe_layer_forward_host": ([ctypes.POINTER(LayerDesc), _I, _P, _P, _P, _P, _P, _P, _P, _P,
+                                ctypes.c_size_t, _P], ctypes.c_int),
     "moe_ffn_pipeline_workspace_size": ([_I, _I, _I, _I, _I], ctypes.c_size_t),
     "moe_ffn_pipeline": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
                           ctypes.c_size_t, _P], ctypes.c_int),
@@ -158,6 +162,16 @@ def _need(t, name, dtype, shape=None, device=None):
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _need_host(t, name, dtype, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype or t.device.type != "cpu" or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} CPU tensor")
+    if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     return t
 
@@ -626,6 +640,50 @@ def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=
                                      _ptr(topk_idx_out), _ptr(gates_out), _ptr(counts_out),
                                      _ptr(ws), ws.numel(), _stream(stream, dev)))
     return Y
+
+
+def moe_host_workspace_size(desc: LayerDesc, with_logits: bool) -> int:
+    return int(load_library().moe_host_workspace_size(ctypes.byref(desc), int(bool(with_logits))))
+
+
+def moe_layer_forward_host(X_host, W1, W2, k, Y_host, score="softmax", renormalize=True,
+                           logits_host=None, Wr=None, w1_scale=None, ws=None, stream=None,
+                           temperature=1.0, min_prob=0.0, **flags):
+    """The layer over len(X_host) batches in host memory (C ABI moe_layer_forward_host).
+
+    X_host / Y_host: lists of [T, d] bf16 CPU tensors (pinned for overlap);
+    logits_host: a list of [T, E] fp32 CPU tensors, or None with Wr given.
+    W1 holds E4M3 codes when w1_scale is given (FP8 mode).  Returns once the
+    work is enqueued; `stream` (default: the current one) waits for the last
+    copy out."""
+    lib = load_library()
+    n = len(X_host)
+    if len(Y_host) != n or (logits_host is not None and len(logits_host) != n):
+        raise ValueError("one output (and logits) tensor per batch")
+    T, d = X_host[0].shape
+    E, f, _ = W1.shape
+    dev = W1.device
+    for i in range(n):
+        _need_host(X_host[i], f"X_host[{i}]", torch.bfloat16, (T, d))
+        _need_host(Y_host[i], f"Y_host[{i}]", torch.bfloat16, (T, d))
+        if logits_host is not None:
+            _need_host(logits_host[i], f"logits_host[{i}]", torch.float32, (T, E))
+    _need(W1, "W1", torch.uint8 if w1_scale is not None else torch.bfloat16, (E, f, d))
+    _need(W2, "W2", torch.bfloat16, (E, d, f), dev)
+    if Wr is not None:
+        _need(Wr, "Wr", torch.bfloat16, (E, d), dev)
+    if w1_scale is not None:
+        _need(w1_scale, "w1_scale", torch.float32, (E,), dev)
+    desc = make_desc(T, d, E, k, f, score, renormalize, temperature, min_prob, **flags)
+    if ws is None:
+        ws = torch.empty(max(moe_host_workspace_size(desc, logits_host is not None), 16),
+                         dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, None, dev)
+    arr = lambda ts: (ctypes.c_void_p * n)(*[t.data_ptr() for t in ts])  # noqa: E731
+    _check(lib.moe_layer_forward_host(ctypes.byref(desc), n, arr(X_host),
+                                      None if logits_host is None else arr(logits_host),
+                                      _ptr(Wr), _ptr(W1), _ptr(w1_scale), _ptr(W2), arr(Y_host),
+                                      _ptr(ws), ws.numel(), _stream(stream, dev)))
 
 
 def moe_selftest_bounded_wait(which: int, limit_us: int, counter=None, stream=None):

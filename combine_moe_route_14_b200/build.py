@@ -49,12 +49,15 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          nvtx: bool = False) -> str:
+    """nvtx=True (or MOE_NVTX=1 in the environment) adds per-stage NVTX ranges."""
+    nvtx = nvtx or os.environ.get("MOE_NVTX") == "1"
+    if not force and not nvtx and up_to_date():
         return LIB
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
-    extra = ["-Xptxas", "-v"] if ptxas_info else []
+    extra = (["-Xptxas", "-v"] if ptxas_info else []) + (["-DMOE_NVTX=1"] if nvtx else [])
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
@@ -83,5 +86,7 @@ if __name__ == "__main__":
     ap.add_argument("--force", action="store_true")
     ap.add_argument("-v", "--verbose", action="store_true")
     ap.add_argument("--ptxas-info", action="store_true")
+    ap.add_argument("--nvtx", action="store_true", help="per-stage NVTX ranges in the layer")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.verbose or a.ptxas_info, ptxas_info=a.ptxas_info))
+    print(build(force=a.force, verbose=a.verbose or a.ptxas_info, ptxas_info=a.ptxas_info,
+                nvtx=a.nvtx))

@@ -9,6 +9,24 @@
 #include "common.cuh"
 #include "launch.h"
 
+// Per-stage NVTX ranges around the layer's launches (build with -DMOE_NVTX=1;
+// header-only NVTX v3, so nothing to link).  A profiler's timeline then shows
+// router / route / layout / dispatch / GEMM-1 / GEMM-2 / combine by name: the
+// kernel-level view of the GPT-4 "2%" article §5.2 (a GPU kernel flame graph
+// of the router and expert GEMM kernels).  Off by default: they cost host time.
+#if MOE_NVTX
+#include <nvtx3/nvToolsExt.h>
+struct NvtxStage {
+  explicit NvtxStage(const char* name) { nvtxRangePushA(name); }
+  ~NvtxStage() { nvtxRangePop(); }
+};
+#define MOE_STAGE(name) NvtxStage moe_nvtx_stage_(name)
+#else
+#define MOE_STAGE(name) \
+  do {                  \
+  } while (0)
+#endif
+
 // Sticky per-device status word set by kernels (MOE_DEV_* bits).
 __device__ uint32_t g_moe_device_status;
 
@@ -263,17 +281,27 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   const bool comb = (d.flags & MOE_LAYER_FUSED_COMBINE) && d.k <= 2;
   const bool fdisp = fused && (d.flags & MOE_LAYER_FUSED_DISPATCH) && !fp8;
 
-  if (Wr) MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, *dev, s), "router_logits");
+  if (Wr) {
+    MOE_STAGE("moe.router_logits");
+    MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, *dev, s), "router_logits");
+  }
   // The routing kernel also clears the tickets, readiness and combine
   // counters (they start at zero in every forward) and, with the combine in
   // GEMM-2's epilogue, writes the zero outputs of tokens whose slots were all
   // dropped (no expert row reaches them).
   const bool drops = d.min_prob > 0.f;
-  MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
-                             d.min_prob, idx, gates, s, (comb && drops) ? Y : nullptr, d.d, ctr,
-                             lc.used),
-           "route");
-  MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s), "layout");
+  {
+    MOE_STAGE("moe.route");
+    MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
+                               d.min_prob, idx, gates, s, (comb && drops) ? Y : nullptr, d.d,
+                               ctr, lc.used),
+             "route");
+  }
+  {
+    MOE_STAGE("moe.layout");
+    MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s),
+             "layout");
+  }
   // The two-launch path keeps the static balanced schedule (measured faster
   // than tickets on uniform tiles); the fused launch always takes tickets.
   moe::GemmExtras ex1, ex2;
@@ -297,11 +325,14 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
       ex2.disp_T = d.T;
       ex2.dready = ctr + lc.disp;
     } else if (fp8) {
+      MOE_STAGE("moe.dispatch");
       MOE_CUDA(moe::launch_dispatch_fp8_rows(X, row_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
                "dispatch_fp8");
     } else {
+      MOE_STAGE("moe.dispatch");
       MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
     }
+    MOE_STAGE("moe.fused_ffn");
     e = moe::launch_fused_ffn(Xe, x_scale, offsets, W1, W1s, W2, d.E, R, d.d, d.f, fp8, H, Ye,
                               ctr + lc.ffn, true, *dev, s, &err, &ex2);
     if (e != cudaSuccess) return gemm_fail(e, err, "fused_ffn");
@@ -319,19 +350,32 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
     e = moe::launch_grouped_gemm_gather(A, x_scale, src_of, d.T, d.k, offsets, W1, W1s, d.E, d.f,
                                         d.d, true, fp8, H, *dev, s, &err);
   } else if (fp8) {
-    MOE_CUDA(moe::launch_dispatch_fp8_rows(X, row_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
-             "dispatch_fp8");
+    {
+      MOE_STAGE("moe.dispatch");
+      MOE_CUDA(moe::launch_dispatch_fp8_rows(X, row_of, d.T, d.d, d.k, Xe, x_scale, *dev, s),
+               "dispatch_fp8");
+    }
+    MOE_STAGE("moe.gemm1");
     e = moe::launch_grouped_gemm_fp8(Xe, x_scale, offsets, W1, W1s, d.E, R, d.f, d.d, true, H,
                                      *dev, s, &err, &ex1);
   } else {
-    MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+    {
+      MOE_STAGE("moe.dispatch");
+      MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+    }
+    MOE_STAGE("moe.gemm1");
     e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err, &ex1);
   }
   if (e != cudaSuccess) return gemm_fail(e, err, "gemm1");
-  e = moe::launch_grouped_gemm(H, offsets, W2, d.E, R, d.d, d.f, false, Ye, *dev, s, &err, &ex2);
+  {
+    MOE_STAGE("moe.gemm2");
+    e = moe::launch_grouped_gemm(H, offsets, W2, d.E, R, d.d, d.f, false, Ye, *dev, s, &err, &ex2);
+  }
   if (e != cudaSuccess) return gemm_fail(e, err, "gemm2");
-  if (!comb)
+  if (!comb) {
+    MOE_STAGE("moe.combine");
     MOE_CUDA(moe::launch_combine(Ye, row_of, gates, d.T, d.d, d.k, Y, *dev, s), "combine");
+  }
   return MOE_OK;
 }
 
@@ -841,6 +885,128 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const void* X, const fl
                              void* ws, size_t ws_bytes, void* stream) {
   return layer_forward(desc, X, logits, Wr, W1, nullptr, W2, Y, topk_idx_out, gates_out,
                        counts_out, ws, ws_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Host-buffer batches (moe_layer_forward_host): per-device streams and events
+// owned by the library, created on first use.
+// ---------------------------------------------------------------------------
+namespace {
+struct HostLanes {
+  std::mutex mu;  // one enqueue at a time per device (the events are shared)
+  bool ready = false;
+  cudaError_t err = cudaSuccess;
+  cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
+  cudaEvent_t entry = nullptr, done = nullptr;
+  cudaEvent_t x_ready[2] = {}, x_free[2] = {}, y_ready[2] = {}, y_free[2] = {};
+};
+HostLanes g_lanes[64];
+
+cudaError_t lanes_init(HostLanes& h) {
+  cudaError_t e = cudaSuccess;
+  auto ev = [&](cudaEvent_t* p) {
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(p, cudaEventDisableTiming);
+  };
+  for (cudaStream_t* st : {&h.h2d, &h.comp, &h.d2h})
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(st, cudaStreamNonBlocking);
+  ev(&h.entry);
+  ev(&h.done);
+  for (int i = 0; i < 2; ++i) {
+    ev(&h.x_ready[i]);
+    ev(&h.x_free[i]);
+    ev(&h.y_ready[i]);
+    ev(&h.y_free[i]);
+  }
+  return e;
+}
+
+struct HostWs {
+  size_t X[2], Y[2], L[2], layer, total;
+};
+HostWs host_ws(const moe_layer_desc& d, bool with_logits) {
+  HostWs w;
+  size_t o = 0;
+  for (int i = 0; i < 2; ++i) {
+    w.X[i] = o; o += up256((size_t)d.T * d.d * 2);
+    w.Y[i] = o; o += up256((size_t)d.T * d.d * 2);
+    w.L[i] = o; o += with_logits ? up256((size_t)d.T * d.E * sizeof(float)) : 0;
+  }
+  w.layer = o;
+  o += layer_ws(d).total;
+  w.total = o;
+  return w;
+}
+}  // namespace
+
+size_t moe_host_workspace_size(const moe_layer_desc* desc, int32_t with_logits) {
+  if (check_desc(desc) != MOE_OK) return 0;
+  return host_ws(*desc, with_logits != 0).total;
+}
+
+moe_status moe_layer_forward_host(const moe_layer_desc* desc, int32_t nbatch,
+                                  const void* const* X_host, const float* const* logits_host,
+                                  const void* Wr, const void* W1, const float* w1_scale,
+                                  const void* W2, void* const* Y_host, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  MOE_TRY(check_desc(desc));
+  const moe_layer_desc d = *desc;
+  if (nbatch < 0) return fail(MOE_ERR_INVALID_ARG, "nbatch must be >= 0");
+  if (nbatch == 0 || d.T == 0) return MOE_OK;
+  if (!X_host || !Y_host) return fail(MOE_ERR_INVALID_ARG, "X_host and Y_host are required");
+  if ((logits_host == nullptr) == (Wr == nullptr))
+    return fail(MOE_ERR_INVALID_ARG, "give exactly one of logits_host and Wr");
+  for (int i = 0; i < nbatch; ++i) {
+    if (!X_host[i] || !Y_host[i] || (logits_host && !logits_host[i]))
+      return fail(MOE_ERR_INVALID_ARG, "batch " + std::to_string(i) + ": a host pointer is NULL");
+  }
+  const bool with_logits = logits_host != nullptr;
+  const HostWs w = host_ws(d, with_logits);
+  if (ws_bytes < w.total) return fail(MOE_ERR_INVALID_ARG, "workspace too small");
+  MOE_TRY(check_ptr(ws, "ws"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  HostLanes& h = g_lanes[dev->device & 63];
+  std::lock_guard<std::mutex> lock(h.mu);
+  if (!h.ready) {
+    h.err = lanes_init(h);
+    h.ready = h.err == cudaSuccess;
+    if (!h.ready) return cuda_fail(h.err, "host-batch streams");
+  }
+  char* base = static_cast<char*>(ws);
+  const size_t xb = (size_t)d.T * d.d * 2, lb = (size_t)d.T * d.E * sizeof(float);
+  cudaStream_t caller = as_stream(stream);
+  // everything enqueued on `stream` before this call comes first
+  MOE_CUDA(cudaEventRecord(h.entry, caller), "record entry");
+  for (cudaStream_t st : {h.h2d, h.comp, h.d2h})
+    MOE_CUDA(cudaStreamWaitEvent(st, h.entry, 0), "wait entry");
+  for (int i = 0; i < nbatch; ++i) {
+    const int s = i & 1;
+    void* Xd = base + w.X[s];
+    void* Yd = base + w.Y[s];
+    float* Ld = with_logits ? reinterpret_cast<float*>(base + w.L[s]) : nullptr;
+    // inputs of batch i into buffer set s, once the forward two batches back
+    // (this call's or a previous call's) has read it
+    MOE_CUDA(cudaStreamWaitEvent(h.h2d, h.x_free[s], 0), "wait x_free");
+    MOE_CUDA(cudaMemcpyAsync(Xd, X_host[i], xb, cudaMemcpyHostToDevice, h.h2d), "copy X");
+    if (with_logits)
+      MOE_CUDA(cudaMemcpyAsync(Ld, logits_host[i], lb, cudaMemcpyHostToDevice, h.h2d),
+               "copy logits");
+    MOE_CUDA(cudaEventRecord(h.x_ready[s], h.h2d), "record x_ready");
+    // the forward, once its inputs are in and Y[s] has been copied out
+    MOE_CUDA(cudaStreamWaitEvent(h.comp, h.x_ready[s], 0), "wait x_ready");
+    MOE_CUDA(cudaStreamWaitEvent(h.comp, h.y_free[s], 0), "wait y_free");
+    MOE_TRY(layer_forward(&d, Xd, Ld, Wr, W1, w1_scale, W2, Yd, nullptr, nullptr, nullptr,
+                          base + w.layer, ws_bytes - w.layer, h.comp));
+    MOE_CUDA(cudaEventRecord(h.x_free[s], h.comp), "record x_free");
+    MOE_CUDA(cudaEventRecord(h.y_ready[s], h.comp), "record y_ready");
+    // the output back to the host
+    MOE_CUDA(cudaStreamWaitEvent(h.d2h, h.y_ready[s], 0), "wait y_ready");
+    MOE_CUDA(cudaMemcpyAsync(Y_host[i], Yd, xb, cudaMemcpyDeviceToHost, h.d2h), "copy Y");
+    MOE_CUDA(cudaEventRecord(h.y_free[s], h.d2h), "record y_free");
+  }
+  MOE_CUDA(cudaEventRecord(h.done, h.d2h), "record done");
+  MOE_CUDA(cudaStreamWaitEvent(caller, h.done, 0), "wait done");
+  return MOE_OK;
 }
 
 moe_status moe_layer_forward_fp8(const moe_layer_desc* desc, const void* X, const float* logits,

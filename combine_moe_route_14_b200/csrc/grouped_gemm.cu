@@ -183,6 +183,7 @@ struct Args {
   const uint8_t* w2_ptr;
   int w_pitch, w2_pitch;
   int w_prefetch;          // weight K-blocks prefetched into L2 ahead (0: none)
+  bool fb_fastest, fb_fastest2;  // tile order of phase 0 / phase 1 (see decode)
   // Dynamic schedule: non-null -> clusters take items from this counter, in
   // item order (zeroed before the launch); null -> static round-robin.
   uint32_t* ticket;
@@ -218,8 +219,13 @@ struct Tile {
 // load requests than one ragged block.)
 __device__ __forceinline__ int token_blocks(int c) { return (c + BN - 1) / BN; }
 
+// fb_fastest = false: an expert's tiles go token block fastest (the CTAs
+// running at once share each weight block through L2); true: feature block
+// fastest (they share each token block instead: every feature-block tile of a
+// token block runs at about the same time, so the token rows are read from
+// DRAM once even when a long K leaves no room in L2 to keep them).
 __device__ __forceinline__ Tile decode(int tile, const int* s_start, const int* s_lo,
-                                       const int* s_hi, int E) {
+                                       const int* s_hi, int E, bool fb_fastest, int n_fb) {
   int lo = 0, hi = E - 1;
   while (lo < hi) {  // last expert whose first tile is <= tile
     const int mid = (lo + hi + 1) >> 1;
@@ -230,8 +236,14 @@ __device__ __forceinline__ Tile decode(int tile, const int* s_start, const int* 
   const int local = tile - s_start[lo];
   const int c = s_hi[lo] - s_lo[lo];
   const int ntb = token_blocks(c);
-  t.fb = local / ntb;
-  const int tb = local - t.fb * ntb;
+  int tb;
+  if (fb_fastest) {
+    tb = local / n_fb;
+    t.fb = local - tb * n_fb;
+  } else {
+    t.fb = local / ntb;
+    tb = local - t.fb * ntb;
+  }
   t.row0 = s_lo[lo] + tb * BN;
   t.ntok = min(BN, c - tb * BN);
   return t;
@@ -418,10 +430,10 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     x -= n_disp;
     if (kFused && x >= tiles0) {
       phase = 1;
-      return decode(x - tiles0, s_start2, s_lo, s_hi, E);
+      return decode(x - tiles0, s_start2, s_lo, s_hi, E, args.fb_fastest2, args.n_fblocks2);
     }
     phase = 0;
-    return decode(x, s_start, s_lo, s_hi, E);
+    return decode(x, s_start, s_lo, s_hi, E, args.fb_fastest, args.n_fblocks);
   };
   // fused form: index of the token block holding a tile's rows
   auto block_of = [&](const Tile& t) -> int {
@@ -1133,6 +1145,14 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
   args.stages = pair == 2 ? gg::stages_for<2>(E) : gg::stages_for<1>(E);
   apply_extras(args, ex);
   if (gelu) args.comb_Y = nullptr;  // the combine belongs to the GEMM without activation
+#ifndef MOE_GEMM2_FB_FASTEST
+#define MOE_GEMM2_FB_FASTEST 0
+#endif
+  // Token block fastest for both GEMMs.  Feature block fastest for GEMM-2
+  // (each block of H shared by its feature-block tiles at once) measured
+  // more DRAM reads on the Mixtral shape (1.66 vs 1.41 GB, the W2 blocks
+  // then being read again) at the same time; it stays a build option.
+  args.fb_fastest = !gelu && MOE_GEMM2_FB_FASTEST;
   // an upper bound on the tile count: every expert adds at most one partial token block
   const long long max_tiles =
       ((long long)(R + gg::BN - 1) / gg::BN + E) * (long long)args.n_fblocks;
@@ -1214,6 +1234,7 @@ cudaError_t launch_fused_ffn(const void* A, const float* a_scale, const int32_t*
   args.N2 = d;
   args.n_fblocks2 = (d + gg::BM * pair - 1) / (gg::BM * pair);
   args.num_kb2 = (f + gg::BK - 1) / gg::BK;
+  args.fb_fastest2 = MOE_GEMM2_FB_FASTEST;
   apply_extras(args, ex);
   // Always the dynamic schedule: tickets are taken in item order, so a tile
   // only ever waits on tiles that running clusters hold (any residency).

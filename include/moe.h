@@ -345,6 +345,38 @@ moe_status moe_layer_forward(const moe_layer_desc* desc, const void* X, const fl
                              void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_layer_forward_host -- moe_layer_forward over `nbatch` batches whose
+ * tokens and outputs live in HOST memory (the end-to-end form of the layer:
+ * the pages' dispatch/combine path starts and ends with token rows that have
+ * to move, ThunderEP blog §1.2 and §5.3 on overlapping transfer with compute).
+ *   Batch i: X_host[i] [T, d] bf16 (and logits_host[i] [T, E] fp32 when the
+ *   router is not given) is copied to the device, the layer runs, and its
+ *   output is copied to Y_host[i] [T, d] bf16 -- one cudaMemcpyAsync per
+ *   copy.  The library orders the work on three streams of its own per
+ *   device (copies in, compute, copies out) with events, and two device
+ *   buffer sets in `ws`, so the copies of neighbouring batches overlap the
+ *   current forward and a batch costs about the slowest of the three.
+ *   All batches share `desc` and the weights (device pointers: Wr or the
+ *   logits_host array, W1, W2; w1_scale non-NULL selects the FP8 mode with
+ *   W1 holding moe_quantize_experts_fp8 codes, as moe_layer_forward_fp8).
+ *   Host buffers should be pinned (page-locked) for the copies to run
+ *   asynchronously; pageable memory gives the same results, serialised.
+ *   The call returns once the work is enqueued.  Work already on `stream`
+ *   runs first, and `stream` waits for the last copy out: synchronising
+ *   `stream` (or enqueueing after this call on it) sees every Y_host[i]
+ *   complete.  The host buffers must stay valid until then.  Calls on one
+ *   device are serialised on the library's streams; they are not for CUDA
+ *   graph capture (the streams are the library's).
+ *   ws: at least moe_host_workspace_size(desc, with_logits) bytes.
+ * ------------------------------------------------------------------------- */
+size_t moe_host_workspace_size(const moe_layer_desc* desc, int32_t with_logits);
+moe_status moe_layer_forward_host(const moe_layer_desc* desc, int32_t nbatch,
+                                  const void* const* X_host, const float* const* logits_host,
+                                  const void* Wr, const void* W1, const float* w1_scale,
+                                  const void* W2, void* const* Y_host, void* ws, size_t ws_bytes,
+                                  void* stream);
+
+/* ---------------------------------------------------------------------------
  * FP8 mode (ThunderEP PCIe blog §3.3 "transport-side bit reduction" and §5.2:
  * the activations a dispatch moves are cast to FP8 with one dynamic
  * per-tensor scale before they move and cast back after, halving the bytes;

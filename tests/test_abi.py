@@ -166,3 +166,20 @@ def test_fused_ffn_checks_on_the_host(lib):
     fused = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, moe.LAYER_FUSED_FFN)
     assert lib.moe_kernel_launches_per_forward(ctypes.byref(fused), 1) == 6  # one GEMM launch
     assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(fused), 1) == 7
+
+
+def test_host_batches_reject_bad_arguments(lib):
+    d = moe.LayerDesc(64, 128, 8, 2, 256, 0, 1, 0)
+    need = lib.moe_host_workspace_size(ctypes.byref(d), 1)
+    assert need > lib.moe_workspace_size(ctypes.byref(d))  # two buffer sets on top
+    p = ctypes.c_void_p(0x10000)
+    arr = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    zero = (ctypes.c_void_p * 2)(0x10000, 0)
+    args = lambda n, X, L, Wr, Y, ws: (ctypes.byref(d), n, X, L, Wr, p, N, p, Y, p, ws, N)  # noqa
+    assert lib.moe_layer_forward_host(*args(-1, arr, arr, N, arr, need)) == INVALID
+    assert lib.moe_layer_forward_host(*args(2, arr, arr, p, arr, need)) == INVALID  # both routers
+    assert lib.moe_layer_forward_host(*args(2, zero, arr, N, arr, need)) == INVALID  # NULL batch
+    assert "batch 1" in _err(lib)
+    assert lib.moe_layer_forward_host(*args(2, arr, arr, N, arr, need - 1)) == INVALID
+    assert "workspace" in _err(lib)
+    assert lib.moe_layer_forward_host(*args(0, N, N, N, N, 0)) == OK  # nothing to do

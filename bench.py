@@ -72,6 +72,7 @@ def stage_model(cfg, counts=None, fp8=False):  # gather form: same algorithmic b
         m["router_logits"] = {"bytes": T * d * 2 + E * d * 2 + T * E * 4, "flops": 2 * T * d * E}
     m["route"] = {"bytes": T * E * 4 + R * 8}
     m["layout"] = {"bytes": R * 4 + R * 8 + (2 * E + 1) * 4}
+    m["route_layout"] = {"bytes": T * E * 4 + R * 8 + R * 8 + (2 * E + 1) * 4}
     m["dispatch"] = {"bytes": T * d * 2 + R * d * 2 + R * 4}
     m["gemm1"] = {"flops": 2 * R * d * f, "bytes": E_act * f * d * 2 + R * d * 2 + R * f * 2}
     m["gemm2"] = {"flops": 2 * R * d * f, "bytes": E_act * d * f * 2 + R * f * 2 + R * d * 2}
@@ -375,7 +376,11 @@ def run_ours(args, cfg, rank, world, local_rank):
         step_us = step_percentiles([vev[i].elapsed_time(vev[i + 1]) for i in range(args.steps)])
 
         # ---- per-stage times: the same kernels, launched stage by stage with events between
-        stage_names = (["router_logits"] if Wr is not None else []) + ["route", "layout"] + (
+        # the layer's bf16 path ranks the slots in its routing kernel (no
+        # layout launch); its staged form is moe_route_layout
+        ranked = not (args.gather or args.fp8 or args.pipeline) and cfg.E <= 32
+        stage_names = (["router_logits"] if Wr is not None else []) + (
+            ["route_layout"] if ranked else ["route", "layout"]) + (
             ["pipeline"] if args.pipeline else
             (["quantize"] if args.gather and args.fp8 else [] if args.gather else ["dispatch"]) +
             (["ffn"] if args.fused else ["gemm1", "gemm2"]) + ["combine"])
@@ -403,6 +408,7 @@ def run_ours(args, cfg, rank, world, local_rank):
             "route": lambda: moe.moe_route_ex(L_buf, cfg.k, cfg.score, cfg.renormalize,
                                               cfg.temperature, cfg.min_prob, idx, g),
             "layout": lambda: moe.moe_layout(idx, cfg.E, counts, offs, row_of, src_of, lws),
+            "route_layout": lambda: route_layout_into(L_buf),
             # the layer's form: walked by token through row_of
             "dispatch": (lambda: moe.moe_dispatch_fp8_by_token(X, row_of, cfg.k, Xe, xs))
                         if args.fp8 else (lambda: moe.moe_dispatch_by_token(X, row_of, cfg.k, Xe)),
@@ -424,6 +430,12 @@ def run_ours(args, cfg, rank, world, local_rank):
             "pipeline": lambda: moe.moe_ffn_pipeline(X, src_of, row_of, g, offs, inp["W1"],
                                                      inp["W2"], Y=Y, ws=pws),
         }
+        def route_layout_into(Lb):
+            r = moe.moe_route_layout(Lb, cfg.k, cfg.score, cfg.renormalize, cfg.temperature,
+                                     cfg.min_prob)
+            for dst, src in zip((idx, g, counts, offs, row_of, src_of), r):
+                dst.copy_(src)
+
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stage_names) + 1)]
                for _ in range(args.steps)]
         # one untimed pass fills every staged buffer (offsets, row_of, ...) before

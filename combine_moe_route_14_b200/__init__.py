@@ -30,7 +30,7 @@ __all__ = [
     "moe_expert_ffn_fused_workspace_size", "moe_expert_ffn_fused", "moe_expert_ffn_fused_fp8",
     "moe_selftest_bounded_wait", "moe_dispatch_by_token", "moe_dispatch_fp8_by_token",
     "moe_ffn_pipeline_workspace_size", "moe_ffn_pipeline", "make_desc",
-    "moe_host_workspace_size", "moe_layer_forward_host",
+    "moe_host_workspace_size", "moe_layer_forward_host", "moe_route_layout",
     "LAYER_GATHER_ON_LOAD", "LAYER_FUSED_FFN", "LAYER_FUSED_COMBINE", "LAYER_FUSED_DISPATCH",
     "LAYER_PIPELINE",
 ]
@@ -103,6 +103,9 @@ _SIG = {
                              ctypes.c_int),
     "moe_expert_ffn_fused_fp8": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P,
                                   ctypes.c_size_t, _P], ctypes.c_int),
+    "moe_route_layout_workspace_size": ([_I, _I], ctypes.c_size_t),
+    "moe_route_layout": ([_P, _I, _I, _I, _I, _I, ctypes.c_float, ctypes.c_float, _P, _P, _P, _P,
+                          _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "moe_host_workspace_size": ([ctypes.POINTER(LayerDesc), _I], ctypes.c_size_t),
     "moe_layer_forward_host": ([ctypes.POINTER(LayerDesc), _I, _P, _P, _P, _P, _P, _P, _P, _P,
                                 ctypes.c_size_t, _P], ctypes.c_int),
@@ -640,6 +643,29 @@ def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=
                                      _ptr(topk_idx_out), _ptr(gates_out), _ptr(counts_out),
                                      _ptr(ws), ws.numel(), _stream(stream, dev)))
     return Y
+
+
+def moe_route_layout(logits, k, score="softmax", renormalize=True, temperature=1.0,
+                     min_prob=0.0, stream=None):
+    """Routing and layout in one pass (C ABI moe_route_layout).
+
+    Returns (topk_idx, gates, counts, offsets, row_of, src_of)."""
+    lib = load_library()
+    T, E = logits.shape
+    dev = logits.device
+    _need(logits, "logits", torch.float32, (T, E))
+    i32 = dict(dtype=torch.int32, device=dev)
+    idx = torch.empty((T, k), **i32)
+    gates = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts, offsets = torch.empty((E,), **i32), torch.empty((E + 1,), **i32)
+    row_of, src_of = torch.empty((T * k,), **i32), torch.empty((T * k,), **i32)
+    ws = torch.empty(max(16, int(lib.moe_route_layout_workspace_size(T, E))), dtype=torch.uint8,
+                     device=dev)
+    _check(lib.moe_route_layout(_ptr(logits), T, E, k, _score(score), int(bool(renormalize)),
+                                float(temperature), float(min_prob), _ptr(idx), _ptr(gates),
+                                _ptr(counts), _ptr(offsets), _ptr(row_of), _ptr(src_of), _ptr(ws),
+                                ws.numel(), _stream(stream, dev)))
+    return idx, gates, counts, offsets, row_of, src_of
 
 
 def moe_host_workspace_size(desc: LayerDesc, with_logits: bool) -> int:

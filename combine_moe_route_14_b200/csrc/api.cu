@@ -146,7 +146,7 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 // Workspace of the fused forward: sub-buffers, each 256-byte aligned.
 struct LayerWs {
   size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, scale, ctr, part,
-      total;
+      lb, total;
 };
 
 // Counter words of the layer workspace (all zeroed by one memset per forward):
@@ -192,6 +192,7 @@ LayerWs layer_ws(const moe_layer_desc& d) {
                                      moe::dispatch_counter_words((int)R) +
                                      moe::combine_counter_words(d.T, d.d)) * sizeof(uint32_t));
   w.part = o;    o += up256(T * d.d * sizeof(float));  // fused combine: fp32 partial rows
+  w.lb = o;      o += up256(moe::route_rank_lookback_words(d.T, d.E) * sizeof(uint32_t));
   w.total = o;
   return w;
 }
@@ -280,6 +281,15 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   const bool gather = (d.flags & MOE_LAYER_GATHER_ON_LOAD) != 0;
   const bool comb = (d.flags & MOE_LAYER_FUSED_COMBINE) && d.k <= 2;
   const bool fdisp = fused && (d.flags & MOE_LAYER_FUSED_DISPATCH) && !fp8;
+  // Routing fused with the layout's ranking, the rows finished by the
+  // token-walking dispatch: the layer's bf16 path (the gathered, dispatch-item
+  // and FP8 forms read src_of before any dispatch kernel, or dispatch
+  // quantised rows, and keep the separate layout kernel).
+  // Up to 32 experts (one look-back per warp of the routing kernel); with
+  // more, the per-expert look-backs of a tile run one after another and the
+  // separate layout kernels measured faster (256 experts: 103 us vs 27 us).
+  const bool ranked = !gather && !fdisp && !fp8 && d.E <= moe::kRankedMaxExperts;
+  uint32_t* lb = reinterpret_cast<uint32_t*>(base + w.lb);
 
   if (Wr) {
     MOE_STAGE("moe.router_logits");
@@ -290,14 +300,24 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   // GEMM-2's epilogue, writes the zero outputs of tokens whose slots were all
   // dropped (no expert row reaches them).
   const bool drops = d.min_prob > 0.f;
-  {
+  if (ranked) {
     MOE_STAGE("moe.route");
-    MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
-                               d.min_prob, idx, gates, s, (comb && drops) ? Y : nullptr, d.d,
-                               ctr, lc.used),
-             "route");
-  }
-  {
+    MOE_CUDA(cudaMemsetAsync(lb, 0, moe::route_rank_lookback_words(d.T, d.E) * sizeof(uint32_t),
+                             s),
+             "memset look-back");
+    MOE_CUDA(moe::launch_route_rank(L, d.T, d.E, d.k, d.score, d.renormalize,
+                                    desc_temperature(d), d.min_prob, idx, gates, row_of, counts,
+                                    offsets, lb, *dev, s, (comb && drops) ? Y : nullptr, d.d, ctr,
+                                    lc.used),
+             "route_rank");
+  } else {
+    {
+      MOE_STAGE("moe.route");
+      MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
+                                 d.min_prob, idx, gates, s, (comb && drops) ? Y : nullptr, d.d,
+                                 ctr, lc.used),
+               "route");
+    }
     MOE_STAGE("moe.layout");
     MOE_CUDA(moe::launch_layout(idx, R, d.E, counts, offsets, row_of, src_of, lws, *dev, s),
              "layout");
@@ -330,7 +350,9 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
                "dispatch_fp8");
     } else {
       MOE_STAGE("moe.dispatch");
-      MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+      MOE_CUDA(moe::launch_dispatch_scatter(X, idx, row_of, offsets, d.T, d.d, d.k, d.E, Xe,
+                                            src_of, *dev, s),
+               "dispatch");
     }
     MOE_STAGE("moe.fused_ffn");
     e = moe::launch_fused_ffn(Xe, x_scale, offsets, W1, W1s, W2, d.E, R, d.d, d.f, fp8, H, Ye,
@@ -361,7 +383,9 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   } else {
     {
       MOE_STAGE("moe.dispatch");
-      MOE_CUDA(moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s), "dispatch");
+      MOE_CUDA(moe::launch_dispatch_scatter(X, idx, row_of, offsets, d.T, d.d, d.k, d.E, Xe,
+                                            src_of, *dev, s),
+               "dispatch");
     }
     MOE_STAGE("moe.gemm1");
     e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err, &ex1);
@@ -493,6 +517,54 @@ moe_status moe_layout(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k, 
   }
   MOE_CUDA(moe::launch_layout(topk_idx, T * k, E, counts, offsets, row_of, src_of, ws, *dev, s),
            "layout");
+  return MOE_OK;
+}
+
+size_t moe_route_layout_workspace_size(int32_t T, int32_t E) {
+  if (T < 0 || E < 1) return 0;
+  return up256(moe::route_rank_lookback_words(T, E) * sizeof(uint32_t));
+}
+
+moe_status moe_route_layout(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
+                            int32_t renormalize, float temperature, float min_prob,
+                            int32_t* topk_idx, float* gates, int32_t* counts, int32_t* offsets,
+                            int32_t* row_of, int32_t* src_of, void* ws, size_t ws_bytes,
+                            void* stream) {
+  MOE_TRY(check_ET(T, E, k));
+  if (score != MOE_SCORE_SOFTMAX && score != MOE_SCORE_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "unknown score");
+  if (renormalize != 0 && renormalize != 1)
+    return fail(MOE_ERR_INVALID_ARG, "renormalize must be 0 or 1");
+  if (!std::isfinite(temperature) || !(temperature > 0.f))
+    return fail(MOE_ERR_INVALID_ARG, "temperature must be > 0");
+  if (!std::isfinite(min_prob)) return fail(MOE_ERR_INVALID_ARG, "min_prob must be finite");
+  MOE_TRY(check_ptr4(counts, "counts"));
+  MOE_TRY(check_ptr4(offsets, "offsets"));
+  cudaStream_t s = as_stream(stream);
+  if (T == 0) {
+    MOE_CUDA(cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), s), "memset counts");
+    MOE_CUDA(cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * sizeof(int32_t), s), "memset offsets");
+    return MOE_OK;
+  }
+  MOE_TRY(check_ptr4(logits, "logits"));
+  MOE_TRY(check_ptr4(topk_idx, "topk_idx"));
+  MOE_TRY(check_ptr4(gates, "gates"));
+  MOE_TRY(check_ptr4(row_of, "row_of"));
+  MOE_TRY(check_ptr4(src_of, "src_of"));
+  if (ws_bytes < moe_route_layout_workspace_size(T, E))
+    return fail(MOE_ERR_INVALID_ARG, "workspace too small");
+  MOE_TRY(check_ptr(ws, "ws"));
+  const moe::DeviceInfo* dev;
+  MOE_TRY(get_dev(&dev));
+  uint32_t* lb = static_cast<uint32_t*>(ws);
+  MOE_CUDA(cudaMemsetAsync(lb, 0, moe::route_rank_lookback_words(T, E) * sizeof(uint32_t), s),
+           "memset look-back");
+  MOE_CUDA(moe::launch_route_rank(logits, T, E, k, score, renormalize, temperature, min_prob,
+                                  topk_idx, gates, row_of, counts, offsets, lb, *dev, s),
+           "route_rank");
+  MOE_CUDA(moe::launch_dispatch_scatter(nullptr, topk_idx, row_of, offsets, T, 8, k, E, nullptr,
+                                        src_of, *dev, s),
+           "rows");
   return MOE_OK;
 }
 
@@ -864,8 +936,13 @@ int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with
       ((f & MOE_LAYER_GATHER_ON_LOAD) || (fused && (f & MOE_LAYER_FUSED_DISPATCH))) ? 0 : 1;
   const int gemms = fused ? 1 : 2;
   const int combine = ((f & MOE_LAYER_FUSED_COMBINE) && desc->k <= 2) ? 0 : 1;
-  return (with_router ? 1 : 0) + 1 + moe::layout_kernel_count((int64_t)desc->T * desc->k) +
-         dispatch + gemms + combine;
+  // the bf16 layer ranks the slots inside the routing kernel (no layout
+  // launch) unless it gathers or dispatches inside the fused FFN
+  const bool ranked = !(f & MOE_LAYER_GATHER_ON_LOAD) &&
+                      !(fused && (f & MOE_LAYER_FUSED_DISPATCH)) &&
+                      desc->E <= moe::kRankedMaxExperts;
+  const int layout = ranked ? 0 : moe::layout_kernel_count((int64_t)desc->T * desc->k);
+  return (with_router ? 1 : 0) + 1 + layout + dispatch + gemms + combine;
 }
 
 int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t with_router) {
@@ -875,7 +952,11 @@ int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t 
   moe_layer_desc d = *desc;
   d.flags &= ~MOE_LAYER_FUSED_DISPATCH;
   const int dispatch = (d.flags & MOE_LAYER_GATHER_ON_LOAD) ? 0 : 1;
-  return moe_kernel_launches_per_forward(&d, with_router) - dispatch +
+  // FP8 mode keeps the separate layout kernel (the bf16 count has none when
+  // it ranks in the routing kernel)
+  const bool ranked = !(d.flags & MOE_LAYER_GATHER_ON_LOAD) && d.E <= moe::kRankedMaxExperts;
+  const int layout = ranked ? moe::layout_kernel_count((int64_t)desc->T * desc->k) : 0;
+  return moe_kernel_launches_per_forward(&d, with_router) - dispatch + layout +
          moe::fp8_dispatch_kernel_count(desc->T);
 }
 

@@ -90,6 +90,59 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
   }
 }
 
+// Token-ordered dispatch that also finishes the layout: slot i = t*k + j of
+// expert e_i = idx[i] with stable rank rank_i (row_of[i] on entry, from the
+// routing's ranking) takes row offsets[e_i] + rank_i.  Writes that row into
+// row_of[i] (in place), src_of[row] = i, and the token row into Xe[row];
+// rows past offsets[E] get src_of = -1.
+__global__ void __launch_bounds__(kGatherWarps * 32)
+    dispatch_scatter_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ idx,
+                            int32_t* __restrict__ row_of, const int32_t* __restrict__ offsets,
+                            int T, int k, int R, int E, int row_vecs, uint4* __restrict__ Xe,
+                            int32_t* __restrict__ src_of, uint32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * kGatherWarps;
+  const int kept = min(max(__ldg(offsets + E), 0), R);
+  for (int r = kept + blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x)
+    src_of[r] = -1;
+  for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
+    int my_row = -1;  // lane j < k: the row of slot j (-1: dropped)
+    if (lane < k) {
+      const int i = t * k + lane;
+      const int e = __ldg(idx + i);
+      if (e >= 0 && e < E) {
+        my_row = __ldg(offsets + e) + row_of[i];
+        if (my_row < 0 || my_row >= R) {
+          flag_error(status, MOE_DEV_BAD_ROW);
+          my_row = -1;
+        }
+      }
+      row_of[i] = my_row;
+      if (my_row >= 0) src_of[my_row] = i;
+    }
+    const uint32_t live = __ballot_sync(0xffffffffu, lane < k && my_row >= 0);
+    if (!live || X == nullptr) continue;  // X null: the rows only (moe_route_layout)
+    const uint4* src = X + (size_t)t * row_vecs;
+    for (int c0 = 0; c0 < row_vecs; c0 += 32 * kCopyUnroll) {
+      uint4 v[kCopyUnroll];
+#pragma unroll
+      for (int u = 0; u < kCopyUnroll; ++u) {
+        const int c = c0 + u * 32 + lane;
+        if (c < row_vecs) v[u] = ld_stream_v4(src + c);
+      }
+      for (uint32_t m = live; m; m &= m - 1) {
+        const int r = __shfl_sync(0xffffffffu, my_row, __ffs(m) - 1);
+        uint4* dst = Xe + (size_t)r * row_vecs;
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+          const int c = c0 + u * 32 + lane;
+          if (c < row_vecs) dst[c] = v[u];
+        }
+      }
+    }
+  }
+}
+
 // Y[t, :] = bf16( sum_{j<k} gates[t, j] * Ye[row_of[t*k + j], :] ), fp32 sum in slot order;
 // a dropped slot (row_of -1) contributes nothing.
 // kK > 0: k known at compile time; kK == 0: runtime k (<= kMaxTopK).
@@ -190,6 +243,16 @@ cudaError_t launch_dispatch_rows(const void* X, const int32_t* row_of, int T, in
   dispatch_rows_kernel<<<gather_grid(T, dev), kGatherWarps * 32, 0, stream>>>(
       static_cast<const uint4*>(X), row_of, T, k, T * k, d / 8, static_cast<uint4*>(Xe),
       dev.status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_scatter(const void* X, const int32_t* idx, int32_t* row_of,
+                                    const int32_t* offsets, int T, int d, int k, int E, void* Xe,
+                                    int32_t* src_of, const DeviceInfo& dev, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  dispatch_scatter_kernel<<<gather_grid(T, dev), kGatherWarps * 32, 0, stream>>>(
+      static_cast<const uint4*>(X), idx, row_of, offsets, T, k, T * k, E, d / 8,
+      static_cast<uint4*>(Xe), src_of, dev.status);
   return cudaGetLastError();
 }
 

@@ -35,6 +35,24 @@ cudaError_t launch_route(const float* L, int T, int E, int k, int score, int ren
                          cudaStream_t stream, void* zero_rows = nullptr, int zero_d = 0,
                          uint32_t* zero_words = nullptr, int n_zero_words = 0);
 
+// Routing fused with the layout's ranking (see route.cu): idx, gates, the
+// stable rank of each kept slot within its expert (into rank[], -1 for a
+// dropped slot), counts and offsets.  lookback: route_rank_lookback_words(T,
+// E) words, zeroed before the launch.
+size_t route_rank_lookback_words(int T, int E);
+constexpr int kRankedMaxExperts = 32;  // the layer ranks in its routing kernel up to this E
+cudaError_t launch_route_rank(const float* L, int T, int E, int k, int score, int renormalize,
+                              float temperature, float min_prob, int32_t* idx, float* gates,
+                              int32_t* rank, int32_t* counts, int32_t* offsets, uint32_t* lookback,
+                              const DeviceInfo& dev, cudaStream_t stream, void* zero_rows = nullptr,
+                              int zero_d = 0, uint32_t* zero_words = nullptr,
+                              int n_zero_words = 0);
+// Token-ordered dispatch finishing the layout from route_rank's ranks
+// (row_of holds the ranks on entry and the rows on return; src_of written).
+cudaError_t launch_dispatch_scatter(const void* X, const int32_t* idx, int32_t* row_of,
+                                    const int32_t* offsets, int T, int d, int k, int E, void* Xe,
+                                    int32_t* src_of, const DeviceInfo& dev, cudaStream_t stream);
+
 size_t layout_workspace_bytes(int64_t R, int E);
 // Number of kernels launch_layout issues for R slots.
 int layout_kernel_count(int64_t R);

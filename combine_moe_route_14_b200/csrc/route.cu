@@ -340,23 +340,12 @@ __device__ __forceinline__ bool better(float v, int e, float bv, int be) {
   return v > bv || (v == bv && e < be);
 }
 
+// One token's routing by one warp: lanes j < k get slot j's expert (or -1
+// when the slot is dropped) and its gate.  Every lane must call it.
 template <int kEPL>
-__global__ void __launch_bounds__(kRouteWarps * 32)
-    route_topk_kernel(const float* __restrict__ L, int T, int E, int k, int score, int renorm,
-                      float inv_temp, float min_prob, int32_t* __restrict__ idx,
-                      float* __restrict__ gates, uint4* __restrict__ zero_rows, int zero_vecs,
-                      uint32_t* __restrict__ zero_words, int n_zero_words) {
-  // side job: clear the caller's counter words (grid-stride; the layer's
-  // later kernels run after this one on the same stream)
-  if (zero_words) {
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero_words;
-         i += gridDim.x * blockDim.x)
-      zero_words[i] = 0u;
-  }
-  const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (t >= T) return;
-  const float* row = L + (size_t)t * E;
+__device__ __forceinline__ void route_token(const float* __restrict__ row, int E, int k, int score,
+                                            int renorm, float inv_temp, float min_prob,
+                                            int lane, int& e_out, float& g_out) {
   float v[kEPL];
 #pragma unroll
   for (int i = 0; i < kEPL; ++i) {
@@ -428,15 +417,210 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   } else {
     g = keep ? prob : 0.f;
   }
-  if (slot) {
-    idx[(size_t)t * k + lane] = keep ? my_e : -1;
-    gates[(size_t)t * k + lane] = g;
-  }
-  // A token with no kept slot gets no expert row, so no later stage writes
-  // its output; when asked, its output row is zeroed here.
-  if (zero_rows && __ballot_sync(0xffffffffu, keep) == 0u) {
+  e_out = keep ? my_e : -1;
+  g_out = g;
+}
+
+// A token with no kept slot gets no expert row, so no later stage writes
+// its output; when asked, its output row is zeroed here.
+__device__ __forceinline__ void zero_row_if_dropped(int e_lane, int k, int lane, uint4* zero_rows,
+                                                    int zero_vecs, int t) {
+  if (zero_rows && __ballot_sync(0xffffffffu, lane < k && e_lane >= 0) == 0u) {
     uint4* row = zero_rows + (size_t)t * zero_vecs;
     for (int c = lane; c < zero_vecs; c += 32) row[c] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+template <int kEPL>
+__global__ void __launch_bounds__(kRouteWarps * 32)
+    route_topk_kernel(const float* __restrict__ L, int T, int E, int k, int score, int renorm,
+                      float inv_temp, float min_prob, int32_t* __restrict__ idx,
+                      float* __restrict__ gates, uint4* __restrict__ zero_rows, int zero_vecs,
+                      uint32_t* __restrict__ zero_words, int n_zero_words) {
+  // side job: clear the caller's counter words (grid-stride; the layer's
+  // later kernels run after this one on the same stream)
+  if (zero_words) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero_words;
+         i += gridDim.x * blockDim.x)
+      zero_words[i] = 0u;
+  }
+  const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= T) return;
+  int e;
+  float g;
+  route_token<kEPL>(L + (size_t)t * E, E, k, score, renorm, inv_temp, min_prob, lane, e, g);
+  if (lane < k) {
+    idx[(size_t)t * k + lane] = e;
+    gates[(size_t)t * k + lane] = g;
+  }
+  zero_row_if_dropped(e, k, lane, zero_rows, zero_vecs, t);
+}
+
+// ---------------------------------------------------------------------------
+// Routing fused with the layout's ranking (the layer's path): each CTA
+// routes a tile of tokens, taken in ticket order, and also gives every kept
+// slot i its stable rank among the slots of its expert:
+//   rank[i] = #{i' < i : e_i' = e_i}            (DySHARP review §3.1 item 3:
+// layout blocks allocated incrementally, in logical order), written into
+// row_of[i].  Within the tile the ranks come from warp match / popcount over
+// the slots in order; across tiles each CTA adds, per expert, the count of
+// all earlier tiles, found with a decoupled look-back (Merrill & Garland,
+// "Single-pass Parallel Prefix Scan with Decoupled Look-back", 2016) over
+// per-tile status words.  The CTA with the last ticket holds the totals and
+// writes counts and offsets.  The token-walking dispatch then turns ranks
+// into rows (row_of[i] = offsets[e_i] + rank[i], src_of[row] = i) while it
+// copies the token rows, so no separate layout launch runs.
+// ---------------------------------------------------------------------------
+// Warps (= tokens) per CTA: 32, or 16 when a lane holds 32 logits (E > 512),
+// which needs more registers than 1024 threads leave.
+__host__ __device__ constexpr int rank_warps(int epl) { return epl >= 32 ? 16 : 32; }
+constexpr uint32_t kLbAggregate = 1u << 30;
+constexpr uint32_t kLbInclusive = 2u << 30;
+constexpr uint32_t kLbValue = (1u << 30) - 1u;
+
+static int rank_tile(int E) { return rank_warps((E + 31) / 32 > 16 ? 32 : 1); }
+int route_rank_tiles(int T, int E) { return (T + rank_tile(E) - 1) / rank_tile(E); }
+size_t route_rank_lookback_words(int T, int E) { return 1 + (size_t)route_rank_tiles(T, E) * E; }
+
+template <int kEPL>
+__global__ void __launch_bounds__(rank_warps(kEPL) * 32)
+    route_rank_kernel(const float* __restrict__ L, int T, int E, int k, int score, int renorm,
+                      float inv_temp, float min_prob, int32_t* __restrict__ idx,
+                      float* __restrict__ gates, int32_t* __restrict__ rank,
+                      int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                      uint32_t* __restrict__ lookback, uint4* __restrict__ zero_rows,
+                      int zero_vecs, uint32_t* __restrict__ zero_words, int n_zero_words,
+                      uint32_t* status) {
+  constexpr int kRankWarps = rank_warps(kEPL);
+  constexpr int kRankTile = kRankWarps;  // one token per warp
+  // shared: keys[kRankTile * k] | run[E] | tile id
+  extern __shared__ int sm[];
+  const int nslot = kRankTile * k;
+  int* keys = sm;
+  int* run = keys + nslot;
+  int* s_tile = run + E;
+  uint32_t* ticket = lookback;          // word 0
+  uint32_t* words = lookback + 1;       // [tiles][E] status words
+  if (zero_words) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero_words;
+         i += gridDim.x * blockDim.x)
+      zero_words[i] = 0u;
+  }
+  if (threadIdx.x == 0) *s_tile = (int)atomicAdd(ticket, 1u);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) run[e] = 0;
+  __syncthreads();
+  const int tile = *s_tile;
+  const int tiles = (int)gridDim.x;
+  const int t0 = tile * kRankTile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // ---- route this tile's tokens, one warp per token
+  {
+    const int t = t0 + warp;
+    int e = -1;
+    float g = 0.f;
+    if (t < T) {
+      route_token<kEPL>(L + (size_t)t * E, E, k, score, renorm, inv_temp, min_prob, lane, e, g);
+      if (lane < k) {
+        idx[(size_t)t * k + lane] = e;
+        gates[(size_t)t * k + lane] = g;
+      }
+      zero_row_if_dropped(e, k, lane, zero_rows, zero_vecs, t);
+    }
+    if (lane < k) keys[warp * k + lane] = t < T ? e : -1;
+  }
+  __syncthreads();
+  // ---- ranks within the tile: warp 0 walks the slots in order, 32 at a time
+  if (warp == 0) {
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int c = 0; c < nslot; c += 32) {
+      const int key = c + lane < nslot ? keys[c + lane] : -1;
+      const uint32_t peers = __match_any_sync(0xffffffffu, key);
+      const int r = key >= 0 ? run[key] + __popc(peers & lt_mask) : -1;
+      __syncwarp();
+      if (key >= 0 && lane == __ffs(peers) - 1) run[key] += __popc(peers);
+      if (c + lane < nslot) keys[c + lane] = key >= 0 ? (key << 20) | r : -1;  // e, local rank
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // ---- per expert: this tile's base among all earlier tiles, by a
+  // warp-wide look-back (one warp per expert; lane l reads tile p - l, so 32
+  // predecessors' status words are in flight at once)
+  for (int e = warp; e < E; e += kRankWarps) {
+    uint32_t* my = words + (size_t)tile * E + e;
+    const uint32_t a = (uint32_t)run[e];
+    uint32_t excl = 0;
+    if (tile == 0) {
+      if (lane == 0) st_release_gpu(my, kLbInclusive | a);
+    } else {
+      if (lane == 0) st_release_gpu(my, kLbAggregate | a);
+      int p = tile - 1;
+      uint64_t tstart = 0;
+      uint32_t spins = 0;
+      bool timed_out = false;
+      while (true) {
+        const int pred = p - lane;
+        // before tile 0: an inclusive prefix of 0
+        const uint32_t sw = pred >= 0 ? ld_acquire_gpu(words + (size_t)pred * E + e) : kLbInclusive;
+        const uint32_t flag = sw & ~kLbValue;
+        const uint32_t inc = __ballot_sync(0xffffffffu, flag == kLbInclusive);
+        const uint32_t pub = __ballot_sync(0xffffffffu, flag != 0u);
+        const int first = inc ? __ffs(inc) - 1 : 31;   // nearest inclusive prefix (or all 32)
+        const uint32_t need = first == 31 ? 0xffffffffu : ((2u << first) - 1u);
+        if ((pub & need) != need) {
+          // a predecessor has not published: its CTA took its ticket earlier,
+          // so it is running; wait, but not forever
+          if (spins == 0) tstart = globaltimer_ns();
+          if ((++spins & 63u) == 0 && globaltimer_ns() - tstart > kWaitLimitNs) {
+            timed_out = true;
+            break;
+          }
+          __nanosleep(32);
+          continue;
+        }
+        uint32_t v = lane <= first ? (sw & kLbValue) : 0u;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        excl += v;
+        if (inc) break;
+        p -= 32;
+      }
+      if (timed_out && lane == 0) flag_error(status, MOE_DEV_TIMEOUT);
+      if (lane == 0) st_release_gpu(my, kLbInclusive | ((excl + a) & kLbValue));
+    }
+    if (lane == 0) {
+      if (tile == tiles - 1) counts[e] = (int)(excl + a);  // the last tile sees every slot
+      run[e] = (int)excl;
+    }
+  }
+  __syncthreads();
+// ---- ranks out (into row_of)
+  for (int i = threadIdx.x; i < nslot; i += blockDim.x) {
+    const int t = t0 + i / k;
+    if (t >= T) continue;
+    const int kv = keys[i];
+    rank[(size_t)t0 * k + i] = kv < 0 ? -1 : run[kv >> 20] + (kv & 0xFFFFF);
+  }
+  // ---- the last tile: offsets = exclusive scan of the counts
+  if (tile == tiles - 1) {
+    __threadfence_block();
+    if (warp == 0) {
+      int base = 0;
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        const int c = e < E ? counts[e] : 0;
+        int incl = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        if (e < E) offsets[e] = base + incl - c;
+        base += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) offsets[E] = base;
+    }
   }
 }
 
@@ -460,6 +644,31 @@ cudaError_t launch_route(const float* L, int T, int E, int k, int score, int ren
   else if (epl <= 16) MOE_ROUTE_LAUNCH(16);
   else MOE_ROUTE_LAUNCH(32);
 #undef MOE_ROUTE_LAUNCH
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_rank(const float* L, int T, int E, int k, int score, int renormalize,
+                              float temperature, float min_prob, int32_t* idx, float* gates,
+                              int32_t* rank, int32_t* counts, int32_t* offsets, uint32_t* lookback,
+                              const DeviceInfo& dev, cudaStream_t stream, void* zero_rows,
+                              int zero_d, uint32_t* zero_words, int n_zero_words) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = route_rank_tiles(T, E);
+  const int epl = (E + 31) / 32;
+  const float inv_temp = 1.0f / temperature;
+  const size_t smem = (size_t)(rank_tile(E) * k + E + 1) * sizeof(int);
+#define MOE_RANK_LAUNCH(N)                                                                     \
+  route_rank_kernel<N><<<blocks, rank_warps(N) * 32, smem, stream>>>(                          \
+      L, T, E, k, score, renormalize, inv_temp, min_prob, idx, gates, rank, counts, offsets,     \
+      lookback, static_cast<uint4*>(zero_rows), zero_d / 8, zero_words, n_zero_words,            \
+      dev.status)
+  if (epl <= 1) MOE_RANK_LAUNCH(1);
+  else if (epl <= 2) MOE_RANK_LAUNCH(2);
+  else if (epl <= 4) MOE_RANK_LAUNCH(4);
+  else if (epl <= 8) MOE_RANK_LAUNCH(8);
+  else if (epl <= 16) MOE_RANK_LAUNCH(16);
+  else MOE_RANK_LAUNCH(32);
+#undef MOE_RANK_LAUNCH
   return cudaGetLastError();
 }
 

@@ -183,6 +183,26 @@ moe_status moe_layout(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k, 
                       size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_route_layout -- moe_route_ex followed by moe_layout, with the layout's
+ * ranking folded into the routing kernel (the layer's own path): each CTA of
+ * the routing kernel ranks its tile's kept slots within their experts, in
+ * slot order, and adds the counts of all earlier tiles found by a decoupled
+ * look-back over per-tile status words (tiles taken in ticket order; every
+ * wait bounded); the last tile writes counts and offsets.  A second short
+ * kernel turns ranks into rows (row_of) and fills src_of.  Two launches
+ * instead of three (one + two past 16384 slots), and no single-CTA pass.
+ *   Arguments and results as moe_route_ex and moe_layout, bit for bit.
+ *   ws: at least moe_route_layout_workspace_size(T, E) bytes (look-back
+ *   status words, zeroed by the call).
+ * ------------------------------------------------------------------------- */
+size_t moe_route_layout_workspace_size(int32_t T, int32_t E);
+moe_status moe_route_layout(const float* logits, int32_t T, int32_t E, int32_t k, int32_t score,
+                            int32_t renormalize, float temperature, float min_prob,
+                            int32_t* topk_idx, float* gates, int32_t* counts, int32_t* offsets,
+                            int32_t* row_of, int32_t* src_of, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_layout_static -- moe_layout without a workspace argument, for callers
  * that cannot allocate device memory.  The pages have no counterpart: this
  * is a convenience of this library, not a step of the method.

@@ -109,14 +109,23 @@ def test_layer_workspace_and_desc_checks(lib):
 
 
 def test_launch_count(lib):
+    # bf16: router, route (with the layout's ranking), dispatch, 2 GEMMs, combine
     d = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 0)
-    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 1) == 7
-    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 0) == 6
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 1) == 6
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 0) == 5
+    # 256 experts: the separate layout (two kernels past 16384 slots)
     d4 = moe.LayerDesc(8192, 7168, 256, 8, 2048, 1, 1, 0)
-    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d4), 0) == 7  # two-kernel layout
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(d4), 0) == 7
+    # FP8: the separate layout kernel, absmax + dispatch
+    assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(d), 1) == 8
+    assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(d4), 0) == 8
+    # gathering: the separate layout, no dispatch kernel
     dg = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, moe.LAYER_GATHER_ON_LOAD)
-    assert lib.moe_kernel_launches_per_forward(ctypes.byref(dg), 1) == 6   # no dispatch kernel
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(dg), 1) == 6
     assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(dg), 1) == 8  # absmax + quantise
+    # the pipeline: route, layout, one persistent FFN (dispatch, GEMMs, combine)
+    dp = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, moe.LAYER_PIPELINE)
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(dp), 1) == 4
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
@@ -164,7 +173,7 @@ def test_fused_ffn_checks_on_the_host(lib):
     assert lib.moe_layer_forward(ctypes.byref(both), p, p, N, p, p, p, N, N, N, p, ws,
                                  N) == UNSUPPORTED
     fused = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, moe.LAYER_FUSED_FFN)
-    assert lib.moe_kernel_launches_per_forward(ctypes.byref(fused), 1) == 6  # one GEMM launch
+    assert lib.moe_kernel_launches_per_forward(ctypes.byref(fused), 1) == 5  # one GEMM launch
     assert lib.moe_kernel_launches_per_forward_fp8(ctypes.byref(fused), 1) == 7
 
 

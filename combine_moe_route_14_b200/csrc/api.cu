@@ -325,6 +325,13 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   // The two-launch path keeps the static balanced schedule (measured faster
   // than tickets on uniform tiles); the fused launch always takes tickets.
   moe::GemmExtras ex1, ex2;
+  // bf16 dispatch: with the ranks from the routing kernel it also turns them
+  // into rows (row_of, src_of); otherwise the layout kernel already did
+  auto dispatch_bf16 = [&]() {
+    return ranked ? moe::launch_dispatch_scatter(X, idx, row_of, offsets, d.T, d.d, d.k, d.E,
+                                                 Xe, src_of, *dev, s)
+                  : moe::launch_dispatch_rows(X, row_of, d.T, d.d, d.k, Xe, *dev, s);
+  };
   if (comb) {
     ex2.comb_Y = Y;
     ex2.comb_src = src_of;
@@ -350,9 +357,7 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
                "dispatch_fp8");
     } else {
       MOE_STAGE("moe.dispatch");
-      MOE_CUDA(moe::launch_dispatch_scatter(X, idx, row_of, offsets, d.T, d.d, d.k, d.E, Xe,
-                                            src_of, *dev, s),
-               "dispatch");
+      MOE_CUDA(dispatch_bf16(), "dispatch");
     }
     MOE_STAGE("moe.fused_ffn");
     e = moe::launch_fused_ffn(Xe, x_scale, offsets, W1, W1s, W2, d.E, R, d.d, d.f, fp8, H, Ye,
@@ -383,9 +388,7 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   } else {
     {
       MOE_STAGE("moe.dispatch");
-      MOE_CUDA(moe::launch_dispatch_scatter(X, idx, row_of, offsets, d.T, d.d, d.k, d.E, Xe,
-                                            src_of, *dev, s),
-               "dispatch");
+      MOE_CUDA(dispatch_bf16(), "dispatch");
     }
     MOE_STAGE("moe.gemm1");
     e = moe::launch_grouped_gemm(Xe, offsets, W1, d.E, R, d.f, d.d, true, H, *dev, s, &err, &ex1);

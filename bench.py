@@ -430,11 +430,13 @@ def run_ours(args, cfg, rank, world, local_rank):
             "pipeline": lambda: moe.moe_ffn_pipeline(X, src_of, row_of, g, offs, inp["W1"],
                                                      inp["W2"], Y=Y, ws=pws),
         }
+        rl_ws = torch.empty(max(16, moe.load_library().moe_route_layout_workspace_size(
+            cfg.T, cfg.E)), dtype=torch.uint8, device=dev)
+
         def route_layout_into(Lb):
-            r = moe.moe_route_layout(Lb, cfg.k, cfg.score, cfg.renormalize, cfg.temperature,
-                                     cfg.min_prob)
-            for dst, src in zip((idx, g, counts, offs, row_of, src_of), r):
-                dst.copy_(src)
+            moe.moe_route_layout(Lb, cfg.k, cfg.score, cfg.renormalize, cfg.temperature,
+                                 cfg.min_prob, out=(idx, g, counts, offs, row_of, src_of),
+                                 ws=rl_ws)
 
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stage_names) + 1)]
                for _ in range(args.steps)]

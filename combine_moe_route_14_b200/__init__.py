@@ -646,21 +646,32 @@ def moe_layer_forward_fp8(X, W1q, w1_scale, W2, k, score="softmax", renormalize=
 
 
 def moe_route_layout(logits, k, score="softmax", renormalize=True, temperature=1.0,
-                     min_prob=0.0, stream=None):
+                     min_prob=0.0, out=None, ws=None, stream=None):
     """Routing and layout in one pass (C ABI moe_route_layout).
 
-    Returns (topk_idx, gates, counts, offsets, row_of, src_of)."""
+    out: optional (topk_idx, gates, counts, offsets, row_of, src_of) tensors to
+    fill.  Returns that tuple."""
     lib = load_library()
     T, E = logits.shape
     dev = logits.device
     _need(logits, "logits", torch.float32, (T, E))
     i32 = dict(dtype=torch.int32, device=dev)
-    idx = torch.empty((T, k), **i32)
-    gates = torch.empty((T, k), dtype=torch.float32, device=dev)
-    counts, offsets = torch.empty((E,), **i32), torch.empty((E + 1,), **i32)
-    row_of, src_of = torch.empty((T * k,), **i32), torch.empty((T * k,), **i32)
-    ws = torch.empty(max(16, int(lib.moe_route_layout_workspace_size(T, E))), dtype=torch.uint8,
-                     device=dev)
+    if out is None:
+        out = (torch.empty((T, k), **i32), torch.empty((T, k), dtype=torch.float32, device=dev),
+               torch.empty((E,), **i32), torch.empty((E + 1,), **i32),
+               torch.empty((T * k,), **i32), torch.empty((T * k,), **i32))
+    idx, gates, counts, offsets, row_of, src_of = out
+    for t, n, dt, shp in ((idx, "topk_idx", torch.int32, (T, k)),
+                          (gates, "gates", torch.float32, (T, k)),
+                          (counts, "counts", torch.int32, (E,)),
+                          (offsets, "offsets", torch.int32, (E + 1,)),
+                          (row_of, "row_of", torch.int32, (T * k,)),
+                          (src_of, "src_of", torch.int32, (T * k,))):
+        _need(t, n, dt, shp, dev)
+    if ws is None:
+        ws = torch.empty(max(16, int(lib.moe_route_layout_workspace_size(T, E))),
+                         dtype=torch.uint8, device=dev)
+    _need(ws, "ws", torch.uint8, None, dev)
     _check(lib.moe_route_layout(_ptr(logits), T, E, k, _score(score), int(bool(renormalize)),
                                 float(temperature), float(min_prob), _ptr(idx), _ptr(gates),
                                 _ptr(counts), _ptr(offsets), _ptr(row_of), _ptr(src_of), _ptr(ws),
@@ -713,7 +724,8 @@ def moe_layer_forward_host(X_host, W1, W2, k, Y_host, score="softmax", renormali
 
 
 def moe_selftest_bounded_wait(which: int, limit_us: int, counter=None, stream=None):
-    """Run one bounded device wait that times out (0: global counter, 1: mbarrier)."""
+    """Run one bounded device wait that times out (0: readiness counts, 1: ring mbarrier,
+    2: combine flag bit, 3: work-item queue mbarrier, cluster scope)."""
     lib = load_library()
     dev = counter.device if counter is not None else torch.device("cuda", torch.cuda.current_device())
     if counter is not None:

@@ -438,10 +438,10 @@ moe_status moe_device_status(uint32_t* bits, int32_t clear) {
 
 moe_status moe_selftest_bounded_wait(int32_t which, uint32_t limit_us, uint32_t* counter,
                                      void* stream) {
-  if (which != 0 && which != 1) return fail(MOE_ERR_INVALID_ARG, "which must be 0 or 1");
+  if (which < 0 || which > 3) return fail(MOE_ERR_INVALID_ARG, "which must be 0, 1, 2 or 3");
   if (limit_us < 1 || limit_us > 10u * 1000u * 1000u)
     return fail(MOE_ERR_INVALID_ARG, "limit_us must be in [1, 10^7]");
-  if (which == 0) MOE_TRY(check_ptr4(counter, "counter"));
+  if (which == 0 || which == 2) MOE_TRY(check_ptr4(counter, "counter"));
   const moe::DeviceInfo* dev;
   MOE_TRY(get_dev(&dev));
   MOE_CUDA(moe::launch_selftest_wait(which, (uint64_t)limit_us * 1000u, counter, *dev,

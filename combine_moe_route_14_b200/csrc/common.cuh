@@ -172,29 +172,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
-// Bounded wait until the counter at p (global memory, written by other CTAs
-// with release semantics or fence + atomic) reaches target; acquire order.
-// Gives up, with MOE_DEV_TIMEOUT and the CTA's abort flag set, after
-// limit_ns, or returns false at once when another role has aborted.
-__device__ __forceinline__ bool wait_count_geq(const uint32_t* p, uint32_t target,
-                                               uint32_t* status, volatile int* abort_flag,
-                                               uint64_t limit_ns = kWaitLimitNs) {
-  if (ld_acquire_gpu(p) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(128);
-    if (ld_acquire_gpu(p) >= target) return true;
-    if ((it & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        flag_error(status, MOE_DEV_TIMEOUT);
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
 // True when every counter p[0..n) has reached target (relaxed loads, all in
 // flight together; no ordering).
 __device__ __forceinline__ bool counts_reached(const uint32_t* p, int n, uint32_t target) {

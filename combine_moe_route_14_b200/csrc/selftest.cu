@@ -9,10 +9,14 @@
 
 namespace moe {
 
-// which = 0: a global counter that nothing increments (the fused FFN's
-//            readiness wait, wait_count_geq);
+// which = 0: global counters that nothing increments (the fused forms'
+//            readiness gates, wait_counts_geq);
 // which = 1: a shared-memory mbarrier that nothing arrives on (the GEMM's
-//            pipeline waits, mbar_wait).
+//            pipeline waits, mbar_wait);
+// which = 2: a flag bit in global memory that nothing sets (the combine
+//            epilogue's wait for a token's first slot, wait_bits_set);
+// which = 3: a shared-memory mbarrier with cluster-scope acquire (the
+//            work-item queue's waits, mbar_wait_cluster).
 __global__ void selftest_wait_kernel(int which, uint64_t limit_ns, uint32_t* counter,
                                      uint32_t* status) {
   __shared__ uint64_t bar;
@@ -20,11 +24,14 @@ __global__ void selftest_wait_kernel(int which, uint64_t limit_ns, uint32_t* cou
   if (threadIdx.x != 0) return;
   abort_flag = 0;
   if (which == 0) {
-    wait_count_geq(counter, 1u, status, &abort_flag, limit_ns);
+    wait_counts_geq(counter, 1, 1u, status, &abort_flag, limit_ns);
+  } else if (which == 2) {
+    wait_bits_set(counter, 0x100u, status, &abort_flag, limit_ns);
   } else {
     mbar_init(&bar, 1);
     fence_mbarrier_init();
-    mbar_wait(&bar, 0, status, &abort_flag, limit_ns);
+    if (which == 1) mbar_wait(&bar, 0, status, &abort_flag, limit_ns);
+    else mbar_wait_cluster(&bar, 0, status, &abort_flag, limit_ns);
   }
 }
 

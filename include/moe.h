@@ -505,10 +505,15 @@ const char* moe_last_error_string(void);
  * can check the failure path without faulting or hanging the GPU: the wait
  * gives up after limit_us microseconds, the kernel sets MOE_DEV_TIMEOUT in
  * the status word and returns; read it with moe_device_status().
- *   which = 0: the global-counter wait of the fused FFN (counter: a device
- *              uint32 holding 0, which nothing increments; caller-owned);
- *   which = 1: the shared-memory mbarrier wait of the grouped GEMM (counter
- *              unused, may be NULL).
+ *   which = 0: the readiness-count wait of the fused forms (counter: a
+ *              device uint32 holding 0, which nothing increments;
+ *              caller-owned);
+ *   which = 1: the shared-memory mbarrier wait of the grouped GEMM's ring
+ *              (counter unused, may be NULL);
+ *   which = 2: the flag wait of the combine in GEMM-2's epilogue (counter: a
+ *              device uint32 holding 0, whose flag bit nothing sets);
+ *   which = 3: the cluster-scope mbarrier wait of the work-item queue
+ *              (counter unused, may be NULL).
  *   1 <= limit_us <= 10^7. */
 moe_status moe_selftest_bounded_wait(int32_t which, uint32_t limit_us, uint32_t* counter,
                                      void* stream);

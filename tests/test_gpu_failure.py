@@ -14,10 +14,11 @@ DEV = "cuda:0"
 TIMEOUT_BIT = 0x2
 
 
-@pytest.mark.parametrize("which", [0, 1])
+# 0: readiness counts, 1: ring mbarrier, 2: combine flag bit, 3: queue mbarrier (cluster scope)
+@pytest.mark.parametrize("which", [0, 1, 2, 3])
 def test_bounded_wait_times_out_and_reports(cuda_lib, which):
     moe.moe_device_status(clear=True)
-    counter = torch.zeros(1, dtype=torch.int32, device=DEV) if which == 0 else None
+    counter = torch.zeros(1, dtype=torch.int32, device=DEV) if which in (0, 2) else None
     t0 = time.perf_counter()
     moe.moe_selftest_bounded_wait(which, 50_000, counter)  # 50 ms
     bits = moe.moe_device_status(clear=True)  # synchronises
@@ -35,6 +36,6 @@ def test_bounded_wait_times_out_and_reports(cuda_lib, which):
 
 def test_selftest_rejects_bad_arguments(cuda_lib):
     with pytest.raises(moe.MoeError):
-        moe.moe_selftest_bounded_wait(2, 1000)
+        moe.moe_selftest_bounded_wait(4, 1000)
     with pytest.raises(moe.MoeError):
         moe.moe_selftest_bounded_wait(1, 0)

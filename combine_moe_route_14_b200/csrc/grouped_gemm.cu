@@ -103,6 +103,38 @@ template <bool kGather, int kPair> struct Roles {
   static constexpr int FULL_ARRIVALS = NW + (kGather ? 1 : NTOK);
 };
 constexpr uint32_t TMEM_COLS = 2 * BN;       // two accumulators
+// Merged last token block (paired CTAs, plain two-launch forms): an expert
+// whose last token block would hold at most kMergeRows rows gives them to
+// the block before it, which then spans up to BN_MAX rows in one tile.  A
+// tile's pace is set by streaming its weight rows, whatever its token count,
+// so a 16-row tail tile costs about as much as a full one; merged, the
+// expert's weight block streams through the ring once instead of twice.  The
+// merged tile issues two MMAs per K step (N = 256 and N = the tail) into
+// BN_MAX accumulator columns.  Accumulators then no longer sit in two fixed
+// halves of TMEM: tiles alternate between a low placement (from column 0)
+// and a high one (ending at column 512), and where two consecutive tiles'
+// columns overlap, the next tile's MMAs wait until the epilogue has drained
+// the shared columns, which it drains first.
+constexpr int kMergeRows = 64;
+// Merging is used when the mean rows per expert is above kMergeMinMeanRows
+// (below it hardly any expert reaches 257 rows, and the variant costs ~1 % on
+// the decode shapes for nothing) and at most kMergeMaxMeanRows.  With few
+// rows per expert the GEMM is bound by streaming each tile's weights and a
+// tail tile doubles that stream.  With many (the Mixtral shape, ~1024 per
+// expert) the GEMM is bound by shared-memory bandwidth at full MMA rate, the
+// tail tile's weights come from L2 beside the full tiles, and a merged tile
+// costs more than the tail tile it replaces: its second MMA reads the weight
+// stage from shared memory again, neighbouring tiles whose columns overlap
+// cannot overlap their MMAs with its epilogue, and the static schedule gives
+// the wider tiles to some clusters only.  Measured on a B200: the fine-grained
+// shape (256 rows per expert) -10 % per GEMM, 1040 rows per expert +27 %.
+constexpr int kMergeMinMeanRows = 128;
+constexpr int kMergeMaxMeanRows = 384;
+constexpr int BN_MAX = BN + kMergeRows;      // 320 accumulator columns at most
+constexpr int kHighMin = 2 * BN - BN_MAX;    // 192: the lowest column a high tile starts at
+// A merged tile's tail rows (up to 32 per CTA) go into a ring of their own,
+// one 4 KB box per K-block beside each slot, so that the ordinary stage
+// layout and its address arithmetic stay as they are.
 constexpr int MAX_STAGES = 8;                // barrier slots; the ring uses Args::stages of them
 constexpr size_t kSmemBudget = 232448;       // B200 opt-in shared memory per block
 constexpr uint64_t kDrainLimitNs = 20ull * 1000ull * 1000ull;  // 20 ms
@@ -138,8 +170,7 @@ template <int kPair> struct Cfg {
   // K-blocks per ring slot: two with paired CTAs (3 slots of 64 KB), one with
   // a single CTA (its 48 KB K-block already leaves only 4 slots)
   static constexpr int KPS = kPair == 2 ? MOE_KPS_PAIR : 1;
-  static constexpr int STAGE = KPS * (A_STAGE + B_STAGE);  // one ring slot
-  static constexpr int NUM_BARS = 2 * MAX_STAGES + 4 + 1 + 2 * kQueue + 1;
+  static constexpr int NUM_BARS = 2 * MAX_STAGES + 4 + 1 + 2 * kQueue + 1 + 2;
   static constexpr int FEAT = BM * kPair;                // output features per tile
 };
 
@@ -149,15 +180,20 @@ __host__ __device__ constexpr size_t fixed_smem(int E) {
   return 1024 /* alignment slack */ + Cfg<kPair>::NUM_BARS * 8 + 16 + kQueue * sizeof(int) +
          (size_t)4 * (E + 1) * sizeof(int);
 }
+// merge: each slot also holds KPS tail boxes (merged last token blocks)
 template <int kPair>
-__host__ __device__ constexpr size_t smem_bytes(int E, int stages) {
-  return fixed_smem<kPair>(E) + (size_t)stages * Cfg<kPair>::STAGE;
+__host__ __device__ constexpr size_t slot_bytes(bool merge) {
+  return (size_t)Cfg<kPair>::KPS * (size_t)(A_STAGE + Cfg<kPair>::B_STAGE + (merge ? B_BOX : 0));
+}
+template <int kPair>
+__host__ __device__ constexpr size_t smem_bytes(int E, int stages, bool merge) {
+  return fixed_smem<kPair>(E) + (size_t)stages * slot_bytes<kPair>(merge);
 }
 // As many stages as fit (more bytes in flight hide more load latency).
 template <int kPair>
-inline int stages_for(int E) {
+inline int stages_for(int E, bool merge = false) {
   const size_t avail = kSmemBudget - fixed_smem<kPair>(E);
-  const int n = (int)(avail / Cfg<kPair>::STAGE);
+  const int n = (int)(avail / slot_bytes<kPair>(merge));
   return n < MAX_STAGES ? n : MAX_STAGES;
 }
 
@@ -214,10 +250,23 @@ struct Tile {
 };
 
 // Token blocks of an expert with c rows: ceil(c / 256) blocks of 256 rows,
-// the last one ragged.  (Splitting c evenly across the blocks was measured
-// slower: the kernel is bound by operand loads, and even blocks cost more
-// load requests than one ragged block.)
-__device__ __forceinline__ int token_blocks(int c) { return (c + BN - 1) / BN; }
+// the last one ragged; with `merge`, a last block of at most kMergeRows rows
+// joins the one before it.  (Splitting c evenly across the blocks was
+// measured slower: the kernel is bound by operand loads, and even blocks
+// cost more load requests than one ragged block.)
+__device__ __forceinline__ int token_blocks(int c, bool merge) {
+  int nb = (c + BN - 1) / BN;
+  if (merge && nb >= 2 && c - (nb - 1) * BN <= kMergeRows) --nb;
+  return nb;
+}
+
+// First TMEM column of a tile's accumulator: buffer 0 (even tiles) at 0,
+// buffer 1 at 256, or with merged blocks ending at column 512 (its width
+// rounded up to 32 columns, the epilogue's chunk), so that consecutive
+// tiles overlap only when their widths add up to more than 512.
+__device__ __forceinline__ int acc_base(int buf, int width, bool merge) {
+  return buf == 0 ? 0 : merge ? 2 * BN - ((width + 31) & ~31) : BN;
+}
 
 // fb_fastest = false: an expert's tiles go token block fastest (the CTAs
 // running at once share each weight block through L2); true: feature block
@@ -225,7 +274,8 @@ __device__ __forceinline__ int token_blocks(int c) { return (c + BN - 1) / BN; }
 // token block runs at about the same time, so the token rows are read from
 // DRAM once even when a long K leaves no room in L2 to keep them).
 __device__ __forceinline__ Tile decode(int tile, const int* s_start, const int* s_lo,
-                                       const int* s_hi, int E, bool fb_fastest, int n_fb) {
+                                       const int* s_hi, int E, bool fb_fastest, int n_fb,
+                                       bool merge) {
   int lo = 0, hi = E - 1;
   while (lo < hi) {  // last expert whose first tile is <= tile
     const int mid = (lo + hi + 1) >> 1;
@@ -235,7 +285,7 @@ __device__ __forceinline__ Tile decode(int tile, const int* s_start, const int* 
   t.e = lo;
   const int local = tile - s_start[lo];
   const int c = s_hi[lo] - s_lo[lo];
-  const int ntb = token_blocks(c);
+  const int ntb = token_blocks(c, merge);
   int tb;
   if (fb_fastest) {
     tb = local / n_fb;
@@ -245,7 +295,7 @@ __device__ __forceinline__ Tile decode(int tile, const int* s_start, const int* 
     tb = local - t.fb * ntb;
   }
   t.row0 = s_lo[lo] + tb * BN;
-  t.ntok = min(BN, c - tb * BN);
+  t.ntok = tb == ntb - 1 ? c - tb * BN : BN;  // up to BN_MAX when merged
   return t;
 }
 
@@ -281,7 +331,8 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
-template <bool kGelu, int kPair, bool kFp8, bool kGather, bool kFused>
+// kMerge: merged last token blocks (paired CTAs, plain forms only)
+template <bool kGelu, int kPair, bool kFp8, bool kGather, bool kFused, bool kMerge>
 __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x,
@@ -295,6 +346,9 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
   constexpr int KB = kFp8 ? BK_FP8 : BK;  // K values per stage (128 bytes of a row)
   const int STAGES = args.stages;
   constexpr int B_STAGE = C::B_STAGE;
+  static_assert(!kMerge || (kPair == 2 && !kGather && !kFused),
+                "merged blocks: paired CTAs, neither gathered nor fused");
+  constexpr bool merge = kMerge;
   // queue readers: the producers and epilogue warps of both CTAs and the
   // leader's MMA warp
   constexpr uint32_t kQReaders = kPair * Ro::NPROD + 1 + kPair * EPI_WARPS;
@@ -303,7 +357,8 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * KPS * A_STAGE;  // slot s, K-block h: sA + (s*KPS + h)*A_STAGE
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * KPS * B_STAGE);
+  uint8_t* sT = sB + STAGES * KPS * B_STAGE;  // merged tails: slot s, K-block h at (s*KPS + h)*B_BOX
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sT + (merge ? STAGES * KPS * B_BOX : 0));
   uint64_t* full = bars;                   // used in the leader CTA: both CTAs' bytes land here
   uint64_t* empty = bars + MAX_STAGES;     // per CTA: the MMAs have read this stage
   uint64_t* tfull = bars + 2 * MAX_STAGES; // per CTA: accumulator ready
@@ -312,6 +367,8 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
   uint64_t* qfull = drain + 1;         // per CTA: queue slot holds the next item
   uint64_t* qempty = qfull + kQueue;   // leader CTA: every reader has taken the slot
   uint64_t* qprod = qempty + kQueue;   // leader CTA: its weight producer has taken an item
+  uint64_t* tearly = qprod + 1;        // leader CTA: both CTAs' epilogues drained the columns
+                                       // the next tile may share (drained first)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
   volatile int* s_queue = reinterpret_cast<volatile int*>(s_tmem + 4);
@@ -335,6 +392,7 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kPair * EPI_WARPS);
+      mbar_init(&tearly[a], kPair * EPI_WARPS);
     }
     mbar_init(drain, 1);
     for (int q = 0; q < kQueue; ++q) {
@@ -375,7 +433,7 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     const int per = (E + 31) / 32;
     const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
     int sum = 0;
-    for (int e = e0; e < e1; ++e) sum += token_blocks(s_hi[e] - s_lo[e]) * args.n_fblocks;
+    for (int e = e0; e < e1; ++e) sum += token_blocks(s_hi[e] - s_lo[e], merge) * args.n_fblocks;
     int incl = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -385,14 +443,14 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     int run = incl - sum;
     for (int e = e0; e < e1; ++e) {
       s_start[e] = run;
-      run += token_blocks(s_hi[e] - s_lo[e]) * args.n_fblocks;
+      run += token_blocks(s_hi[e] - s_lo[e], merge) * args.n_fblocks;
     }
     if (lane == 31) s_start[E] = incl;
     if (kFused) {  // GEMM-2's tiles: same token blocks, n_fblocks2 feature blocks each
       run = (incl - sum) / args.n_fblocks * args.n_fblocks2;
       for (int e = e0; e < e1; ++e) {
         s_start2[e] = run;
-        run += token_blocks(s_hi[e] - s_lo[e]) * args.n_fblocks2;
+        run += token_blocks(s_hi[e] - s_lo[e], merge) * args.n_fblocks2;
       }
       if (lane == 31) s_start2[E] = incl / args.n_fblocks * args.n_fblocks2;
     }
@@ -430,10 +488,11 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     x -= n_disp;
     if (kFused && x >= tiles0) {
       phase = 1;
-      return decode(x - tiles0, s_start2, s_lo, s_hi, E, args.fb_fastest2, args.n_fblocks2);
+      return decode(x - tiles0, s_start2, s_lo, s_hi, E, args.fb_fastest2, args.n_fblocks2,
+                    merge);
     }
     phase = 0;
-    return decode(x, s_start, s_lo, s_hi, E, args.fb_fastest, args.n_fblocks);
+    return decode(x, s_start, s_lo, s_hi, E, args.fb_fastest, args.n_fblocks, merge);
   };
   // fused form: index of the token block holding a tile's rows
   auto block_of = [&](const Tile& t) -> int {
@@ -442,6 +501,7 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
   // the leader's barriers as cluster addresses (the CTA's own when kPair == 1)
   const uint32_t full_lead = kPair == 2 ? cluster_map(smem_u32(full), 0) : smem_u32(full);
   const uint32_t tempty_lead = kPair == 2 ? cluster_map(smem_u32(tempty), 0) : smem_u32(tempty);
+  const uint32_t tearly_lead = kPair == 2 ? cluster_map(smem_u32(tearly), 0) : smem_u32(tearly);
   const uint32_t qempty_lead = kPair == 2 ? cluster_map(smem_u32(qempty), 0) : smem_u32(qempty);
 
   // Static schedule: every role computes this cluster's i-th item itself.
@@ -584,15 +644,22 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
         }
       }
       const int nmma = (t.ntok + 15) & ~15;
-      const int half = nmma / kPair;  // token rows staged by this CTA (a multiple of 8)
+      // a merged tile's first 256 rows, then its tail (a second MMA)
+      const int nmain = (kMerge && nmma > BN) ? BN : nmma;
+      const int half = nmain / kPair;  // token rows staged by this CTA (a multiple of 8)
       const bool wide = half >= kWideMin;
       const int nbox = (half + B_BOX_ROWS - 1) / B_BOX_ROWS;
       // wide boxes of 128 rows: one with paired CTAs (half <= 128), up to two
       // with a single CTA (half <= 256); the stage holds BN / kPair rows
       const int nwide = (half + B_WIDE_ROWS - 1) / B_WIDE_ROWS;
+      // merged tile: this CTA's half of the tail (8..32 rows), one 32-row box
+      // in the tail ring (a merged tile's first half-tile is 128 rows: wide)
+      const int half2 = (nmma - nmain) / kPair;
+      const int nbox2 = (kMerge && half2 > 0) ? 1 : 0;
       const uint32_t bytes = is_w ? (uint32_t)(kPair * A_STAGE)
-                                  : (uint32_t)kPair * (wide ? nwide * B_WIDE_ROWS * BK * 2
-                                                            : nbox * B_BOX);
+                                  : (uint32_t)kPair * ((wide ? nwide * B_WIDE_ROWS * BK * 2
+                                                             : nbox * B_BOX) +
+                                                       nbox2 * B_BOX);
       const int wy = t.e * Np + t.fb * C::FEAT + (int)rank * BM;
       // weight prefetch: this CTA's 128 weight rows, 4 per lane
       const uint8_t* wrow = (p1 ? args.w2_ptr : args.w_ptr) +
@@ -700,6 +767,9 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
               for (int j = 0; j < nwide; ++j)
                 tma_load_2d_cg<kPair>(sB + (s * KPS + hh) * B_STAGE + j * B_WIDE_ROWS * 128,
                                       map_xw, kb * kbv, by + j * B_WIDE_ROWS, fb_addr, pol);
+              if (kMerge && nbox2)  // a merged tile's tail rows, into the tail ring
+                tma_load_2d_cg<kPair>(sT + (s * KPS + hh) * B_BOX, map_x, kb * kbv,
+                                      t.row0 + BN + (int)rank * half2, fb_addr, pol);
             } else {
               for (int j = 0; j < nbox; ++j)
                 tma_load_2d_cg<kPair>(sB + (s * KPS + hh) * B_STAGE + j * B_BOX, map_x, kb * kbv,
@@ -738,6 +808,7 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
       int s = 0;
       uint32_t ph = 0;
       int it = 0;  // GEMM tiles so far (selects the accumulator)
+      int prev_lo = 0, prev_hi = 0;  // TMEM columns of the previous tile's accumulator
       bool ok = true;
       for (int qi = 0; ok; ++qi) {
         int x;
@@ -750,33 +821,70 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
         const bool f8 = kFp8 && !p1;  // GEMM-2 of the fused form is bf16
         const int nkb = p1 ? args.num_kb2 : args.num_kb;
         const uint32_t nmma = (uint32_t)((t.ntok + 15) & ~15);
-        const uint32_t idesc = f8 ? idesc_e4m3_f32((uint32_t)C::FEAT, nmma)
-                                  : idesc_bf16_f32((uint32_t)C::FEAT, nmma);
+        // a merged tile (nmma > 256): N = 256, then N = the tail at column +256
+        const uint32_t n1 = (kMerge && nmma > (uint32_t)BN) ? (uint32_t)BN : nmma;
+        const uint32_t n2 = kMerge ? nmma - n1 : 0u;
+        const uint32_t idesc = f8 ? idesc_e4m3_f32((uint32_t)C::FEAT, n1)
+                                  : idesc_bf16_f32((uint32_t)C::FEAT, n1);
+        const uint32_t idesc2 = n2 == 0 ? 0u
+                                : f8 ? idesc_e4m3_f32((uint32_t)C::FEAT, n2)
+                                     : idesc_bf16_f32((uint32_t)C::FEAT, n2);
         const int acc = it & 1;
         const uint32_t aph = (uint32_t)((it >> 1) & 1);
+        const int base = acc_base(acc, (int)nmma, merge);
+        // the tile before this one used the other buffer: if their columns
+        // overlap, wait until its epilogue has drained the shared ones
+        const bool shares = kMerge && it > 0 && prev_lo < base + (int)nmma && base < prev_hi;
+        const uint32_t pph = (uint32_t)(((it - 1) >> 1) & 1);
+        prev_lo = base;
+        prev_hi = base + (int)nmma;
         ++it;
         ok = warp_wait(&tempty[acc], aph ^ 1u, args.status, s_abort);
+        if (ok && shares) ok = warp_wait(&tearly[acc ^ 1], pph, args.status, s_abort);
         if (!ok) break;
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)base;
         for (int ks = 0; ks * KPS < nkb; ++ks) {
           const int nsub = min(KPS, nkb - ks * KPS);
           ok = warp_wait(&full[s], ph, args.status, s_abort);
           if (!ok) break;
           tc_fence_after_sync();
           if (lane == 0) {
-            for (int hh = 0; hh < nsub; ++hh) {
-              const int kb = ks * KPS + hh;
-              const uint32_t a0 = smem_u32(sA + (s * KPS + hh) * A_STAGE);
-              const uint32_t b0 = smem_u32(sB + (s * KPS + hh) * B_STAGE);
+            if (!kMerge || n2 == 0) {
+              for (int hh = 0; hh < nsub; ++hh) {
+                const int kb = ks * KPS + hh;
+                const uint32_t a0 = smem_u32(sA + (s * KPS + hh) * A_STAGE);
+                const uint32_t b0 = smem_u32(sB + (s * KPS + hh) * B_STAGE);
 #pragma unroll
-              for (int kk = 0; kk < 128 / UMMA_K_BYTES; ++kk) {
-                const uint64_t ad = smem_desc_k128(a0 + kk * UMMA_K_BYTES);
-                const uint64_t bd = smem_desc_k128(b0 + kk * UMMA_K_BYTES);
-                if (f8)
-                  tc_mma_e4m3<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
-                else
-                  tc_mma_bf16<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                for (int kk = 0; kk < 128 / UMMA_K_BYTES; ++kk) {
+                  const uint64_t ad = smem_desc_k128(a0 + kk * UMMA_K_BYTES);
+                  const uint64_t bd = smem_desc_k128(b0 + kk * UMMA_K_BYTES);
+                  if (f8)
+                    tc_mma_e4m3<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                  else
+                    tc_mma_bf16<kPair>(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                }
+              }
+            } else {  // merged tile: N = 256, then the tail from the tail ring
+              for (int hh = 0; hh < nsub; ++hh) {
+                const int kb = ks * KPS + hh;
+                const uint32_t a0 = smem_u32(sA + (s * KPS + hh) * A_STAGE);
+                const uint32_t b0 = smem_u32(sB + (s * KPS + hh) * B_STAGE);
+                const uint32_t t0 = smem_u32(sT + (s * KPS + hh) * B_BOX);
+#pragma unroll
+                for (int kk = 0; kk < 128 / UMMA_K_BYTES; ++kk) {
+                  const uint64_t ad = smem_desc_k128(a0 + kk * UMMA_K_BYTES);
+                  const uint64_t bd = smem_desc_k128(b0 + kk * UMMA_K_BYTES);
+                  const uint64_t td = smem_desc_k128(t0 + kk * UMMA_K_BYTES);
+                  const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+                  if (f8) {
+                    tc_mma_e4m3<kPair>(d_tmem, ad, bd, idesc, accum);
+                    tc_mma_e4m3<kPair>(d_tmem + (uint32_t)BN, ad, td, idesc2, accum);
+                  } else {
+                    tc_mma_bf16<kPair>(d_tmem, ad, bd, idesc, accum);
+                    tc_mma_bf16<kPair>(d_tmem + (uint32_t)BN, ad, td, idesc2, accum);
+                  }
+                }
               }
             }
             // the stage is free (in both CTAs) once these MMAs have read it
@@ -806,8 +914,9 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;              // TMEM lane quarter this warp may access
-    // which span of the tile's 256 token columns (EPI_WARPS / 4 spans)
-    constexpr int SPAN = BN / (EPI_WARPS / 4);
+    // the tile's 32-column chunks are dealt out round robin over NSPAN warps
+    // per lane quarter: this warp takes chunks hsel, hsel + NSPAN, ...
+    constexpr int NSPAN = EPI_WARPS / 4;
     const int hsel = (warp - Ro::EPI0) >> 2;
     int it = 0;  // GEMM tiles so far
     for (int qi = 0;; ++qi) {
@@ -859,15 +968,24 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       ++it;
+      const int nmma = (t.ntok + 15) & ~15;
+      const int base = acc_base(acc, nmma, merge);
+      // Columns of this accumulator (relative to base) that the next tile may
+      // reuse, drained first: a low tile's from column 192 on (a high tile
+      // starts there at the earliest), a high tile's below column 320 (where
+      // a low tile ends at the latest).  None without merged blocks.
+      const int ov0 = acc == 0 ? kHighMin : 0;
+      const int ov1 = !merge ? 0 : acc == 0 ? nmma : BN_MAX - base;
       if (!warp_wait(&tfull[acc], aph, args.status, s_abort)) break;
       tc_fence_after_sync();
       // this lane's output feature; the warp covers 32 consecutive features
       const int f0 = t.fb * C::FEAT + (int)rank * BM + q * 32;
       const int f = f0 + lane;
       const float sc = f8 ? __ldg(args.a_scale) * __ldg(args.w_scale + t.e) : 1.0f;
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      const int c_end = min(t.ntok, hsel * SPAN + SPAN);
-      for (int c0 = hsel * SPAN; c0 < c_end; c0 += 32) {
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)base;
+      const int nch = (t.ntok + 31) >> 5;
+      // one 32-column chunk of the accumulator: tokens c0 .. c0 + 31
+      auto drain_chunk = [&](const int c0) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + (uint32_t)c0, v);
         tmem_wait_ld();
@@ -886,12 +1004,12 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
               if (j < jmax) col[(size_t)j * N] = to_bf16_bits(x);
             }
           }
-          continue;
+          return;
         }
         // ---- combine: lane j describes token column j of this chunk.  A warp
         // whose 32 features all lie past N (last feature block) has nothing
         // to write, and its counter index would name the next token's word.
-        if (f0 >= N) continue;
+        if (f0 >= N) return;
         int tok = 0, mode = 0;  // mode 1: the token's only kept slot; 2: one of two
         float g = 0.f;
         if (lane < jmax) {
@@ -930,7 +1048,7 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
         if (second) {  // the partner slot's flag, then its partial
           bool got = true;
           if ((second >> lane) & 1u) got = wait_bits_set(cw, 0x100u, args.status, s_abort);
-          if (!__all_sync(0xffffffffu, got)) continue;
+          if (!__all_sync(0xffffffffu, got)) return;
           __threadfence();
           // the partners' partial rows, 8 loads in flight at a time
 #pragma unroll
@@ -953,6 +1071,21 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
             }
           }
         }
+      };
+      if constexpr (!kMerge) {  // each warp a contiguous span of the tile's columns
+        constexpr int SPAN = BN / NSPAN;
+        const int c_end = min(t.ntok, hsel * SPAN + SPAN);
+        for (int c0 = hsel * SPAN; c0 < c_end; c0 += 32) drain_chunk(c0);
+      } else {
+        // chunks dealt out round robin; first those the next tile may reuse,
+        // then a tearly arrival, then the others
+        for (int ch = hsel; ch < nch; ch += NSPAN)
+          if (ch * 32 + 32 > ov0 && ch * 32 < ov1) drain_chunk(ch * 32);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tearly_lead + (uint32_t)acc * 8u);
+        for (int ch = hsel; ch < nch; ch += NSPAN)
+          if (!(ch * 32 + 32 > ov0 && ch * 32 < ov1)) drain_chunk(ch * 32);
       }
       if (kFused && !p1) {  // publish this warp's part of H for GEMM-2's tiles
         __threadfence();
@@ -1028,16 +1161,17 @@ struct KernelSlot {
   cudaError_t err = cudaSuccess;
   int max_clusters = 0;  // co-resident clusters (pairs) or CTAs of this kernel
 };
-static KernelSlot g_slots[64][32];
+static KernelSlot g_slots[64][64];
 
-template <bool kGelu, int kPair, bool kFp8, bool kGather, bool kFused = false>
+template <bool kGelu, int kPair, bool kFp8, bool kGather, bool kFused = false, bool kMerge = false>
 static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm_x,
                                   const CUtensorMap& tm_xw, const gg::Args& args, long long max_tiles, const DeviceInfo& dev,
                                   cudaStream_t stream, const CUtensorMap* tm2 = nullptr) {
-  auto kern = gg::grouped_gemm_kernel<kGelu, kPair, kFp8, kGather, kFused>;
+  auto kern = gg::grouped_gemm_kernel<kGelu, kPair, kFp8, kGather, kFused, kMerge>;
   const size_t smem_max = gg::kSmemBudget;  // one attribute for every E
   const int slot =
-      (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0) + (kFp8 ? 4 : 0) + (kGather ? 8 : 0) + (kFused ? 16 : 0);
+      (kGelu ? 1 : 0) + (kPair == 2 ? 2 : 0) + (kFp8 ? 4 : 0) + (kGather ? 8 : 0) + (kFused ? 16 : 0) +
+      (kMerge ? 32 : 0);
   KernelSlot& ks = g_slots[dev.device & 63][slot];
   std::call_once(ks.once, [&] {
     ks.err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_max);
@@ -1072,7 +1206,7 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3((unsigned)(units * kPair), 1, 1);
   cfg.blockDim = dim3(gg::Roles<kGather, kPair>::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = gg::smem_bytes<kPair>(args.E, args.stages);
+  cfg.dynamicSmemBytes = gg::smem_bytes<kPair>(args.E, args.stages, kMerge);
   cfg.stream = stream;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -1143,6 +1277,21 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
   const int kb = kFp8 ? gg::BK_FP8 : gg::BK;
   args.num_kb = (K + kb - 1) / kb;
   args.stages = pair == 2 ? gg::stages_for<2>(E) : gg::stages_for<1>(E);
+#ifndef MOE_MERGE_TAILS
+#define MOE_MERGE_TAILS 1
+#endif
+  // Merged last token blocks (paired CTAs, tokens by rows, few rows per
+  // expert): each slot also holds 4 KB tail boxes, which costs no ring slot
+  // as long as as many slots still fit (E up to ~600).
+  bool merge = false;
+  if (MOE_MERGE_TAILS && pair == 2 && !gather && (long long)R > (long long)gg::kMergeMinMeanRows * E &&
+      (long long)R <= (long long)gg::kMergeMaxMeanRows * E) {
+    const int st = gg::stages_for<2>(E, true);
+    if (st >= args.stages) {
+      merge = true;
+      args.stages = st;
+    }
+  }
   apply_extras(args, ex);
   if (gelu) args.comb_Y = nullptr;  // the combine belongs to the GEMM without activation
 #ifndef MOE_GEMM2_FB_FASTEST
@@ -1158,6 +1307,11 @@ static cudaError_t launch_gemm(const void* A, const float* a_scale, const int32_
       ((long long)(R + gg::BN - 1) / gg::BN + E) * (long long)args.n_fblocks;
 #define MOE_GG_LAUNCH(G, P, GA) \
   launch_variant<G, P, kFp8, GA>(tm_w, tm_x, tm_xw, args, max_tiles, dev, stream)
+  if (merge)
+    return gelu ? launch_variant<true, 2, kFp8, false, false, true>(tm_w, tm_x, tm_xw, args,
+                                                                     max_tiles, dev, stream)
+                : launch_variant<false, 2, kFp8, false, false, true>(tm_w, tm_x, tm_xw, args,
+                                                                      max_tiles, dev, stream);
   if (gather) {
     if (pair == 2) return gelu ? MOE_GG_LAUNCH(true, 2, true) : MOE_GG_LAUNCH(false, 2, true);
     return gelu ? MOE_GG_LAUNCH(true, 1, true) : MOE_GG_LAUNCH(false, 1, true);

@@ -166,6 +166,7 @@ FP8_GEMM_CASES = [
     ([1030, 990, 1024], 256, 320, True),
     ([300, 129, 97], 128, 256, True),                  # one CTA per tile, > 128 rows per tile
     ([320, 321, 272, 576], 256, 256, True),            # short last token blocks (64, 65, 16 rows)
+    ([300, 256, 320, 200, 576, 17] * 16, 768, 256, True),  # merged blocks, several tiles per cluster
 ]
 
 

@@ -369,6 +369,12 @@ GEMM_CASES = [
     ([300, 0, 129, 256, 97, 128], 128, 64, True),
     ([700], 64, 200, False),
     ([1000, 3], 96, 136, True),
+    # merged last blocks (a tail of at most 64 rows joins the block before it:
+    # tiles of 257..320 rows) mixed with ordinary ones, enough tiles that each
+    # cluster runs several in a row: the accumulator placement alternates and
+    # a wide tile shares TMEM columns with its neighbour
+    ([300, 256, 320, 200, 576, 17, 64, 288] * 12, 1024, 128, True),
+    ([290, 260, 321, 512, 33] * 24, 512, 192, False),
 ]
 
 

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <cstdlib>
 #include <mutex>
 #include <string>
 
@@ -57,6 +58,14 @@ cudaError_t g_dev_err[kMaxDevices];
 int set_last_error(int status, const std::string& msg) {
   g_last_error = msg;
   return status;
+}
+
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* v = std::getenv("MOE_PDL");
+    return !(v && v[0] == '0');
+  }();
+  return on;
 }
 
 const DeviceInfo* current_device_info(std::string* err) {

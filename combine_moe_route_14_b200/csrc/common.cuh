@@ -22,6 +22,22 @@ __device__ __forceinline__ void flag_error(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+// Programmatic dependent launch.  pdl_wait: wait until the stream
+// predecessor grid has completed and its memory operations are visible (a
+// no-op for a kernel launched without the attribute); every thread calls it
+// before its first global access.  pdl_release: this CTA lets the grid's
+// dependents be scheduled (once every CTA has released or exited).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Short kernels release at once: their dependents' blocks then take the SMs
+// their own blocks leave and start their set-up.
+__device__ __forceinline__ void pdl_wait_and_release() {
+  pdl_wait();
+  pdl_release();
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -21,6 +21,7 @@ constexpr int kCopyUnroll = 8;   // 16-byte vectors in flight per lane
 __global__ void __launch_bounds__(kGatherWarps * 32)
     dispatch_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ src_of, int R,
                     int k, int row_vecs, uint4* __restrict__ Xe, uint32_t* status) {
+  pdl_wait_and_release();
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * kGatherWarps;
   for (int r = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); r < R; r += nwarps) {
@@ -56,6 +57,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
 __global__ void __launch_bounds__(kGatherWarps * 32)
     dispatch_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ row_of, int T,
                          int k, int R, int row_vecs, uint4* __restrict__ Xe, uint32_t* status) {
+  pdl_wait_and_release();
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * kGatherWarps;
   for (int t = blockIdx.x * kGatherWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
@@ -100,6 +102,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
                             int32_t* __restrict__ row_of, const int32_t* __restrict__ offsets,
                             int T, int k, int R, int E, int row_vecs, uint4* __restrict__ Xe,
                             int32_t* __restrict__ src_of, uint32_t* status) {
+  pdl_wait_and_release();
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * kGatherWarps;
   const int kept = min(max(__ldg(offsets + E), 0), R);
@@ -151,6 +154,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32)
     combine_kernel(const uint4* __restrict__ Ye, const int32_t* __restrict__ row_of,
                    const float* __restrict__ gates, int T, int R, int k_rt, int row_vecs,
                    uint4* __restrict__ Y, uint32_t* status) {
+  pdl_wait_and_release();
   constexpr int kSlots = kK > 0 ? kK : kMaxTopK;
   constexpr int kUnroll = kK > 0 ? (kK >= 4 ? 2 : 4) : 1;
   const int k = kK > 0 ? kK : k_rt;
@@ -232,17 +236,18 @@ cudaError_t launch_dispatch(const void* X, const int32_t* src_of, int T, int d, 
                             const DeviceInfo& dev, cudaStream_t stream) {
   const int R = T * k;
   if (R == 0) return cudaSuccess;
-  dispatch_kernel<<<gather_grid(R, dev), kGatherWarps * 32, 0, stream>>>(
-      static_cast<const uint4*>(X), src_of, R, k, d / 8, static_cast<uint4*>(Xe), dev.status);
+  launch_kernel(dispatch_kernel, dim3(gather_grid(R, dev)), dim3(kGatherWarps * 32), 0, stream,
+                static_cast<const uint4*>(X), src_of, R, k, d / 8, static_cast<uint4*>(Xe),
+                dev.status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dispatch_rows(const void* X, const int32_t* row_of, int T, int d, int k,
                                  void* Xe, const DeviceInfo& dev, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  dispatch_rows_kernel<<<gather_grid(T, dev), kGatherWarps * 32, 0, stream>>>(
-      static_cast<const uint4*>(X), row_of, T, k, T * k, d / 8, static_cast<uint4*>(Xe),
-      dev.status);
+  launch_kernel(dispatch_rows_kernel, dim3(gather_grid(T, dev)), dim3(kGatherWarps * 32), 0,
+                stream, static_cast<const uint4*>(X), row_of, T, k, T * k, d / 8,
+                static_cast<uint4*>(Xe), dev.status);
   return cudaGetLastError();
 }
 
@@ -250,9 +255,9 @@ cudaError_t launch_dispatch_scatter(const void* X, const int32_t* idx, int32_t* 
                                     const int32_t* offsets, int T, int d, int k, int E, void* Xe,
                                     int32_t* src_of, const DeviceInfo& dev, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  dispatch_scatter_kernel<<<gather_grid(T, dev), kGatherWarps * 32, 0, stream>>>(
-      static_cast<const uint4*>(X), idx, row_of, offsets, T, k, T * k, E, d / 8,
-      static_cast<uint4*>(Xe), src_of, dev.status);
+  launch_kernel(dispatch_scatter_kernel, dim3(gather_grid(T, dev)), dim3(kGatherWarps * 32), 0,
+                stream, static_cast<const uint4*>(X), idx, row_of, offsets, T, k, T * k, E,
+                d / 8, static_cast<uint4*>(Xe), src_of, dev.status);
   return cudaGetLastError();
 }
 
@@ -265,19 +270,24 @@ cudaError_t launch_combine(const void* Ye, const int32_t* row_of, const float* g
   const int R = T * k;
   switch (k) {
     case 1:
-      combine_kernel<1><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      launch_kernel(combine_kernel<1>, dim3(grid), dim3(kGatherWarps * 32), 0, stream, ye,
+                    row_of, gates, T, R, k, d / 8, y, dev.status);
       break;
     case 2:
-      combine_kernel<2><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      launch_kernel(combine_kernel<2>, dim3(grid), dim3(kGatherWarps * 32), 0, stream, ye,
+                    row_of, gates, T, R, k, d / 8, y, dev.status);
       break;
     case 4:
-      combine_kernel<4><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      launch_kernel(combine_kernel<4>, dim3(grid), dim3(kGatherWarps * 32), 0, stream, ye,
+                    row_of, gates, T, R, k, d / 8, y, dev.status);
       break;
     case 8:
-      combine_kernel<8><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      launch_kernel(combine_kernel<8>, dim3(grid), dim3(kGatherWarps * 32), 0, stream, ye,
+                    row_of, gates, T, R, k, d / 8, y, dev.status);
       break;
     default:
-      combine_kernel<0><<<grid, kGatherWarps * 32, 0, stream>>>(ye, row_of, gates, T, R, k, d / 8, y, dev.status);
+      launch_kernel(combine_kernel<0>, dim3(grid), dim3(kGatherWarps * 32), 0, stream, ye,
+                    row_of, gates, T, R, k, d / 8, y, dev.status);
   }
   return cudaGetLastError();
 }

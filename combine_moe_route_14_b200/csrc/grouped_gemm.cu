@@ -417,6 +417,11 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
     tmem_alloc<kPair>(s_tmem, TMEM_COLS);
     tmem_relinquish<kPair>();
   }
+  // The set-up above touches no global memory; from here on the kernel reads
+  // its stream predecessors' results.  The GEMM releases its dependents only
+  // at its end: their blocks would otherwise wait beside its warps for the
+  // whole launch (measured on the fine-grained shape: +3 % per layer).
+  pdl_wait();
   // Expert row ranges, clamped into [0, R) so that malformed offsets can
   // only produce wrong numbers, never out-of-range stores.
   bool bad_offsets = false;
@@ -1100,6 +1105,7 @@ __global__ void __launch_bounds__(Roles<kGather, kPair>::THREADS, 1)
 
   tc_fence_before_sync();
   __syncthreads();
+  pdl_release();
   if (kPair == 2) cluster_sync();  // no CTA leaves while its peer may still signal it
   if (warp == Ro::MMA) {
     tc_fence_after_sync();
@@ -1199,17 +1205,19 @@ static cudaError_t launch_variant(const CUtensorMap& tm_w, const CUtensorMap& tm
   if (ks.max_clusters < 1) return cudaErrorInvalidConfiguration;
   const long long units = max_tiles < ks.max_clusters ? max_tiles : ks.max_clusters;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kPair;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.gridDim = dim3((unsigned)(units * kPair), 1, 1);
   cfg.blockDim = dim3(gg::Roles<kGather, kPair>::THREADS, 1, 1);
   cfg.dynamicSmemBytes = gg::smem_bytes<kPair>(args.E, args.stages, kMerge);
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   // the fused form's GEMM-2 maps; the other forms pass copies they never read
   const CUtensorMap& w2 = tm2 ? tm2[0] : tm_w;
   const CUtensorMap& x2 = tm2 ? tm2[1] : tm_x;

@@ -6,8 +6,37 @@
 #include <stdint.h>
 
 #include <string>
+#include <utility>
 
 namespace moe {
+
+// Programmatic dependent launch.  Every kernel of the library starts with
+// griddepcontrol.wait (it reads nothing a stream predecessor writes, and
+// writes nothing it reads, before that point) and then lets its own
+// dependents launch.  Launched with the stream-serialisation attribute, a
+// kernel's blocks are therefore scheduled while its predecessor's last
+// blocks run, and its launch latency and set-up overlap them; the wait keeps
+// the stream order of every memory access.  MOE_PDL=0 in the environment
+// launches without the attribute (plain stream order).
+bool pdl_enabled();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  if (pdl_enabled()) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Limits checked by the ABI before any launch.
 constexpr int kMaxExperts = 1024;

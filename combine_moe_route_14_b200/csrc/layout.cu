@@ -219,6 +219,7 @@ __device__ void scan_over_warps(int* hist, int E, int* agg) {
 __global__ void __launch_bounds__(kLayoutThreads)
     layout_single_kernel(const int32_t* __restrict__ idx, int R, int E, int32_t* counts,
                          int32_t* offsets, int32_t* row_of, int32_t* src_of, uint32_t* status) {
+  pdl_wait_and_release();
   extern __shared__ int smem_i[];
   int* keys = smem_i;
   int* hist = keys + R;
@@ -254,6 +255,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
 __global__ void __launch_bounds__(kLayoutThreads)
     layout_hist_kernel(const int32_t* __restrict__ idx, int R, int E, int32_t* counts,
                        uint32_t* lookback, uint32_t* ticket, uint32_t* status) {
+  pdl_wait_and_release();
   extern __shared__ int smem_i[];
   int* hist = smem_i;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -283,6 +285,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
                           const int32_t* __restrict__ counts, int32_t* offsets, int32_t* row_of,
                           int32_t* src_of, uint32_t* lookback, uint32_t* ticket,
                           uint32_t* status) {
+  pdl_wait_and_release();
   extern __shared__ int smem_i[];
   int* keys = smem_i;
   int* hist = keys + kTile;
@@ -388,8 +391,8 @@ cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (err != cudaSuccess) return err;
     }
-    layout_single_kernel<<<1, kLayoutThreads, smem, stream>>>(idx, R, E, counts, offsets, row_of,
-                                                              src_of, dev.status);
+    launch_kernel(layout_single_kernel, dim3(1), dim3(kLayoutThreads), smem, stream, idx, R, E,
+                  counts, offsets, row_of, src_of, dev.status);
     return cudaGetLastError();
   }
   uint32_t* ticket = static_cast<uint32_t*>(ws);
@@ -397,8 +400,8 @@ cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int
   const int tiles = num_tiles(R);
   cudaError_t err = cudaMemsetAsync(counts, 0, (size_t)E * sizeof(int32_t), stream);
   if (err != cudaSuccess) return err;
-  layout_hist_kernel<<<tiles, kLayoutThreads, (size_t)E * sizeof(int), stream>>>(
-      idx, R, E, counts, lookback, ticket, dev.status);
+  launch_kernel(layout_hist_kernel, dim3(tiles), dim3(kLayoutThreads), (size_t)E * sizeof(int),
+                stream, idx, R, E, counts, lookback, ticket, dev.status);
   err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const size_t smem = (size_t)(kTile + kLayoutWarps * E + E + E + 1 + 33 + 1) * sizeof(int);
@@ -407,7 +410,7 @@ cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int
                                (int)smem);
     if (err != cudaSuccess) return err;
   }
-  layout_scatter_kernel<<<tiles, kLayoutThreads, smem, stream>>>(
+  launch_kernel(layout_scatter_kernel, dim3(tiles), dim3(kLayoutThreads), smem, stream,
       idx, R, E, counts, offsets, row_of, src_of, lookback, ticket, dev.status);
   return cudaGetLastError();
 }

@@ -50,6 +50,7 @@ __device__ __forceinline__ uint2 quant8(uint4 v, float inv) {
 // the launcher zeroes) with an integer atomicMax on its fp32 bits.
 __global__ void __launch_bounds__(kQThreads)
     amax_kernel(const uint4* __restrict__ X, size_t vecs, uint32_t* amax_bits) {
+  pdl_wait_and_release();
   const uint4* p = X + (size_t)blockIdx.y * vecs;
   uint32_t m2 = 0;  // two 16-bit magnitudes
   const size_t stride = (size_t)gridDim.x * kQThreads;
@@ -92,6 +93,7 @@ __global__ void __launch_bounds__(kQThreads)
 __global__ void __launch_bounds__(kQThreads)
     quantize_kernel(const uint4* __restrict__ W, size_t vecs, const float* __restrict__ amax,
                     uint2* __restrict__ Wq, float* scale_out) {
+  pdl_wait_and_release();
   const float inv = inv_scale_of(amax[blockIdx.y]);
   if (scale_out && blockIdx.x == 0 && threadIdx.x == 0)
     scale_out[blockIdx.y] = scale_of(amax[blockIdx.y]);
@@ -111,6 +113,7 @@ __global__ void __launch_bounds__(kQThreads)
 
 // amax -> dequantisation scale, in place.
 __global__ void scale_finalize_kernel(float* s, int n) {
+  pdl_wait_and_release();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) s[i] = scale_of(s[i]);
 }
@@ -125,6 +128,7 @@ __global__ void __launch_bounds__(kDispWarps * 32)
     dispatch_fp8_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ src_of, int R,
                         int k, int row_vecs, float* x_scale, uint2* __restrict__ Xeq,
                         uint32_t* status) {
+  pdl_wait_and_release();
   const float amax = x_scale[1];
   const float inv = inv_scale_of(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) x_scale[0] = scale_of(amax);
@@ -160,6 +164,7 @@ __global__ void __launch_bounds__(kDispWarps * 32)
     dispatch_fp8_rows_kernel(const uint4* __restrict__ X, const int32_t* __restrict__ row_of,
                              int T, int k, int row_vecs, float* x_scale, uint2* __restrict__ Xeq,
                              uint32_t* status) {
+  pdl_wait_and_release();
   const float amax = x_scale[1];
   const float inv = inv_scale_of(amax);
   if (blockIdx.x == 0 && threadIdx.x == 0) x_scale[0] = scale_of(amax);
@@ -210,7 +215,7 @@ static cudaError_t launch_amax(const void* X, size_t vecs, int groups, float* am
   cudaError_t e = cudaMemsetAsync(amax, 0, (size_t)groups * sizeof(float), stream);
   if (e != cudaSuccess) return e;
   if (vecs == 0) return cudaSuccess;
-  amax_kernel<<<dim3(stream_grid(vecs, groups, dev), groups), kQThreads, 0, stream>>>(
+  launch_kernel(amax_kernel, dim3(stream_grid(vecs, groups, dev), groups), dim3(kQThreads), 0, stream,
       static_cast<const uint4*>(X), vecs, reinterpret_cast<uint32_t*>(amax));
   return cudaGetLastError();
 }
@@ -221,11 +226,12 @@ cudaError_t launch_quantize_experts(const void* W, int E, int64_t per_expert, vo
   cudaError_t e = launch_amax(W, vecs, E, scales, dev, stream);
   if (e != cudaSuccess) return e;
   if (vecs > 0) {
-    quantize_kernel<<<dim3(stream_grid(vecs, E, dev), E), kQThreads, 0, stream>>>(
-        static_cast<const uint4*>(W), vecs, scales, static_cast<uint2*>(Wq), nullptr);
+    launch_kernel(quantize_kernel, dim3(stream_grid(vecs, E, dev), E), dim3(kQThreads), 0, stream,
+      static_cast<const uint4*>(W), vecs, scales, static_cast<uint2*>(Wq), nullptr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  scale_finalize_kernel<<<(E + 255) / 256, 256, 0, stream>>>(scales, E);
+  launch_kernel(scale_finalize_kernel, dim3((E + 255) / 256), dim3(256), 0, stream,
+      scales, E);
   return cudaGetLastError();
 }
 
@@ -235,7 +241,7 @@ cudaError_t launch_quantize_tensor(const void* X, int64_t n, void* Xq, float* x_
   cudaError_t e = launch_amax(X, vecs, 1, x_scale + 1, dev, stream);
   if (e != cudaSuccess) return e;
   // n == 0 still runs one CTA so that x_scale[0] is written
-  quantize_kernel<<<stream_grid(vecs, 1, dev), kQThreads, 0, stream>>>(
+  launch_kernel(quantize_kernel, dim3(stream_grid(vecs, 1, dev)), dim3(kQThreads), 0, stream,
       static_cast<const uint4*>(X), vecs, x_scale + 1, static_cast<uint2*>(Xq), x_scale);
   return cudaGetLastError();
 }
@@ -250,7 +256,7 @@ cudaError_t launch_dispatch_fp8(const void* X, const int32_t* src_of, int T, int
   const int cap = dev.sm_count * 8;
   const int grid = need < 1 ? 1 : (need < cap ? need : cap);
   // R == 0 still runs one CTA so that x_scale[0] is written
-  dispatch_fp8_kernel<<<grid, kDispWarps * 32, 0, stream>>>(
+  launch_kernel(dispatch_fp8_kernel, dim3(grid), dim3(kDispWarps * 32), 0, stream,
       static_cast<const uint4*>(X), src_of, R, k, d / 8, x_scale, static_cast<uint2*>(Xeq),
       dev.status);
   return cudaGetLastError();
@@ -265,7 +271,7 @@ cudaError_t launch_dispatch_fp8_rows(const void* X, const int32_t* row_of, int T
   const int cap = dev.sm_count * 8;
   const int grid = need < 1 ? 1 : (need < cap ? need : cap);
   // T == 0 still runs one CTA so that x_scale[0] is written
-  dispatch_fp8_rows_kernel<<<grid, kDispWarps * 32, 0, stream>>>(
+  launch_kernel(dispatch_fp8_rows_kernel, dim3(grid), dim3(kDispWarps * 32), 0, stream,
       static_cast<const uint4*>(X), row_of, T, k, d / 8, x_scale, static_cast<uint2*>(Xeq),
       dev.status);
   return cudaGetLastError();

@@ -104,6 +104,7 @@ template <int kG, bool kWs>
 __global__ void __launch_bounds__(kRouterThreads, kG == 1 ? 2 : 1)
     router_logits_kernel(const uint8_t* __restrict__ X, const uint4* __restrict__ Wr, int T,
                          int d, int E, float* __restrict__ L, uint32_t* status) {
+  pdl_wait_and_release();
   static_assert(!kWs || kG == 1, "Wr is staged for one n-tile only");
   extern __shared__ __align__(128) uint8_t smem_r[];
   uint8_t* ring = smem_r;
@@ -308,14 +309,14 @@ cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, in
   const uint8_t* x = static_cast<const uint8_t*>(X);
   const uint4* w = static_cast<const uint4*>(Wr);
   if (ws)
-    router_logits_kernel<1, true><<<blocks, kRouterThreads, smem, stream>>>(x, w, T, d, E, L,
-                                                                            dev.status);
+    launch_kernel(router_logits_kernel<1, true>, dim3(blocks), dim3(kRouterThreads), smem, stream,
+                  x, w, T, d, E, L, dev.status);
   else if (gmax == 1)
-    router_logits_kernel<1, false><<<blocks, kRouterThreads, smem, stream>>>(x, w, T, d, E, L,
-                                                                             dev.status);
+    launch_kernel(router_logits_kernel<1, false>, dim3(blocks), dim3(kRouterThreads), smem,
+                  stream, x, w, T, d, E, L, dev.status);
   else
-    router_logits_kernel<kRouterGroup, false><<<blocks, kRouterThreads, smem, stream>>>(
-        x, w, T, d, E, L, dev.status);
+    launch_kernel(router_logits_kernel<kRouterGroup, false>, dim3(blocks), dim3(kRouterThreads),
+                  smem, stream, x, w, T, d, E, L, dev.status);
   return cudaGetLastError();
 }
 
@@ -437,6 +438,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
                       float inv_temp, float min_prob, int32_t* __restrict__ idx,
                       float* __restrict__ gates, uint4* __restrict__ zero_rows, int zero_vecs,
                       uint32_t* __restrict__ zero_words, int n_zero_words) {
+  pdl_wait_and_release();
   // side job: clear the caller's counter words (grid-stride; the layer's
   // later kernels run after this one on the same stream)
   if (zero_words) {
@@ -492,6 +494,7 @@ __global__ void __launch_bounds__(rank_warps(kEPL) * 32)
                       uint32_t* __restrict__ lookback, uint4* __restrict__ zero_rows,
                       int zero_vecs, uint32_t* __restrict__ zero_words, int n_zero_words,
                       uint32_t* status) {
+  pdl_wait_and_release();
   constexpr int kRankWarps = rank_warps(kEPL);
   constexpr int kRankTile = kRankWarps;  // one token per warp
   // shared: keys[kRankTile * k] | run[E] | tile id
@@ -633,10 +636,9 @@ cudaError_t launch_route(const float* L, int T, int E, int k, int score, int ren
   const int epl = (E + 31) / 32;
   const float inv_temp = 1.0f / temperature;
 #define MOE_ROUTE_LAUNCH(N)                                                                    \
-  route_topk_kernel<N><<<blocks, kRouteWarps * 32, 0, stream>>>(L, T, E, k, score, renormalize, \
-                                                                inv_temp, min_prob, idx, gates, \
-                                                                static_cast<uint4*>(zero_rows), \
-                                                                zero_d / 8, zero_words, n_zero_words)
+  launch_kernel(route_topk_kernel<N>, dim3(blocks), dim3(kRouteWarps * 32), 0, stream, L, T, E,  \
+                k, score, renormalize, inv_temp, min_prob, idx, gates,                           \
+                static_cast<uint4*>(zero_rows), zero_d / 8, zero_words, n_zero_words)
   if (epl <= 1) MOE_ROUTE_LAUNCH(1);
   else if (epl <= 2) MOE_ROUTE_LAUNCH(2);
   else if (epl <= 4) MOE_ROUTE_LAUNCH(4);
@@ -658,10 +660,10 @@ cudaError_t launch_route_rank(const float* L, int T, int E, int k, int score, in
   const float inv_temp = 1.0f / temperature;
   const size_t smem = (size_t)(rank_tile(E) * k + E + 1) * sizeof(int);
 #define MOE_RANK_LAUNCH(N)                                                                     \
-  route_rank_kernel<N><<<blocks, rank_warps(N) * 32, smem, stream>>>(                          \
-      L, T, E, k, score, renormalize, inv_temp, min_prob, idx, gates, rank, counts, offsets,     \
-      lookback, static_cast<uint4*>(zero_rows), zero_d / 8, zero_words, n_zero_words,            \
-      dev.status)
+  launch_kernel(route_rank_kernel<N>, dim3(blocks), dim3(rank_warps(N) * 32), smem, stream, L, T, \
+                E, k, score, renormalize, inv_temp, min_prob, idx, gates, rank, counts, offsets, \
+                lookback, static_cast<uint4*>(zero_rows), zero_d / 8, zero_words, n_zero_words,  \
+                dev.status)
   if (epl <= 1) MOE_RANK_LAUNCH(1);
   else if (epl <= 2) MOE_RANK_LAUNCH(2);
   else if (epl <= 4) MOE_RANK_LAUNCH(4);

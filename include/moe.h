@@ -38,6 +38,13 @@
  *     T*k < 2^30.  T == 0 is a valid no-op.
  *   - Threads may call the library concurrently; calls on streams that run at
  *     the same time must not share output buffers or workspaces.
+ *   - Kernels are launched as programmatic dependents of their stream
+ *     predecessor (cudaLaunchAttributeProgrammaticStreamSerialization): a
+ *     kernel's blocks may be scheduled before the previous kernel on the
+ *     stream has finished, and wait (griddepcontrol.wait) before their first
+ *     global memory access, so stream order holds for every access.  The
+ *     environment variable MOE_PDL=0, read once per process, launches them
+ *     without the attribute.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

@@ -121,3 +121,39 @@ def test_layer_fused_ffn_is_bitwise_the_default_layer(name, fp8):
         ref = O.layer_forward(bits(inp["X"]), bits(inp["W1"]), bits(inp["W2"]), cfg.k, cfg.score,
                               cfg.renormalize, logits=inp["logits"].numpy())
         np.testing.assert_array_less(np.abs(f64(outs[1]) - ref["Y"]).max(), O.tolerance(ref["Y"]))
+
+
+@pytest.mark.parametrize("form", ["fused", "pipeline"])
+def test_fused_forms_share_the_gpu_with_another_stream(form):
+    """Tiles come from an atomic ticket in dependency order, so a tile only
+    waits on tiles that running clusters hold: the persistent kernel finishes
+    with the right bytes, and no wait runs out, while a long, bounded stream
+    of GEMMs on another stream holds SMs when it starts."""
+    counts = np.array([2048, 0, 2048, 4096])
+    E, R, d, f = len(counts), int(counts.sum()), 512, 1024
+    offsets = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)).to(DEV)
+    Xe = I.random_bf16((R, d), 34, "Xe").to(DEV)
+    W1 = I.random_bf16((E, f, d), 34, "W1", 0.05).to(DEV)
+    W2 = I.random_bf16((E, d, f), 34, "W2", 0.05).to(DEV)
+    run = (lambda: moe.moe_expert_ffn_fused(Xe, offsets, W1, W2)[1]) if form == "fused" else None
+    if form == "pipeline":
+        cfg = I.workload("tiny")
+        inp = I.make_layer_inputs(cfg, 34, device=DEV)
+        dv = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        layer = moe.MoeLayer(dv["W1"], dv["W2"], cfg.k, cfg.score, cfg.renormalize,
+                             pipeline=True)
+        run = lambda: layer(dv["X"], logits=dv["logits"])
+    ref = run().clone()
+    torch.cuda.synchronize()
+    a = torch.randn(4096, 4096, device=DEV, dtype=torch.bfloat16)
+    side = torch.cuda.Stream(DEV)
+    outs = []
+    for _ in range(3):
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(40):  # ~40 bounded GEMMs, a few ms in all
+                a = torch.tanh(a @ a)
+        outs.append(run().clone())
+    torch.cuda.synchronize()
+    for o in outs:
+        assert same(o, ref)

@@ -109,11 +109,20 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def code_sha256(text: str) -> str:
+    """sha256 of C++/CUDA source with its comments and blank space removed:
+    the same for two versions that differ only in comments or layout."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return hashlib.sha256(" ".join(text.split()).encode()).hexdigest()
+
+
 def ncu_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it still matches the source.
+    """DRAM bytes per launch from a committed ncu summary, if it still matches the code.
 
     profiles/<kernel>_<workload>.md carries 'traffic_bytes_per_launch:' and
-    'source_sha256:' lines; a changed kernel source voids the figure.
+    'code_sha256:' lines (the grouped GEMM source's code_sha256 when the
+    counters were taken); any change to the kernel's code voids the figure.
     """
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     src = os.path.join(ROOT, "combine_moe_route_14_b200", "csrc", "grouped_gemm.cu")
@@ -121,10 +130,10 @@ def ncu_traffic(kernel: str, workload: str):
         return None
     text = open(path).read()
     mt = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    ms = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    ms = re.search(r"code_sha256:\s*([0-9a-f]{64})", text)
     if not mt or not ms:
         return None
-    if hashlib.sha256(open(src, "rb").read()).hexdigest() != ms.group(1):
+    if code_sha256(open(src).read()) != ms.group(1):
         return None
     return float(mt.group(1))
 

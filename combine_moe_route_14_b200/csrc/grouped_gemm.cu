@@ -121,13 +121,13 @@ constexpr int kMergeRows = 64;
 // the decode shapes for nothing) and at most kMergeMaxMeanRows.  With few
 // rows per expert the GEMM is bound by streaming each tile's weights and a
 // tail tile doubles that stream.  With many (the Mixtral shape, ~1024 per
-// expert) the GEMM is bound by shared-memory bandwidth at full MMA rate, the
-// tail tile's weights come from L2 beside the full tiles, and a merged tile
-// costs more than the tail tile it replaces: its second MMA reads the weight
-// stage from shared memory again, neighbouring tiles whose columns overlap
-// cannot overlap their MMAs with its epilogue, and the static schedule gives
-// the wider tiles to some clusters only.  Measured on a B200: the fine-grained
-// shape (256 rows per expert) -10 % per GEMM, 1040 rows per expert +27 %.
+// expert) the GEMM runs near its tensor rate, the tail tile's weights come
+// from L2 beside the full tiles, and a merged tile costs more than the tail
+// tile it replaces: its second, narrow MMA per K step reads the weight stage
+// again, neighbouring tiles whose columns overlap cannot overlap their MMAs
+// with its epilogue, and the static schedule gives the wider tiles to some
+// clusters only.  Measured on a B200: the fine-grained shape (256 rows per
+// expert) -10 % per GEMM, 1040 rows per expert +27 %.
 constexpr int kMergeMinMeanRows = 128;
 constexpr int kMergeMaxMeanRows = 384;
 constexpr int BN_MAX = BN + kMergeRows;      // 320 accumulator columns at most

@@ -45,22 +45,33 @@ def _fake_tree(tmp_path, src_text, recorded_sha, traffic=123456789):
     prof = tmp_path / "profiles"
     prof.mkdir()
     (prof / "grouped_gemm_gelu_mixtral.md").write_text(
-        f"# summary\n\nsource_sha256: {recorded_sha}\n\ntraffic_bytes_per_launch: {traffic}\n")
+        f"# summary\n\ncode_sha256: {recorded_sha}\n\ntraffic_bytes_per_launch: {traffic}\n")
 
 
-def test_ncu_traffic_needs_the_recorded_source(tmp_path, monkeypatch):
-    src = "// kernel source\n"
-    sha = hashlib.sha256(src.encode()).hexdigest()
-    _fake_tree(tmp_path, src, sha)
+KERNEL = "__global__ void k(int* p) {\n  p[0] = 1;  // store\n}\n"
+
+
+def test_ncu_traffic_needs_the_recorded_code(tmp_path, monkeypatch):
+    _fake_tree(tmp_path, KERNEL, bench.code_sha256(KERNEL))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.ncu_traffic("grouped_gemm_gelu", "mixtral") == 123456789.0
     assert bench.ncu_traffic("grouped_gemm_gelu", "fine_grained") is None  # no summary
 
 
-def test_ncu_traffic_is_void_once_the_kernel_changed(tmp_path, monkeypatch):
-    old = hashlib.sha256(b"// the kernel that was profiled\n").hexdigest()
-    _fake_tree(tmp_path, "// an edited kernel\n", old)
+def test_ncu_traffic_survives_comment_and_layout_edits(tmp_path, monkeypatch):
+    edited = "/* a note */\n__global__ void k(int* p)\n{\n    p[0] = 1;   // the store\n}\n"
+    _fake_tree(tmp_path, edited, bench.code_sha256(KERNEL))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("grouped_gemm_gelu", "mixtral") == 123456789.0
+
+
+def test_ncu_traffic_is_void_once_the_kernel_changed(tmp_path, monkeypatch):
+    _fake_tree(tmp_path, KERNEL.replace("p[0] = 1", "p[0] = 2"), bench.code_sha256(KERNEL))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("grouped_gemm_gelu", "mixtral") is None
+    # the raw file hash (the older record format) no longer matches either
+    _fake_tree(tmp_path / "raw", KERNEL, hashlib.sha256(KERNEL.encode()).hexdigest())
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path / "raw"))
     assert bench.ncu_traffic("grouped_gemm_gelu", "mixtral") is None
 
 

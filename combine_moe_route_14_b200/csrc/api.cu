@@ -953,7 +953,7 @@ int32_t moe_kernel_launches_per_forward(const moe_layer_desc* desc, int32_t with
   const bool ranked = !(f & MOE_LAYER_GATHER_ON_LOAD) &&
                       !(fused && (f & MOE_LAYER_FUSED_DISPATCH)) &&
                       desc->E <= moe::kRankedMaxExperts;
-  const int layout = ranked ? 0 : moe::layout_kernel_count((int64_t)desc->T * desc->k);
+  const int layout = ranked ? 0 : moe::layout_kernel_count((int64_t)desc->T * desc->k, desc->E);
   return (with_router ? 1 : 0) + 1 + layout + dispatch + gemms + combine;
 }
 
@@ -967,7 +967,7 @@ int32_t moe_kernel_launches_per_forward_fp8(const moe_layer_desc* desc, int32_t 
   // FP8 mode keeps the separate layout kernel (the bf16 count has none when
   // it ranks in the routing kernel)
   const bool ranked = !(d.flags & MOE_LAYER_GATHER_ON_LOAD) && d.E <= moe::kRankedMaxExperts;
-  const int layout = ranked ? moe::layout_kernel_count((int64_t)desc->T * desc->k) : 0;
+  const int layout = ranked ? moe::layout_kernel_count((int64_t)desc->T * desc->k, desc->E) : 0;
   return moe_kernel_launches_per_forward(&d, with_router) - dispatch + layout +
          moe::fp8_dispatch_kernel_count(desc->T);
 }

@@ -84,7 +84,7 @@ cudaError_t launch_dispatch_scatter(const void* X, const int32_t* idx, int32_t* 
 
 size_t layout_workspace_bytes(int64_t R, int E);
 // Number of kernels launch_layout issues for R slots.
-int layout_kernel_count(int64_t R);
+int layout_kernel_count(int64_t R, int E);
 cudaError_t launch_layout(const int32_t* idx, int R, int E, int32_t* counts, int32_t* offsets,
                           int32_t* row_of, int32_t* src_of, void* ws, const DeviceInfo& dev,
                           cudaStream_t stream);

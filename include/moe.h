@@ -197,7 +197,9 @@ moe_status moe_layout(const int32_t* topk_idx, int32_t T, int32_t E, int32_t k, 
  * look-back over per-tile status words (tiles taken in ticket order; every
  * wait bounded); the last tile writes counts and offsets.  A second short
  * kernel turns ranks into rows (row_of) and fills src_of.  Two launches
- * instead of three (one + two past 16384 slots), and no single-CTA pass.
+ * instead of two or three (moe_route, then one layout kernel up to 8192 slots
+ * with at most 32 experts or 4096 otherwise, two past that), and no
+ * single-CTA pass.
  *   Arguments and results as moe_route_ex and moe_layout, bit for bit.
  *   ws: at least moe_route_layout_workspace_size(T, E) bytes (look-back
  *   status words, zeroed by the call).

@@ -113,7 +113,7 @@ def test_launch_count(lib):
     d = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, 0)
     assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 1) == 6
     assert lib.moe_kernel_launches_per_forward(ctypes.byref(d), 0) == 5
-    # 256 experts: the separate layout (two kernels past 16384 slots)
+    # 256 experts: the separate layout (two kernels past 4096 slots)
     d4 = moe.LayerDesc(8192, 7168, 256, 8, 2048, 1, 1, 0)
     assert lib.moe_kernel_launches_per_forward(ctypes.byref(d4), 0) == 7
     # FP8: the separate layout kernel, absmax + dispatch
@@ -126,6 +126,12 @@ def test_launch_count(lib):
     # the pipeline: route, layout, one persistent FFN (dispatch, GEMMs, combine)
     dp = moe.LayerDesc(4096, 4096, 8, 2, 14336, 0, 1, moe.LAYER_PIPELINE)
     assert lib.moe_kernel_launches_per_forward(ctypes.byref(dp), 1) == 4
+    # the layout's one-CTA path: up to 8192 slots with at most 32 experts, 4096 otherwise
+    for T, E, one_cta in [(4096, 8, True), (4097, 8, False), (2048, 64, True), (2049, 64, False)]:
+        dl = moe.LayerDesc(T, 256, E, 2, 256, 0, 1, moe.LAYER_GATHER_ON_LOAD)
+        # router, route, layout (1 or 2), GEMM-1 (gathering), GEMM-2, combine
+        assert lib.moe_kernel_launches_per_forward(ctypes.byref(dl), 1) == (6 if one_cta else 7)
+        assert (lib.moe_layout_workspace_size(T, E, 2) == 0) == one_cta
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

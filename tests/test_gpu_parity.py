@@ -186,18 +186,21 @@ def test_router_logits_parity(T, d, E):
 LAYOUT_CASES = [
     # (T, E, k, skew)
     (256, 8, 2, 0.0),
-    (4096, 8, 2, 0.0),        # 8192 slots: one-block path
+    (4096, 8, 2, 0.0),        # 8192 slots, 8 experts: one-block path at its limit
     (4096, 8, 1, 2.5),        # skewed
-    (8192, 256, 8, 0.0),      # 65536 slots: histogram + decoupled look-back
-    (8193, 256, 2, 0.0),      # 16386 slots: just past the one-block limit, ragged last tile
+    (8192, 256, 8, 0.0),      # 65536 slots: histogram + decoupled look-back, 32 tiles
+    (8193, 256, 2, 0.0),      # 16386 slots: ragged last tile
     (20000, 7, 3, 1.0),       # several tiles, few experts
     (10, 256, 4, 0.0),        # mostly empty experts
     (3000, 1024, 16, 0.0),    # max experts and k, multi-block
     (50, 1024, 2, 0.0),
     (1, 1, 1, 0.0),
     (999, 1, 1, 0.0),
-    (5461, 16, 3, 0.0),       # 16383 slots, E = 16: one-block path near its limit
-    (4096, 12, 4, 1.5),       # 16384 slots exactly (the one-block limit), skewed
+    (5461, 16, 3, 0.0),       # 16383 slots, E = 16: multi-block, ragged last tile
+    (4096, 12, 4, 1.5),       # 16384 slots exactly, skewed
+    (2731, 32, 3, 0.0),       # 8193 slots, 32 experts: just past the one-block limit
+    (2048, 33, 2, 0.0),       # 4096 slots, 33 experts: one-block path at its limit
+    (2049, 64, 2, 0.0),       # 4098 slots, 64 experts: just past it
     (3000, 17, 2, 0.0),       # E = 17
 ]
 

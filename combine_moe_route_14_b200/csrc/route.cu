@@ -337,8 +337,18 @@ cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, in
 constexpr int kRouteWarps = 8;
 constexpr int kNoPick = 0x7fffffff;  // larger than every expert id
 
-__device__ __forceinline__ bool better(float v, int e, float bv, int be) {
-  return v > bv || (v == bv && e < be);
+// Order-preserving key of a logit for the warp-wide maximum: a larger logit
+// has a larger key, and +0 and -0 share one (they tie, as floats do).  -inf
+// and NaN, which are never chosen, have key 0, below every candidate
+// (-FLT_MAX has key 0x00800000).
+__device__ __forceinline__ uint32_t logit_key(float x) {
+  if (!(x >= -FLT_MAX)) return 0u;  // -inf or NaN
+  if (x == 0.f) x = 0.f;            // -0 -> +0
+  const uint32_t b = __float_as_uint(x);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 // One token's routing by one warp: lanes j < k get slot j's expert (or -1
@@ -348,43 +358,42 @@ __device__ __forceinline__ void route_token(const float* __restrict__ row, int E
                                             int renorm, float inv_temp, float min_prob,
                                             int lane, int& e_out, float& g_out) {
   float v[kEPL];
+  uint32_t key[kEPL];  // 0: not a candidate (past E, -inf, NaN, or taken)
 #pragma unroll
   for (int i = 0; i < kEPL; ++i) {
     const int e = lane + 32 * i;
     v[i] = (e < E) ? __ldg(row + e) : -FLT_MAX;
+    key[i] = (e < E) ? logit_key(v[i]) : 0u;
   }
-  uint32_t taken = 0;
   float my_v = 0.f;  // lane j < k: logit of slot j
   int my_e = 0;      // lane j < k: expert of slot j
 #pragma unroll
   for (int j = 0; j < kMaxTopK; ++j) {
     if (j < k) {
-      float bv = -FLT_MAX;
+      // this lane's best: the largest key, the lowest expert id among equals
+      // (ids grow with i, so a strictly larger key replaces)
+      uint32_t bk = 0u;
       int be = kNoPick;
 #pragma unroll
-      for (int i = 0; i < kEPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !((taken >> i) & 1u) && better(v[i], e, bv, be)) {
-          bv = v[i];
-          be = e;
+      for (int i = 0; i < kEPL; ++i)
+        if (key[i] > bk) {
+          bk = key[i];
+          be = lane + 32 * i;
         }
+      // the warp's largest key, then the lowest id holding it (ties -> lower id)
+      const uint32_t gk = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t ge = __reduce_min_sync(0xffffffffu,
+                                            (gk != 0u && bk == gk) ? (uint32_t)be : 0xffffffffu);
+      // no candidate left (every remaining logit is -inf or NaN): the slot
+      // keeps kNoPick and is dropped below
+      const int pick = gk != 0u ? (int)ge : kNoPick;
+      if (lane == j) {
+        my_v = gk != 0u ? key_logit(gk) : -FLT_MAX;
+        my_e = pick;
       }
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-        if (better(ov, oe, bv, be)) {
-          bv = ov;
-          be = oe;
-        }
-      }
-      // be stays kNoPick when no candidate is left (every remaining logit
-      // is -inf or NaN): the slot is dropped below
-      if (lane == j) {
-        my_v = bv;
-        my_e = be;
-      }
-      if (be < E && (be & 31) == lane) taken |= 1u << (be >> 5);
+      for (int i = 0; i < kEPL; ++i)  // taken (unrolled: key[] stays in registers)
+        if (pick == lane + 32 * i) key[i] = 0u;
     }
   }
   // Gates.  z = logit / temperature; the largest chosen logit is lane 0's.

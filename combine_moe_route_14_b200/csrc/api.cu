@@ -155,7 +155,7 @@ cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 // Workspace of the fused forward: sub-buffers, each 256-byte aligned.
 struct LayerWs {
   size_t logits, idx, gates, counts, offsets, row_of, src_of, layout, Xe, H, Ye, scale, ctr, part,
-      lb, total;
+      lb, lpart, total;
 };
 
 // Counter words of the layer workspace (all zeroed by one memset per forward):
@@ -202,6 +202,10 @@ LayerWs layer_ws(const moe_layer_desc& d) {
                                      moe::combine_counter_words(d.T, d.d)) * sizeof(uint32_t));
   w.part = o;    o += up256(T * d.d * sizeof(float));  // fused combine: fp32 partial rows
   w.lb = o;      o += up256(moe::route_rank_lookback_words(d.T, d.E) * sizeof(uint32_t));
+  // split router's partial logits (small batches on the ranked path)
+  w.lpart = o;
+  if (d.T <= moe::kSplitMaxT && d.E <= moe::kRankedMaxExperts)
+    o += up256((size_t)moe::router_split_count(d.d) * T * d.E * sizeof(float));
   w.total = o;
   return w;
 }
@@ -300,9 +304,24 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   const bool ranked = !gather && !fdisp && !fp8 && d.E <= moe::kRankedMaxExperts;
   uint32_t* lb = reinterpret_cast<uint32_t*>(base + w.lb);
 
+  // The ranked routing's look-back words start at zero in every forward: the
+  // router kernel clears them as a side job, or a memset when the logits are
+  // given.  Small batches (up to 32 experts) take the split router, whose
+  // partial logits the routing kernel sums; every form of the layer does, so
+  // the forms route on the same logits.
+  const int lb_words = ranked ? (int)moe::route_rank_lookback_words(d.T, d.E) : 0;
+  const bool split = Wr && d.T <= moe::kSplitMaxT && d.E <= moe::kRankedMaxExperts;
+  const int nsplit = split ? moe::router_split_count(d.d) : 1;
+  const float* Lr = split ? reinterpret_cast<const float*>(base + w.lpart) : L;
   if (Wr) {
     MOE_STAGE("moe.router_logits");
-    MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, *dev, s), "router_logits");
+    if (split)
+      MOE_CUDA(moe::launch_router_split(X, Wr, d.T, d.d, d.E, const_cast<float*>(Lr), *dev, s,
+                                        lb, lb_words),
+               "router_split");
+    else
+      MOE_CUDA(moe::launch_router_logits(X, Wr, d.T, d.d, d.E, L, *dev, s, lb, lb_words),
+               "router_logits");
   }
   // The routing kernel also clears the tickets, readiness and combine
   // counters (they start at zero in every forward) and, with the combine in
@@ -311,20 +330,19 @@ moe_status layer_forward(const moe_layer_desc* desc, const void* X, const float*
   const bool drops = d.min_prob > 0.f;
   if (ranked) {
     MOE_STAGE("moe.route");
-    MOE_CUDA(cudaMemsetAsync(lb, 0, moe::route_rank_lookback_words(d.T, d.E) * sizeof(uint32_t),
-                             s),
-             "memset look-back");
-    MOE_CUDA(moe::launch_route_rank(L, d.T, d.E, d.k, d.score, d.renormalize,
+    if (!Wr)
+      MOE_CUDA(cudaMemsetAsync(lb, 0, (size_t)lb_words * sizeof(uint32_t), s), "memset look-back");
+    MOE_CUDA(moe::launch_route_rank(Lr, d.T, d.E, d.k, d.score, d.renormalize,
                                     desc_temperature(d), d.min_prob, idx, gates, row_of, counts,
                                     offsets, lb, *dev, s, (comb && drops) ? Y : nullptr, d.d, ctr,
-                                    lc.used),
+                                    lc.used, nsplit),
              "route_rank");
   } else {
     {
       MOE_STAGE("moe.route");
-      MOE_CUDA(moe::launch_route(L, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
+      MOE_CUDA(moe::launch_route(Lr, d.T, d.E, d.k, d.score, d.renormalize, desc_temperature(d),
                                  d.min_prob, idx, gates, s, (comb && drops) ? Y : nullptr, d.d,
-                                 ctr, lc.used),
+                                 ctr, lc.used, nsplit),
                "route");
     }
     MOE_STAGE("moe.layout");

@@ -54,15 +54,17 @@ struct DeviceInfo {
 // the message in *err.
 const DeviceInfo* current_device_info(std::string* err);
 
+// zero_words (optional): n_zero_words words cleared by the same launch.
 cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, int E, float* L,
-                                 const DeviceInfo& dev, cudaStream_t stream);
+                                 const DeviceInfo& dev, cudaStream_t stream,
+                                 uint32_t* zero_words = nullptr, int n_zero_words = 0);
 
 // zero_rows (optional): [T, zero_d] bf16 rows zeroed for tokens with no kept slot.
 // zero_words (optional): n_zero_words counter words cleared by the same launch.
 cudaError_t launch_route(const float* L, int T, int E, int k, int score, int renormalize,
                          float temperature, float min_prob, int32_t* idx, float* gates,
                          cudaStream_t stream, void* zero_rows = nullptr, int zero_d = 0,
-                         uint32_t* zero_words = nullptr, int n_zero_words = 0);
+                         uint32_t* zero_words = nullptr, int n_zero_words = 0, int nsplit = 1);
 
 // Routing fused with the layout's ranking (see route.cu): idx, gates, the
 // stable rank of each kept slot within its expert (into rank[], -1 for a
@@ -70,12 +72,19 @@ cudaError_t launch_route(const float* L, int T, int E, int k, int score, int ren
 // E) words, zeroed before the launch.
 size_t route_rank_lookback_words(int T, int E);
 constexpr int kRankedMaxExperts = 32;  // the layer ranks in its routing kernel up to this E
+// Split router (small batches, ranked path): partial logits P[s][T][E] over
+// router_split_count(d) column slices, summed by the routing kernel.
+constexpr int kSplitMaxT = 64;
+int router_split_count(int d);
+cudaError_t launch_router_split(const void* X, const void* Wr, int T, int d, int E, float* P,
+                                const DeviceInfo& dev, cudaStream_t stream,
+                                uint32_t* zero_words = nullptr, int n_zero_words = 0);
 cudaError_t launch_route_rank(const float* L, int T, int E, int k, int score, int renormalize,
                               float temperature, float min_prob, int32_t* idx, float* gates,
                               int32_t* rank, int32_t* counts, int32_t* offsets, uint32_t* lookback,
                               const DeviceInfo& dev, cudaStream_t stream, void* zero_rows = nullptr,
                               int zero_d = 0, uint32_t* zero_words = nullptr,
-                              int n_zero_words = 0);
+                              int n_zero_words = 0, int nsplit = 1);
 // Token-ordered dispatch finishing the layout from route_rank's ranks
 // (row_of holds the ranks on entry and the rows on return; src_of written).
 cudaError_t launch_dispatch_scatter(const void* X, const int32_t* idx, int32_t* row_of,

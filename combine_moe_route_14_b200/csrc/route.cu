@@ -103,8 +103,12 @@ __device__ __forceinline__ bool router_warp_wait(uint64_t* bar, uint32_t parity,
 template <int kG, bool kWs>
 __global__ void __launch_bounds__(kRouterThreads, kG == 1 ? 2 : 1)
     router_logits_kernel(const uint8_t* __restrict__ X, const uint4* __restrict__ Wr, int T,
-                         int d, int E, float* __restrict__ L, uint32_t* status) {
+                         int d, int E, float* __restrict__ L, uint32_t* status,
+                         uint32_t* __restrict__ zero_words, int n_zero_words) {
   pdl_wait_and_release();
+  // side job: clear the next kernel's counter words (saves a memset launch)
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero_words; i += gridDim.x * blockDim.x)
+    zero_words[i] = 0u;
   static_assert(!kWs || kG == 1, "Wr is staged for one n-tile only");
   extern __shared__ __align__(128) uint8_t smem_r[];
   uint8_t* ring = smem_r;
@@ -277,7 +281,8 @@ struct RouterSlot {
 static RouterSlot g_router[64];
 
 cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, int E, float* L,
-                                 const DeviceInfo& dev, cudaStream_t stream) {
+                                 const DeviceInfo& dev, cudaStream_t stream, uint32_t* zero_words,
+                                 int n_zero_words) {
   if (T == 0) return cudaSuccess;
   const int ntiles = (E + 7) / 8;
   const int gmax = ntiles < kRouterGroup ? ntiles : kRouterGroup;  // n-tiles per pass
@@ -310,13 +315,111 @@ cudaError_t launch_router_logits(const void* X, const void* Wr, int T, int d, in
   const uint4* w = static_cast<const uint4*>(Wr);
   if (ws)
     launch_kernel(router_logits_kernel<1, true>, dim3(blocks), dim3(kRouterThreads), smem, stream,
-                  x, w, T, d, E, L, dev.status);
+                  x, w, T, d, E, L, dev.status, zero_words, n_zero_words);
   else if (gmax == 1)
     launch_kernel(router_logits_kernel<1, false>, dim3(blocks), dim3(kRouterThreads), smem,
-                  stream, x, w, T, d, E, L, dev.status);
+                  stream, x, w, T, d, E, L, dev.status, zero_words, n_zero_words);
   else
     launch_kernel(router_logits_kernel<kRouterGroup, false>, dim3(blocks), dim3(kRouterThreads),
-                  smem, stream, x, w, T, d, E, L, dev.status);
+                  smem, stream, x, w, T, d, E, L, dev.status, zero_words, n_zero_words);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Split router for small batches (T <= kSplitMaxT, E <= 32): the router
+// linear over column slices of kSplitCols, one CTA per slice, each writing
+// its partial logits P[s][t][e]; the routing kernel adds the partials of a
+// logit in slice order (deterministic).  With a handful of tokens the whole
+// router is one CTA streaming X and Wr (two DRAM round trips and a reduction
+// in one SM); split, every slice's bytes arrive at once.  The sums are fp32
+// in a different order from router_logits_kernel, so the logits may differ
+// in the last bits.
+//   A CTA stages the slice of X (T rows, zero-padded to 64) and of Wr (E rows,
+// zero-padded to 32) in shared memory, rows padded by 16 bytes so that a
+// quarter-warp's 8 rows fall in distinct banks, and 8 warps take the
+// (16-token, 8-expert) tiles with mma.sync m16n8k16 over the slice.
+// ---------------------------------------------------------------------------
+constexpr int kSplitCols = 256;                       // bf16 columns per slice
+constexpr int kSplitWords = kSplitCols / 2 + 4;       // 32-bit words per staged row (+16 B)
+constexpr int kSplitRowsX = kSplitMaxT;               // 64
+constexpr int kSplitRowsW = 32;
+constexpr size_t kSplitSmem = (size_t)(kSplitRowsX + kSplitRowsW) * kSplitWords * 4;
+
+__global__ void __launch_bounds__(256)
+    router_split_kernel(const uint4* __restrict__ X, const uint4* __restrict__ Wr, int T, int d,
+                        int E, float* __restrict__ P, uint32_t* __restrict__ zero_words,
+                        int n_zero_words) {
+  pdl_wait_and_release();
+  extern __shared__ uint32_t sw[];
+  uint32_t* xs = sw;                                // [64][kSplitWords]
+  uint32_t* ws = sw + kSplitRowsX * kSplitWords;    // [32][kSplitWords]
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n_zero_words; i += gridDim.x * blockDim.x)
+    zero_words[i] = 0u;
+  const int s = blockIdx.x;
+  const int c0 = s * kSplitCols;
+  const int nvec = min(kSplitCols, d - c0) / 8;     // 16-byte vectors of a row in this slice
+  const int row_vecs = d / 8;
+  constexpr int kVecs = kSplitCols / 8;             // 32
+  for (int i = threadIdx.x; i < (kSplitRowsX + kSplitRowsW) * kVecs; i += blockDim.x) {
+    const int r = i / kVecs, v = i - r * kVecs;
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (r < kSplitRowsX) {
+      if (r < T && v < nvec) val = __ldg(X + (size_t)r * row_vecs + c0 / 8 + v);
+      *reinterpret_cast<uint4*>(xs + r * kSplitWords + v * 4) = val;
+    } else {
+      const int e = r - kSplitRowsX;
+      if (e < E && v < nvec) val = __ldg(Wr + (size_t)e * row_vecs + c0 / 8 + v);
+      *reinterpret_cast<uint4*>(ws + e * kSplitWords + v * 4) = val;
+    }
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntt = (T + 15) / 16, nte = (E + 7) / 8;
+  for (int tile = warp; tile < ntt * nte; tile += 8) {
+    const int tt = tile / nte, te = tile - tt * nte;
+    const int ra = tt * 16 + (lane >> 2), rb = te * 8 + (lane >> 2);
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int kk = 0; kk < kSplitCols / 16; ++kk) {
+      // A (16 x 16, row-major): rows ra and ra + 8, k pairs (lane%4)*2 and +8;
+      // B (16 x 8, column-major = Wr rows): expert rb, the same k pairs
+      const int w0 = kk * 8 + (lane & 3);
+      const uint32_t a0 = xs[ra * kSplitWords + w0], a1 = xs[(ra + 8) * kSplitWords + w0];
+      const uint32_t a2 = xs[ra * kSplitWords + w0 + 4], a3 = xs[(ra + 8) * kSplitWords + w0 + 4];
+      const uint32_t b0 = ws[rb * kSplitWords + w0], b1 = ws[rb * kSplitWords + w0 + 4];
+      mma_bf16_16816(c, a0, a1, a2, a3, b0, b1);
+    }
+    // c[0], c[1]: token ra, experts te*8 + (lane%4)*2 + {0, 1}; c[2], c[3]: token ra + 8
+    const int e0 = te * 8 + (lane & 3) * 2;
+    float* out = P + (size_t)s * T * E;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int t = ra + 8 * h;
+      if (t < T) {
+        if (e0 < E) out[(size_t)t * E + e0] = c[2 * h];
+        if (e0 + 1 < E) out[(size_t)t * E + e0 + 1] = c[2 * h + 1];
+      }
+    }
+  }
+}
+
+int router_split_count(int d) { return (d + kSplitCols - 1) / kSplitCols; }
+
+static RouterSlot g_router_split[64];
+
+cudaError_t launch_router_split(const void* X, const void* Wr, int T, int d, int E, float* P,
+                                const DeviceInfo& dev, cudaStream_t stream,
+                                uint32_t* zero_words, int n_zero_words) {
+  if (T == 0) return cudaSuccess;
+  RouterSlot& rs = g_router_split[dev.device & 63];
+  std::call_once(rs.once, [&] {
+    rs.err = cudaFuncSetAttribute(router_split_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSplitSmem);
+  });
+  if (rs.err != cudaSuccess) return rs.err;
+  launch_kernel(router_split_kernel, dim3(router_split_count(d)), dim3(256), kSplitSmem, stream,
+                static_cast<const uint4*>(X), static_cast<const uint4*>(Wr), T, d, E, P,
+                zero_words, n_zero_words);
   return cudaGetLastError();
 }
 
@@ -354,15 +457,23 @@ __device__ __forceinline__ float key_logit(uint32_t key) {
 // One token's routing by one warp: lanes j < k get slot j's expert (or -1
 // when the slot is dropped) and its gate.  Every lane must call it.
 template <int kEPL>
+// The token's logits are row[e], or with nsplit > 1 the sum over s in order
+// of the partial logits row[s * split_stride + e] (the split router's).
 __device__ __forceinline__ void route_token(const float* __restrict__ row, int E, int k, int score,
                                             int renorm, float inv_temp, float min_prob,
-                                            int lane, int& e_out, float& g_out) {
+                                            int lane, int& e_out, float& g_out, int nsplit = 1,
+                                            size_t split_stride = 0) {
   float v[kEPL];
   uint32_t key[kEPL];  // 0: not a candidate (past E, -inf, NaN, or taken)
 #pragma unroll
   for (int i = 0; i < kEPL; ++i) {
     const int e = lane + 32 * i;
-    v[i] = (e < E) ? __ldg(row + e) : -FLT_MAX;
+    float x = -FLT_MAX;
+    if (e < E) {
+      x = __ldg(row + e);
+      for (int sp = 1; sp < nsplit; ++sp) x += __ldg(row + (size_t)sp * split_stride + e);
+    }
+    v[i] = x;
     key[i] = (e < E) ? logit_key(v[i]) : 0u;
   }
   float my_v = 0.f;  // lane j < k: logit of slot j
@@ -446,7 +557,7 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
     route_topk_kernel(const float* __restrict__ L, int T, int E, int k, int score, int renorm,
                       float inv_temp, float min_prob, int32_t* __restrict__ idx,
                       float* __restrict__ gates, uint4* __restrict__ zero_rows, int zero_vecs,
-                      uint32_t* __restrict__ zero_words, int n_zero_words) {
+                      uint32_t* __restrict__ zero_words, int n_zero_words, int nsplit) {
   pdl_wait_and_release();
   // side job: clear the caller's counter words (grid-stride; the layer's
   // later kernels run after this one on the same stream)
@@ -460,7 +571,8 @@ __global__ void __launch_bounds__(kRouteWarps * 32)
   if (t >= T) return;
   int e;
   float g;
-  route_token<kEPL>(L + (size_t)t * E, E, k, score, renorm, inv_temp, min_prob, lane, e, g);
+  route_token<kEPL>(L + (size_t)t * E, E, k, score, renorm, inv_temp, min_prob, lane, e, g, nsplit,
+                    (size_t)T * E);
   if (lane < k) {
     idx[(size_t)t * k + lane] = e;
     gates[(size_t)t * k + lane] = g;
@@ -502,7 +614,7 @@ __global__ void __launch_bounds__(rank_warps(kEPL) * 32)
                       int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                       uint32_t* __restrict__ lookback, uint4* __restrict__ zero_rows,
                       int zero_vecs, uint32_t* __restrict__ zero_words, int n_zero_words,
-                      uint32_t* status) {
+                      uint32_t* status, int nsplit) {
   pdl_wait_and_release();
   constexpr int kRankWarps = rank_warps(kEPL);
   constexpr int kRankTile = kRankWarps;  // one token per warp
@@ -532,7 +644,8 @@ __global__ void __launch_bounds__(rank_warps(kEPL) * 32)
     int e = -1;
     float g = 0.f;
     if (t < T) {
-      route_token<kEPL>(L + (size_t)t * E, E, k, score, renorm, inv_temp, min_prob, lane, e, g);
+      route_token<kEPL>(L + (size_t)t * E, E, k, score, renorm, inv_temp, min_prob, lane, e, g,
+                        nsplit, (size_t)T * E);
       if (lane < k) {
         idx[(size_t)t * k + lane] = e;
         gates[(size_t)t * k + lane] = g;
@@ -639,7 +752,7 @@ __global__ void __launch_bounds__(rank_warps(kEPL) * 32)
 cudaError_t launch_route(const float* L, int T, int E, int k, int score, int renormalize,
                          float temperature, float min_prob, int32_t* idx, float* gates,
                          cudaStream_t stream, void* zero_rows, int zero_d, uint32_t* zero_words,
-                         int n_zero_words) {
+                         int n_zero_words, int nsplit) {
   if (T == 0) return cudaSuccess;
   const int blocks = (T + kRouteWarps - 1) / kRouteWarps;
   const int epl = (E + 31) / 32;
@@ -647,7 +760,7 @@ cudaError_t launch_route(const float* L, int T, int E, int k, int score, int ren
 #define MOE_ROUTE_LAUNCH(N)                                                                    \
   launch_kernel(route_topk_kernel<N>, dim3(blocks), dim3(kRouteWarps * 32), 0, stream, L, T, E,  \
                 k, score, renormalize, inv_temp, min_prob, idx, gates,                           \
-                static_cast<uint4*>(zero_rows), zero_d / 8, zero_words, n_zero_words)
+                static_cast<uint4*>(zero_rows), zero_d / 8, zero_words, n_zero_words, nsplit)
   if (epl <= 1) MOE_ROUTE_LAUNCH(1);
   else if (epl <= 2) MOE_ROUTE_LAUNCH(2);
   else if (epl <= 4) MOE_ROUTE_LAUNCH(4);
@@ -662,7 +775,7 @@ cudaError_t launch_route_rank(const float* L, int T, int E, int k, int score, in
                               float temperature, float min_prob, int32_t* idx, float* gates,
                               int32_t* rank, int32_t* counts, int32_t* offsets, uint32_t* lookback,
                               const DeviceInfo& dev, cudaStream_t stream, void* zero_rows,
-                              int zero_d, uint32_t* zero_words, int n_zero_words) {
+                              int zero_d, uint32_t* zero_words, int n_zero_words, int nsplit) {
   if (T == 0) return cudaSuccess;
   const int blocks = route_rank_tiles(T, E);
   const int epl = (E + 31) / 32;
@@ -672,7 +785,7 @@ cudaError_t launch_route_rank(const float* L, int T, int E, int k, int score, in
   launch_kernel(route_rank_kernel<N>, dim3(blocks), dim3(rank_warps(N) * 32), smem, stream, L, T, \
                 E, k, score, renormalize, inv_temp, min_prob, idx, gates, rank, counts, offsets, \
                 lookback, static_cast<uint4*>(zero_rows), zero_d / 8, zero_words, n_zero_words,  \
-                dev.status)
+                dev.status, nsplit)
   if (epl <= 1) MOE_RANK_LAUNCH(1);
   else if (epl <= 2) MOE_RANK_LAUNCH(2);
   else if (epl <= 4) MOE_RANK_LAUNCH(4);

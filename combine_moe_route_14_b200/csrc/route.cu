@@ -471,7 +471,16 @@ __device__ __forceinline__ void route_token(const float* __restrict__ row, int E
     float x = -FLT_MAX;
     if (e < E) {
       x = __ldg(row + e);
-      for (int sp = 1; sp < nsplit; ++sp) x += __ldg(row + (size_t)sp * split_stride + e);
+      // partials 1 .. nsplit-1, eight loads in flight, added in slice order
+      for (int s0 = 1; s0 < nsplit; s0 += 8) {
+        float p[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          p[u] = s0 + u < nsplit ? __ldg(row + (size_t)(s0 + u) * split_stride + e) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (s0 + u < nsplit) x += p[u];
+      }
     }
     v[i] = x;
     key[i] = (e < E) ? logit_key(v[i]) : 0u;

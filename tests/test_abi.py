@@ -198,3 +198,19 @@ def test_host_batches_reject_bad_arguments(lib):
     assert lib.moe_layer_forward_host(*args(2, arr, arr, N, arr, need - 1)) == INVALID
     assert "workspace" in _err(lib)
     assert lib.moe_layer_forward_host(*args(0, N, N, N, N, 0)) == OK  # nothing to do
+
+
+def test_workspace_holds_the_split_routers_partial_logits(lib):
+    """At T <= 64 with up to 32 experts the layer's router writes one partial
+    logit per 256-column slice (summed by the routing kernel), so the
+    workspace holds slices * T * E floats there and not past either limit."""
+    def ws(T, d, E):
+        return lib.moe_workspace_size(ctypes.byref(moe.LayerDesc(T, d, E, 2, 256, 0, 1, 0)))
+    part = 16 * 64 * 32 * 4  # d = 4096: 16 slices, 64 tokens, 32 experts
+    # a 33rd expert adds a few hundred bytes of per-expert data but drops the partials
+    assert part - 4096 < ws(64, 4096, 32) - ws(64, 4096, 33) <= part
+    # a 65th token adds one token's buffers like a 64th does, but drops the
+    # 16 * 64 * 8 floats of partials of an 8-expert layer
+    step64 = ws(64, 4096, 8) - ws(63, 4096, 8)
+    step65 = ws(65, 4096, 8) - ws(64, 4096, 8)
+    assert abs((step64 - step65) - 16 * 64 * 8 * 4) <= 4096
